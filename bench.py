@@ -1,0 +1,420 @@
+"""Throughput of the gated delta-rule recurrence on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One "step" is one chunked prefill (decay, grams, UT solve, WY factors, the
+sequential state pass and the output/final-state write) of the H = 16,
+d = 128, T = 8192 workload: B = 8 sequences, per-channel decay, decoupled
+per-channel erase and write gates, bf16 inputs, float32 state with a random
+N(0, 0.1) initial state.  `value` is tokens/s (B*T per step) over all ranks.
+The same line carries the decode step's HBM bandwidth (batch 256, H = 32,
+d = 128, float32 state read and written in place), the roofline fraction of
+the prefill kernel, the float64 oracle's throughput on this host, the
+end-to-end figure through host buffers, and the SM clocks seen while timing.
+
+Under torchrun each rank runs its own B = 8 batch (weak scaling, no
+collective on the data path); the barrier and the max-over-ranks timing use
+torch.distributed.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PREFILL = "gdn2_bf16"
+DECODE = "decode_bf16"
+METRIC = "gated delta-rule tokens/s at H=16,d=128,T=8k; % of roofline; decode GB/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def prefill_bytes(wl) -> int:
+    """Algorithmic HBM bytes of one prefill: every input read once, o written
+    once, s0 read and S_T written once (no intermediates)."""
+    e = 2 if wl.dtype == "bf16" else 4
+    th = wl.B * wl.T * wl.H
+    per_th = e * (2 * wl.dk + wl.dv)                         # q, k, v
+    per_th += e * (wl.dk if wl.decay == "vector" else 1)       # a
+    per_th += e * (wl.dk if wl.erase == "vector" else 1)       # b
+    if wl.write != "shared":
+        per_th += e * (wl.dv if wl.write == "vector" else 1)   # w
+    per_th += e * wl.dv                                        # o
+    state = 4 * wl.B * wl.H * wl.dk * wl.dv
+    return th * per_th + state * (2 if wl.random_s0 else 1)
+
+
+def prefill_flops(wl) -> int:
+    """Tensor-core flops of the chunked form per token-head, counted 2mnk:
+    8 d^2 + 16 C d + C^2 with decoupled vector gates."""
+    d, C = wl.dk, wl.chunk
+    return wl.B * wl.T * wl.H * (8 * d * d + 16 * C * d + C * C)
+
+
+def decode_bytes(wl) -> int:
+    e = 2 if wl.dtype == "bf16" else 4
+    per = 8 * wl.dk * wl.dv + e * (4 * wl.dk + 3 * wl.dv)
+    return wl.B * wl.H * per
+
+
+class ClockSampler:
+    """nvidia-smi SM clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="gdr_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        names = ["active_mask", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i in range(1, 5)
+                          if r[3][i].lower() in ("active", "1")})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "samples": len(rows),
+                "samples_under_load": len(loaded), "reasons": reasons}
+
+
+# --------------------------------------------------------------- the oracle arm
+
+def oracle_throughput(wl, seed: int, target_s: float = 10.0):
+    """float64 oracle on a bounded sample of the prefill workload: every
+    (b, h) of the batch over the first T_s tokens, T_s sized for about
+    `target_s` seconds.  Returns (tokens/s, cores, sample description)."""
+    import oracle
+    from gated_delta_rule_154_b200 import workload as W
+
+    cores = oracle.max_threads()
+    cal = wl.replace(T=64)
+    x = W.make_prefill(cal, seed=seed)
+    f = lambda k: W.as_f32(x[k], wl.dtype)
+    t = time.perf_counter()
+    oracle.forward(f("q"), f("k"), f("v"), f("a"), f("b"),
+                   f("w") if x["w"] is not None else f("b"), x["s0"])
+    per_tok = (time.perf_counter() - t) / cal.T
+    Ts = int(max(64, min(wl.T, round(target_s / max(per_tok, 1e-9)))))
+    sub = wl.replace(T=Ts)
+    x = W.make_prefill(sub, seed=seed)
+    f = lambda k: W.as_f32(x[k], wl.dtype)
+    t = time.perf_counter()
+    oracle.forward(f("q"), f("k"), f("v"), f("a"), f("b"),
+                   f("w") if x["w"] is not None else f("b"), x["s0"])
+    dt = time.perf_counter() - t
+    sample = "all %d (b,h) pairs x first %d of %d tokens (%d token-heads), float64" % (
+        wl.B * wl.H, Ts, wl.T, wl.B * wl.H * Ts)
+    return wl.B * Ts / dt, cores, sample, dt
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from gated_delta_rule_154_b200 import workload as W
+    wl = W.WORKLOADS[PREFILL]
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, cores, sample, dt = oracle_throughput(wl, seed=0, target_s=args.ref_seconds)
+        if i >= args.warmup:
+            vals.append((v, dt))
+    value = statistics.median(v for v, _ in vals)
+    ms = statistics.median(dt for _, dt in vals) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "%s: B=%d T=%d H=%d dk=dv=%d chunk=%d, bf16 inputs (exact in f64)"
+                   % (wl.name, wl.B, wl.T, wl.H, wl.dk, wl.chunk)},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ the GPU arm
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from gated_delta_rule_154_b200 import api
+    from gated_delta_rule_154_b200 import workload as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks, peak_src = load_peaks()
+    wl = W.WORKLOADS[PREFILL]
+    if args.T:
+        wl = wl.replace(T=args.T)
+    inp = W.make_prefill(wl, seed=rank)
+
+    def dev_t(x, dtype):
+        if x is None:
+            return None
+        if dtype == "bf16":
+            return torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(dev)
+
+    d = {k: dev_t(inp[k], wl.dtype) for k in ("q", "k", "v", "a", "b", "w")}
+    d["s0"] = dev_t(inp["s0"], "f32")
+    o = torch.empty((wl.B, wl.T, wl.H, wl.dv), dtype=d["q"].dtype, device=dev)
+    sT = torch.empty((wl.B, wl.H, wl.dk, wl.dv), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        api.forward_chunked(d["q"], d["k"], d["v"], d["a"], d["b"], d["w"], d["s0"],
+                            chunk=wl.chunk, out=o, s_final=sT, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize()
+    if api.last_device_error(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    clk = clocks.summary()
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    ms_step = total_ms / args.steps
+    if api.last_device_error(stream) != 0:
+        raise RuntimeError("device error during the timed region")
+
+    tokens_step = wl.B * wl.T * world
+    value = tokens_step / (ms_step * 1e-3)
+    alg_bytes = prefill_bytes(wl)
+    avg_launch_s = statistics.mean(launch_ms) * 1e-3
+    achieved = alg_bytes / avg_launch_s / 1e9
+    hbm_peak = float(peaks["hbm_gbs"])
+    flops = prefill_flops(wl)
+    t_tc = flops / (float(peaks["bf16_tflops"]) * 1e12)
+
+    # ---- end to end through host buffers: pinned host inputs -> device ->
+    # the library call -> o and S_T back to pinned host memory, every step.
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in d.items()}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    s_host = torch.empty(sT.shape, dtype=sT.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = o_host.numel() * o_host.element_size() + s_host.numel() * s_host.element_size()
+    scratch = {k: (None if v is None else torch.empty_like(v)) for k, v in d.items()}
+
+    def e2e_step():
+        for k, v in host.items():
+            if v is not None:
+                scratch[k].copy_(v, non_blocking=True)
+        api.forward_chunked(scratch["q"], scratch["k"], scratch["v"], scratch["a"],
+                            scratch["b"], scratch["w"], scratch["s0"], chunk=wl.chunk,
+                            out=o, s_final=sT, stream=stream)
+        o_host.copy_(o, non_blocking=True)
+        s_host.copy_(sT, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    with torch.cuda.stream(stream):
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1)) / e2e_steps
+    del scratch, host
+
+    # ---- decode: batch 256, H = 32, d = 128, float32 state in place
+    dec = None
+    if not args.no_decode:
+        dwl = W.WORKLOADS[DECODE]
+        state = torch.from_numpy(W.make_decode_state(dwl, seed=rank)).to(dev)
+        pool = []
+        for s in range(1, args.decode_pool + 1):
+            x = W.make_decode_step(dwl, s, seed=rank)
+            pool.append({k: dev_t(x[k], dwl.dtype) for k in ("q", "k", "v", "a", "b", "w")})
+        od = torch.empty((dwl.B, dwl.H, dwl.dv), dtype=torch.bfloat16, device=dev)
+
+        def dstep(i):
+            p = pool[i % len(pool)]
+            api.decode_step(p["q"], p["k"], p["v"], p["a"], p["b"], p["w"], state, out=od,
+                            stream=stream)
+
+        with torch.cuda.stream(stream):
+            for i in range(10):
+                dstep(i)
+            torch.cuda.synchronize()
+            barrier()
+            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            d0.record(stream)
+            for i in range(args.decode_steps):
+                dstep(i)
+            d1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+        dms = max_over_ranks(d0.elapsed_time(d1)) / args.decode_steps
+        if api.last_device_error(stream) != 0:
+            raise RuntimeError("device error during decode timing")
+        gbs = decode_bytes(dwl) / (dms * 1e-3) / 1e9
+        dec = {"workload": "%s: batch %d, H=%d, dk=dv=%d, bf16 inputs, f32 state in place"
+                           % (dwl.name, dwl.B, dwl.H, dwl.dk),
+               "steps": args.decode_steps, "us_per_step": dms * 1e3,
+               "GB/s": gbs, "frac_of_hbm": gbs / hbm_peak,
+               "bytes_per_step": decode_bytes(dwl),
+               "tokens/s": dwl.B * world / (dms * 1e-3)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample, _ = oracle_throughput(wl, seed=0, target_s=args.ref_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": sample}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "%s: B=%d T=%d H=%d dk=dv=%d chunk=%d, per-channel decay, "
+                               "decoupled vector erase/write gates, s0~N(0,0.1)"
+                               % (wl.name, wl.B, wl.T, wl.H, wl.dk, wl.chunk),
+                   "global_batch": wl.B * world, "seq_len": wl.T, "heads": wl.H,
+                   "parallelism": "dp%d (independent sequences per rank)" % world,
+                   "l2": "inputs (%.2f GB per rank) larger than L2" % (alg_bytes / 1e9)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None,
+                     "peak_source": "%s hbm_gbs" % peak_src,
+                     "algorithmic_bytes_per_launch": alg_bytes,
+                     "tensor_flops_per_launch": flops,
+                     "t_tensor_min_us": t_tc * 1e6,
+                     "t_hbm_min_us": alg_bytes / (hbm_peak * 1e9) * 1e6},
+        "decode": dec,
+        "e2e": {"value": tokens_step / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "cpu_baseline": cpu,
+        "gpu_launches": args.steps * 1,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--T", type=int, default=0, help="override the sequence length")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--decode-pool", type=int, default=2)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,150 @@
+"""torch-facing calls of the gated delta-rule library.
+
+Argument marshalling only: every step of the recurrence runs in libgdr.so's
+CUDA kernels.  torch supplies device memory and the current stream.
+
+Shapes (row-major, contiguous, on one CUDA device):
+    prefill  q, k [B, T, H, dk]; v [B, T, H, dv]; a, b [B, T, H, dk] or
+             [B, T, H] (scalar gate) or None (gate == 1); w [B, T, H, dv] or
+             [B, T, H] or None; s0 [B, H, dk, dv] float32 or None (zeros)
+    decode   the same without the T axis; state [B, H, dk, dv] float32,
+             updated in place
+q, k, v, the gates and o share one dtype (torch.float32 or torch.bfloat16).
+"""
+
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+
+_DT = {torch.float32: _lib.F32, torch.bfloat16: _lib.BF16}
+
+
+def _ptr(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _check(t: Optional[torch.Tensor], name: str, dtype, device, shapes):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+    if t.dtype != dtype:
+        raise ValueError("%s has dtype %s, expected %s" % (name, t.dtype, dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if tuple(t.shape) not in [tuple(s) for s in shapes]:
+        raise ValueError("%s has shape %s, expected one of %s" % (name, tuple(t.shape), shapes))
+
+
+def _gate_kind(g: Optional[torch.Tensor], ndim_vector: int) -> int:
+    if g is None:
+        return _lib.GATE_ONE
+    return _lib.GATE_VECTOR if g.dim() == ndim_vector else _lib.GATE_SCALAR
+
+
+def make_desc(B, T, H, dk, dv, chunk, dtype, a_kind, b_kind, w_kind) -> _lib.GdrDesc:
+    return _lib.GdrDesc(B, T, H, dk, dv, chunk, dtype, a_kind, b_kind, w_kind)
+
+
+def desc_for(q, v, a, b, w, chunk: int = 64, decode: bool = False) -> _lib.GdrDesc:
+    if decode:
+        B, H, dk = q.shape
+        T = 1
+        nd = 3
+    else:
+        B, T, H, dk = q.shape
+        nd = 4
+    dv = v.shape[-1]
+    return make_desc(B, T, H, dk, dv, chunk, _DT[q.dtype], _gate_kind(a, nd),
+                     _gate_kind(b, nd), _gate_kind(w, nd))
+
+
+def workspace_size(desc: _lib.GdrDesc) -> int:
+    return _lib.workspace_size(desc)
+
+
+def forward_chunked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                    a: Optional[torch.Tensor] = None, b: Optional[torch.Tensor] = None,
+                    w: Optional[torch.Tensor] = None, s0: Optional[torch.Tensor] = None,
+                    *, chunk: int = 64, out: Optional[torch.Tensor] = None,
+                    s_final: Optional[torch.Tensor] = None, return_final: bool = True,
+                    workspace: Optional[torch.Tensor] = None,
+                    stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Causal chunked prefill.  Returns (o [B, T, H, dv], S_T [B, H, dk, dv] or None)."""
+    if q.dtype not in _DT:
+        raise ValueError("q must be float32 or bfloat16")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    _check(q, "q", dt, dev, [(B, T, H, dk)])
+    _check(k, "k", dt, dev, [(B, T, H, dk)])
+    _check(v, "v", dt, dev, [(B, T, H, dv)])
+    _check(a, "a", dt, dev, [(B, T, H, dk), (B, T, H)])
+    _check(b, "b", dt, dev, [(B, T, H, dk), (B, T, H)])
+    _check(w, "w", dt, dev, [(B, T, H, dv), (B, T, H)])
+    _check(s0, "s0", torch.float32, dev, [(B, H, dk, dv)])
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    _check(out, "out", dt, dev, [(B, T, H, dv)])
+    if s_final is None and return_final:
+        s_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    _check(s_final, "s_final", torch.float32, dev, [(B, H, dk, dv)])
+    desc = desc_for(q, v, a, b, w, chunk)
+    need = _lib.workspace_size(desc)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.forward_chunked(desc, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(w),
+                              _ptr(s0), _ptr(out), _ptr(s_final), _ptr(workspace), ws_bytes,
+                              _stream_handle(stream))
+    if st != _lib.OK:
+        raise _lib.GdrError(st, "gdr_forward_chunked")
+    return out, s_final
+
+
+def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                a: Optional[torch.Tensor], b: Optional[torch.Tensor],
+                w: Optional[torch.Tensor], state: torch.Tensor, *,
+                out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One decode step; `state` is updated in place.  Returns o [B, H, dv]."""
+    if q.dtype not in _DT:
+        raise ValueError("q must be float32 or bfloat16")
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    _check(q, "q", dt, dev, [(B, H, dk)])
+    _check(k, "k", dt, dev, [(B, H, dk)])
+    _check(v, "v", dt, dev, [(B, H, dv)])
+    _check(a, "a", dt, dev, [(B, H, dk), (B, H)])
+    _check(b, "b", dt, dev, [(B, H, dk), (B, H)])
+    _check(w, "w", dt, dev, [(B, H, dv), (B, H)])
+    _check(state, "state", torch.float32, dev, [(B, H, dk, dv)])
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=dt, device=dev)
+    _check(out, "out", dt, dev, [(B, H, dv)])
+    desc = desc_for(q, v, a, b, w, decode=True)
+    st = _lib.decode_step(desc, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(w),
+                          _ptr(state), _ptr(out), _stream_handle(stream))
+    if st != _lib.OK:
+        raise _lib.GdrError(st, "gdr_decode_step")
+    return out
+
+
+def last_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status."""
+    return _lib.last_device_error(_stream_handle(stream))
+
+
+Desc = _lib.GdrDesc

@@ -1,0 +1,156 @@
+// decode.cu -- single-token decode step of the gated delta rule.
+//
+// Per (batch, head), with the state S [dk, dv] float32 in HBM:
+//     e_j   = sum_i a_i k_i S_ij                   (key read of the decayed state)
+//     S_ij <- a_i S_ij - b_i k_i e_j + k_i w_j v_j  (decay, erase, write)
+//     o_j   = sum_i q_i S_ij                        (read-out of the new state)
+// FG^2-GDN page (gist.science 2604.19021), section 2 "Methodology", update
+// rule, with Gated DeltaNet-2's decoupled erase/write gates (needhelp.icu,
+// gates table).  The fixed-size state is the whole decode memory (Gated
+// DeltaNet-2 page, "The attention bottleneck": O(1) decode memory).
+//
+// The step is bound by HBM: every state element is read once and written
+// once, 8 bytes per element, against ~6 flops.  One CTA owns one head: its
+// 256 threads load the whole 64 KB state into registers with 16-byte loads
+// (each warp reads whole 512-byte rows), reduce e over the key axis (in
+// registers, then across warps through shared memory), update in registers,
+// store the new state with 16-byte stores, and reduce o the same way.
+#include "common.cuh"
+
+namespace gdr {
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(256, 2)
+decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                   const Tin* __restrict__ v, const Tin* __restrict__ a,
+                   const Tin* __restrict__ b, const Tin* __restrict__ w,
+                   int a_kind, int b_kind, int w_kind,
+                   float* __restrict__ state, Tin* __restrict__ o) {
+    constexpr int NT = 256;
+    constexpr int TPR = DV / 4;     // threads per state row (one float4 each)
+    constexpr int RS = NT / TPR;    // rows handled side by side
+    constexpr int RPT = DK / RS;    // rows per thread
+    static_assert(DV % 4 == 0 && NT % TPR == 0 && DK % RS == 0, "shape");
+
+    __shared__ float qs[DK], ks[DK], as_[DK], bks[DK];
+    __shared__ float us[DV];
+    __shared__ __align__(16) float red[RS][DV];
+
+    const int tid = threadIdx.x;
+    const long long bh = blockIdx.x;  // (b * H + h)
+    const int cg = tid % TPR;         // column group: columns 4cg .. 4cg+3
+    const int rs = tid / TPR;         // row set: rows rs, rs + RS, ...
+
+    float* S = state + bh * (long long)DK * DV;
+
+    // Issue the state loads first so they are in flight while the small
+    // inputs are staged.
+    float4 s[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r)
+        s[r] = *reinterpret_cast<const float4*>(S + (size_t)(rs + RS * r) * DV + 4 * cg);
+
+    for (int i = tid; i < DK; i += NT) {
+        const long long vb = bh * DK;
+        const float kv = to_f32(k[vb + i]);
+        qs[i] = to_f32(q[vb + i]);
+        ks[i] = kv;
+        as_[i] = gate_value(a, a_kind, bh, vb, i);
+        bks[i] = gate_value(b, b_kind, bh, vb, i) * kv;
+    }
+    for (int j = tid; j < DV; j += NT) {
+        const long long vb = bh * DV;
+        us[j] = gate_value(w, w_kind, bh, vb, j) * to_f32(v[vb + j]);
+    }
+    __syncthreads();
+
+    // e partial over this thread's rows.
+    float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const int i = rs + RS * r;
+        const float c = as_[i] * ks[i];
+        e.x = fmaf(c, s[r].x, e.x);
+        e.y = fmaf(c, s[r].y, e.y);
+        e.z = fmaf(c, s[r].z, e.z);
+        e.w = fmaf(c, s[r].w, e.w);
+    }
+    *reinterpret_cast<float4*>(&red[rs][4 * cg]) = e;
+    __syncthreads();
+    e = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int x = 0; x < RS; ++x) {
+        const float4 p = *reinterpret_cast<const float4*>(&red[x][4 * cg]);
+        e.x += p.x; e.y += p.y; e.z += p.z; e.w += p.w;
+    }
+    const float4 u = *reinterpret_cast<const float4*>(&us[4 * cg]);
+    __syncthreads();  // everyone has read red[] before it is reused for o
+
+    float4 op = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const int i = rs + RS * r;
+        const float ai = as_[i], bki = bks[i], ki = ks[i], qi = qs[i];
+        float4 n;
+        n.x = fmaf(ai, s[r].x, fmaf(-bki, e.x, ki * u.x));
+        n.y = fmaf(ai, s[r].y, fmaf(-bki, e.y, ki * u.y));
+        n.z = fmaf(ai, s[r].z, fmaf(-bki, e.z, ki * u.z));
+        n.w = fmaf(ai, s[r].w, fmaf(-bki, e.w, ki * u.w));
+        *reinterpret_cast<float4*>(S + (size_t)i * DV + 4 * cg) = n;
+        op.x = fmaf(qi, n.x, op.x);
+        op.y = fmaf(qi, n.y, op.y);
+        op.z = fmaf(qi, n.z, op.z);
+        op.w = fmaf(qi, n.w, op.w);
+    }
+    *reinterpret_cast<float4*>(&red[rs][4 * cg]) = op;
+    __syncthreads();
+    if (rs == 0) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int x = 0; x < RS; ++x) {
+            const float4 p = *reinterpret_cast<const float4*>(&red[x][4 * cg]);
+            acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
+        }
+        Tin* od = o + bh * DV + 4 * cg;
+        od[0] = from_f32<Tin>(acc.x);
+        od[1] = from_f32<Tin>(acc.y);
+        od[2] = from_f32<Tin>(acc.z);
+        od[3] = from_f32<Tin>(acc.w);
+    }
+}
+
+template <typename Tin, int DK, int DV>
+static cudaError_t launch_decode_t(const gdr_desc& d, const void* q, const void* k,
+                                   const void* v, const void* a, const void* b,
+                                   const void* w, float* state, void* o,
+                                   cudaStream_t stream) {
+    const unsigned grid = (unsigned)((long long)d.B * d.H);
+    decode_step_kernel<Tin, DK, DV><<<grid, 256, 0, stream>>>(
+        (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)a, (const Tin*)b,
+        (const Tin*)w, (int)d.decay, (int)d.erase, (int)d.write, state, (Tin*)o);
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+static cudaError_t launch_decode_d(const gdr_desc& d, const void* q, const void* k,
+                                   const void* v, const void* a, const void* b,
+                                   const void* w, float* state, void* o,
+                                   cudaStream_t stream) {
+    if (d.dk == 128 && d.dv == 128)
+        return launch_decode_t<Tin, 128, 128>(d, q, k, v, a, b, w, state, o, stream);
+    if (d.dk == 128 && d.dv == 64)
+        return launch_decode_t<Tin, 128, 64>(d, q, k, v, a, b, w, state, o, stream);
+    if (d.dk == 64 && d.dv == 128)
+        return launch_decode_t<Tin, 64, 128>(d, q, k, v, a, b, w, state, o, stream);
+    return launch_decode_t<Tin, 64, 64>(d, q, k, v, a, b, w, state, o, stream);
+}
+
+cudaError_t launch_decode(const gdr_desc& d, const void* q, const void* k, const void* v,
+                          const void* a, const void* b, const void* w, float* state,
+                          void* o, cudaStream_t stream) {
+    if (d.in_dtype == GDR_BF16)
+        return launch_decode_d<__nv_bfloat16>(d, q, k, v, a, b, w, state, o, stream);
+    return launch_decode_d<float>(d, q, k, v, a, b, w, state, o, stream);
+}
+
+}  // namespace gdr

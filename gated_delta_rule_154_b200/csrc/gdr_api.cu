@@ -1,0 +1,169 @@
+// gdr_api.cu -- the C ABI of libgdr.so: argument checks, kernel choice,
+// device error word.  Declarations and contracts are in include/gdr.h.
+#include <mutex>
+
+#include "common.cuh"
+
+namespace gdr {
+cudaError_t launch_decode(const gdr_desc& d, const void* q, const void* k, const void* v,
+                          const void* a, const void* b, const void* w, float* state,
+                          void* o, cudaStream_t stream);
+cudaError_t launch_chunked_simt(const gdr_desc& d, const void* q, const void* k,
+                                const void* v, const void* a, const void* b, const void* w,
+                                const float* s0, void* o, float* s_final, cudaStream_t st);
+bool chunked_tc_supports(const gdr_desc& d);
+cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, const void* v,
+                              const void* a, const void* b, const void* w, const float* s0,
+                              void* o, float* s_final, int* err_word, cudaStream_t st);
+}  // namespace gdr
+
+// One error word per device (each device holds its own copy of the symbol).
+static __device__ int g_gdr_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int* g_err_ptr[kMaxDevices];
+
+// Device address of this device's error word (looked up once per device).
+cudaError_t error_word(int** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_err_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_gdr_error_word);
+        if (e != cudaSuccess) return e;
+        g_err_ptr[dev] = static_cast<int*>(p);
+    }
+    *out = g_err_ptr[dev];
+    return cudaSuccess;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_gate(int g) { return g == GDR_GATE_ONE || g == GDR_GATE_SCALAR || g == GDR_GATE_VECTOR; }
+
+// Checks shared by both entry points; `T_axis` tells whether T is part of the
+// tensor shapes (prefill) or fixed to 1 (decode).
+gdr_status check_desc(const gdr_desc* d) {
+    if (!d) return GDR_ERR_INVALID_ARG;
+    if (d->B < 1 || d->H < 1 || d->T < 0) return GDR_ERR_INVALID_ARG;
+    if ((long long)d->B * d->H > 0x7fffffffLL) return GDR_ERR_INVALID_ARG;
+    if ((long long)d->B * d->T > (1LL << 40)) return GDR_ERR_INVALID_ARG;
+    if (!(d->dk == 64 || d->dk == 128) || !(d->dv == 64 || d->dv == 128))
+        return GDR_ERR_INVALID_ARG;
+    if (!(d->chunk == 16 || d->chunk == 32 || d->chunk == 64)) return GDR_ERR_INVALID_ARG;
+    if (!(d->in_dtype == GDR_F32 || d->in_dtype == GDR_BF16)) return GDR_ERR_INVALID_ARG;
+    if (!valid_gate(d->decay) || !valid_gate(d->erase) || !valid_gate(d->write))
+        return GDR_ERR_INVALID_ARG;
+    return GDR_OK;
+}
+
+gdr_status check_ptr(const void* p, bool required) {
+    if (!p) return required ? GDR_ERR_INVALID_ARG : GDR_OK;
+    return aligned16(p) ? GDR_OK : GDR_ERR_INVALID_ARG;
+}
+
+gdr_status check_inputs(const gdr_desc* d, bool have_tokens, const void* q, const void* k,
+                        const void* v, const void* a, const void* b, const void* w,
+                        const void* o) {
+    gdr_status s;
+    if ((s = check_ptr(q, have_tokens)) != GDR_OK) return s;
+    if ((s = check_ptr(k, have_tokens)) != GDR_OK) return s;
+    if ((s = check_ptr(v, have_tokens)) != GDR_OK) return s;
+    if ((s = check_ptr(o, have_tokens)) != GDR_OK) return s;
+    if ((s = check_ptr(a, have_tokens && d->decay != GDR_GATE_ONE)) != GDR_OK) return s;
+    if ((s = check_ptr(b, have_tokens && d->erase != GDR_GATE_ONE)) != GDR_OK) return s;
+    if ((s = check_ptr(w, have_tokens && d->write != GDR_GATE_ONE)) != GDR_OK) return s;
+    return GDR_OK;
+}
+
+// The float32 kernel takes every (dk, dv, chunk) the checks admit.
+bool simt_supports(const gdr_desc&) { return true; }
+
+}  // namespace
+
+extern "C" {
+
+int gdr_version(void) { return 0x000100; }
+
+const char* gdr_status_string(gdr_status s) {
+    switch (s) {
+        case GDR_OK: return "GDR_OK";
+        case GDR_ERR_INVALID_ARG: return "GDR_ERR_INVALID_ARG";
+        case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED";
+        case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE";
+        case GDR_ERR_CUDA: return "GDR_ERR_CUDA";
+        case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT";
+        case GDR_ERR_RANGE: return "GDR_ERR_RANGE";
+    }
+    return "GDR_UNKNOWN_STATUS";
+}
+
+size_t gdr_workspace_size(const gdr_desc* d) {
+    if (check_desc(d) != GDR_OK) return 0;
+    return 0;  // every kernel keeps its intermediates on chip
+}
+
+gdr_status gdr_forward_chunked(const gdr_desc* d, const void* q, const void* k, const void* v,
+                               const void* a, const void* b, const void* w, const float* s0,
+                               void* o, float* s_final, void* workspace, size_t ws_bytes,
+                               gdr_stream_t stream) {
+    gdr_status s = check_desc(d);
+    if (s != GDR_OK) return s;
+    const bool have_tokens = d->T > 0;
+    if ((s = check_inputs(d, have_tokens, q, k, v, a, b, w, o)) != GDR_OK) return s;
+    if ((s = check_ptr(s0, false)) != GDR_OK) return s;
+    if ((s = check_ptr(s_final, false)) != GDR_OK) return s;
+    const size_t need = gdr_workspace_size(d);
+    if (need > 0 && (workspace == nullptr || ws_bytes < need)) return GDR_ERR_WORKSPACE;
+    if (workspace && !aligned16(workspace)) return GDR_ERR_INVALID_ARG;
+
+    if (d->T == 0 && s_final == nullptr) return GDR_OK;  // nothing to compute or write
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (gdr::chunked_tc_supports(*d)) {
+        int* err = nullptr;
+        if ((e = error_word(&err)) != cudaSuccess) return GDR_ERR_CUDA;
+        e = gdr::launch_chunked_tc(*d, q, k, v, a, b, w, s0, o, s_final, err, st);
+    } else if (simt_supports(*d)) {
+        e = gdr::launch_chunked_simt(*d, q, k, v, a, b, w, s0, o, s_final, st);
+    } else {
+        return GDR_ERR_UNSUPPORTED;
+    }
+    return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+gdr_status gdr_decode_step(const gdr_desc* d, const void* q, const void* k, const void* v,
+                           const void* a, const void* b, const void* w, float* state, void* o,
+                           gdr_stream_t stream) {
+    gdr_status s = check_desc(d);
+    if (s != GDR_OK) return s;
+    if (d->T != 1) return GDR_ERR_INVALID_ARG;
+    if ((s = check_inputs(d, true, q, k, v, a, b, w, o)) != GDR_OK) return s;
+    if ((s = check_ptr(state, true)) != GDR_OK) return s;
+    cudaError_t e = gdr::launch_decode(*d, q, k, v, a, b, w, state, o,
+                                       reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+gdr_status gdr_last_device_error(gdr_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_gdr_error_word, sizeof(int)) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    if (word == 0) return GDR_OK;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_gdr_error_word, &zero, sizeof(int)) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    if (word & gdr::kErrTimeout) return GDR_ERR_TIMEOUT;
+    return GDR_ERR_RANGE;
+}
+
+}  // extern "C"

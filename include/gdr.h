@@ -1,0 +1,148 @@
+/*
+ * gdr.h -- C ABI of the gated delta-rule recurrence library (libgdr.so),
+ * CUDA kernels for NVIDIA B200 (sm_100a).
+ *
+ * The operation.  Per (batch b, head h), with a state S in R^{dk x dv} whose
+ * rows index key channels and columns index value channels, each token t does
+ *
+ *     S'  = Diag(a_t) S_{t-1}                          decay
+ *     S_t = S' - (b_t * k_t)(k_t^T S') + k_t (w_t * v_t)^T   erase, then write
+ *     o_t = S_t^T q_t                                   read-out
+ *
+ * Sources: the update rule and its order (decay, erase from the decayed state,
+ * write) -- page "FG^2-GDN: Enhancing Long-Context Gated Delta Networks with
+ * Doubly Fine-Grained Control" (gist.science 2604.19021), section 2
+ * "Methodology", FG2-GDN update rule; the decoupled per-channel erase gate b_t
+ * (key side) and write gate w_t (value side) with KDA's per-channel decay --
+ * page "Gated DeltaNet-2: decoupling erase and write in linear attention"
+ * (needhelp.icu), the gates table; scalar decay (Gated DeltaNet) versus
+ * per-channel decay (KDA) -- FG^2-GDN page, section 1 "Problem statement";
+ * the chunkwise-parallel (WY) evaluation used by gdr_forward_chunked --
+ * FG^2-GDN page, section 2 (rank-1 Householder structure kept for WY chunked
+ * training) and section 3 (DPLR structure, KDA-style chunked kernels); the
+ * fixed-size state that replaces a KV cache and makes decoding O(1) in memory
+ * -- Gated DeltaNet-2 page, "The attention bottleneck".  The read-out with the
+ * updated state, no 1/sqrt(dk) on q, and q, k normalised by the caller are
+ * readings where the pages print no equation.
+ *
+ * Conventions shared by every entry point.
+ *   - Tensors are dense, row-major, contiguous, in device memory owned by the
+ *     caller: q, k [B, T, H, dk]; v, o [B, T, H, dv]; vector gates a, b
+ *     [B, T, H, dk] and w [B, T, H, dv]; scalar gates [B, T, H] (one value per
+ *     token and head); states [B, H, dk, dv] in float32.
+ *   - q, k, v, the gates and o share in_dtype (float32 or bf16); the state is
+ *     always float32.  Arithmetic is float32 (tensor-core products take bf16
+ *     operands with float32 accumulation on the bf16 path).
+ *   - q and k are expected L2-normalised by the caller; a_t in (0, 1].
+ *   - Every pointer the call reads or writes must be 16-byte aligned.
+ *   - The library allocates nothing and keeps no per-call state.  Calls are
+ *     asynchronous on `stream` (0 = the legacy default stream).
+ *   - Argument errors are reported synchronously, before anything is
+ *     launched; nothing is written in that case.  A failed launch returns
+ *     GDR_ERR_CUDA.  Faults found on the device (a bounded wait that ran out,
+ *     decay outside the supported range) are recorded in a per-device error
+ *     word read by gdr_last_device_error().  No C++ exception crosses the ABI.
+ *   - Concurrent calls on distinct buffers are safe.
+ */
+#ifndef GDR_H_
+#define GDR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *gdr_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    GDR_OK = 0,
+    GDR_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, bad enum */
+    GDR_ERR_UNSUPPORTED = 2, /* valid, but no kernel for this combination  */
+    GDR_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required  */
+    GDR_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed        */
+    GDR_ERR_TIMEOUT = 5,     /* device: a bounded wait ran out              */
+    GDR_ERR_RANGE = 6        /* device: decay too strong for the chunk form */
+} gdr_status;
+
+typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
+
+/* How a gate is given.  ONE: the gate is identically 1 and its pointer is
+ * ignored (may be NULL).  SCALAR: one value per (b, t, h), [B, T, H].
+ * VECTOR: one value per channel, [B, T, H, dk] for a and b, [B, T, H, dv]
+ * for w. */
+typedef enum { GDR_GATE_ONE = 0, GDR_GATE_SCALAR = 1, GDR_GATE_VECTOR = 2 } gdr_gate;
+
+typedef struct {
+    int B, T, H;          /* batch, tokens, heads; B, H >= 1, T >= 0        */
+    int dk, dv;           /* 64 or 128 each                                 */
+    int chunk;            /* chunk length of the chunked form: 16, 32 or 64 */
+    gdr_dtype in_dtype;   /* dtype of q, k, v, a, b, w and o                */
+    gdr_gate decay;       /* a */
+    gdr_gate erase;       /* b */
+    gdr_gate write;       /* w; b and w may be the same tensor (shared beta) */
+} gdr_desc;
+
+/* Bytes of device workspace gdr_forward_chunked needs for `desc` (0 if none,
+ * or if desc is invalid).  Pure host function, no CUDA call. */
+size_t gdr_workspace_size(const gdr_desc *desc);
+
+/*
+ * Causal prefill over T tokens by the chunkwise-parallel form: per chunk of
+ * `chunk` tokens, cumulative decay, intra-chunk gram matrices, a triangular
+ * (UT-transform) solve for the erase terms, and a sequential pass over
+ * chunks that carries S in float32.  Equal, up to rounding, to running the
+ * recurrence above token by token.
+ *
+ *   q, k, v, a, b, w  inputs as described above (a/b/w ignored when ONE)
+ *   s0       [B, H, dk, dv] float32 initial state, or NULL for zeros
+ *   o        [B, T, H, dv] in_dtype, written
+ *   s_final  [B, H, dk, dv] float32 final state, or NULL (not written);
+ *            may equal s0 (in-place update)
+ *   workspace, ws_bytes  device scratch of gdr_workspace_size(desc) bytes
+ *            (NULL / 0 when that is 0)
+ *
+ * Supported: dk, dv in {64, 128}; float32 inputs with chunk in {16, 32, 64}
+ * (chunk <= 32 when dk = 128); bf16 inputs with chunk 64 and dk = dv = 128 on
+ * the tensor-core kernel, and the float32 kernel's chunk sizes otherwise.
+ * Other valid descriptors return GDR_ERR_UNSUPPORTED.
+ *
+ * Decay range: within each chunk the products of a over any run of tokens
+ * must stay representable in float32 after the kernel's factorisation
+ * (about exp(-80) over half a chunk per channel on the bf16 tensor-core
+ * kernel); outside it the device error word reports GDR_ERR_RANGE.
+ */
+gdr_status gdr_forward_chunked(const gdr_desc *desc, const void *q, const void *k,
+                               const void *v, const void *a, const void *b,
+                               const void *w, const float *s0, void *o,
+                               float *s_final, void *workspace, size_t ws_bytes,
+                               gdr_stream_t stream);
+
+/*
+ * One decode step (desc->T must be 1): reads and rewrites `state` in place.
+ * Shapes drop the T axis: q, k, a, b [B, H, dk] (scalar gates [B, H]);
+ * v, w [B, H, dv]; state [B, H, dk, dv] float32; o [B, H, dv] in_dtype.
+ * Each state element is read once and written once.
+ */
+gdr_status gdr_decode_step(const gdr_desc *desc, const void *q, const void *k,
+                           const void *v, const void *a, const void *b,
+                           const void *w, float *state, void *o,
+                           gdr_stream_t stream);
+
+/* Synchronises `stream`, returns the status recorded on the device since the
+ * previous call (GDR_OK if none) and clears it.  GDR_ERR_CUDA if the
+ * synchronisation itself failed. */
+gdr_status gdr_last_device_error(gdr_stream_t stream);
+
+/* Static, human-readable name of a status. */
+const char *gdr_status_string(gdr_status status);
+
+/* Library version, e.g. 0x000100 for 0.1.0. */
+int gdr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H_ */

@@ -1,0 +1,106 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/gdr.h declares, and rejects bad arguments on the host before any CUDA
+call (no compute call is made here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_154_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "gdr.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdr_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_documented_calls():
+    names = _declared_functions()
+    for n in ("gdr_forward_chunked", "gdr_decode_step", "gdr_workspace_size",
+              "gdr_status_string", "gdr_last_device_error"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    assert set(_lib.EXPORTS) <= set(_declared_functions())
+
+
+def test_status_strings(lib):
+    assert _lib.status_string(_lib.OK) == "GDR_OK"
+    assert _lib.status_string(_lib.ERR_RANGE) == "GDR_ERR_RANGE"
+    assert _lib.status_string(99) == "GDR_UNKNOWN_STATUS"
+    assert lib.gdr_version() >= 0x000100
+
+
+def _desc(**kw):
+    base = dict(B=2, T=128, H=4, dk=128, dv=128, chunk=64, in_dtype=_lib.BF16,
+                decay=_lib.GATE_VECTOR, erase=_lib.GATE_VECTOR, write=_lib.GATE_VECTOR)
+    base.update(kw)
+    return _lib.GdrDesc(**base)
+
+
+def test_workspace_is_host_only_and_zero(lib):
+    assert _lib.workspace_size(_desc()) == 0
+    assert lib.gdr_workspace_size(None) == 0
+
+
+P = 1 << 20  # a 16-byte-aligned fake address: never dereferenced, checks fail first
+
+
+@pytest.mark.parametrize("field,value", [
+    ("B", 0), ("H", 0), ("T", -1), ("dk", 96), ("dv", 32), ("chunk", 48),
+    ("in_dtype", 7), ("decay", 3), ("erase", -1), ("write", 5)])
+def test_bad_descriptor_rejected(lib, field, value):
+    d = _desc(**{field: value})
+    st = _lib.forward_chunked(d, P, P, P, P, P, P, 0, P, 0, 0, 0, 0)
+    assert st == _lib.ERR_INVALID_ARG
+    d.T = 1
+    setattr(d, field, value)
+    if field != "T":
+        st = _lib.decode_step(d, P, P, P, P, P, P, P, P, 0)
+        assert st == _lib.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("which", range(7))
+def test_null_or_misaligned_pointer_rejected(lib, which):
+    ptrs = [P] * 7  # q k v a b w o
+    for bad in (0, P + 8):
+        p = list(ptrs)
+        p[which] = bad
+        q, k, v, a, b, w, o = p
+        assert _lib.forward_chunked(_desc(), q, k, v, a, b, w, 0, o, 0, 0, 0, 0) == _lib.ERR_INVALID_ARG
+        assert _lib.decode_step(_desc(T=1), q, k, v, a, b, w, P, o, 0) == _lib.ERR_INVALID_ARG
+
+
+def test_misaligned_state_rejected(lib):
+    assert _lib.forward_chunked(_desc(), P, P, P, P, P, P, P + 4, P, 0, 0, 0, 0) == _lib.ERR_INVALID_ARG
+    assert _lib.forward_chunked(_desc(), P, P, P, P, P, P, 0, P, P + 4, 0, 0, 0) == _lib.ERR_INVALID_ARG
+    assert _lib.decode_step(_desc(T=1), P, P, P, P, P, P, 0, P, 0) == _lib.ERR_INVALID_ARG
+
+
+def test_decode_needs_t_equal_one(lib):
+    assert _lib.decode_step(_desc(T=2), P, P, P, P, P, P, P, P, 0) == _lib.ERR_INVALID_ARG
+
+
+def test_gate_one_needs_no_pointer_and_empty_is_a_no_op(lib):
+    # T = 0 with no final state: nothing to do, no CUDA call, GDR_OK.
+    d = _desc(T=0, decay=_lib.GATE_ONE, erase=_lib.GATE_ONE, write=_lib.GATE_ONE)
+    assert _lib.forward_chunked(d, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0) == _lib.OK
+
+
+def test_null_descriptor(lib):
+    assert lib.gdr_forward_chunked(None, *([None] * 9), None, 0, None) == _lib.ERR_INVALID_ARG
+    assert lib.gdr_decode_step(None, *([None] * 9)) == _lib.ERR_INVALID_ARG

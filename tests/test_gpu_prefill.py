@@ -1,0 +1,177 @@
+"""GPU parity of the chunked prefill against the float64 oracle, through the
+library's C ABI (via the thin torch binding), plus the properties the
+recurrence fixes at any size: chunk-size invariance, resume, head
+permutation, in-place state, empty input, and agreement with the decode
+kernel run token by token.
+
+Tolerances (max |x - ref| / max |ref| per tensor): 1e-4 for float32 inputs,
+2e-2 for bf16 inputs (state float32 in both)."""
+
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_154_b200 import api
+from gated_delta_rule_154_b200 import workload as W
+from gpu_helpers import (TOL, gpu_prefill, inputs_to_dev, oracle_prefill, rel_err, to_dev,
+                         to_host)
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_full(wl, inp, chunk=None):
+    o, s = gpu_prefill(wl, inp, chunk)
+    o_ref, s_ref = oracle_prefill(wl, inp)
+    eo, es = rel_err(to_host(o), o_ref), rel_err(to_host(s), s_ref)
+    assert eo <= TOL[wl.dtype] and es <= TOL[wl.dtype], (wl.name, chunk, eo, es)
+    return eo, es
+
+
+def test_gdn_fp32_full_workload():
+    """Gated DeltaNet, scalar gates, float32: B=1 H=2 T=256 d=64 chunk 64."""
+    wl = W.WORKLOADS["gdn_fp32"]
+    _check_full(wl, W.make_prefill(wl))
+
+
+@pytest.mark.parametrize("name", ["gdn_fp32", "kda_bf16", "gdn2_bf16", "long_bf16"])
+@pytest.mark.parametrize("T", [64, 200, 333])
+def test_small_shapes_every_gate_kind(name, T):
+    """Reduced B/H/T of each prefill workload, with ragged tails."""
+    wl = W.WORKLOADS[name].replace(B=2, H=3, T=T)
+    _check_full(wl, W.make_prefill(wl, seed=T))
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 64), (64, 128), (128, 128)])
+def test_chunk_sizes_and_head_dims_fp32(chunk, dk, dv):
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=150, dk=dk, dv=dv, dtype="f32", chunk=chunk)
+    _check_full(wl, W.make_prefill(wl, seed=chunk + dk + dv))
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_chunk_sizes_bf16(chunk):
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=300, chunk=chunk)
+    _check_full(wl, W.make_prefill(wl, seed=7))
+
+
+def test_gate_one_everywhere():
+    """a = b = w = 1 given as GATE_ONE (no gate tensors): plain DeltaNet."""
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=130, dtype="f32")
+    inp = W.make_prefill(wl, seed=3)
+    d = inputs_to_dev(inp, wl)
+    o, s = api.forward_chunked(d["q"], d["k"], d["v"], None, None, None, d["s0"], chunk=64)
+    ones_k = np.ones_like(inp["a"])
+    ref = dict(inp, a=ones_k, b=ones_k, w=np.ones_like(inp["w"]))
+    o_ref, s_ref = oracle_prefill(wl, ref)
+    assert rel_err(to_host(o), o_ref) <= 1e-4 and rel_err(to_host(s), s_ref) <= 1e-4
+
+
+def test_chunk_size_invariance_fp32():
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=2, H=2, T=256, dtype="f32")
+    inp = W.make_prefill(wl, seed=11)
+    o16, s16 = gpu_prefill(wl, inp, 16)
+    o64, s64 = gpu_prefill(wl, inp, 64)
+    assert rel_err(to_host(o16), to_host(o64)) <= 1e-4
+    assert rel_err(to_host(s16), to_host(s64)) <= 1e-4
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_resume_split_sequence(dtype):
+    """forward(T1) then forward(T2, s0 = S_T1) equals forward(T1 + T2)."""
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=2, H=2, T=320, dtype=dtype)
+    inp = W.make_prefill(wl, seed=5)
+    d = inputs_to_dev(inp, wl)
+    o, s = api.forward_chunked(d["q"], d["k"], d["v"], d["a"], d["b"], d["w"], d["s0"])
+    c = 192
+    part = lambda x, sl: x[:, sl].contiguous()
+    o1, s1 = api.forward_chunked(*(part(d[k], slice(0, c)) for k in "qkvabw"), d["s0"])
+    o2, s2 = api.forward_chunked(*(part(d[k], slice(c, None)) for k in "qkvabw"), s1)
+    tol = TOL[dtype]
+    assert rel_err(to_host(torch.cat([o1, o2], 1)), to_host(o)) <= tol
+    assert rel_err(to_host(s2), to_host(s)) <= tol
+
+
+def test_head_permutation():
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=4, T=100)
+    inp = W.make_prefill(wl, seed=9)
+    d = inputs_to_dev(inp, wl)
+    perm = torch.tensor([2, 0, 3, 1], device="cuda")
+    o, s = api.forward_chunked(d["q"], d["k"], d["v"], d["a"], d["b"], d["w"], d["s0"])
+    p = lambda x: x.index_select(2, perm).contiguous()
+    op, sp = api.forward_chunked(*(p(d[k]) for k in "qkvabw"), d["s0"].index_select(1, perm).contiguous())
+    assert torch.equal(op, o.index_select(2, perm))
+    assert torch.equal(sp, s.index_select(1, perm))
+
+
+def test_in_place_final_state_and_no_final_state():
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=130)
+    inp = W.make_prefill(wl, seed=2)
+    d = inputs_to_dev(inp, wl)
+    o, s = api.forward_chunked(d["q"], d["k"], d["v"], d["a"], d["b"], d["w"], d["s0"])
+    st = d["s0"].clone()
+    o2, s2 = api.forward_chunked(d["q"], d["k"], d["v"], d["a"], d["b"], d["w"], st, s_final=st)
+    assert s2.data_ptr() == st.data_ptr()
+    assert torch.equal(o2, o) and torch.equal(st, s)
+    o3, s3 = api.forward_chunked(d["q"], d["k"], d["v"], d["a"], d["b"], d["w"], d["s0"],
+                                 return_final=False)
+    assert s3 is None and torch.equal(o3, o)
+
+
+def test_empty_sequence_returns_initial_state():
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=2, H=2, T=0)
+    inp = W.make_prefill(wl.replace(T=1), seed=1)
+    s0 = to_dev(inp["s0"], "f32")
+    e = lambda d: torch.empty((2, 0, 2, d), dtype=torch.bfloat16, device="cuda")
+    o, s = api.forward_chunked(e(128), e(128), e(128), e(128), e(128), e(128), s0)
+    torch.cuda.synchronize()
+    assert o.shape == (2, 0, 2, 128) and torch.equal(s, s0)
+    o, s = api.forward_chunked(e(128), e(128), e(128), e(128), e(128), e(128), None)
+    assert torch.count_nonzero(s) == 0
+
+
+def test_matches_decode_kernel_token_by_token():
+    """The chunked kernel and the decode kernel run step by step agree."""
+    wl = W.WORKLOADS["kda_bf16"].replace(B=2, H=2, T=70, dtype="f32")
+    inp = W.make_prefill(wl, seed=4)
+    d = inputs_to_dev(inp, wl)
+    o, s = api.forward_chunked(d["q"], d["k"], d["v"], d["a"], d["b"], d["w"], None)
+    state = torch.zeros_like(s)
+    outs = []
+    for t in range(wl.T):
+        g = lambda x: x[:, t].contiguous()
+        outs.append(api.decode_step(g(d["q"]), g(d["k"]), g(d["v"]), g(d["a"]), g(d["b"]),
+                                    g(d["w"]), state))
+    torch.cuda.synchronize()
+    assert rel_err(to_host(torch.stack(outs, 1)), to_host(o)) <= 1e-4
+    assert rel_err(to_host(state), to_host(s)) <= 1e-4
+
+
+def test_no_device_error_recorded():
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=64)
+    gpu_prefill(wl, W.make_prefill(wl))
+    assert api.last_device_error() == 0
+
+
+# ------------------------------------------------- full-size workloads (sampled)
+
+def _sample_heads(wl, n, seed):
+    rng = np.random.default_rng(seed)
+    all_heads = [(b, h) for b in range(wl.B) for h in range(wl.H)]
+    idx = rng.choice(len(all_heads), size=min(n, len(all_heads)), replace=False)
+    return [all_heads[i] for i in sorted(idx)]
+
+
+@pytest.mark.parametrize("name,n_heads", [("kda_bf16", 6), ("gdn2_bf16", 6), ("long_bf16", 3)])
+def test_full_size_sampled_heads(name, n_heads):
+    """Full workload on the GPU in the bench's launch configuration; the oracle
+    recomputes a seeded sample of whole heads (every token, final state)."""
+    wl = W.WORKLOADS[name]
+    inp = W.make_prefill(wl, seed=0)
+    o, s = gpu_prefill(wl, inp)
+    heads = _sample_heads(wl, n_heads, 123)
+    o_ref, s_ref = oracle_prefill(wl, inp, heads=heads)
+    for i, (b, h) in enumerate(heads):
+        eo = rel_err(to_host(o[b, :, h]), o_ref[i])
+        es = rel_err(to_host(s[b, h]), s_ref[i])
+        assert eo <= TOL[wl.dtype] and es <= TOL[wl.dtype], (name, b, h, eo, es)
+    assert np.isfinite(to_host(o)).all() and np.isfinite(to_host(s)).all()
