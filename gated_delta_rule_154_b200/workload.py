@@ -85,7 +85,7 @@ WORKLOADS: Dict[str, Workload] = {
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float32 to bf16 (round-to-nearest-even); returns uint16 bits."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    u = np.array(x, dtype=np.float32, order="C").view(np.uint32)
     rounding = ((u >> 16) & np.uint32(1)) + np.uint32(0x7FFF)
     return ((u + rounding) >> 16).astype(np.uint16)
 

@@ -175,3 +175,50 @@ def test_full_size_sampled_heads(name, n_heads):
         es = rel_err(to_host(s[b, h]), s_ref[i])
         assert eo <= TOL[wl.dtype] and es <= TOL[wl.dtype], (name, b, h, eo, es)
     assert np.isfinite(to_host(o)).all() and np.isfinite(to_host(s)).all()
+
+
+# ------------------------------------------- tensor-core kernel specific checks
+
+@pytest.mark.parametrize("name", ["kda_bf16", "gdn2_bf16"])
+def test_tensor_core_kernel_matches_float32_kernel(name):
+    """bf16 inputs, chunk 64 runs on the tcgen05 kernel; chunk 32 on the
+    float32 CUDA-core kernel.  Same inputs, same recurrence."""
+    wl = W.WORKLOADS[name].replace(B=2, H=4, T=517)
+    inp = W.make_prefill(wl, seed=17)
+    o64, s64 = gpu_prefill(wl, inp, 64)
+    o32, s32 = gpu_prefill(wl, inp, 32)
+    assert rel_err(to_host(o64), to_host(o32)) <= TOL["bf16"]
+    assert rel_err(to_host(s64), to_host(s32)) <= TOL["bf16"]
+
+
+def test_tensor_core_scalar_decay_and_gate_one():
+    """Scalar decay, no erase gate (b = 1), scalar write gate, bf16."""
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=3, T=190, decay="scalar", erase="scalar",
+                                          write="scalar")
+    inp = W.make_prefill(wl, seed=23)
+    d = inputs_to_dev(inp, wl)
+    o, s = api.forward_chunked(d["q"], d["k"], d["v"], d["a"], None, d["w"], d["s0"], chunk=64)
+    torch.cuda.synchronize()
+    ref = dict(inp, b=np.full_like(inp["b"], W.f32_to_bf16_bits(np.float32(1.0))))
+    o_ref, s_ref = oracle_prefill(wl, ref)
+    assert rel_err(to_host(o), o_ref) <= TOL["bf16"]
+    assert rel_err(to_host(s), s_ref) <= TOL["bf16"]
+    assert api.last_device_error() == 0
+
+
+def test_decay_beyond_tensor_core_range_is_reported():
+    """A decay strong enough that exp(decay over half a chunk) leaves float
+    range is flagged as GDR_ERR_RANGE on the tensor-core kernel, and the
+    error word is cleared once read."""
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=64)
+    inp = W.make_prefill(wl, seed=1)
+    a = inp["a"].copy()
+    a[0, :, 1, 5] = W.f32_to_bf16_bits(np.full(64, 0.01, np.float32))  # log(0.01)*32 < -80
+    inp = dict(inp, a=a)
+    gpu_prefill(wl, inp, 64)
+    assert api.last_device_error() == 6   # GDR_ERR_RANGE
+    assert api.last_device_error() == 0
+    # the float32 kernel (chunk 32) has no such limit and matches the oracle
+    o, s = gpu_prefill(wl, inp, 32)
+    o_ref, s_ref = oracle_prefill(wl, inp)
+    assert rel_err(to_host(o), o_ref) <= TOL["bf16"] and rel_err(to_host(s), s_ref) <= TOL["bf16"]
