@@ -249,5 +249,52 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar_saddr, uint32_t p
     }
 }
 
+// ------------------------------------------------------------- TMA loads
+
+// Arm `bar` for one arrival plus `bytes` of asynchronous transactions.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar_saddr, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_saddr),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// 4-D tiled bulk-tensor load into shared memory, completion counted on `bar`
+// in bytes.  Coordinates are innermost first.  (Plain load: no multicast.)
+__device__ __forceinline__ void tma_load_4d(uint32_t dst_saddr, const void* tmap, int c0, int c1,
+                                            int c2, int c3, uint32_t bar_saddr) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst_saddr),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+        "r"(bar_saddr)
+        : "memory");
+}
+
+// 4-D tiled bulk-tensor store from shared memory (bulk-group completion).
+// Rows past the tensor's extent are not written.
+__device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src_saddr, int c0, int c1,
+                                             int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group "
+        "[%0, {%2, %3, %4, %5}], [%1];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+        "r"(src_saddr), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until every committed bulk store has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until every committed bulk store has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
 }  // namespace tc
 }  // namespace gdr
