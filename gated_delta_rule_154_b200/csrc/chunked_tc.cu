@@ -8,7 +8,7 @@
 //   A_kb[r,s] = sum_c k_rc b_sc k_sc gamma_rc/gamma_sc     (strictly lower)
 //   A_qk[r,s], A_qb[r,s] the same with q_r for k_r          (lower, diagonal in)
 //   T  = (I + A_kb)^{-1}                 UT transform (unit lower triangular)
-//   E  = T (Kh S0 + A_kk U),             Kh = gamma*K   (row r: S'_r^T k_r)
+//   R  = Kh S0 + A_kk U,  E = T R        Kh = gamma*K   (row r of E: S'_r^T k_r)
 //   O  = Qh S0 + A_qk U - A_qb E,        Qh = gamma*Q
 //   S  = gamma_C * S0 + Kt^T U - Bt^T E, Kt = (gamma_C/gamma)*K, Bt = b*Kt
 // This is the WY / UT-transform evaluation of the rank-1 Householder-like
@@ -20,26 +20,26 @@
 //
 // Scaling around the middle token m = 31.  With g_m = gamma_m per channel:
 //   K' = (gamma/g_m)*K, Q' = (gamma/g_m)*Q, K" = (g_m/gamma)*K, B" = b*K"
-// the grams are [K';Q'] [K";B"]^T, and with the state kept as
-// S~ = Diag(g_m) S0 the same four tiles serve every other product:
-//   E^T  = S~^T (T K')^T + (A_kk U)^T T^T
-//   O^T  = S~^T Q'^T + U^T A_qk^T - E^T A_qb^T
-//   S~^T <- S~^T + U^T K" - E^T B"      then S_new = Diag(gamma_C/g_m) S~.
-// Every factor is exp of the decay accumulated over at most half a chunk.  If
-// that exceeds exp(80) in some channel the factors leave float range; the
-// kernel then sets GDR_ERR_RANGE in the device error word (the float32
-// CUDA-core kernel, chunk <= 32, has no such limit).
+// and the state kept as S~ = Diag(g_m) S0, one 128 x 128 accumulator X holds
+// [R; O] (rows 0-63 tokens of R, rows 64-127 tokens of O):
+//   X   = [K'; Q'] S~ + [A_kk; A_qk] U          (R and the first terms of O)
+//   X  += [T - I; 0] R                           (rows 0-63 become E = T R)
+//   X  += [0; -A_qb] E                           (rows 64-127 become O)
+//   S~ += K"^T U - B"^T E,   S_new = Diag(gamma_C/g_m) S~
+// and the grams are [K';Q'] [K";B"]^T.  Every factor is a ratio of decay
+// products over at most half a chunk; if one leaves float range (decay
+// stronger than about exp(-80) over half a chunk, or an exact zero) the
+// kernel sets GDR_ERR_RANGE in the device error word (the float32 CUDA-core
+// kernel, chunk <= 32, has no such limit).
 //
-// State-side products are formed transposed so that every product has
-// M = 128 (tensor-memory lane = value channel j).  S~^T stays in float32 in
-// tensor memory for the whole sequence; a bf16 copy in shared memory is the
-// MMA operand.  One CTA (16 warps) owns one (batch, head) and walks its
-// chunks in order.  Raw q/k/v and vector gates arrive by TMA as 64-token x
+// One CTA (16 warps) owns one (batch, head) and walks its chunks in order;
+// S~ stays in float32 in tensor memory (lane = key channel) for the whole
+// sequence.  Raw q/k/v and vector gates arrive by TMA as 64-token x
 // 64-channel boxes, 128-byte swizzled, i.e. already in the operand layout of
-// tc_common.cuh; the next chunk's q and k are fetched while the current one
-// is processed, and o leaves by a TMA store.  Products are tcgen05.mma issued
-// by one thread; the cumulative decay, the UT solve and the conversions run
-// on the CUDA cores with 16-byte shared-memory accesses.
+// tc_common.cuh, each prefetched as soon as its destination is free; o leaves
+// by a TMA store.  Products are tcgen05.mma issued by one thread; the decay
+// products, the UT solve and the conversions run on the CUDA cores with
+// 16-byte shared-memory accesses.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -58,44 +58,39 @@ constexpr int NT = 512;      // threads per CTA (16 warps)
 
 // ---- shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_RAW = 0;         // raw k (rows 0-63) and q (rows 64-127), 2 panels
-constexpr uint32_t OFF_X1 = 32768;      // [K'; Q'] 128 rows x 128; o staging at the end
-constexpr uint32_t OFF_X2 = 65536;      // [K"; B"] 128 rows x 128 (raw a, b land here)
-constexpr uint32_t OFF_U = 98304;       // U = w*v [s][j] (raw v lands here)
-constexpr uint32_t OFF_L = 114688;      // A_kk strictly lower [r][s] (raw w lands at L..AQK)
-constexpr uint32_t OFF_AQK = 122880;    // A_qk lower [r][s]
-constexpr uint32_t OFF_AQB = 131072;    // -A_qb lower [r][s]
-constexpr uint32_t OFF_T = 139264;      // T [r][s] bf16
-constexpr uint32_t OFF_S0T = 147456;    // S~^T [j][i] bf16, 2 panels
-constexpr uint32_t OFF_R = 180224;      // scratch region, 36 KB:
-constexpr uint32_t OFF_REL = OFF_R;             //  P1: log(gamma_r) partial sums, float [64][128]
-constexpr uint32_t OFF_QT = OFF_R + 32768;      //  P1: quarter totals, float [4][128]
-constexpr uint32_t OFF_OFS = OFF_R + 34816;     //  P1: per-quarter offsets, float [4][128]
-constexpr uint32_t OFF_NS = OFF_R;              //  P4-P5: A_kb, float [64][65]
-constexpr uint32_t OFF_TS = OFF_R + 16640;      //  P5: T, float [64][65]
-constexpr uint32_t OFF_PS = OFF_R + 33280;      //  P5: float [3][256]
-constexpr uint32_t OFF_W = OFF_R;               //  P7-P8: (T K')^T [i][r]
-constexpr uint32_t OFF_ZT = OFF_R + 16384;      //  P7-P8: (A_kk U)^T [j][s]
-constexpr uint32_t OFF_ET = OFF_R;              //  P9-P10: E^T [j][r]
-constexpr uint32_t OFF_SMALL = OFF_R + 36864;   // 217088
+constexpr uint32_t OFF_X1 = 32768;      // [K'; Q'] 128 x 128 (raw a, b land here)
+constexpr uint32_t OFF_X2 = 65536;      // [K"; B"] 128 x 128
+constexpr uint32_t OFF_U = 98304;       // U = w*v [s][j] 64 x 128 (raw v lands here)
+constexpr uint32_t OFF_LQ = 114688;     // [A_kk; A_qk] 128 x 64 (raw w lands here)
+constexpr uint32_t OFF_Z3 = 131072;     // [T - I; 0; -A_qb] 192 x 64
+constexpr uint32_t OFF_S0 = 155648;     // S~ [i][j] bf16 128 x 128; o staging 64 x 128
+constexpr uint32_t OFF_R = 188416;      // scratch region, 38 KB:
+constexpr uint32_t OFF_REL = OFF_R;             //  P1: decay products, float [64][128]
+constexpr uint32_t OFF_QT = OFF_R + 32768;      //  P1: quarter products, float [4][128]
+constexpr uint32_t OFF_OFS = OFF_R + 34816;     //  P1: per-quarter factors, float [4][128]
+constexpr uint32_t OFF_NS = OFF_R;              //  P4-P5: A_kb, float [64][68]
+constexpr uint32_t OFF_TS = OFF_R + 17408;      //  P5: T, float [64][68]
+constexpr uint32_t OFF_PS = OFF_R + 34816;      //  P5: float [3][16][16]
+constexpr uint32_t OFF_RB = OFF_R;              //  P6: R bf16 [s][j] 64 x 128
+constexpr uint32_t OFF_EB = OFF_R + 16384;      //  P7: E bf16 [s][j] 64 x 128
+constexpr uint32_t OFF_SMALL = OFF_R + 38912;   // 227328
 constexpr uint32_t OFF_FCUR = OFF_SMALL;        // float[128]: state scale this chunk
 constexpr uint32_t OFF_FPREV = OFF_SMALL + 512; // float[128]: gamma_C/g_m of last chunk
 constexpr uint32_t OFF_SCA = OFF_SMALL + 1024;  // float[3][64]: scalar a, b, w
-constexpr uint32_t OFF_BAR = OFF_SMALL + 1792;  // 3 mbarriers: mma, kq, rest
-constexpr uint32_t OFF_TSLOT = OFF_BAR + 24;
-constexpr uint32_t OFF_ABORT = OFF_BAR + 28;
-constexpr uint32_t SMEM_USED = OFF_BAR + 32;
+constexpr uint32_t OFF_BAR = OFF_SMALL + 1792;  // 4 mbarriers: mma, kq, ab, vw
+constexpr uint32_t OFF_TSLOT = OFF_BAR + 32;
+constexpr uint32_t OFF_ABORT = OFF_BAR + 36;
+constexpr uint32_t SMEM_USED = OFF_BAR + 40;
 constexpr size_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory");
+static_assert(OFF_PS + 3 * 256 * 4 <= OFF_SMALL, "solve scratch");
 
-constexpr int NSP = 65;  // row stride (floats) of the solve's float tiles
+constexpr int NSP = 68;  // row stride (floats) of the solve's float tiles (16-byte rows)
 
 // ---- tensor-memory columns (512 allocated)
 constexpr uint32_t TM_G = 0;     // gram 128 x 128
-constexpr uint32_t TM_W = 128;   // (T K')^T 128 x 64
-constexpr uint32_t TM_Z = 192;   // (A_kk U)^T 128 x 64
-constexpr uint32_t TM_E = 256;   // E^T  128 x 64
-constexpr uint32_t TM_O = 320;   // O^T  128 x 64
-constexpr uint32_t TM_S = 384;   // S~^T 128 x 128, float32 state
+constexpr uint32_t TM_X = 128;   // [R -> E; O] 128 x 128
+constexpr uint32_t TM_S = 256;   // S~ 128 x 128 (lane = key channel), float32 state
 
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait
 constexpr uint32_t BOX_BYTES = 64 * 128;     // one 64 x 64 bf16 TMA box
@@ -109,15 +104,7 @@ __device__ __forceinline__ float ld_bf16_sm(const uint8_t* base, uint32_t off) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
 }
 
-// 8 bf16 (one 16-byte chunk) <-> 8 floats
-__device__ __forceinline__ void unpack8(uint4 u, float* f) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int x = 0; x < 4; ++x) {
-        f[2 * x] = __uint_as_float(w[x] << 16);
-        f[2 * x + 1] = __uint_as_float(w[x] & 0xFFFF0000u);
-    }
-}
+// 8 floats -> 8 bf16 (one 16-byte chunk)
 __device__ __forceinline__ uint4 pack8(const float* f) {
     uint4 u;
     u.x = tc::pack_bf16x2(f[0], f[1]);
@@ -126,40 +113,34 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
     u.w = tc::pack_bf16x2(f[6], f[7]);
     return u;
 }
+// 8 packed bf16 products, each rounded once to bf16
+__device__ __forceinline__ uint32_t mul2(uint32_t x, uint32_t y) {
+    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&x),
+                               *reinterpret_cast<__nv_bfloat162*>(&y));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint4 mul8(uint4 x, uint4 y) {
+    return make_uint4(mul2(x.x, y.x), mul2(x.y, y.y), mul2(x.z, y.z), mul2(x.w, y.w));
+}
+__device__ __forceinline__ uint4 splat8(float v) {
+    const uint32_t p = tc::pack_bf16x2(v, v);
+    return make_uint4(p, p, p, p);
+}
+// Reciprocal to about 1 ulp (one SFU op); its results are rounded to bf16.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 
 // ---------------------------------------------------------------- UT solve
 // T = (I + N)^{-1}, N strictly lower 64 x 64 in NS, T into TS (both float,
 // row stride NSP).  The four 16 x 16 diagonal blocks by right-looking
 // substitution, then the off-diagonal blocks level by level:
 //   T_IJ = -T_II * P,  P = sum_{s in blocks J..I-1} N[I rows][s] T[s][J cols].
-template <int LVL>
-__device__ __forceinline__ void ut_level(const float* NS, float* TS, float* PS, int tid) {
-    constexpr int NB = 4 - LVL;
-    for (int x = tid; x < NB * 256; x += NT) {
-        const int b = x >> 8, e = x & 255, rho = e >> 4, kap = e & 15;
-        const int I = LVL + b, J = b;
-        const float* nr = NS + (16 * I + rho) * NSP + 16 * J;
-        const float* tc_ = TS + (16 * J) * NSP + 16 * J + kap;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int s = 0; s < 16 * LVL; ++s) acc[s & 3] = fmaf(nr[s], tc_[s * NSP], acc[s & 3]);
-        PS[x] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-    }
-    __syncthreads();
-    for (int x = tid; x < NB * 256; x += NT) {
-        const int b = x >> 8, e = x & 255, rho = e >> 4, kap = e & 15;
-        const int I = LVL + b, J = b;
-        const float* tr = TS + (16 * I + rho) * NSP + 16 * I;  // row of T_II (zero above diag)
-        const float* pc = PS + (b << 8) + kap;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int sg = 0; sg < 16; ++sg) acc[sg & 3] = fmaf(tr[sg], pc[sg << 4], acc[sg & 3]);
-        TS[(16 * I + rho) * NSP + 16 * J + kap] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
-    }
-    __syncthreads();
-}
-
-__device__ void ut_solve(const float* NS, float* TS, float* PS, int tid) {
+__device__ __forceinline__ void ut_diag(const float* NS, float* TS, int tid) {
     if (tid < 64) {
         const int I = tid >> 4, c = tid & 15;
         const float* nb = NS + (16 * I) * NSP + 16 * I;
@@ -176,14 +157,67 @@ __device__ void ut_solve(const float* NS, float* TS, float* PS, int tid) {
         for (int r = 0; r < 16; ++r) TS[(16 * I + r) * NSP + 16 * I + c] = x[r];
     }
     __syncthreads();
-    ut_level<1>(NS, TS, PS, tid);
-    ut_level<2>(NS, TS, PS, tid);
-    ut_level<3>(NS, TS, PS, tid);
+}
+
+// One level: blocks (I, J = I - LVL).  A thread owns four consecutive columns
+// of one row of one block, so every shared load is 16 bytes.
+template <int LVL>
+__device__ __forceinline__ void ut_level(const float* NS, float* TS, float* PS, int tid) {
+    constexpr int NB = 4 - LVL;
+    const int b = tid >> 6, rho = (tid >> 2) & 15, k4 = tid & 3;
+    const bool on = tid < NB * 64;
+    const int I = LVL + b, J = b;
+    if (on) {
+        const float* nr = NS + (16 * I + rho) * NSP + 16 * J;
+        const float* tcol = TS + (16 * J) * NSP + 16 * J + 4 * k4;
+        float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+#pragma unroll
+        for (int s4 = 0; s4 < 4 * LVL; ++s4) {
+            const float4 n4 = ld4(nr + 4 * s4);
+            const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float4 t4 = ld4(tcol + (4 * s4 + u) * NSP);
+                float4& A = acc[u & 1];
+                A.x = fmaf(nv[u], t4.x, A.x);
+                A.y = fmaf(nv[u], t4.y, A.y);
+                A.z = fmaf(nv[u], t4.z, A.z);
+                A.w = fmaf(nv[u], t4.w, A.w);
+            }
+        }
+        st4(PS + b * 256 + rho * 16 + 4 * k4,
+            make_float4(acc[0].x + acc[1].x, acc[0].y + acc[1].y, acc[0].z + acc[1].z,
+                        acc[0].w + acc[1].w));
+    }
+    __syncthreads();
+    if (on) {
+        const float* tr = TS + (16 * I + rho) * NSP + 16 * I;  // row of T_II (zero above diag)
+        const float* pc = PS + b * 256 + 4 * k4;
+        float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) {
+            const float4 t4 = ld4(tr + 4 * s4);
+            const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float4 p4 = ld4(pc + (4 * s4 + u) * 16);
+                float4& A = acc[u & 1];
+                A.x = fmaf(tv[u], p4.x, A.x);
+                A.y = fmaf(tv[u], p4.y, A.y);
+                A.z = fmaf(tv[u], p4.z, A.z);
+                A.w = fmaf(tv[u], p4.w, A.w);
+            }
+        }
+        st4(TS + (16 * I + rho) * NSP + 16 * J + 4 * k4,
+            make_float4(-(acc[0].x + acc[1].x), -(acc[0].y + acc[1].y), -(acc[0].z + acc[1].z),
+                        -(acc[0].w + acc[1].w)));
+    }
+    __syncthreads();
 }
 
 // ---------------------------------------------------------------- TMA issue
-// Group "kq": raw k and q into the RAW tile.  Group "rest": vector a and b
-// into X2, v into U, vector w into L..AQK.
+// Group "kq": raw k and q into RAW.  Group "ab": vector a and b into X1.
+// Group "vw": v into U and vector w into LQ.
 __device__ __forceinline__ void issue_kq(const TcMaps& m, uint32_t sbase, int t0, int hi, int bi,
                                          uint32_t bar) {
     tc::mbar_arrive_expect_tx(bar, 4 * BOX_BYTES);
@@ -194,17 +228,32 @@ __device__ __forceinline__ void issue_kq(const TcMaps& m, uint32_t sbase, int t0
     }
 }
 
-__device__ __forceinline__ void issue_rest(const TcMaps& m, uint32_t sbase, int t0, int hi,
-                                           int bi, bool va, bool vb, bool vw, uint32_t bar) {
-    const uint32_t nbox = 2u * (1u + (va ? 1u : 0u) + (vb ? 1u : 0u) + (vw ? 1u : 0u));
-    tc::mbar_arrive_expect_tx(bar, nbox * BOX_BYTES);
+__device__ __forceinline__ void issue_ab(const TcMaps& m, uint32_t sbase, int t0, int hi, int bi,
+                                         bool va, bool vb, uint32_t bar) {
+    tc::mbar_arrive_expect_tx(bar, 2u * ((va ? 1u : 0u) + (vb ? 1u : 0u)) * BOX_BYTES);
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+        if (va) tc::tma_load_4d(sbase + OFF_X1 + p * 16384, &m.a, 64 * p, hi, t0, bi, bar);
+        if (vb) tc::tma_load_4d(sbase + OFF_X1 + p * 16384 + 8192, &m.b, 64 * p, hi, t0, bi, bar);
+    }
+}
+
+__device__ __forceinline__ void issue_vw(const TcMaps& m, uint32_t sbase, int t0, int hi, int bi,
+                                         bool vw, uint32_t bar) {
+    tc::mbar_arrive_expect_tx(bar, 2u * (1u + (vw ? 1u : 0u)) * BOX_BYTES);
 #pragma unroll
     for (int p = 0; p < 2; ++p) {
         tc::tma_load_4d(sbase + OFF_U + p * 8192, &m.v, 64 * p, hi, t0, bi, bar);
-        if (va) tc::tma_load_4d(sbase + OFF_X2 + p * 16384, &m.a, 64 * p, hi, t0, bi, bar);
-        if (vb) tc::tma_load_4d(sbase + OFF_X2 + p * 16384 + 8192, &m.b, 64 * p, hi, t0, bi, bar);
-        if (vw) tc::tma_load_4d(sbase + OFF_L + p * 8192, &m.w, 64 * p, hi, t0, bi, bar);
+        if (vw) tc::tma_load_4d(sbase + OFF_LQ + p * 8192, &m.w, 64 * p, hi, t0, bi, bar);
     }
+}
+
+// One thread waits on `bar`; the CTA barrier that follows releases the rest.
+__device__ __forceinline__ void wait_then_sync(uint32_t bar, uint32_t parity, int tid,
+                                               volatile int* abort_s) {
+    if (tid == 0 && !tc::mbar_wait_bounded(bar, parity, WAIT_NS)) *abort_s = 1;
+    __syncthreads();
+    tc::fence_after_sync();
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -229,13 +278,14 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
     volatile int* abort_s = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
     const uint32_t bar_mma = sbase + OFF_BAR;
     const uint32_t bar_kq = sbase + OFF_BAR + 8;
-    const uint32_t bar_rs = sbase + OFF_BAR + 16;
+    const uint32_t bar_ab = sbase + OFF_BAR + 16;
+    const uint32_t bar_vw = sbase + OFF_BAR + 24;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
-    const int quarter = warp & 3;               // tensor-memory lanes 32*quarter ..
-    const int cb = warp >> 2;                   // 32-column block this warp reads
-    const int lane_j = 32 * quarter + (tid & 31);  // tensor-memory lane of this thread
+    const int quarter = warp & 3;                  // tensor-memory lanes 32*quarter ..
+    const int cb = warp >> 2;                      // 32-column block this warp reads
+    const int lane_t = 32 * quarter + (tid & 31);  // tensor-memory lane of this thread
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
 
     const int bh = blockIdx.x;
@@ -243,11 +293,13 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
     const size_t soff = (size_t)bh * D * D;
     const bool va = a_kind == GDR_GATE_VECTOR, vb = b_kind == GDR_GATE_VECTOR,
                vw = w_kind == GDR_GATE_VECTOR;
+    const bool has_ab = va || vb;
 
     if (tid == 0) {
         tc::mbar_init(bar_mma, 1);
         tc::mbar_init(bar_kq, 1);
-        tc::mbar_init(bar_rs, 1);
+        tc::mbar_init(bar_ab, 1);
+        tc::mbar_init(bar_vw, 1);
         tc::mbar_fence_init();
         *abort_s = 0;
         tc::tma_prefetch_desc(&maps.q);
@@ -256,16 +308,20 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
         tc::tma_prefetch_desc(&maps.o);
     }
     if (tid < D) fprev[tid] = 1.0f;
+    // the middle 64 rows of Z3 stay zero for the whole sequence
+    *reinterpret_cast<uint4*>(sm + OFF_Z3 + 8192 + 16 * tid) = make_uint4(0u, 0u, 0u, 0u);
     if (warp == 0) tc::tmem_alloc(sbase + OFF_TSLOT, 512);
+    tc::fence_async_smem();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + OFF_TSLOT);
-    uint32_t ph_mma = 0, ph_kq = 0, ph_rs = 0;
+    uint32_t ph_mma = 0, ph_kq = 0, ph_ab = 0, ph_vw = 0;
 
     if (tid == 0 && T > 0) {
         issue_kq(maps, sbase, 0, hi, bi, bar_kq);
-        issue_rest(maps, sbase, 0, hi, bi, va, vb, vw, bar_rs);
+        if (has_ab) issue_ab(maps, sbase, 0, hi, bi, va, vb, bar_ab);
+        issue_vw(maps, sbase, 0, hi, bi, vw, bar_vw);
     }
     // scalar gates of the next chunk, loaded a chunk ahead
     float a_nx = 1.f, b_nx = 1.f, w_nx = 1.f;
@@ -281,12 +337,21 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
     };
     if (T > 0) load_scalars(0);
 
-    // ---- initial state S0^T (unscaled) into tensor memory
+    // ---- initial state S0 (unscaled) into tensor memory: lane i, columns j
     {
         const int c0 = 32 * cb;
         float vals[32];
+        if (s0) {
+            const float4* src = reinterpret_cast<const float4*>(s0 + soff + (size_t)lane_t * D + c0);
 #pragma unroll
-        for (int x = 0; x < 32; ++x) vals[x] = s0 ? s0[soff + (size_t)(c0 + x) * D + lane_j] : 0.0f;
+            for (int x = 0; x < 8; ++x) {
+                const float4 v4 = src[x];
+                vals[4 * x] = v4.x; vals[4 * x + 1] = v4.y; vals[4 * x + 2] = v4.z; vals[4 * x + 3] = v4.w;
+            }
+        } else {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) vals[x] = 0.f;
+        }
         tc::tmem_st32(tmem + lane_off + TM_S + c0, vals);
         tc::tmem_wait_st();
     }
@@ -298,54 +363,60 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
         const int n = min(C, T - t0);
         const bool has_next = t0 + C < T;
 
-        // ================= P1: wait for the chunk, cumulative decay, operands
+        // ================= P1: wait for the chunk, decay products, operands
         if (tid < C) {
             sca[tid] = a_nx;
             sca[64 + tid] = b_nx;
             sca[128 + tid] = w_nx;
         }
-        if (tid == 0) tc::bulk_wait_read();  // the previous o store has left X1
-        if (!tc::mbar_wait_bounded(bar_kq, ph_kq, WAIT_NS)) *abort_s = 1;
-        if (!tc::mbar_wait_bounded(bar_rs, ph_rs, WAIT_NS)) *abort_s = 1;
+        if (tid == 0) {
+            tc::bulk_wait_read();  // the previous o store has left the staging tile
+            bool ok = tc::mbar_wait_bounded(bar_kq, ph_kq, WAIT_NS);
+            if (has_ab) ok = ok && tc::mbar_wait_bounded(bar_ab, ph_ab, WAIT_NS);
+            ok = ok && tc::mbar_wait_bounded(bar_vw, ph_vw, WAIT_NS);
+            if (!ok) *abort_s = 1;
+        }
         ph_kq ^= 1;
-        ph_rs ^= 1;
+        ph_ab ^= has_ab ? 1 : 0;
+        ph_vw ^= 1;
         __syncthreads();
+        // ================= P1a:
         {
-            // pass A: log-decay partial sums over 16-token quarters, channel i
+            // pass A: products of a over 16-token quarters, channel i
             const int i = tid & 127, qr = tid >> 7;
             const int pch = i >> 6, cc = i & 63;
             const uint32_t colb = ((uint32_t)(cc & 7) << 1);
             const int chunk8 = cc >> 3;
-            float run = 0.f, first = 0.f;
+            float run = 1.f, first = 1.f;
+            const uint8_t* acol = sm + OFF_X1 + (uint32_t)pch * 16384u + colb;
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 const int r = 16 * qr + u;
-                float g = 0.f;
-                if (a_kind != GDR_GATE_ONE && r < n) {
-                    const float av =
-                        va ? ld_bf16_sm(sm + OFF_X2, (uint32_t)pch * 16384u + (uint32_t)r * 128u +
-                                                         ((uint32_t)(chunk8 ^ (r & 7)) << 4) + colb)
-                           : sca[r];
-                    g = safe_log_decay(av);
-                }
-                run += g;
-                if (u == 0) first = run;
+                const float raw = va ? ld_bf16_sm(acol, (uint32_t)r * 128u +
+                                                            ((uint32_t)(chunk8 ^ (r & 7)) << 4))
+                                     : sca[r];
+                const float av = (a_kind != GDR_GATE_ONE && r < n) ? raw : 1.f;
+                run *= av;
+                if (u == 0) first = av;
                 REL[r * D + i] = run;
             }
             QT[qr * D + i] = run;
             __syncthreads();
-            // pass B: per-quarter offsets so that REL + OFS = log(gamma_r / g_m)
+            // pass B: factors so that REL * OFS = gamma_r / g_m
             const float q0 = QT[i], q1 = QT[D + i], q2 = QT[2 * D + i], q3 = QT[3 * D + i];
-            const float T0 = q0 + q1, T1 = q2 + q3;
-            const float pre = (qr > 0 ? q0 : 0.f) + (qr > 1 ? q1 : 0.f) + (qr > 2 ? q2 : 0.f);
-            OFS[qr * D + i] = pre - T0;
+            const float gm = q0 * q1;        // g_m = gamma_31
+            const float gcm = q2 * q3;       // gamma_C / g_m
+            const float inv = rcp_approx(gm);
+            OFS[qr * D + i] = qr == 0 ? inv : qr == 1 ? q0 * inv : qr == 2 ? 1.f : q2;
             if (qr == 0) {
-                fcur[i] = fprev[i] * __expf(T0);   // scale of S~ this chunk
-                fprev[i] = __expf(T1);             // gamma_C / g_m, applied next chunk
-                if (a_kind != GDR_GATE_ONE && (first - T0 > 80.f || T1 < -80.f))
+                fcur[i] = fprev[i] * gm;   // scale of S~ this chunk
+                fprev[i] = gcm;            // applied next chunk
+                // the largest factors, gamma_0/g_m and g_m/gamma_63, must stay in range
+                if (a_kind != GDR_GATE_ONE && !(gm > 0.f && first <= gm * 1e35f && gcm >= 1e-35f))
                     atomicOr(err_word, kErrRange);
             }
             __syncthreads();
+            // ================= P1c:
             // pass C: scaled operands, 8 channels (16 bytes) per access
 #pragma unroll 1
             for (int it = tid; it < C * 16; it += NT) {
@@ -354,238 +425,219 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                 const uint32_t otop = (uint32_t)p * 16384u + swz;  // rows 0-63 of 128-row tiles
                 const uint32_t obot = otop + 8192u;                // rows 64-127
                 const uint32_t o64 = (uint32_t)p * 8192u + swz;    // 64-row tiles
-                float kf[8], qf[8], bf[8], vf[8], wf[8], rel[8];
-                unpack8(*reinterpret_cast<const uint4*>(sm + OFF_RAW + otop), kf);
-                unpack8(*reinterpret_cast<const uint4*>(sm + OFF_RAW + obot), qf);
-                unpack8(*reinterpret_cast<const uint4*>(sm + OFF_U + o64), vf);
-                if (vb) {
-                    unpack8(*reinterpret_cast<const uint4*>(sm + OFF_X2 + obot), bf);
-                } else {
+                const uint4 k4 = *reinterpret_cast<const uint4*>(sm + OFF_RAW + otop);
+                const uint4 q4 = *reinterpret_cast<const uint4*>(sm + OFF_RAW + obot);
+                const uint4 v4 = *reinterpret_cast<const uint4*>(sm + OFF_U + o64);
+                const uint4 b4 = vb ? *reinterpret_cast<const uint4*>(sm + OFF_X1 + obot)
+                                    : splat8(sca[64 + r]);
+                const uint4 w4 = vw ? *reinterpret_cast<const uint4*>(sm + OFF_LQ + o64)
+                                    : splat8(sca[128 + r]);
+                const float* rp = REL + r * D + 8 * c16;
+                const float* op = OFS + (r >> 4) * D + 8 * c16;
+                const float4 r0 = ld4(rp), r1 = ld4(rp + 4), f0 = ld4(op), f1 = ld4(op + 4);
+                float e1[8] = {r0.x * f0.x, r0.y * f0.y, r0.z * f0.z, r0.w * f0.w,
+                               r1.x * f1.x, r1.y * f1.y, r1.z * f1.z, r1.w * f1.w};
+                float e1i[8];
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) bf[x] = sca[64 + r];
-                }
-                if (vw) {
-                    unpack8(*reinterpret_cast<const uint4*>(sm + OFF_L + o64), wf);
-                } else {
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) wf[x] = sca[128 + r];
-                }
-                const float4* rp = reinterpret_cast<const float4*>(REL + r * D + 8 * c16);
-                const float4* op = reinterpret_cast<const float4*>(OFS + (r >> 4) * D + 8 * c16);
-                const float4 r0 = rp[0], r1 = rp[1], f0 = op[0], f1 = op[1];
-                rel[0] = r0.x + f0.x; rel[1] = r0.y + f0.y; rel[2] = r0.z + f0.z; rel[3] = r0.w + f0.w;
-                rel[4] = r1.x + f1.x; rel[5] = r1.y + f1.y; rel[6] = r1.z + f1.z; rel[7] = r1.w + f1.w;
-                float o1[8], o2[8], o3[8], o4[8], o5[8];
-#pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    const float e1 = __expf(rel[x]);
-                    const float e1i = __expf(-rel[x]);
-                    o1[x] = kf[x] * e1;
-                    o2[x] = qf[x] * e1;
-                    o3[x] = kf[x] * e1i;
-                    o4[x] = bf[x] * kf[x] * e1i;
-                    o5[x] = wf[x] * vf[x];
-                }
-                *reinterpret_cast<uint4*>(sm + OFF_X1 + otop) = pack8(o1);
-                *reinterpret_cast<uint4*>(sm + OFF_X1 + obot) = pack8(o2);
-                *reinterpret_cast<uint4*>(sm + OFF_X2 + otop) = pack8(o3);
-                *reinterpret_cast<uint4*>(sm + OFF_X2 + obot) = pack8(o4);
-                *reinterpret_cast<uint4*>(sm + OFF_U + o64) = pack8(o5);
+                for (int x = 0; x < 8; ++x) e1i[x] = rcp_approx(e1[x]);
+                const uint4 e4 = pack8(e1), ei4 = pack8(e1i);
+                const uint4 kk1 = mul8(k4, e4);   // K'
+                const uint4 kk2 = mul8(k4, ei4);  // K"
+                *reinterpret_cast<uint4*>(sm + OFF_X1 + otop) = kk1;
+                *reinterpret_cast<uint4*>(sm + OFF_X1 + obot) = mul8(q4, e4);    // Q'
+                *reinterpret_cast<uint4*>(sm + OFF_X2 + otop) = kk2;
+                *reinterpret_cast<uint4*>(sm + OFF_X2 + obot) = mul8(b4, kk2);  // B"
+                *reinterpret_cast<uint4*>(sm + OFF_U + o64) = mul8(w4, v4);     // U
             }
         }
         tc::fence_async_smem();
         __syncthreads();
         if (*abort_s) break;
-        // the RAW tile is free: fetch the next chunk's k and q now
-        if (tid == 0 && has_next) issue_kq(maps, sbase, t0 + C, hi, bi, bar_kq);
+        if (tid == 0) {
+            // the RAW tile is free: fetch the next chunk's k and q now
+            if (has_next) issue_kq(maps, sbase, t0 + C, hi, bi, bar_kq);
+            // gram [K';Q'] [K";B"]^T needs no state: start it under the rescale
+            tc::fence_after_sync();
+            const uint32_t idKK = tc::idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                tc::mma_bf16(tmem + TM_G, tc::desc_kmajor(sbase + OFF_X1, 16384, kk),
+                             tc::desc_kmajor(sbase + OFF_X2, 16384, kk), idKK, kk > 0);
+        }
 
-        // ================= P2: S~^T <- S~^T * f (column i), bf16 copy to smem
+        // ================= P2: S~ <- f_i S~ (lane i), bf16 copy to smem
         tc::fence_after_sync();
         {
             const int c0 = 32 * cb;
+            const float f = fcur[lane_t];
             float vals[32];
             tc::tmem_ld32(tmem + lane_off + TM_S + c0, vals);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int x = 0; x < 32; ++x) vals[x] *= fcur[c0 + x];
+            for (int x = 0; x < 32; ++x) vals[x] *= f;
             tc::tmem_st32(tmem + lane_off + TM_S + c0, vals);
-            tc::store_row32_bf16(sm + OFF_S0T + (cb >> 1) * 16384, lane_j, cb & 1, vals);
+            tc::store_row32_bf16(sm + OFF_S0 + (cb >> 1) * 16384, lane_t, cb & 1, vals);
             tc::tmem_wait_st();
         }
         tc::fence_async_smem();
         tc::fence_before_sync();
         __syncthreads();
 
-        // ================= P3: gram [K';Q'] [K";B"]^T
+        // ================= P3: X = [K';Q'] S~, S~ += K"^T U (gram already issued)
         if (tid == 0) {
             tc::fence_after_sync();
-            const uint32_t id = tc::idesc_bf16(128, 128, 0, 0);
+            const uint32_t idKM = tc::idesc_bf16(128, 128, 0, 1);
+            const uint32_t idMM = tc::idesc_bf16(128, 128, 1, 1);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-                tc::mma_bf16(tmem + TM_G, tc::desc_kmajor(sbase + OFF_X1, 16384, kk),
-                             tc::desc_kmajor(sbase + OFF_X2, 16384, kk), id, kk > 0);
+                tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_X1, 16384, kk),
+                             tc::desc_mnmajor(sbase + OFF_S0, 16384, kk), idKM, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                tc::mma_bf16(tmem + TM_S, tc::desc_mnmajor(sbase + OFF_X2, 16384, kk),
+                             tc::desc_mnmajor(sbase + OFF_U, 8192, kk), idMM, true);
             tc::mma_commit(bar_mma);
         }
-        if (!tc::mbar_wait_bounded(bar_mma, ph_mma, WAIT_NS)) *abort_s = 1;
+        wait_then_sync(bar_mma, ph_mma, tid, abort_s);
         ph_mma ^= 1;
-        tc::fence_after_sync();
+        // X1 is free: fetch the next chunk's vector a and b
+        if (tid == 0 && has_next && has_ab) issue_ab(maps, sbase, t0 + C, hi, bi, va, vb, bar_ab);
 
         // ================= P4: read the gram; masked blocks out
         {
-            float vals[32];
-            tc::tmem_ld32(tmem + lane_off + TM_G + 32 * cb, vals);
-            tc::tmem_wait_ld();
-            const bool top = lane_j < 64;  // rows of K' (else Q')
-            const int r = top ? lane_j : lane_j - 64;
+            // This warp's 32 x 32 block lies below (mode < 0), on (0) or above
+            // (> 0) the diagonal of its 64 x 64 gram block: warp-uniform.
+            const int mode = (cb & 1) - (quarter & 1);
+            const bool top = lane_t < 64;  // rows of K' (else Q')
+            const int r = top ? lane_t : lane_t - 64;
             const int s0c = 32 * (cb & 1);  // first s of this column block
-            if (cb < 2) {
-                // A_kk (strictly lower) or A_qk (lower incl. diagonal)
+            float vals[32];
+            if (mode > 0) {
 #pragma unroll
-                for (int x = 0; x < 32; ++x)
-                    vals[x] = (top ? (s0c + x < r) : (s0c + x <= r)) ? vals[x] : 0.f;
-                tc::store_row32_bf16(sm + (top ? OFF_L : OFF_AQK), r, cb & 1, vals);
+                for (int x = 0; x < 32; ++x) vals[x] = 0.f;
+            } else {
+                tc::tmem_ld32(tmem + lane_off + TM_G + 32 * cb, vals);
+                tc::tmem_wait_ld();
+                if (mode == 0) {
+                    // strictly lower for the K' rows, diagonal included for Q'
+                    const int lim = top ? r - s0c : r - s0c + 1;
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) vals[x] = x < lim ? vals[x] : 0.f;
+                }
+            }
+            if (cb < 2) {
+                tc::store_row32_bf16(sm + OFF_LQ, lane_t, cb & 1, vals);   // [A_kk; A_qk]
             } else if (top) {
                 float* nrow = NS + r * NSP + s0c;
 #pragma unroll
-                for (int x = 0; x < 32; ++x) nrow[x] = (s0c + x < r) ? vals[x] : 0.f;
+                for (int x = 0; x < 32; x += 4)
+                    st4(nrow + x, make_float4(vals[x], vals[x + 1], vals[x + 2], vals[x + 3]));
             } else {
 #pragma unroll
-                for (int x = 0; x < 32; ++x) vals[x] = (s0c + x <= r) ? -vals[x] : 0.f;
-                tc::store_row32_bf16(sm + OFF_AQB, r, cb & 1, vals);
+                for (int x = 0; x < 32; ++x) vals[x] = -vals[x];
+                tc::store_row32_bf16(sm + OFF_Z3, 128 + r, cb & 1, vals);  // -A_qb
             }
         }
+        tc::fence_async_smem();
         tc::fence_before_sync();
         __syncthreads();
+        // X += [A_kk; A_qk] U: runs under the solve
+        if (tid == 0) {
+            tc::fence_after_sync();
+            const uint32_t idKM = tc::idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_LQ, 16384, kk),
+                             tc::desc_mnmajor(sbase + OFF_U, 8192, kk), idKM, true);
+            tc::mma_commit(bar_mma);
+        }
         if (*abort_s) break;
 
         // ================= P5: UT transform T = (I + A_kb)^{-1}
-        ut_solve(NS, TS, PS, tid);
+        ut_diag(NS, TS, tid);
+        // ================= P5b:
+        ut_level<1>(NS, TS, PS, tid);
+        // ================= P5c:
+        ut_level<2>(NS, TS, PS, tid);
+        ut_level<3>(NS, TS, PS, tid);
+        // ================= P5d:
         {
-            const int r = tid >> 3, ch = tid & 7;  // 64 rows x 8 chunks of 8
+            const int r = tid >> 3, ch = tid & 7;  // T - I, 64 rows x 8 chunks of 8
             float vals[8];
             const float* trow = TS + r * NSP + 8 * ch;
 #pragma unroll
-            for (int x = 0; x < 8; ++x) vals[x] = (8 * ch + x <= r) ? trow[x] : 0.f;
-            *reinterpret_cast<uint4*>(sm + OFF_T + r * 128 + ((ch ^ (r & 7)) << 4)) = pack8(vals);
+            for (int x = 0; x < 8; ++x) vals[x] = (8 * ch + x < r) ? trow[x] : 0.f;
+            *reinterpret_cast<uint4*>(sm + OFF_Z3 + r * 128 + ((ch ^ (r & 7)) << 4)) = pack8(vals);
         }
         tc::fence_async_smem();
-        __syncthreads();
 
-        // ================= P6: (T K')^T = K'^T T^T and (A_kk U)^T = U^T A_kk^T
-        if (tid == 0) {
-            tc::fence_after_sync();
-            const uint32_t id = tc::idesc_bf16(128, 64, 1, 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                tc::mma_bf16(tmem + TM_W, tc::desc_mnmajor(sbase + OFF_X1, 16384, kk),
-                             tc::desc_kmajor(sbase + OFF_T, 8192, kk), id, kk > 0);
-                tc::mma_bf16(tmem + TM_Z, tc::desc_mnmajor(sbase + OFF_U, 8192, kk),
-                             tc::desc_kmajor(sbase + OFF_L, 8192, kk), id, kk > 0);
-            }
-            tc::mma_commit(bar_mma);
-        }
-        if (!tc::mbar_wait_bounded(bar_mma, ph_mma, WAIT_NS)) *abort_s = 1;
+        // ================= P6: R -> bf16; X += [T - I; 0] R (rows 0-63 become E)
+        wait_then_sync(bar_mma, ph_mma, tid, abort_s);
         ph_mma ^= 1;
-        tc::fence_after_sync();
-
-        // ================= P7: (T K')^T -> smem [i][r], (A_kk U)^T -> smem [j][s]
-        {
-            float vals[32];
-            tc::tmem_ld32(tmem + lane_off + TM_W + 32 * cb, vals);  // TM_Z = TM_W + 64
-            tc::tmem_wait_ld();
-            tc::store_row32_bf16(sm + (cb < 2 ? OFF_W : OFF_ZT), lane_j, cb & 1, vals);
-        }
-        tc::fence_async_smem();
-        tc::fence_before_sync();
-        __syncthreads();
-
-        // ================= P8: E^T = S~^T (T K')^T + (A_kk U)^T T^T
-        if (tid == 0) {
-            tc::fence_after_sync();
-            const uint32_t id1 = tc::idesc_bf16(128, 64, 0, 1);
-            const uint32_t id2 = tc::idesc_bf16(128, 64, 0, 0);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                tc::mma_bf16(tmem + TM_E, tc::desc_kmajor(sbase + OFF_S0T, 16384, kk),
-                             tc::desc_mnmajor(sbase + OFF_W, 16384, kk), id1, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_E, tc::desc_kmajor(sbase + OFF_ZT, 16384, kk),
-                             tc::desc_kmajor(sbase + OFF_T, 8192, kk), id2, true);
-            tc::mma_commit(bar_mma);
-        }
-        if (!tc::mbar_wait_bounded(bar_mma, ph_mma, WAIT_NS)) *abort_s = 1;
-        ph_mma ^= 1;
-        tc::fence_after_sync();
-
-        // ================= P9: E^T -> smem [j][r]
-        if (cb < 2) {
-            float vals[32];
-            tc::tmem_ld32(tmem + lane_off + TM_E + 32 * cb, vals);
-            tc::tmem_wait_ld();
-            tc::store_row32_bf16(sm + OFF_ET, lane_j, cb, vals);
-        }
-        tc::fence_async_smem();
-        tc::fence_before_sync();
-        __syncthreads();
-
-        // ================= P10: O^T and the state update
-        if (tid == 0) {
-            tc::fence_after_sync();
-            const uint32_t idKK = tc::idesc_bf16(128, 64, 0, 0);
-            const uint32_t idMK = tc::idesc_bf16(128, 64, 1, 0);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                tc::mma_bf16(tmem + TM_O, tc::desc_kmajor(sbase + OFF_S0T, 16384, kk),
-                             tc::desc_kmajor(sbase + OFF_X1 + 8192, 16384, kk), idKK, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_O, tc::desc_mnmajor(sbase + OFF_U, 8192, kk),
-                             tc::desc_kmajor(sbase + OFF_AQK, 8192, kk), idMK, true);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_O, tc::desc_kmajor(sbase + OFF_ET, 16384, kk),
-                             tc::desc_kmajor(sbase + OFF_AQB, 8192, kk), idKK, true);
-            const uint32_t idMM = tc::idesc_bf16(128, 128, 1, 1);
-            const uint32_t idKMn = tc::idesc_bf16(128, 128, 0, 1) | IDESC_NEG_B;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_S, tc::desc_mnmajor(sbase + OFF_U, 8192, kk),
-                             tc::desc_mnmajor(sbase + OFF_X2, 16384, kk), idMM, true);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_S, tc::desc_kmajor(sbase + OFF_ET, 16384, kk),
-                             tc::desc_mnmajor(sbase + OFF_X2 + 8192, 16384, kk), idKMn, true);
-            tc::mma_commit(bar_mma);
-        }
-        if (!tc::mbar_wait_bounded(bar_mma, ph_mma, WAIT_NS)) *abort_s = 1;
-        ph_mma ^= 1;
-        tc::fence_after_sync();
-        // X2, U, L..AQK are free: fetch the next chunk's v and vector gates
-        if (tid == 0 && has_next) issue_rest(maps, sbase, t0 + C, hi, bi, va, vb, vw, bar_rs);
+        // U and LQ are free: fetch the next chunk's v and vector w
+        if (tid == 0 && has_next) issue_vw(maps, sbase, t0 + C, hi, bi, vw, bar_vw);
         if (has_next) load_scalars(t0 + C);
-
-        // ================= P11: O^T -> [token][channel] tile in X1 -> TMA store
-        if (cb < 2) {
+        if (quarter < 2) {
             float vals[32];
-            tc::tmem_ld32(tmem + lane_off + TM_O + 32 * cb, vals);
+            tc::tmem_ld32(tmem + lane_off + TM_X + 32 * cb, vals);
             tc::tmem_wait_ld();
-            const int j = lane_j, pj = j >> 6, cj = j & 63;
-#pragma unroll
-            for (int x = 0; x < 32; ++x) {
-                const int r = 32 * cb + x;
-                const uint32_t off = (uint32_t)pj * 8192u + (uint32_t)r * 128u +
-                                     ((uint32_t)(((cj >> 3) ^ (r & 7))) << 4) +
-                                     ((uint32_t)(cj & 7) << 1);
-                *reinterpret_cast<__nv_bfloat16*>(sm + OFF_X1 + off) = __float2bfloat16_rn(vals[x]);
-            }
+            tc::store_row32_bf16(sm + OFF_RB + (cb >> 1) * 8192, lane_t, cb & 1, vals);
         }
         tc::fence_async_smem();
         tc::fence_before_sync();
         __syncthreads();
         if (tid == 0) {
-            tc::tma_store_4d(&maps.o, sbase + OFF_X1, 0, hi, t0, bi);
-            tc::tma_store_4d(&maps.o, sbase + OFF_X1 + 8192, 64, hi, t0, bi);
+            tc::fence_after_sync();
+            const uint32_t idKM = tc::idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_Z3, 8192, kk),
+                             tc::desc_mnmajor(sbase + OFF_RB, 8192, kk), idKM, true);
+            tc::mma_commit(bar_mma);
+        }
+        wait_then_sync(bar_mma, ph_mma, tid, abort_s);
+        ph_mma ^= 1;
+
+        // ================= P7: E -> bf16; X += [0; -A_qb] E; S~ -= B"^T E
+        if (quarter < 2) {
+            float vals[32];
+            tc::tmem_ld32(tmem + lane_off + TM_X + 32 * cb, vals);
+            tc::tmem_wait_ld();
+            tc::store_row32_bf16(sm + OFF_EB + (cb >> 1) * 8192, lane_t, cb & 1, vals);
+        }
+        tc::fence_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            tc::fence_after_sync();
+            const uint32_t idKM = tc::idesc_bf16(128, 128, 0, 1);
+            const uint32_t idMMn = tc::idesc_bf16(128, 128, 1, 1) | IDESC_NEG_B;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_Z3 + 8192, 8192, kk),
+                             tc::desc_mnmajor(sbase + OFF_EB, 8192, kk), idKM, true);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                tc::mma_bf16(tmem + TM_S, tc::desc_mnmajor(sbase + OFF_X2 + 8192, 16384, kk),
+                             tc::desc_mnmajor(sbase + OFF_EB, 8192, kk), idMMn, true);
+            tc::mma_commit(bar_mma);
+        }
+        wait_then_sync(bar_mma, ph_mma, tid, abort_s);
+        ph_mma ^= 1;
+
+        // ================= P8: O (rows 64-127 of X) -> staging tile -> TMA store
+        if (quarter >= 2) {
+            float vals[32];
+            tc::tmem_ld32(tmem + lane_off + TM_X + 32 * cb, vals);
+            tc::tmem_wait_ld();
+            tc::store_row32_bf16(sm + OFF_S0 + (cb >> 1) * 8192, lane_t - 64, cb & 1, vals);
+        }
+        tc::fence_async_smem();
+        tc::fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            tc::tma_store_4d(&maps.o, sbase + OFF_S0, 0, hi, t0, bi);
+            tc::tma_store_4d(&maps.o, sbase + OFF_S0 + 8192, 64, hi, t0, bi);
             tc::bulk_commit();
         }
         if (*abort_s) break;
@@ -598,18 +650,22 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
         if (tid == 0) {
             tc::mbar_wait_bounded(bar_mma, ph_mma, WAIT_NS);
             tc::mbar_wait_bounded(bar_kq, ph_kq, WAIT_NS);
-            tc::mbar_wait_bounded(bar_rs, ph_rs, WAIT_NS);
+            if (has_ab) tc::mbar_wait_bounded(bar_ab, ph_ab, WAIT_NS);
+            tc::mbar_wait_bounded(bar_vw, ph_vw, WAIT_NS);
         }
         __syncthreads();
     } else if (s_final) {
         tc::fence_after_sync();
         const int c0 = 32 * cb;
+        const float f = fprev[lane_t];
         float vals[32];
         tc::tmem_ld32(tmem + lane_off + TM_S + c0, vals);
         tc::tmem_wait_ld();
+        float4* dst = reinterpret_cast<float4*>(s_final + soff + (size_t)lane_t * D + c0);
 #pragma unroll
-        for (int x = 0; x < 32; ++x)
-            s_final[soff + (size_t)(c0 + x) * D + lane_j] = vals[x] * fprev[c0 + x];
+        for (int x = 0; x < 8; ++x)
+            dst[x] = make_float4(vals[4 * x] * f, vals[4 * x + 1] * f, vals[4 * x + 2] * f,
+                                 vals[4 * x + 3] * f);
     }
     tc::fence_before_sync();
     __syncthreads();
