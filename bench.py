@@ -170,8 +170,10 @@ def run_reference(args):
     from gated_delta_rule_154_b200 import workload as W
     wl = W.WORKLOADS[PREFILL]
     vals = []
+    # each step is a bounded sample so the whole run stays within a few minutes
+    per_step = min(args.ref_seconds, 150.0 / max(1, args.warmup + args.steps))
     for i in range(args.warmup + args.steps):
-        v, cores, sample, dt = oracle_throughput(wl, seed=0, target_s=args.ref_seconds)
+        v, cores, sample, dt = oracle_throughput(wl, seed=0, target_s=per_step)
         if i >= args.warmup:
             vals.append((v, dt))
     value = statistics.median(v for v, _ in vals)
@@ -193,6 +195,37 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------ rank plumbing
+
+class Ranks:
+    """Barrier and max-over-ranks timing over whatever process group is
+    initialised (NCCL on GPUs; gloo in the CPU tests).  A world of one needs
+    no process group."""
+
+    def __init__(self, world: int, device=None):
+        self.world = world
+        self.device = device
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, x: float) -> float:
+        if self.world == 1:
+            return x
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own batch (weak scaling): seed = rank."""
+    return rank
+
+
 # ------------------------------------------------------------------ the GPU arm
 
 def run_gpu(args):
@@ -212,22 +245,15 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks(world, dev)
+    barrier = ranks.barrier
+    max_over_ranks = ranks.max
 
     peaks, peak_src = load_peaks()
     wl = W.WORKLOADS[PREFILL]
     if args.T:
         wl = wl.replace(T=args.T)
-    inp = W.make_prefill(wl, seed=rank)
+    inp = W.make_prefill(wl, seed=rank_seed(rank))
 
     def dev_t(x, dtype):
         if x is None:
@@ -322,10 +348,12 @@ def run_gpu(args):
     dec = None
     if not args.no_decode:
         dwl = W.WORKLOADS[DECODE]
-        state = torch.from_numpy(W.make_decode_state(dwl, seed=rank)).to(dev)
+        if args.decode_batch:
+            dwl = dwl.replace(B=args.decode_batch)
+        state = torch.from_numpy(W.make_decode_state(dwl, seed=rank_seed(rank))).to(dev)
         pool = []
         for s in range(1, args.decode_pool + 1):
-            x = W.make_decode_step(dwl, s, seed=rank)
+            x = W.make_decode_step(dwl, s, seed=rank_seed(rank))
             pool.append({k: dev_t(x[k], dwl.dtype) for k in ("q", "k", "v", "a", "b", "w")})
         od = torch.empty((dwl.B, dwl.H, dwl.dv), dtype=torch.bfloat16, device=dev)
 
@@ -405,6 +433,7 @@ def main():
     ap.add_argument("--T", type=int, default=0, help="override the sequence length")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--decode-pool", type=int, default=2)
+    ap.add_argument("--decode-batch", type=int, default=0, help="override the decode batch")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=10.0)
