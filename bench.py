@@ -47,6 +47,30 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
+def measured_traffic():
+    """DRAM bytes per prefill launch from the committed ncu summary, or None
+    when the kernel sources changed since that capture."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "chunked_tc_gdn2_bf16_T1024.md")
+    if not os.path.exists(prof):
+        return None
+    fields = {}
+    for line in open(prof):
+        if ":" in line and not line.startswith(("|", "#", " ")):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    csrc = os.path.join(ROOT, "gated_delta_rule_154_b200", "csrc")
+    h = hashlib.sha256()
+    for name in ("chunked_tc.cu", "tc_common.cuh"):
+        h.update(open(os.path.join(csrc, name), "rb").read())
+    if fields.get("source_sha256") != h.hexdigest():
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch_scaled"])
+    except (KeyError, ValueError):
+        return None
+
+
 def prefill_bytes(wl) -> int:
     """Algorithmic HBM bytes of one prefill: every input read once, o written
     once, s0 read and S_T written once (no intermediates)."""
@@ -407,7 +431,10 @@ def run_gpu(args):
                    "parallelism": "dp%d (independent sequences per rank)" % world,
                    "l2": "inputs (%.2f GB per rank) larger than L2" % (alg_bytes / 1e9)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None,
+                     "frac": achieved / hbm_peak,
+                     "traffic": measured_traffic() if (wl.T == 8192 and world >= 1) else None,
+                     "traffic_source": "ncu dram__bytes_read+write at T=1024 scaled x8 "
+                                       "(profiles/chunked_tc_gdn2_bf16_T1024.md)",
                      "peak_source": "%s hbm_gbs" % peak_src,
                      "algorithmic_bytes_per_launch": alg_bytes,
                      "tensor_flops_per_launch": flops,
