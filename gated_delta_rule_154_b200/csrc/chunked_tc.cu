@@ -159,58 +159,66 @@ __device__ __forceinline__ void ut_diag(const float* NS, float* TS, int tid) {
     __syncthreads();
 }
 
-// One level: blocks (I, J = I - LVL).  A thread owns four consecutive columns
-// of one row of one block, so every shared load is 16 bytes.
+// tf32 operand of mma.sync (round to nearest, ties away)
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+// D(16x8) += A(16x8) B(8x8), tf32 inputs, float32 accumulate (one warp).
+__device__ __forceinline__ void mma_tf32_16x8x8(float* d, const uint32_t* a, const uint32_t* b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// One level: blocks (I, J = I - LVL), each 16 x 16, two warps per block (one
+// per 8-column half).  The 16 x 16 x 16k block products are tiny and
+// latency-bound, so they use the warp-level mma.sync tensor path in tf32
+// (T is rounded to bf16 afterwards); the chunk's large products stay on
+// tcgen05.  Fragments: g = lane/4, t = lane%4; A rows g, g+8 and columns
+// t, t+4; B rows t, t+4 and column g; D rows g, g+8 and columns 2t, 2t+1.
 template <int LVL>
 __device__ __forceinline__ void ut_level(const float* NS, float* TS, float* PS, int tid) {
     constexpr int NB = 4 - LVL;
-    const int b = tid >> 6, rho = (tid >> 2) & 15, k4 = tid & 3;
-    const bool on = tid < NB * 64;
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+    const int b = warp >> 1, nt = warp & 1;
+    const bool on = warp < 2 * NB;
     const int I = LVL + b, J = b;
     if (on) {
-        const float* nr = NS + (16 * I + rho) * NSP + 16 * J;
-        const float* tcol = TS + (16 * J) * NSP + 16 * J + 4 * k4;
-        float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+        // P[:, 8nt..8nt+7] = N[I rows][16J .. 16I) T[16J .. 16I)[J cols]
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        const float* n0 = NS + (16 * I + g) * NSP + 16 * J + t;
+        const float* t0 = TS + (16 * J + t) * NSP + 16 * J + 8 * nt + g;
 #pragma unroll
-        for (int s4 = 0; s4 < 4 * LVL; ++s4) {
-            const float4 n4 = ld4(nr + 4 * s4);
-            const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float4 t4 = ld4(tcol + (4 * s4 + u) * NSP);
-                float4& A = acc[u & 1];
-                A.x = fmaf(nv[u], t4.x, A.x);
-                A.y = fmaf(nv[u], t4.y, A.y);
-                A.z = fmaf(nv[u], t4.z, A.z);
-                A.w = fmaf(nv[u], t4.w, A.w);
-            }
+        for (int ks = 0; ks < 2 * LVL; ++ks) {
+            const uint32_t af[4] = {to_tf32(n0[8 * ks]), to_tf32(n0[8 * NSP + 8 * ks]),
+                                    to_tf32(n0[8 * ks + 4]), to_tf32(n0[8 * NSP + 8 * ks + 4])};
+            const uint32_t bfr[2] = {to_tf32(t0[(8 * ks) * NSP]), to_tf32(t0[(8 * ks + 4) * NSP])};
+            mma_tf32_16x8x8(d, af, bfr);
         }
-        st4(PS + b * 256 + rho * 16 + 4 * k4,
-            make_float4(acc[0].x + acc[1].x, acc[0].y + acc[1].y, acc[0].z + acc[1].z,
-                        acc[0].w + acc[1].w));
+        float* pp = PS + b * 256 + 8 * nt + 2 * t;
+        *reinterpret_cast<float2*>(pp + g * 16) = make_float2(d[0], d[1]);
+        *reinterpret_cast<float2*>(pp + (g + 8) * 16) = make_float2(d[2], d[3]);
     }
     __syncthreads();
     if (on) {
-        const float* tr = TS + (16 * I + rho) * NSP + 16 * I;  // row of T_II (zero above diag)
-        const float* pc = PS + b * 256 + 4 * k4;
-        float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+        // T_IJ[:, 8nt..] = -T_II P[:, 8nt..]
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        const float* a0p = TS + (16 * I + g) * NSP + 16 * I + t;
+        const float* b0p = PS + b * 256 + t * 16 + 8 * nt + g;
 #pragma unroll
-        for (int s4 = 0; s4 < 4; ++s4) {
-            const float4 t4 = ld4(tr + 4 * s4);
-            const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float4 p4 = ld4(pc + (4 * s4 + u) * 16);
-                float4& A = acc[u & 1];
-                A.x = fmaf(tv[u], p4.x, A.x);
-                A.y = fmaf(tv[u], p4.y, A.y);
-                A.z = fmaf(tv[u], p4.z, A.z);
-                A.w = fmaf(tv[u], p4.w, A.w);
-            }
+        for (int ks = 0; ks < 2; ++ks) {
+            const uint32_t af[4] = {to_tf32(a0p[8 * ks]), to_tf32(a0p[8 * NSP + 8 * ks]),
+                                    to_tf32(a0p[8 * ks + 4]), to_tf32(a0p[8 * NSP + 8 * ks + 4])};
+            const uint32_t bfr[2] = {to_tf32(b0p[(8 * ks) * 16]), to_tf32(b0p[(8 * ks + 4) * 16])};
+            mma_tf32_16x8x8(d, af, bfr);
         }
-        st4(TS + (16 * I + rho) * NSP + 16 * J + 4 * k4,
-            make_float4(-(acc[0].x + acc[1].x), -(acc[0].y + acc[1].y), -(acc[0].z + acc[1].z),
-                        -(acc[0].w + acc[1].w)));
+        float* tp = TS + (16 * I + g) * NSP + 16 * J + 8 * nt + 2 * t;
+        *reinterpret_cast<float2*>(tp) = make_float2(-d[0], -d[1]);
+        *reinterpret_cast<float2*>(tp + 8 * NSP) = make_float2(-d[2], -d[3]);
     }
     __syncthreads();
 }
