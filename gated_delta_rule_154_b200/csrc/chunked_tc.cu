@@ -61,23 +61,25 @@ constexpr uint32_t OFF_RAW = 0;         // raw k (rows 0-63) and q (rows 64-127)
 constexpr uint32_t OFF_X1 = 32768;      // [K'; Q'] 128 x 128 (raw a, b land here)
 constexpr uint32_t OFF_X2 = 65536;      // [K"; B"] 128 x 128
 constexpr uint32_t OFF_U = 98304;       // U = w*v [s][j] 64 x 128 (raw v lands here)
-constexpr uint32_t OFF_LQ = 114688;     // [A_kk; A_qk] 128 x 64 (raw w lands here)
+constexpr uint32_t OFF_LQ = 114688;     // [A_kk; A_qk] 128 x 64; then R bf16 [s][j] 64 x 128
+                                        // (raw w lands here)
 constexpr uint32_t OFF_Z3 = 131072;     // [T - I; 0; -A_qb] 192 x 64
-constexpr uint32_t OFF_S0 = 155648;     // S~ [i][j] bf16 128 x 128; o staging 64 x 128
-constexpr uint32_t OFF_R = 188416;      // scratch region, 38 KB:
-constexpr uint32_t OFF_REL = OFF_R;             //  P1: decay products, float [64][128]
-constexpr uint32_t OFF_QT = OFF_R + 32768;      //  P1: quarter products, float [4][128]
-constexpr uint32_t OFF_OFS = OFF_R + 34816;     //  P1: per-quarter factors, float [4][128]
+constexpr uint32_t OFF_S0 = 155648;     // S~ [i][j] bf16 128 x 128; before it, the next
+                                        // chunk's decay factors:
+constexpr uint32_t OFF_E1 = OFF_S0;             //  gamma_r/g_m, bf16 [64][128]
+constexpr uint32_t OFF_E1I = OFF_S0 + 16384;    //  g_m/gamma_r, bf16 [64][128]
+constexpr uint32_t OFF_R = 188416;      // scratch region:
 constexpr uint32_t OFF_NS = OFF_R;              //  P4-P5: A_kb, float [64][68]
 constexpr uint32_t OFF_TS = OFF_R + 17408;      //  P5: T, float [64][68]
 constexpr uint32_t OFF_PS = OFF_R + 34816;      //  P5: float [3][16][16]
-constexpr uint32_t OFF_RB = OFF_R;              //  P6: R bf16 [s][j] 64 x 128
+constexpr uint32_t OFF_OST = OFF_R;             //  P8: o staging [r][j] 64 x 128
 constexpr uint32_t OFF_EB = OFF_R + 16384;      //  P7: E bf16 [s][j] 64 x 128
-constexpr uint32_t OFF_SMALL = OFF_R + 38912;   // 227328
+constexpr uint32_t OFF_SMALL = OFF_R + 37888;   // 226304
 constexpr uint32_t OFF_FCUR = OFF_SMALL;        // float[128]: state scale this chunk
 constexpr uint32_t OFF_FPREV = OFF_SMALL + 512; // float[128]: gamma_C/g_m of last chunk
-constexpr uint32_t OFF_SCA = OFF_SMALL + 1024;  // float[3][64]: scalar a, b, w
-constexpr uint32_t OFF_BAR = OFF_SMALL + 1792;  // 4 mbarriers: mma, kq, ab, vw
+constexpr uint32_t OFF_SCA = OFF_SMALL + 1024;  // float[2][3][64]: scalar a, b, w (2 chunks)
+constexpr uint32_t OFF_QT = OFF_SMALL + 2560;   // float[4][128]: 16-token group products
+constexpr uint32_t OFF_BAR = OFF_SMALL + 4608;  // 4 mbarriers: mma, kq, ab, vw
 constexpr uint32_t OFF_TSLOT = OFF_BAR + 32;
 constexpr uint32_t OFF_ABORT = OFF_BAR + 36;
 constexpr uint32_t SMEM_USED = OFF_BAR + 40;
@@ -99,10 +101,6 @@ constexpr uint32_t IDESC_NEG_B = 1u << 14;   // negate the B operand
 struct TcMaps {
     CUtensorMap q, k, v, a, b, w, o;  // a/b/w only meaningful for vector gates
 };
-
-__device__ __forceinline__ float ld_bf16_sm(const uint8_t* base, uint32_t off) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
-}
 
 // 8 floats -> 8 bf16 (one 16-byte chunk)
 __device__ __forceinline__ uint4 pack8(const float* f) {
@@ -132,12 +130,16 @@ __device__ __forceinline__ float rcp_approx(float x) {
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 __device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+
+// Barrier over one half of the CTA: id 1 = warps 0-7, id 2 = warps 8-15.
+__device__ __forceinline__ void half_sync(int id) {
+    asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");
+}
 
 // ---------------------------------------------------------------- UT solve
 // T = (I + N)^{-1}, N strictly lower 64 x 64 in NS, T into TS (both float,
-// row stride NSP).  The four 16 x 16 diagonal blocks by right-looking
+// row stride NSP); run by warps 0-7 (barrier id 1).  The four 16 x 16 diagonal blocks by right-looking
 // substitution, then the off-diagonal blocks level by level:
 //   T_IJ = -T_II * P,  P = sum_{s in blocks J..I-1} N[I rows][s] T[s][J cols].
 __device__ __forceinline__ void ut_diag(const float* NS, float* TS, int tid) {
@@ -156,7 +158,7 @@ __device__ __forceinline__ void ut_diag(const float* NS, float* TS, int tid) {
 #pragma unroll
         for (int r = 0; r < 16; ++r) TS[(16 * I + r) * NSP + 16 * I + c] = x[r];
     }
-    __syncthreads();
+    half_sync(1);
 }
 
 // tf32 operand of mma.sync (round to nearest, ties away)
@@ -203,7 +205,7 @@ __device__ __forceinline__ void ut_level(const float* NS, float* TS, float* PS, 
         *reinterpret_cast<float2*>(pp + g * 16) = make_float2(d[0], d[1]);
         *reinterpret_cast<float2*>(pp + (g + 8) * 16) = make_float2(d[2], d[3]);
     }
-    __syncthreads();
+    half_sync(1);
     if (on) {
         // T_IJ[:, 8nt..] = -T_II P[:, 8nt..]
         float d[4] = {0.f, 0.f, 0.f, 0.f};
@@ -220,7 +222,7 @@ __device__ __forceinline__ void ut_level(const float* NS, float* TS, float* PS, 
         *reinterpret_cast<float2*>(tp) = make_float2(-d[0], -d[1]);
         *reinterpret_cast<float2*>(tp + 8 * NSP) = make_float2(-d[2], -d[3]);
     }
-    __syncthreads();
+    half_sync(1);
 }
 
 // ---------------------------------------------------------------- TMA issue
@@ -256,6 +258,69 @@ __device__ __forceinline__ void issue_vw(const TcMaps& m, uint32_t sbase, int t0
     }
 }
 
+// Decay factors of one chunk, run by warps 8-15 (barrier id 2; u = tid - 256):
+// per key channel the products gamma_r of a over the chunk, g_m = gamma_31,
+// written as bf16 pairs gamma_r/g_m (E1) and g_m/gamma_r (E1I) [64][128];
+// fcur = fprev * g_m (scale of S~ this chunk), fprev = gamma_63/g_m; and the
+// range check of the factorisation.  Thread (pair p2 of channels, quarter q4)
+// walks 16 tokens.
+__device__ __forceinline__ void decay_pass(uint8_t* sm, int u, bool va, int a_kind, int n,
+                                           const float* sca_a, float* QT, float* fcur,
+                                           float* fprev, int* err_word) {
+    const int p2 = u & 63, q4 = u >> 6;
+    const uint32_t aoff = (uint32_t)(p2 >> 5) * 16384u + 4u * (uint32_t)(p2 & 3);
+    const int ach = (p2 & 31) >> 2;
+    float loc0[16], loc1[16];
+    float run0 = 1.f, run1 = 1.f;
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+        const int r = 16 * q4 + x;
+        float a0, a1;
+        if (va) {
+            const uint32_t pr = *reinterpret_cast<const uint32_t*>(
+                sm + OFF_X1 + aoff + (uint32_t)r * 128u + ((uint32_t)(ach ^ (r & 7)) << 4));
+            a0 = __uint_as_float(pr << 16);
+            a1 = __uint_as_float(pr & 0xFFFF0000u);
+        } else {
+            a0 = a1 = sca_a[r];
+        }
+        const bool live = a_kind != GDR_GATE_ONE && r < n;
+        run0 *= live ? a0 : 1.f;
+        run1 *= live ? a1 : 1.f;
+        loc0[x] = run0;
+        loc1[x] = run1;
+    }
+    *reinterpret_cast<float2*>(QT + q4 * D + 2 * p2) = make_float2(run0, run1);
+    half_sync(2);
+    float pre0 = 1.f, pre1 = 1.f, gm0 = 1.f, gm1 = 1.f, gc0 = 1.f, gc1 = 1.f;
+#pragma unroll
+    for (int gg = 0; gg < 4; ++gg) {
+        const float2 qv = *reinterpret_cast<const float2*>(QT + gg * D + 2 * p2);
+        if (gg < q4) { pre0 *= qv.x; pre1 *= qv.y; }
+        if (gg < 2) { gm0 *= qv.x; gm1 *= qv.y; } else { gc0 *= qv.x; gc1 *= qv.y; }
+    }
+    const float f0 = pre0 * rcp_approx(gm0), f1 = pre1 * rcp_approx(gm1);
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+        const int r = 16 * q4 + x;
+        const float e0 = loc0[x] * f0, e1v = loc1[x] * f1;
+        *reinterpret_cast<uint32_t*>(sm + OFF_E1 + r * 256 + 4 * p2) = tc::pack_bf16x2(e0, e1v);
+        *reinterpret_cast<uint32_t*>(sm + OFF_E1I + r * 256 + 4 * p2) =
+            tc::pack_bf16x2(rcp_approx(e0), rcp_approx(e1v));
+    }
+    if (q4 == 0) {
+        const int i = 2 * p2;
+        fcur[i] = fprev[i] * gm0;
+        fcur[i + 1] = fprev[i + 1] * gm1;
+        fprev[i] = gc0;
+        fprev[i + 1] = gc1;
+        // the largest factors, gamma_0/g_m and g_m/gamma_63, must stay in range
+        const bool ok0 = gm0 > 0.f && loc0[0] <= gm0 * 1e35f && gc0 >= 1e-35f;
+        const bool ok1 = gm1 > 0.f && loc1[0] <= gm1 * 1e35f && gc1 >= 1e-35f;
+        if (a_kind != GDR_GATE_ONE && !(ok0 && ok1)) atomicOr(err_word, kErrRange);
+    }
+}
+
 // One thread waits on `bar`; the CTA barrier that follows releases the rest.
 __device__ __forceinline__ void wait_then_sync(uint32_t bar, uint32_t parity, int tid,
                                                volatile int* abort_s) {
@@ -274,15 +339,13 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = tc::smem_u32(sm);
-    float* REL = reinterpret_cast<float*>(sm + OFF_REL);
     float* QT = reinterpret_cast<float*>(sm + OFF_QT);
-    float* OFS = reinterpret_cast<float*>(sm + OFF_OFS);
     float* NS = reinterpret_cast<float*>(sm + OFF_NS);
     float* TS = reinterpret_cast<float*>(sm + OFF_TS);
     float* PS = reinterpret_cast<float*>(sm + OFF_PS);
     float* fcur = reinterpret_cast<float*>(sm + OFF_FCUR);
     float* fprev = reinterpret_cast<float*>(sm + OFF_FPREV);
-    float* sca = reinterpret_cast<float*>(sm + OFF_SCA);
+    float* sca_all = reinterpret_cast<float*>(sm + OFF_SCA);  // [2][3][64]
     volatile int* abort_s = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
     const uint32_t bar_mma = sbase + OFF_BAR;
     const uint32_t bar_kq = sbase + OFF_BAR + 8;
@@ -331,19 +394,19 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
         if (has_ab) issue_ab(maps, sbase, 0, hi, bi, va, vb, bar_ab);
         issue_vw(maps, sbase, 0, hi, bi, vw, bar_vw);
     }
-    // scalar gates of the next chunk, loaded a chunk ahead
-    float a_nx = 1.f, b_nx = 1.f, w_nx = 1.f;
-    auto load_scalars = [&](int t0n) {
+    // scalar gates of chunk starting at t0n into buffer `buf` (1.0 past T)
+    auto load_scalars = [&](int t0n, int buf) {
         if (tid < C) {
             const int nn = min(C, T - t0n);
             const long long tok = ((long long)bi * T + t0n + tid) * H + hi;
             const bool in = tid < nn;
-            a_nx = (a_kind == GDR_GATE_SCALAR && in) ? to_f32(a[tok]) : 1.f;
-            b_nx = (b_kind == GDR_GATE_SCALAR && in) ? to_f32(b[tok]) : 1.f;
-            w_nx = (w_kind == GDR_GATE_SCALAR && in) ? to_f32(w[tok]) : 1.f;
+            float* sc = sca_all + buf * 192;
+            sc[tid] = (a_kind == GDR_GATE_SCALAR && in) ? to_f32(a[tok]) : 1.f;
+            sc[64 + tid] = (b_kind == GDR_GATE_SCALAR && in) ? to_f32(b[tok]) : 1.f;
+            sc[128 + tid] = (w_kind == GDR_GATE_SCALAR && in) ? to_f32(w[tok]) : 1.f;
         }
     };
-    if (T > 0) load_scalars(0);
+    if (T > 0) load_scalars(0, 0);
 
     // ---- initial state S0 (unscaled) into tensor memory: lane i, columns j
     {
@@ -365,67 +428,37 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
     }
     tc::fence_before_sync();
     __syncthreads();
+    // decay factors of the first chunk (later chunks get theirs under the
+    // previous chunk's UT solve)
+    if (T > 0 && warp >= 8) {
+        if (tid == 256 && has_ab && !tc::mbar_wait_bounded(bar_ab, ph_ab, WAIT_NS)) *abort_s = 1;
+        half_sync(2);
+        decay_pass(sm, tid - 256, va, a_kind, min(C, T), sca_all, QT, fcur, fprev, err_word);
+    }
+    ph_ab ^= (T > 0 && has_ab) ? 1 : 0;
+    __syncthreads();
 
 #pragma unroll 1
     for (int t0 = 0; t0 < T; t0 += C) {
         const int n = min(C, T - t0);
         const bool has_next = t0 + C < T;
+        const int cur = (t0 / C) & 1;
+        const float* sca = sca_all + cur * 192;
 
-        // ================= P1: wait for the chunk, decay products, operands
-        if (tid < C) {
-            sca[tid] = a_nx;
-            sca[64 + tid] = b_nx;
-            sca[128 + tid] = w_nx;
-        }
+        // ================= P1: wait for the chunk's tiles, scaled operands
         if (tid == 0) {
             tc::bulk_wait_read();  // the previous o store has left the staging tile
             bool ok = tc::mbar_wait_bounded(bar_kq, ph_kq, WAIT_NS);
-            if (has_ab) ok = ok && tc::mbar_wait_bounded(bar_ab, ph_ab, WAIT_NS);
             ok = ok && tc::mbar_wait_bounded(bar_vw, ph_vw, WAIT_NS);
             if (!ok) *abort_s = 1;
         }
         ph_kq ^= 1;
-        ph_ab ^= has_ab ? 1 : 0;
         ph_vw ^= 1;
         __syncthreads();
-        // ================= P1a:
+        // ================= P1c:
         {
-            // pass A: products of a over 16-token quarters, channel i
-            const int i = tid & 127, qr = tid >> 7;
-            const int pch = i >> 6, cc = i & 63;
-            const uint32_t colb = ((uint32_t)(cc & 7) << 1);
-            const int chunk8 = cc >> 3;
-            float run = 1.f, first = 1.f;
-            const uint8_t* acol = sm + OFF_X1 + (uint32_t)pch * 16384u + colb;
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int r = 16 * qr + u;
-                const float raw = va ? ld_bf16_sm(acol, (uint32_t)r * 128u +
-                                                            ((uint32_t)(chunk8 ^ (r & 7)) << 4))
-                                     : sca[r];
-                const float av = (a_kind != GDR_GATE_ONE && r < n) ? raw : 1.f;
-                run *= av;
-                if (u == 0) first = av;
-                REL[r * D + i] = run;
-            }
-            QT[qr * D + i] = run;
-            __syncthreads();
-            // pass B: factors so that REL * OFS = gamma_r / g_m
-            const float q0 = QT[i], q1 = QT[D + i], q2 = QT[2 * D + i], q3 = QT[3 * D + i];
-            const float gm = q0 * q1;        // g_m = gamma_31
-            const float gcm = q2 * q3;       // gamma_C / g_m
-            const float inv = rcp_approx(gm);
-            OFS[qr * D + i] = qr == 0 ? inv : qr == 1 ? q0 * inv : qr == 2 ? 1.f : q2;
-            if (qr == 0) {
-                fcur[i] = fprev[i] * gm;   // scale of S~ this chunk
-                fprev[i] = gcm;            // applied next chunk
-                // the largest factors, gamma_0/g_m and g_m/gamma_63, must stay in range
-                if (a_kind != GDR_GATE_ONE && !(gm > 0.f && first <= gm * 1e35f && gcm >= 1e-35f))
-                    atomicOr(err_word, kErrRange);
-            }
-            __syncthreads();
-            // ================= P1c:
-            // pass C: scaled operands, 8 channels (16 bytes) per access
+            // K' = e1*k, Q' = e1*q, K" = k/e1, B" = b*K", U = w*v, 8 channels
+            // (16 bytes) per access, packed bf16 products
 #pragma unroll 1
             for (int it = tid; it < C * 16; it += NT) {
                 const int r = it >> 4, c16 = it & 15, p = c16 >> 3, ch = c16 & 7;
@@ -440,15 +473,8 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                                     : splat8(sca[64 + r]);
                 const uint4 w4 = vw ? *reinterpret_cast<const uint4*>(sm + OFF_LQ + o64)
                                     : splat8(sca[128 + r]);
-                const float* rp = REL + r * D + 8 * c16;
-                const float* op = OFS + (r >> 4) * D + 8 * c16;
-                const float4 r0 = ld4(rp), r1 = ld4(rp + 4), f0 = ld4(op), f1 = ld4(op + 4);
-                float e1[8] = {r0.x * f0.x, r0.y * f0.y, r0.z * f0.z, r0.w * f0.w,
-                               r1.x * f1.x, r1.y * f1.y, r1.z * f1.z, r1.w * f1.w};
-                float e1i[8];
-#pragma unroll
-                for (int x = 0; x < 8; ++x) e1i[x] = rcp_approx(e1[x]);
-                const uint4 e4 = pack8(e1), ei4 = pack8(e1i);
+                const uint4 e4 = *reinterpret_cast<const uint4*>(sm + OFF_E1 + r * 256 + 16 * c16);
+                const uint4 ei4 = *reinterpret_cast<const uint4*>(sm + OFF_E1I + r * 256 + 16 * c16);
                 const uint4 kk1 = mul8(k4, e4);   // K'
                 const uint4 kk2 = mul8(k4, ei4);  // K"
                 *reinterpret_cast<uint4*>(sm + OFF_X1 + otop) = kk1;
@@ -508,8 +534,9 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
         }
         wait_then_sync(bar_mma, ph_mma, tid, abort_s);
         ph_mma ^= 1;
-        // X1 is free: fetch the next chunk's vector a and b
+        // X1 is free: fetch the next chunk's vector a and b; its scalar gates
         if (tid == 0 && has_next && has_ab) issue_ab(maps, sbase, t0 + C, hi, bi, va, vb, bar_ab);
+        if (has_next) load_scalars(t0 + C, cur ^ 1);
 
         // ================= P4: read the gram; masked blocks out
         {
@@ -561,50 +588,68 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
         }
         if (*abort_s) break;
 
-        // ================= P5: UT transform T = (I + A_kb)^{-1}
-        ut_diag(NS, TS, tid);
-        // ================= P5b:
-        ut_level<1>(NS, TS, PS, tid);
-        // ================= P5c:
-        ut_level<2>(NS, TS, PS, tid);
-        ut_level<3>(NS, TS, PS, tid);
-        // ================= P5d:
-        {
-            const int r = tid >> 3, ch = tid & 7;  // T - I, 64 rows x 8 chunks of 8
-            float vals[8];
-            const float* trow = TS + r * NSP + 8 * ch;
+        // ================= P5: warps 0-7: UT transform T = (I + A_kb)^{-1};
+        //                       warps 8-15: R -> bf16, next chunk's decay factors
+        if (warp < 8) {
+            ut_diag(NS, TS, tid);
+            ut_level<1>(NS, TS, PS, tid);
+            ut_level<2>(NS, TS, PS, tid);
+            ut_level<3>(NS, TS, PS, tid);
+            {
+                const int r = tid >> 2, c4 = tid & 3;  // T - I, 64 rows x 4 x 16 columns
 #pragma unroll
-            for (int x = 0; x < 8; ++x) vals[x] = (8 * ch + x < r) ? trow[x] : 0.f;
-            *reinterpret_cast<uint4*>(sm + OFF_Z3 + r * 128 + ((ch ^ (r & 7)) << 4)) = pack8(vals);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int ch = 2 * c4 + hh;
+                    float vals[8];
+                    const float* trow = TS + r * NSP + 8 * ch;
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) vals[x] = (8 * ch + x < r) ? trow[x] : 0.f;
+                    *reinterpret_cast<uint4*>(sm + OFF_Z3 + r * 128 + ((ch ^ (r & 7)) << 4)) = pack8(vals);
+                }
+            }
+            tc::fence_async_smem();
+        } else {
+            if (tid == 256 && !tc::mbar_wait_bounded(bar_mma, ph_mma, WAIT_NS)) *abort_s = 1;
+            half_sync(2);
+            tc::fence_after_sync();
+            if (quarter < 2) {   // lanes 0-63 of X hold R; each warp takes 64 columns
+                const int c0 = 64 * (cb - 2);
+                float vals[32];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    tc::tmem_ld32(tmem + lane_off + TM_X + c0 + 32 * hh, vals);
+                    tc::tmem_wait_ld();
+                    tc::store_row32_bf16(sm + OFF_LQ + (c0 >> 6) * 8192, lane_t, hh, vals);
+                }
+            }
+            tc::fence_async_smem();
+            if (has_next) {
+                if (tid == 256 && has_ab &&
+                    !tc::mbar_wait_bounded(bar_ab, ph_ab, WAIT_NS)) *abort_s = 1;
+                half_sync(2);
+                decay_pass(sm, tid - 256, va, a_kind, min(C, T - t0 - C), sca_all + (cur ^ 1) * 192,
+                           QT, fcur, fprev, err_word);
+            }
         }
-        tc::fence_async_smem();
-
-        // ================= P6: R -> bf16; X += [T - I; 0] R (rows 0-63 become E)
-        wait_then_sync(bar_mma, ph_mma, tid, abort_s);
         ph_mma ^= 1;
-        // U and LQ are free: fetch the next chunk's v and vector w
-        if (tid == 0 && has_next) issue_vw(maps, sbase, t0 + C, hi, bi, vw, bar_vw);
-        if (has_next) load_scalars(t0 + C);
-        if (quarter < 2) {
-            float vals[32];
-            tc::tmem_ld32(tmem + lane_off + TM_X + 32 * cb, vals);
-            tc::tmem_wait_ld();
-            tc::store_row32_bf16(sm + OFF_RB + (cb >> 1) * 8192, lane_t, cb & 1, vals);
-        }
-        tc::fence_async_smem();
+        ph_ab ^= (has_next && has_ab) ? 1 : 0;
         tc::fence_before_sync();
         __syncthreads();
+
+        // ================= P6: X += [T - I; 0] R (rows 0-63 become E)
         if (tid == 0) {
             tc::fence_after_sync();
             const uint32_t idKM = tc::idesc_bf16(128, 128, 0, 1);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_Z3, 8192, kk),
-                             tc::desc_mnmajor(sbase + OFF_RB, 8192, kk), idKM, true);
+                             tc::desc_mnmajor(sbase + OFF_LQ, 8192, kk), idKM, true);
             tc::mma_commit(bar_mma);
         }
         wait_then_sync(bar_mma, ph_mma, tid, abort_s);
         ph_mma ^= 1;
+        // U and LQ are free: fetch the next chunk's v and vector w
+        if (tid == 0 && has_next) issue_vw(maps, sbase, t0 + C, hi, bi, vw, bar_vw);
 
         // ================= P7: E -> bf16; X += [0; -A_qb] E; S~ -= B"^T E
         if (quarter < 2) {
@@ -638,14 +683,14 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             float vals[32];
             tc::tmem_ld32(tmem + lane_off + TM_X + 32 * cb, vals);
             tc::tmem_wait_ld();
-            tc::store_row32_bf16(sm + OFF_S0 + (cb >> 1) * 8192, lane_t - 64, cb & 1, vals);
+            tc::store_row32_bf16(sm + OFF_OST + (cb >> 1) * 8192, lane_t - 64, cb & 1, vals);
         }
         tc::fence_async_smem();
         tc::fence_before_sync();
         __syncthreads();
         if (tid == 0) {
-            tc::tma_store_4d(&maps.o, sbase + OFF_S0, 0, hi, t0, bi);
-            tc::tma_store_4d(&maps.o, sbase + OFF_S0 + 8192, 64, hi, t0, bi);
+            tc::tma_store_4d(&maps.o, sbase + OFF_OST, 0, hi, t0, bi);
+            tc::tma_store_4d(&maps.o, sbase + OFF_OST + 8192, 64, hi, t0, bi);
             tc::bulk_commit();
         }
         if (*abort_s) break;
