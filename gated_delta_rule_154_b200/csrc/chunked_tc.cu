@@ -54,38 +54,39 @@ namespace {
 
 constexpr int C = 64;        // chunk length
 constexpr int D = 128;       // dk = dv
-constexpr int NT = 512;      // threads per CTA (16 warps)
+constexpr int NTC = 512;     // compute threads (warps 0-15)
+constexpr int NT = NTC + 32; // + one warp that issues every TMA copy and tensor-core product
 
-// ---- shared memory map (bytes from a 1024-aligned base)
+// ---- shared memory map (bytes from a 1024-aligned base).  Operand tiles are
+// 64-column panels of 128-byte swizzled rows; "rows r" below are tokens.
 constexpr uint32_t OFF_RAW = 0;         // raw k (rows 0-63) and q (rows 64-127), 2 panels
-constexpr uint32_t OFF_X1 = 32768;      // [K'; Q'] 128 x 128 (raw a, b land here)
-constexpr uint32_t OFF_X2 = 65536;      // [K"; B"] 128 x 128
+constexpr uint32_t OFF_X1 = 32768;      // raw vector a and b land here (rows 0-63 / 64-127),
+                                        // replaced in place by [K'; Q'] 128 x 128
+constexpr uint32_t OFF_X2 = 65536;      // [K"; B"] 128 x 128; between the state products
+                                        // and P6 the K" rows hold R (bf16)
 constexpr uint32_t OFF_U = 98304;       // U = w*v [s][j] 64 x 128 (raw v lands here)
-constexpr uint32_t OFF_LQ = 114688;     // [A_kk; A_qk] 128 x 64; then R bf16 [s][j] 64 x 128
-                                        // (raw w lands here)
+constexpr uint32_t OFF_W = 114688;      // raw vector w 64 x 128
 constexpr uint32_t OFF_Z3 = 131072;     // [T - I; 0; -A_qb] 192 x 64
-constexpr uint32_t OFF_S0 = 155648;     // S~ [i][j] bf16 128 x 128; before it, the next
-                                        // chunk's decay factors:
-constexpr uint32_t OFF_E1 = OFF_S0;             //  gamma_r/g_m, bf16 [64][128]
-constexpr uint32_t OFF_E1I = OFF_S0 + 16384;    //  g_m/gamma_r, bf16 [64][128]
+constexpr uint32_t OFF_S0 = 155648;     // S~ [i][j] bf16 128 x 128
 constexpr uint32_t OFF_R = 188416;      // scratch region:
+constexpr uint32_t OFF_QT = OFF_R;              //  P1: float [8][128], 8-token products
 constexpr uint32_t OFF_NS = OFF_R;              //  P4-P5: A_kb, float [64][68]
 constexpr uint32_t OFF_TS = OFF_R + 17408;      //  P5: T, float [64][68]
-constexpr uint32_t OFF_PS = OFF_R + 34816;      //  P5: float [3][16][16]
-constexpr uint32_t OFF_OST = OFF_R;             //  P8: o staging [r][j] 64 x 128
-constexpr uint32_t OFF_EB = OFF_R + 16384;      //  P7: E bf16 [s][j] 64 x 128
+constexpr uint32_t OFF_PS = OFF_R + 34816;      //  P5: float [2][16][16]
+constexpr uint32_t OFF_EB = OFF_R;              //  P7: E bf16 [s][j] 64 x 128
+constexpr uint32_t OFF_OST = OFF_R + 16384;     //  P8: o staging [r][j] 64 x 128
 constexpr uint32_t OFF_SMALL = OFF_R + 37888;   // 226304
 constexpr uint32_t OFF_FCUR = OFF_SMALL;        // float[128]: state scale this chunk
 constexpr uint32_t OFF_FPREV = OFF_SMALL + 512; // float[128]: gamma_C/g_m of last chunk
 constexpr uint32_t OFF_SCA = OFF_SMALL + 1024;  // float[2][3][64]: scalar a, b, w (2 chunks)
-constexpr uint32_t OFF_QT = OFF_SMALL + 2560;   // float[4][128]: 16-token group products
-constexpr uint32_t OFF_BAR = OFF_SMALL + 4608;  // 4 mbarriers: mma, kq, ab, vw
-constexpr uint32_t OFF_TSLOT = OFF_BAR + 32;
-constexpr uint32_t OFF_ABORT = OFF_BAR + 36;
-constexpr uint32_t SMEM_USED = OFF_BAR + 40;
+constexpr uint32_t OFF_BAR = OFF_SMALL + 2560;  // NBAR mbarriers (see the kernel)
+constexpr int NBAR = 14;
+constexpr uint32_t OFF_TSLOT = OFF_BAR + 8 * NBAR;
+constexpr uint32_t OFF_ABORT = OFF_TSLOT + 4;
+constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
 constexpr size_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory");
-static_assert(OFF_PS + 3 * 256 * 4 <= OFF_SMALL, "solve scratch");
+static_assert(OFF_PS + 2 * 256 * 4 <= OFF_SMALL, "solve scratch");
 
 constexpr int NSP = 68;  // row stride (floats) of the solve's float tiles (16-byte rows)
 
@@ -93,6 +94,7 @@ constexpr int NSP = 68;  // row stride (floats) of the solve's float tiles (16-b
 constexpr uint32_t TM_G = 0;     // gram 128 x 128
 constexpr uint32_t TM_X = 128;   // [R -> E; O] 128 x 128
 constexpr uint32_t TM_S = 256;   // S~ 128 x 128 (lane = key channel), float32 state
+constexpr uint32_t TM_AQ = 384;  // A operand [A_kk; A_qk] 128 x 64 bf16 (32 columns)
 
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait
 constexpr uint32_t BOX_BYTES = 64 * 128;     // one 64 x 64 bf16 TMA box
@@ -102,27 +104,11 @@ struct TcMaps {
     CUtensorMap q, k, v, a, b, w, o;  // a/b/w only meaningful for vector gates
 };
 
-// 8 floats -> 8 bf16 (one 16-byte chunk)
-__device__ __forceinline__ uint4 pack8(const float* f) {
-    uint4 u;
-    u.x = tc::pack_bf16x2(f[0], f[1]);
-    u.y = tc::pack_bf16x2(f[2], f[3]);
-    u.z = tc::pack_bf16x2(f[4], f[5]);
-    u.w = tc::pack_bf16x2(f[6], f[7]);
-    return u;
-}
-// 8 packed bf16 products, each rounded once to bf16
+// Two packed bf16 products, each rounded once to bf16
 __device__ __forceinline__ uint32_t mul2(uint32_t x, uint32_t y) {
     __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&x),
                                *reinterpret_cast<__nv_bfloat162*>(&y));
     return *reinterpret_cast<uint32_t*>(&r);
-}
-__device__ __forceinline__ uint4 mul8(uint4 x, uint4 y) {
-    return make_uint4(mul2(x.x, y.x), mul2(x.y, y.y), mul2(x.z, y.z), mul2(x.w, y.w));
-}
-__device__ __forceinline__ uint4 splat8(float v) {
-    const uint32_t p = tc::pack_bf16x2(v, v);
-    return make_uint4(p, p, p, p);
 }
 // Reciprocal to about 1 ulp (one SFU op); its results are rounded to bf16.
 __device__ __forceinline__ float rcp_approx(float x) {
@@ -132,33 +118,63 @@ __device__ __forceinline__ float rcp_approx(float x) {
 }
 __device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 
-// Barrier over one half of the CTA: id 1 = warps 0-7, id 2 = warps 8-15.
+// Named barriers: id 1 = the 16 compute warps, id 2 = warps 0-7, id 3 =
+// warps 8-15.  (Id 0, __syncthreads, includes the issuing warp.)
+__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
 __device__ __forceinline__ void half_sync(int id) {
     asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");
 }
 
 // ---------------------------------------------------------------- UT solve
-// T = (I + N)^{-1}, N strictly lower 64 x 64 in NS, T into TS (both float,
-// row stride NSP); run by warps 0-7 (barrier id 1).  The four 16 x 16 diagonal blocks by right-looking
-// substitution, then the off-diagonal blocks level by level:
-//   T_IJ = -T_II * P,  P = sum_{s in blocks J..I-1} N[I rows][s] T[s][J cols].
-__device__ __forceinline__ void ut_diag(const float* NS, float* TS, int tid) {
+// T = (I + N)^{-1}, N = A_kb strictly lower 64 x 64 (float, row stride NSP, in
+// NS), by the 2 x 2 block recursion of a unit lower triangular inverse,
+//   [[T1, 0], [T21, T2]] with T21 = -T2 N21 T1,
+// applied at 16 and at 32 rows: the four 16 x 16 diagonal inverses by
+// substitution, then two rounds for the 16 x 16 blocks (1,0) and (3,2), then
+// two for the 32 x 32 block below the diagonal.  Run by warps 0-7 (barrier
+// id 2).  Each finished block also goes, as bf16 T - I, into rows 0-63 of
+// the Z3 operand; the blocks above the diagonal of those rows stay zero.
+
+// One element of T - I into the 128-byte swizzled Z3 rows.
+__device__ __forceinline__ void z3_put(uint8_t* z3, int row, int col, float v) {
+    *reinterpret_cast<__nv_bfloat16*>(z3 + row * 128 + (((col >> 3) ^ (row & 7)) << 4) +
+                                      2 * (col & 7)) = __float2bfloat16_rn(v);
+}
+__device__ __forceinline__ void z3_put2(uint8_t* z3, int row, int col, float v0, float v1) {
+    *reinterpret_cast<uint32_t*>(z3 + row * 128 + (((col >> 3) ^ (row & 7)) << 4) +
+                                 2 * (col & 7)) = tc::pack_bf16x2(v0, v1);
+}
+
+__device__ __forceinline__ void ut_diag(const float* NS, float* TS, uint8_t* z3, int tid) {
     if (tid < 64) {
+        // column c of the inverse of diagonal block I: x_r = [r == c] - sum_{s<r} N_rs x_s,
+        // each row of N read as 16-byte vectors, two partial sums per row
         const int I = tid >> 4, c = tid & 15;
         const float* nb = NS + (16 * I) * NSP + 16 * I;
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.0f : 0.0f;
 #pragma unroll
-        for (int s = 0; s < 15; ++s) {
-            const float xs = x[s];
+        for (int r = 1; r < 16; ++r) {
+            const float* row = nb + r * NSP;
+            float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-            for (int r = s + 1; r < 16; ++r) x[r] = fmaf(-nb[r * NSP + s], xs, x[r]);
+            for (int s4 = 0; 4 * s4 < r; ++s4) {
+                const float4 v = *reinterpret_cast<const float4*>(row + 4 * s4);
+                if (4 * s4 + 0 < r) acc0 = fmaf(v.x, x[4 * s4 + 0], acc0);
+                if (4 * s4 + 1 < r) acc1 = fmaf(v.y, x[4 * s4 + 1], acc1);
+                if (4 * s4 + 2 < r) acc0 = fmaf(v.z, x[4 * s4 + 2], acc0);
+                if (4 * s4 + 3 < r) acc1 = fmaf(v.w, x[4 * s4 + 3], acc1);
+            }
+            x[r] -= acc0 + acc1;
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) TS[(16 * I + r) * NSP + 16 * I + c] = x[r];
+        for (int r = 0; r < 16; ++r) {
+            TS[(16 * I + r) * NSP + 16 * I + c] = x[r];
+            z3_put(z3, 16 * I + r, 16 * I + c, r > c ? x[r] : 0.f);
+        }
     }
-    half_sync(1);
+    half_sync(2);
 }
 
 // tf32 operand of mma.sync (round to nearest, ties away)
@@ -176,65 +192,89 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float* d, const uint32_t* a, con
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// One level: blocks (I, J = I - LVL), each 16 x 16, two warps per block (one
-// per 8-column half).  The 16 x 16 x 16k block products are tiny and
-// latency-bound, so they use the warp-level mma.sync tensor path in tf32
-// (T is rounded to bf16 afterwards); the chunk's large products stay on
-// tcgen05.  Fragments: g = lane/4, t = lane%4; A rows g, g+8 and columns
-// t, t+4; B rows t, t+4 and column g; D rows g, g+8 and columns 2t, 2t+1.
-template <int LVL>
-__device__ __forceinline__ void ut_level(const float* NS, float* TS, float* PS, int tid) {
-    constexpr int NB = 4 - LVL;
-    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-    const int b = warp >> 1, nt = warp & 1;
-    const bool on = warp < 2 * NB;
-    const int I = LVL + b, J = b;
-    if (on) {
-        // P[:, 8nt..8nt+7] = N[I rows][16J .. 16I) T[16J .. 16I)[J cols]
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
-        const float* n0 = NS + (16 * I + g) * NSP + 16 * J + t;
-        const float* t0 = TS + (16 * J + t) * NSP + 16 * J + 8 * nt + g;
+// d = A(16 x 8KS) B(8KS x 8) for float tiles in shared memory (A at its
+// (0,0) with row stride lda, B likewise with ldb).  The block products of
+// the solve are tiny and latency-bound, so they use the warp-level mma.sync
+// path in tf32 (T is rounded to bf16 afterwards); the chunk's large products
+// stay on tcgen05.  Fragments: g = lane/4, t = lane%4; A rows g, g+8 and
+// columns t, t+4; B rows t, t+4 and column g; D rows g, g+8, columns 2t, 2t+1.
+template <int KS>
+__device__ __forceinline__ void tile_16x8(float* d, const float* A, int lda, const float* Bm,
+                                          int ldb, int g, int t) {
+    d[0] = d[1] = d[2] = d[3] = 0.f;
 #pragma unroll
-        for (int ks = 0; ks < 2 * LVL; ++ks) {
-            const uint32_t af[4] = {to_tf32(n0[8 * ks]), to_tf32(n0[8 * NSP + 8 * ks]),
-                                    to_tf32(n0[8 * ks + 4]), to_tf32(n0[8 * NSP + 8 * ks + 4])};
-            const uint32_t bfr[2] = {to_tf32(t0[(8 * ks) * NSP]), to_tf32(t0[(8 * ks + 4) * NSP])};
-            mma_tf32_16x8x8(d, af, bfr);
-        }
+    for (int ks = 0; ks < KS; ++ks) {
+        const float* a0 = A + g * lda + 8 * ks + t;
+        const float* b0 = Bm + (8 * ks + t) * ldb + g;
+        const uint32_t af[4] = {to_tf32(a0[0]), to_tf32(a0[8 * lda]), to_tf32(a0[4]),
+                                to_tf32(a0[8 * lda + 4])};
+        const uint32_t bfr[2] = {to_tf32(b0[0]), to_tf32(b0[4 * ldb])};
+        mma_tf32_16x8x8(d, af, bfr);
+    }
+}
+
+__device__ __forceinline__ void ut_solve(float* NS, float* TS, float* PS, uint8_t* z3, int tid) {
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+    ut_diag(NS, TS, z3, tid);
+    // blocks (1,0) and (3,2): P = N_IJ T_JJ, then T_IJ = -T_II P (warps 0-3)
+    const int b = warp >> 1, nt = warp & 1;
+    const int I = 2 * b + 1, J = 2 * b;
+    float d[4];
+    if (warp < 4) {
+        tile_16x8<2>(d, NS + (16 * I) * NSP + 16 * J, NSP, TS + (16 * J) * NSP + 16 * J + 8 * nt,
+                     NSP, g, t);
         float* pp = PS + b * 256 + 8 * nt + 2 * t;
         *reinterpret_cast<float2*>(pp + g * 16) = make_float2(d[0], d[1]);
         *reinterpret_cast<float2*>(pp + (g + 8) * 16) = make_float2(d[2], d[3]);
     }
-    half_sync(1);
-    if (on) {
-        // T_IJ[:, 8nt..] = -T_II P[:, 8nt..]
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
-        const float* a0p = TS + (16 * I + g) * NSP + 16 * I + t;
-        const float* b0p = PS + b * 256 + t * 16 + 8 * nt + g;
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-            const uint32_t af[4] = {to_tf32(a0p[8 * ks]), to_tf32(a0p[8 * NSP + 8 * ks]),
-                                    to_tf32(a0p[8 * ks + 4]), to_tf32(a0p[8 * NSP + 8 * ks + 4])};
-            const uint32_t bfr[2] = {to_tf32(b0p[(8 * ks) * 16]), to_tf32(b0p[(8 * ks + 4) * 16])};
-            mma_tf32_16x8x8(d, af, bfr);
-        }
-        float* tp = TS + (16 * I + g) * NSP + 16 * J + 8 * nt + 2 * t;
-        *reinterpret_cast<float2*>(tp) = make_float2(-d[0], -d[1]);
-        *reinterpret_cast<float2*>(tp + 8 * NSP) = make_float2(-d[2], -d[3]);
+    half_sync(2);
+    if (warp < 4) {
+        tile_16x8<2>(d, TS + (16 * I) * NSP + 16 * I, NSP, PS + b * 256 + 8 * nt, 16, g, t);
+        const int row = 16 * I + g, col = 16 * J + 8 * nt + 2 * t;
+        *reinterpret_cast<float2*>(TS + row * NSP + col) = make_float2(-d[0], -d[1]);
+        *reinterpret_cast<float2*>(TS + (row + 8) * NSP + col) = make_float2(-d[2], -d[3]);
+        z3_put2(z3, row, col, -d[0], -d[1]);
+        z3_put2(z3, row + 8, col, -d[2], -d[3]);
     }
-    half_sync(1);
+    half_sync(2);
+    // Y = N21 T1 (rows 32-63 of N, columns 0-31), kept in the unused upper
+    // right quadrant of NS: block (i, j) sums over the blocks s = j..1 of T1.
+    const int i2 = warp >> 2, j2 = (warp >> 1) & 1;
+    {
+        const float* A = NS + (32 + 16 * i2) * NSP + 16 * j2;
+        const float* Bm = TS + (16 * j2) * NSP + 16 * j2 + 8 * nt;
+        if (j2 == 0) tile_16x8<4>(d, A, NSP, Bm, NSP, g, t);
+        else tile_16x8<2>(d, A, NSP, Bm, NSP, g, t);
+        float* yp = NS + (16 * i2 + g) * NSP + 32 + 16 * j2 + 8 * nt + 2 * t;
+        *reinterpret_cast<float2*>(yp) = make_float2(d[0], d[1]);
+        *reinterpret_cast<float2*>(yp + 8 * NSP) = make_float2(d[2], d[3]);
+    }
+    half_sync(2);
+    // T21 = -T2 Y: block (i, j) sums T2[i][s] Y[s][j] over s = 0..i
+    {
+        const float* A = TS + (32 + 16 * i2) * NSP + 32;
+        const float* Bm = NS + 32 + 16 * j2 + 8 * nt;
+        if (i2 == 0) tile_16x8<2>(d, A, NSP, Bm, NSP, g, t);
+        else tile_16x8<4>(d, A, NSP, Bm, NSP, g, t);
+        const int row = 32 + 16 * i2 + g, col = 16 * j2 + 8 * nt + 2 * t;
+        *reinterpret_cast<float2*>(TS + row * NSP + col) = make_float2(-d[0], -d[1]);
+        *reinterpret_cast<float2*>(TS + (row + 8) * NSP + col) = make_float2(-d[2], -d[3]);
+        z3_put2(z3, row, col, -d[0], -d[1]);
+        z3_put2(z3, row + 8, col, -d[2], -d[3]);
+    }
 }
 
 // ---------------------------------------------------------------- TMA issue
-// Group "kq": raw k and q into RAW.  Group "ab": vector a and b into X1.
-// Group "vw": v into U and vector w into LQ.
-__device__ __forceinline__ void issue_kq(const TcMaps& m, uint32_t sbase, int t0, int hi, int bi,
-                                         uint32_t bar) {
-    tc::mbar_arrive_expect_tx(bar, 4 * BOX_BYTES);
+// Group "kqw": raw k and q into RAW, vector w into W.  Group "ab": vector a
+// and b into X1.  Group "v": v into U.
+__device__ __forceinline__ void issue_kqw(const TcMaps& m, uint32_t sbase, int t0, int hi, int bi,
+                                          bool vw, uint32_t bar) {
+    tc::mbar_arrive_expect_tx(bar, 2u * (2u + (vw ? 1u : 0u)) * BOX_BYTES);
 #pragma unroll
     for (int p = 0; p < 2; ++p) {
         tc::tma_load_4d(sbase + OFF_RAW + p * 16384, &m.k, 64 * p, hi, t0, bi, bar);
         tc::tma_load_4d(sbase + OFF_RAW + p * 16384 + 8192, &m.q, 64 * p, hi, t0, bi, bar);
+        if (vw) tc::tma_load_4d(sbase + OFF_W + p * 8192, &m.w, 64 * p, hi, t0, bi, bar);
     }
 }
 
@@ -248,86 +288,122 @@ __device__ __forceinline__ void issue_ab(const TcMaps& m, uint32_t sbase, int t0
     }
 }
 
-__device__ __forceinline__ void issue_vw(const TcMaps& m, uint32_t sbase, int t0, int hi, int bi,
-                                         bool vw, uint32_t bar) {
-    tc::mbar_arrive_expect_tx(bar, 2u * (1u + (vw ? 1u : 0u)) * BOX_BYTES);
+__device__ __forceinline__ void issue_v(const TcMaps& m, uint32_t sbase, int t0, int hi, int bi,
+                                        uint32_t bar) {
+    tc::mbar_arrive_expect_tx(bar, 2u * BOX_BYTES);
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
+    for (int p = 0; p < 2; ++p)
         tc::tma_load_4d(sbase + OFF_U + p * 8192, &m.v, 64 * p, hi, t0, bi, bar);
-        if (vw) tc::tma_load_4d(sbase + OFF_LQ + p * 8192, &m.w, 64 * p, hi, t0, bi, bar);
-    }
 }
 
-// Decay factors of one chunk, run by warps 8-15 (barrier id 2; u = tid - 256):
-// per key channel the products gamma_r of a over the chunk, g_m = gamma_31,
-// written as bf16 pairs gamma_r/g_m (E1) and g_m/gamma_r (E1I) [64][128];
-// fcur = fprev * g_m (scale of S~ this chunk), fprev = gamma_63/g_m; and the
-// range check of the factorisation.  Thread (pair p2 of channels, quarter q4)
-// walks 16 tokens.
-__device__ __forceinline__ void decay_pass(uint8_t* sm, int u, bool va, int a_kind, int n,
-                                           const float* sca_a, float* QT, float* fcur,
-                                           float* fprev, int* err_word) {
-    const int p2 = u & 63, q4 = u >> 6;
-    const uint32_t aoff = (uint32_t)(p2 >> 5) * 16384u + 4u * (uint32_t)(p2 & 3);
-    const int ach = (p2 & 31) >> 2;
-    float loc0[16], loc1[16];
+// Decay factors and scaled operands of one chunk, all 512 compute threads.  Thread
+// (channel pair p2, token octet q8) forms the running products of a over its
+// 8 tokens for channels 2*p2, 2*p2 + 1; after one exchange of octet totals
+// (QT) it has gamma_r/g_m and g_m/gamma_r for its tokens (g_m = gamma_31) and
+// writes, one bf16 pair per token (4-byte accesses, a warp covering one
+// 128-byte row of a panel):
+//   K' = (gamma/g_m) k, Q' = (gamma/g_m) q   over raw a, b in X1
+//   K" = (g_m/gamma) k, B" = b K"            into X2
+//   U  = w v                                 over raw v
+// Octet-0 threads also update the state scales, fcur = fprev * g_m and
+// fprev = gamma_63/g_m, and check that the largest factors, gamma_0/g_m and
+// g_m/gamma_63, stay in float range.  `mid` runs between the two halves (after
+// the exchange barrier), before anything is written to X2.
+template <typename Mid>
+__device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool vb, bool vw,
+                                             int a_kind, int n, const float* sca, float* QT,
+                                             float* fcur, float* fprev, int* err_word,
+                                             Mid&& mid) {
+    const int p2 = tid & 63, q8 = tid >> 6;
+    const uint32_t pnl = (uint32_t)(p2 >> 5);
+    const int ch = (p2 & 31) >> 2;                 // 16-byte chunk of the pair in its panel
+    const uint32_t cofs = 4u * (uint32_t)(p2 & 3);  // byte of the pair in its chunk
+    // the pair of a per token as two bf16 (1.0 past the chunk or for GATE_ONE;
+    // scalar gates came from bf16, so the pair is exact)
+    uint32_t apr[8];
+    float loc0[8], loc1[8];
     float run0 = 1.f, run1 = 1.f;
 #pragma unroll
-    for (int x = 0; x < 16; ++x) {
-        const int r = 16 * q4 + x;
-        float a0, a1;
-        if (va) {
-            const uint32_t pr = *reinterpret_cast<const uint32_t*>(
-                sm + OFF_X1 + aoff + (uint32_t)r * 128u + ((uint32_t)(ach ^ (r & 7)) << 4));
-            a0 = __uint_as_float(pr << 16);
-            a1 = __uint_as_float(pr & 0xFFFF0000u);
-        } else {
-            a0 = a1 = sca_a[r];
-        }
-        const bool live = a_kind != GDR_GATE_ONE && r < n;
-        run0 *= live ? a0 : 1.f;
-        run1 *= live ? a1 : 1.f;
+    for (int x = 0; x < 8; ++x) {
+        const int r = 8 * q8 + x;
+        uint32_t pr = va ? *reinterpret_cast<const uint32_t*>(
+                               sm + OFF_X1 + pnl * 16384u + (uint32_t)r * 128u +
+                               ((uint32_t)(ch ^ (r & 7)) << 4) + cofs)
+                         : tc::pack_bf16x2(sca[r], sca[r]);
+        apr[x] = (a_kind != GDR_GATE_ONE && r < n) ? pr : 0x3F803F80u;
+        run0 *= __uint_as_float(apr[x] << 16);
+        run1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
         loc0[x] = run0;
         loc1[x] = run1;
     }
-    *reinterpret_cast<float2*>(QT + q4 * D + 2 * p2) = make_float2(run0, run1);
-    half_sync(2);
+    *reinterpret_cast<float2*>(QT + q8 * D + 2 * p2) = make_float2(run0, run1);
+    compute_sync();
+    mid();
     float pre0 = 1.f, pre1 = 1.f, gm0 = 1.f, gm1 = 1.f, gc0 = 1.f, gc1 = 1.f;
 #pragma unroll
-    for (int gg = 0; gg < 4; ++gg) {
+    for (int gg = 0; gg < 8; ++gg) {
         const float2 qv = *reinterpret_cast<const float2*>(QT + gg * D + 2 * p2);
-        if (gg < q4) { pre0 *= qv.x; pre1 *= qv.y; }
-        if (gg < 2) { gm0 *= qv.x; gm1 *= qv.y; } else { gc0 *= qv.x; gc1 *= qv.y; }
+        if (gg < q8) { pre0 *= qv.x; pre1 *= qv.y; }
+        if (gg < 4) { gm0 *= qv.x; gm1 *= qv.y; } else { gc0 *= qv.x; gc1 *= qv.y; }
     }
+    // gamma_r/g_m = loc_x * f;  g_m/gamma_r = h * prod_{i > x} a_i  (within the octet)
     const float f0 = pre0 * rcp_approx(gm0), f1 = pre1 * rcp_approx(gm1);
+    const float h0 = gm0 * rcp_approx(pre0 * run0), h1 = gm1 * rcp_approx(pre1 * run1);
+    float rev0 = 1.f, rev1 = 1.f;
 #pragma unroll
-    for (int x = 0; x < 16; ++x) {
-        const int r = 16 * q4 + x;
-        const float e0 = loc0[x] * f0, e1v = loc1[x] * f1;
-        *reinterpret_cast<uint32_t*>(sm + OFF_E1 + r * 256 + 4 * p2) = tc::pack_bf16x2(e0, e1v);
-        *reinterpret_cast<uint32_t*>(sm + OFF_E1I + r * 256 + 4 * p2) =
-            tc::pack_bf16x2(rcp_approx(e0), rcp_approx(e1v));
+    for (int x = 7; x >= 0; --x) {
+        const int r = 8 * q8 + x;
+        const uint32_t sw = (uint32_t)r * 128u + ((uint32_t)(ch ^ (r & 7)) << 4) + cofs;
+        const uint32_t o128 = pnl * 16384u + sw, o64 = pnl * 8192u + sw;
+        const uint32_t e = tc::pack_bf16x2(loc0[x] * f0, loc1[x] * f1);
+        const uint32_t ei = tc::pack_bf16x2(h0 * rev0, h1 * rev1);
+        rev0 *= __uint_as_float(apr[x] << 16);
+        rev1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
+        const uint32_t k2 = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW + o128);
+        const uint32_t q2 = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW + o128 + 8192u);
+        const uint32_t b2 = vb ? *reinterpret_cast<const uint32_t*>(sm + OFF_X1 + o128 + 8192u)
+                               : tc::pack_bf16x2(sca[64 + r], sca[64 + r]);
+        const uint32_t v2 = *reinterpret_cast<const uint32_t*>(sm + OFF_U + o64);
+        const uint32_t w2 = vw ? *reinterpret_cast<const uint32_t*>(sm + OFF_W + o64)
+                               : tc::pack_bf16x2(sca[128 + r], sca[128 + r]);
+        const uint32_t kk2 = mul2(k2, ei);                                       // K"
+        *reinterpret_cast<uint32_t*>(sm + OFF_X1 + o128) = mul2(k2, e);          // K'
+        *reinterpret_cast<uint32_t*>(sm + OFF_X1 + o128 + 8192u) = mul2(q2, e);  // Q'
+        *reinterpret_cast<uint32_t*>(sm + OFF_X2 + o128) = kk2;
+        *reinterpret_cast<uint32_t*>(sm + OFF_X2 + o128 + 8192u) = mul2(b2, kk2);  // B"
+        *reinterpret_cast<uint32_t*>(sm + OFF_U + o64) = mul2(w2, v2);             // U
     }
-    if (q4 == 0) {
+    if (q8 == 0) {
         const int i = 2 * p2;
         fcur[i] = fprev[i] * gm0;
         fcur[i + 1] = fprev[i + 1] * gm1;
         fprev[i] = gc0;
         fprev[i + 1] = gc1;
-        // the largest factors, gamma_0/g_m and g_m/gamma_63, must stay in range
         const bool ok0 = gm0 > 0.f && loc0[0] <= gm0 * 1e35f && gc0 >= 1e-35f;
         const bool ok1 = gm1 > 0.f && loc1[0] <= gm1 * 1e35f && gc1 >= 1e-35f;
         if (a_kind != GDR_GATE_ONE && !(ok0 && ok1)) atomicOr(err_word, kErrRange);
     }
 }
 
-// One thread waits on `bar`; the CTA barrier that follows releases the rest.
+// Compute thread 0 waits on `bar`; the compute barrier that follows releases
+// the other compute threads.
 __device__ __forceinline__ void wait_then_sync(uint32_t bar, uint32_t parity, int tid,
                                                volatile int* abort_s) {
     if (tid == 0 && !tc::mbar_wait_bounded(bar, parity, WAIT_NS)) *abort_s = 1;
-    __syncthreads();
+    compute_sync();
     tc::fence_after_sync();
 }
+
+// Barriers (8 bytes each from OFF_BAR).  TMA arrivals and tensor-core
+// commits complete the first group; the compute threads tell the issuing
+// warp that an operand set is in place through the second (thread 0 arrives
+// after a compute barrier).
+enum : uint32_t {
+    B_KQW, B_AB, B_V,              // raw k, q, w / a, b / v landed
+    B_G, B_XAU, B_E, B_ST, B_FIN,  // products done: gram / X, S~, A U / E / O, S~ / all
+    R_OP, R_P2, R_P4, R_P5, R_E, R_O  // ready for: gram / X, S~ / A U / E / O, S~ / o store
+};
+static_assert(R_O + 1 == NBAR, "barrier count");
 
 __global__ void __launch_bounds__(NT, 1)
 chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
@@ -347,10 +423,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
     float* fprev = reinterpret_cast<float*>(sm + OFF_FPREV);
     float* sca_all = reinterpret_cast<float*>(sm + OFF_SCA);  // [2][3][64]
     volatile int* abort_s = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
-    const uint32_t bar_mma = sbase + OFF_BAR;
-    const uint32_t bar_kq = sbase + OFF_BAR + 8;
-    const uint32_t bar_ab = sbase + OFF_BAR + 16;
-    const uint32_t bar_vw = sbase + OFF_BAR + 24;
+    auto bar = [&](uint32_t id) { return sbase + OFF_BAR + 8u * id; };
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -367,348 +440,333 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
     const bool has_ab = va || vb;
 
     if (tid == 0) {
-        tc::mbar_init(bar_mma, 1);
-        tc::mbar_init(bar_kq, 1);
-        tc::mbar_init(bar_ab, 1);
-        tc::mbar_init(bar_vw, 1);
+#pragma unroll 1
+        for (int i = 0; i < NBAR; ++i) tc::mbar_init(bar(i), 1);
         tc::mbar_fence_init();
         *abort_s = 0;
-        tc::tma_prefetch_desc(&maps.q);
-        tc::tma_prefetch_desc(&maps.k);
-        tc::tma_prefetch_desc(&maps.v);
-        tc::tma_prefetch_desc(&maps.o);
     }
     if (tid < D) fprev[tid] = 1.0f;
-    // the middle 64 rows of Z3 stay zero for the whole sequence
-    *reinterpret_cast<uint4*>(sm + OFF_Z3 + 8192 + 16 * tid) = make_uint4(0u, 0u, 0u, 0u);
+    // rows 64-127 of Z3 and the 16 x 16 blocks above the diagonal of T - I
+    // (its rows 0-63) stay zero for the whole sequence
+    if (tid < NTC) {
+        const int r = tid >> 3, c16 = tid & 7;
+        if ((c16 >> 1) > (r >> 4))
+            *reinterpret_cast<uint4*>(sm + OFF_Z3 + r * 128 + ((c16 ^ (r & 7)) << 4)) =
+                make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(sm + OFF_Z3 + 8192 + 16 * tid) = make_uint4(0u, 0u, 0u, 0u);
+    }
     if (warp == 0) tc::tmem_alloc(sbase + OFF_TSLOT, 512);
     tc::fence_async_smem();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + OFF_TSLOT);
-    uint32_t ph_mma = 0, ph_kq = 0, ph_ab = 0, ph_vw = 0;
 
-    if (tid == 0 && T > 0) {
-        issue_kq(maps, sbase, 0, hi, bi, bar_kq);
-        if (has_ab) issue_ab(maps, sbase, 0, hi, bi, va, vb, bar_ab);
-        issue_vw(maps, sbase, 0, hi, bi, vw, bar_vw);
-    }
-    // scalar gates of chunk starting at t0n into buffer `buf` (1.0 past T)
-    auto load_scalars = [&](int t0n, int buf) {
-        if (tid < C) {
-            const int nn = min(C, T - t0n);
-            const long long tok = ((long long)bi * T + t0n + tid) * H + hi;
-            const bool in = tid < nn;
-            float* sc = sca_all + buf * 192;
-            sc[tid] = (a_kind == GDR_GATE_SCALAR && in) ? to_f32(a[tok]) : 1.f;
-            sc[64 + tid] = (b_kind == GDR_GATE_SCALAR && in) ? to_f32(b[tok]) : 1.f;
-            sc[128 + tid] = (w_kind == GDR_GATE_SCALAR && in) ? to_f32(w[tok]) : 1.f;
-        }
-    };
-    if (T > 0) load_scalars(0, 0);
-
-    // ---- initial state S0 (unscaled) into tensor memory: lane i, columns j
-    {
-        const int c0 = 32 * cb;
-        float vals[32];
-        if (s0) {
-            const float4* src = reinterpret_cast<const float4*>(s0 + soff + (size_t)lane_t * D + c0);
-#pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                const float4 v4 = src[x];
-                vals[4 * x] = v4.x; vals[4 * x + 1] = v4.y; vals[4 * x + 2] = v4.z; vals[4 * x + 3] = v4.w;
-            }
-        } else {
-#pragma unroll
-            for (int x = 0; x < 32; ++x) vals[x] = 0.f;
-        }
-        tc::tmem_st32(tmem + lane_off + TM_S + c0, vals);
-        tc::tmem_wait_st();
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    // decay factors of the first chunk (later chunks get theirs under the
-    // previous chunk's UT solve)
-    if (T > 0 && warp >= 8) {
-        if (tid == 256 && has_ab && !tc::mbar_wait_bounded(bar_ab, ph_ab, WAIT_NS)) *abort_s = 1;
-        half_sync(2);
-        decay_pass(sm, tid - 256, va, a_kind, min(C, T), sca_all, QT, fcur, fprev, err_word);
-    }
-    ph_ab ^= (T > 0 && has_ab) ? 1 : 0;
-    __syncthreads();
-
-#pragma unroll 1
-    for (int t0 = 0; t0 < T; t0 += C) {
-        const int n = min(C, T - t0);
-        const bool has_next = t0 + C < T;
-        const int cur = (t0 / C) & 1;
-        const float* sca = sca_all + cur * 192;
-
-        // ================= P1: wait for the chunk's tiles, scaled operands
-        if (tid == 0) {
-            tc::bulk_wait_read();  // the previous o store has left the staging tile
-            bool ok = tc::mbar_wait_bounded(bar_kq, ph_kq, WAIT_NS);
-            ok = ok && tc::mbar_wait_bounded(bar_vw, ph_vw, WAIT_NS);
-            if (!ok) *abort_s = 1;
-        }
-        ph_kq ^= 1;
-        ph_vw ^= 1;
-        __syncthreads();
-        // ================= P1c:
-        {
-            // K' = e1*k, Q' = e1*q, K" = k/e1, B" = b*K", U = w*v, 8 channels
-            // (16 bytes) per access, packed bf16 products
-#pragma unroll 1
-            for (int it = tid; it < C * 16; it += NT) {
-                const int r = it >> 4, c16 = it & 15, p = c16 >> 3, ch = c16 & 7;
-                const uint32_t swz = ((uint32_t)(ch ^ (r & 7)) << 4) + (uint32_t)r * 128u;
-                const uint32_t otop = (uint32_t)p * 16384u + swz;  // rows 0-63 of 128-row tiles
-                const uint32_t obot = otop + 8192u;                // rows 64-127
-                const uint32_t o64 = (uint32_t)p * 8192u + swz;    // 64-row tiles
-                const uint4 k4 = *reinterpret_cast<const uint4*>(sm + OFF_RAW + otop);
-                const uint4 q4 = *reinterpret_cast<const uint4*>(sm + OFF_RAW + obot);
-                const uint4 v4 = *reinterpret_cast<const uint4*>(sm + OFF_U + o64);
-                const uint4 b4 = vb ? *reinterpret_cast<const uint4*>(sm + OFF_X1 + obot)
-                                    : splat8(sca[64 + r]);
-                const uint4 w4 = vw ? *reinterpret_cast<const uint4*>(sm + OFF_LQ + o64)
-                                    : splat8(sca[128 + r]);
-                const uint4 e4 = *reinterpret_cast<const uint4*>(sm + OFF_E1 + r * 256 + 16 * c16);
-                const uint4 ei4 = *reinterpret_cast<const uint4*>(sm + OFF_E1I + r * 256 + 16 * c16);
-                const uint4 kk1 = mul8(k4, e4);   // K'
-                const uint4 kk2 = mul8(k4, ei4);  // K"
-                *reinterpret_cast<uint4*>(sm + OFF_X1 + otop) = kk1;
-                *reinterpret_cast<uint4*>(sm + OFF_X1 + obot) = mul8(q4, e4);    // Q'
-                *reinterpret_cast<uint4*>(sm + OFF_X2 + otop) = kk2;
-                *reinterpret_cast<uint4*>(sm + OFF_X2 + obot) = mul8(b4, kk2);  // B"
-                *reinterpret_cast<uint4*>(sm + OFF_U + o64) = mul8(w4, v4);     // U
-            }
-        }
-        tc::fence_async_smem();
-        __syncthreads();
-        if (*abort_s) break;
-        if (tid == 0) {
-            // the RAW tile is free: fetch the next chunk's k and q now
-            if (has_next) issue_kq(maps, sbase, t0 + C, hi, bi, bar_kq);
-            // gram [K';Q'] [K";B"]^T needs no state: start it under the rescale
-            tc::fence_after_sync();
+    if (warp == NTC / 32) {
+        // ======================= issuing warp (one thread)
+        if ((tid & 31) == 0 && T > 0) {
+            tc::tma_prefetch_desc(&maps.q);
+            tc::tma_prefetch_desc(&maps.k);
+            tc::tma_prefetch_desc(&maps.v);
+            tc::tma_prefetch_desc(&maps.o);
+            uint32_t ph = 0;               // phase of the per-chunk barriers
+            uint32_t n_kqw = 0, n_ab = 0, n_v = 0;
+            issue_kqw(maps, sbase, 0, hi, bi, vw, bar(B_KQW)); ++n_kqw;
+            if (has_ab) { issue_ab(maps, sbase, 0, hi, bi, va, vb, bar(B_AB)); ++n_ab; }
+            issue_v(maps, sbase, 0, hi, bi, bar(B_V)); ++n_v;
+            auto wait_ready = [&](uint32_t id) {
+                if (!tc::mbar_wait_bounded(bar(id), ph, WAIT_NS)) { *abort_s = 1; return false; }
+                tc::fence_after_sync();
+                return *abort_s == 0;
+            };
             const uint32_t idKK = tc::idesc_bf16(128, 128, 0, 0);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                tc::mma_bf16(tmem + TM_G, tc::desc_kmajor(sbase + OFF_X1, 16384, kk),
-                             tc::desc_kmajor(sbase + OFF_X2, 16384, kk), idKK, kk > 0);
-        }
-
-        // ================= P2: S~ <- f_i S~ (lane i), bf16 copy to smem
-        tc::fence_after_sync();
-        {
-            const int c0 = 32 * cb;
-            const float f = fcur[lane_t];
-            float vals[32];
-            tc::tmem_ld32(tmem + lane_off + TM_S + c0, vals);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) vals[x] *= f;
-            tc::tmem_st32(tmem + lane_off + TM_S + c0, vals);
-            tc::store_row32_bf16(sm + OFF_S0 + (cb >> 1) * 16384, lane_t, cb & 1, vals);
-            tc::tmem_wait_st();
-        }
-        tc::fence_async_smem();
-        tc::fence_before_sync();
-        __syncthreads();
-
-        // ================= P3: X = [K';Q'] S~, S~ += K"^T U (gram already issued)
-        if (tid == 0) {
-            tc::fence_after_sync();
             const uint32_t idKM = tc::idesc_bf16(128, 128, 0, 1);
             const uint32_t idMM = tc::idesc_bf16(128, 128, 1, 1);
+            // o of the chunk before t0 leaves by TMA once its staging tile is written
+            auto store_o = [&](int t0o, uint32_t parity) {
+                if (!tc::mbar_wait_bounded(bar(R_O), parity, WAIT_NS)) { *abort_s = 1; return false; }
+                tc::tma_store_4d(&maps.o, sbase + OFF_OST, 0, hi, t0o, bi);
+                tc::tma_store_4d(&maps.o, sbase + OFF_OST + 8192, 64, hi, t0o, bi);
+                tc::bulk_commit();
+                return true;
+            };
+            int t0 = 0;
+#pragma unroll 1
+            for (; t0 < T; t0 += C, ph ^= 1) {
+                const bool has_next = t0 + C < T;
+                if (t0 > 0 && !store_o(t0 - C, ph ^ 1)) break;
+                // operands of the chunk are in place; raw k, q, w are consumed
+                if (!wait_ready(R_OP)) break;
+                if (has_next) { issue_kqw(maps, sbase, t0 + C, hi, bi, vw, bar(B_KQW)); ++n_kqw; }
+                // gram [K';Q'] [K";B"]^T
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-                tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_X1, 16384, kk),
-                             tc::desc_mnmajor(sbase + OFF_S0, 16384, kk), idKM, kk > 0);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16(tmem + TM_G, tc::desc_kmajor(sbase + OFF_X1, 16384, kk),
+                                 tc::desc_kmajor(sbase + OFF_X2, 16384, kk), idKK, kk > 0);
+                tc::bulk_wait_read();  // the o store has left its staging tile (NS reuses it)
+                tc::mma_commit(bar(B_G));
+                // X = [K';Q'] S~, S~ += K"^T U
+                if (!wait_ready(R_P2)) break;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_S, tc::desc_mnmajor(sbase + OFF_X2, 16384, kk),
-                             tc::desc_mnmajor(sbase + OFF_U, 8192, kk), idMM, true);
-            tc::mma_commit(bar_mma);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_X1, 16384, kk),
+                                 tc::desc_mnmajor(sbase + OFF_S0, 16384, kk), idKM, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_S, tc::desc_mnmajor(sbase + OFF_X2, 16384, kk),
+                                 tc::desc_mnmajor(sbase + OFF_U, 8192, kk), idMM, true);
+                // X += [A_kk; A_qk] U
+                if (!wait_ready(R_P4)) break;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16_ts(tmem + TM_X, tmem + TM_AQ + 8 * kk,
+                                    tc::desc_mnmajor(sbase + OFF_U, 8192, kk), idKM, true);
+                tc::mma_commit(bar(B_XAU));
+                if (has_next) {
+                    // X1 and U are free once these products are done
+                    if (!tc::mbar_wait_bounded(bar(B_XAU), ph, WAIT_NS)) { *abort_s = 1; break; }
+                    if (has_ab) { issue_ab(maps, sbase, t0 + C, hi, bi, va, vb, bar(B_AB)); ++n_ab; }
+                    issue_v(maps, sbase, t0 + C, hi, bi, bar(B_V)); ++n_v;
+                }
+                // X += [T - I; 0] R (rows 0-63 become E)
+                if (!wait_ready(R_P5)) break;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_Z3, 8192, kk),
+                                 tc::desc_mnmajor(sbase + OFF_X2, 16384, kk), idKM, true);
+                tc::mma_commit(bar(B_E));
+                // X += [0; -A_qb] E (rows 64-127 become O); S~ -= B"^T E
+                if (!wait_ready(R_E)) break;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_Z3 + 8192, 8192, kk),
+                                 tc::desc_mnmajor(sbase + OFF_EB, 8192, kk), idKM, true);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_S, tc::desc_mnmajor(sbase + OFF_X2 + 8192, 16384, kk),
+                                 tc::desc_mnmajor(sbase + OFF_EB, 8192, kk),
+                                 idMM | IDESC_NEG_B, true);
+                tc::mma_commit(bar(B_ST));
+            }
+            if (t0 >= T && *abort_s == 0) store_o(t0 - C, ph ^ 1);  // the last chunk's o
+            // nothing of this CTA may still be in flight when it exits
+            tc::mma_commit(bar(B_FIN));
+            tc::mbar_wait_bounded(bar(B_FIN), 0, WAIT_NS);
+            if (n_kqw) tc::mbar_wait_bounded(bar(B_KQW), (n_kqw - 1) & 1, WAIT_NS);
+            if (n_ab) tc::mbar_wait_bounded(bar(B_AB), (n_ab - 1) & 1, WAIT_NS);
+            if (n_v) tc::mbar_wait_bounded(bar(B_V), (n_v - 1) & 1, WAIT_NS);
+            tc::bulk_wait_all();
         }
-        wait_then_sync(bar_mma, ph_mma, tid, abort_s);
-        ph_mma ^= 1;
-        // X1 is free: fetch the next chunk's vector a and b; its scalar gates
-        if (tid == 0 && has_next && has_ab) issue_ab(maps, sbase, t0 + C, hi, bi, va, vb, bar_ab);
-        if (has_next) load_scalars(t0 + C, cur ^ 1);
+    } else {
+        // ======================= compute warps
+        // scalar gates of chunk starting at t0n into buffer `buf` (1.0 past T)
+        auto load_scalars = [&](int t0n, int buf) {
+            if (tid < C) {
+                const int nn = min(C, T - t0n);
+                const long long tok = ((long long)bi * T + t0n + tid) * H + hi;
+                const bool in = tid < nn;
+                float* sc = sca_all + buf * 192;
+                sc[tid] = (a_kind == GDR_GATE_SCALAR && in) ? to_f32(a[tok]) : 1.f;
+                sc[64 + tid] = (b_kind == GDR_GATE_SCALAR && in) ? to_f32(b[tok]) : 1.f;
+                sc[128 + tid] = (w_kind == GDR_GATE_SCALAR && in) ? to_f32(w[tok]) : 1.f;
+            }
+        };
+        if (T > 0) load_scalars(0, 0);
 
-        // ================= P4: read the gram; masked blocks out
+        // ---- initial state S0 (unscaled) into tensor memory: lane i, columns j
         {
-            // This warp's 32 x 32 block lies below (mode < 0), on (0) or above
-            // (> 0) the diagonal of its 64 x 64 gram block: warp-uniform.
-            const int mode = (cb & 1) - (quarter & 1);
-            const bool top = lane_t < 64;  // rows of K' (else Q')
-            const int r = top ? lane_t : lane_t - 64;
-            const int s0c = 32 * (cb & 1);  // first s of this column block
+            const int c0 = 32 * cb;
             float vals[32];
-            if (mode > 0) {
+            if (s0) {
+                const float4* src =
+                    reinterpret_cast<const float4*>(s0 + soff + (size_t)lane_t * D + c0);
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const float4 v4 = src[x];
+                    vals[4 * x] = v4.x; vals[4 * x + 1] = v4.y;
+                    vals[4 * x + 2] = v4.z; vals[4 * x + 3] = v4.w;
+                }
+            } else {
 #pragma unroll
                 for (int x = 0; x < 32; ++x) vals[x] = 0.f;
-            } else {
-                tc::tmem_ld32(tmem + lane_off + TM_G + 32 * cb, vals);
-                tc::tmem_wait_ld();
-                if (mode == 0) {
-                    // strictly lower for the K' rows, diagonal included for Q'
-                    const int lim = top ? r - s0c : r - s0c + 1;
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) vals[x] = x < lim ? vals[x] : 0.f;
-                }
             }
-            if (cb < 2) {
-                tc::store_row32_bf16(sm + OFF_LQ, lane_t, cb & 1, vals);   // [A_kk; A_qk]
-            } else if (top) {
-                float* nrow = NS + r * NSP + s0c;
-#pragma unroll
-                for (int x = 0; x < 32; x += 4)
-                    st4(nrow + x, make_float4(vals[x], vals[x + 1], vals[x + 2], vals[x + 3]));
-            } else {
-#pragma unroll
-                for (int x = 0; x < 32; ++x) vals[x] = -vals[x];
-                tc::store_row32_bf16(sm + OFF_Z3, 128 + r, cb & 1, vals);  // -A_qb
-            }
+            tc::tmem_st32(tmem + lane_off + TM_S + c0, vals);
+            tc::tmem_wait_st();
         }
-        tc::fence_async_smem();
-        tc::fence_before_sync();
-        __syncthreads();
-        // X += [A_kk; A_qk] U: runs under the solve
-        if (tid == 0) {
-            tc::fence_after_sync();
-            const uint32_t idKM = tc::idesc_bf16(128, 128, 0, 1);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_LQ, 16384, kk),
-                             tc::desc_mnmajor(sbase + OFF_U, 8192, kk), idKM, true);
-            tc::mma_commit(bar_mma);
-        }
-        if (*abort_s) break;
-
-        // ================= P5: warps 0-7: UT transform T = (I + A_kb)^{-1};
-        //                       warps 8-15: R -> bf16, next chunk's decay factors
-        if (warp < 8) {
-            ut_diag(NS, TS, tid);
-            ut_level<1>(NS, TS, PS, tid);
-            ut_level<2>(NS, TS, PS, tid);
-            ut_level<3>(NS, TS, PS, tid);
-            {
-                const int r = tid >> 2, c4 = tid & 3;  // T - I, 64 rows x 4 x 16 columns
+        uint32_t ph = 0;  // phase of the per-chunk barriers
+        // O (rows 64-127 of X) -> bf16 staging tile, by the warps of lanes 64-127
+        auto read_o = [&] {
+            if (quarter >= 2) {
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    const int ch = 2 * c4 + hh;
-                    float vals[8];
-                    const float* trow = TS + r * NSP + 8 * ch;
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) vals[x] = (8 * ch + x < r) ? trow[x] : 0.f;
-                    *reinterpret_cast<uint4*>(sm + OFF_Z3 + r * 128 + ((ch ^ (r & 7)) << 4)) = pack8(vals);
-                }
-            }
-            tc::fence_async_smem();
-        } else {
-            if (tid == 256 && !tc::mbar_wait_bounded(bar_mma, ph_mma, WAIT_NS)) *abort_s = 1;
-            half_sync(2);
-            tc::fence_after_sync();
-            if (quarter < 2) {   // lanes 0-63 of X hold R; each warp takes 64 columns
-                const int c0 = 64 * (cb - 2);
-                float vals[32];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    tc::tmem_ld32(tmem + lane_off + TM_X + c0 + 32 * hh, vals);
+                    float vals[16];
+                    tc::tmem_ld16(tmem + lane_off + TM_X + 32 * cb + 16 * hh, vals);
                     tc::tmem_wait_ld();
-                    tc::store_row32_bf16(sm + OFF_LQ + (c0 >> 6) * 8192, lane_t, hh, vals);
+                    tc::store_row16_bf16(sm + OFF_OST + (cb >> 1) * 8192, lane_t - 64,
+                                         2 * (cb & 1) + hh, vals);
+                }
+            }
+        };
+        // after the compute barrier that follows, thread 0 signals `id`
+        auto signal = [&](uint32_t id) {
+            compute_sync();
+            if (tid == 0) tc::mbar_arrive(bar(id));
+        };
+
+#pragma unroll 1
+        for (int t0 = 0; t0 < T; t0 += C, ph ^= 1) {
+            const bool has_next = t0 + C < T;
+            const int cur = (t0 / C) & 1;
+            const float* sca = sca_all + cur * 192;
+
+            // ================= P1: the chunk's raw tiles; decay factors, scaled operands
+            if (tid == 0) {
+                bool ok = tc::mbar_wait_bounded(bar(B_KQW), ph, WAIT_NS);
+                ok = ok && (!has_ab || tc::mbar_wait_bounded(bar(B_AB), ph, WAIT_NS));
+                ok = ok && tc::mbar_wait_bounded(bar(B_V), ph, WAIT_NS);
+                if (!ok) *abort_s = 1;
+            }
+            compute_sync();
+            if (*abort_s) break;
+            // ================= P1c:
+            operand_pass(sm, tid, va, vb, vw, a_kind, min(C, T - t0), sca, QT, fcur, fprev,
+                         err_word, [&] {
+                             if (t0 == 0) return;
+                             // the last chunk's state update has read X2 and EB and
+                             // finished its O: O -> staging tile for the issuing warp
+                             wait_then_sync(bar(B_ST), ph ^ 1, tid, abort_s);
+                             read_o();
+                         });
+            tc::fence_async_smem();
+            compute_sync();
+            if (tid == 0) {
+                if (t0 > 0) tc::mbar_arrive(bar(R_O));
+                tc::mbar_arrive(bar(R_OP));
+            }
+
+            // ================= P2: S~ <- f_i S~ (lane i), bf16 copy to smem
+            {
+                const int c0 = 32 * cb;
+                const float f = fcur[lane_t];
+                float vals[32];
+                tc::fence_after_sync();
+                tc::tmem_ld32(tmem + lane_off + TM_S + c0, vals);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) vals[x] *= f;
+                tc::tmem_st32(tmem + lane_off + TM_S + c0, vals);
+                tc::store_row32_bf16(sm + OFF_S0 + (cb >> 1) * 16384, lane_t, cb & 1, vals);
+                tc::tmem_wait_st();
+            }
+            tc::fence_async_smem();
+            tc::fence_before_sync();
+            signal(R_P2);
+
+            // ================= P3: the X and S~ products run under the gram readout
+            if (has_next) load_scalars(t0 + C, cur ^ 1);
+            wait_then_sync(bar(B_G), ph, tid, abort_s);
+
+            // ================= P4: read the gram; masked blocks out
+            {
+                // This warp's 32 x 32 block lies below (mode < 0), on (0) or above
+                // (> 0) the diagonal of its 64 x 64 gram block: warp-uniform.
+                const int mode = (cb & 1) - (quarter & 1);
+                const bool top = lane_t < 64;  // rows of K' (else Q')
+                const int r = top ? lane_t : lane_t - 64;
+                const int s0c = 32 * (cb & 1);  // first s of this column block
+                float vals[32];
+                if (mode > 0) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) vals[x] = 0.f;
+                } else {
+                    tc::tmem_ld32(tmem + lane_off + TM_G + 32 * cb, vals);
+                    tc::tmem_wait_ld();
+                    if (mode == 0) {
+                        // strictly lower for the K' rows, diagonal included for Q'
+                        const int lim = top ? r - s0c : r - s0c + 1;
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) vals[x] = x < lim ? vals[x] : 0.f;
+                    }
+                }
+                if (cb < 2) {
+                    // [A_kk; A_qk] -> tensor memory (A operand of the next product)
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int x = 0; x < 16; ++x)
+                        packed[x] = tc::pack_bf16x2(vals[2 * x], vals[2 * x + 1]);
+                    tc::tmem_st16(tmem + lane_off + TM_AQ + 16 * (cb & 1), packed);
+                    tc::tmem_wait_st();
+                } else if (top) {
+                    float* nrow = NS + r * NSP + s0c;
+#pragma unroll
+                    for (int x = 0; x < 32; x += 4)
+                        st4(nrow + x, make_float4(vals[x], vals[x + 1], vals[x + 2], vals[x + 3]));
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) vals[x] = -vals[x];
+                    tc::store_row32_bf16(sm + OFF_Z3, 128 + r, cb & 1, vals);  // -A_qb
                 }
             }
             tc::fence_async_smem();
-            if (has_next) {
-                if (tid == 256 && has_ab &&
-                    !tc::mbar_wait_bounded(bar_ab, ph_ab, WAIT_NS)) *abort_s = 1;
-                half_sync(2);
-                decay_pass(sm, tid - 256, va, a_kind, min(C, T - t0 - C), sca_all + (cur ^ 1) * 192,
-                           QT, fcur, fprev, err_word);
+            tc::fence_before_sync();
+            signal(R_P4);
+
+            // ================= P5: warps 0-7: UT transform T = (I + A_kb)^{-1};
+            //                       warps 8-15: R -> bf16
+            if (warp < 8) {
+                ut_solve(NS, TS, PS, sm + OFF_Z3, tid);
+                tc::fence_async_smem();
+            } else {
+                if (tid == 256 && !tc::mbar_wait_bounded(bar(B_XAU), ph, WAIT_NS)) *abort_s = 1;
+                half_sync(3);
+                tc::fence_after_sync();
+                if (quarter < 2) {   // lanes 0-63 of X hold R; each warp takes 64 columns
+                    const int c0 = 64 * (cb - 2);
+                    float vals[32];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        tc::tmem_ld32(tmem + lane_off + TM_X + c0 + 32 * hh, vals);
+                        tc::tmem_wait_ld();
+                        // into the K" rows of X2, read by now
+                        tc::store_row32_bf16(sm + OFF_X2 + (c0 >> 6) * 16384, lane_t, hh, vals);
+                    }
+                }
+                tc::fence_async_smem();
             }
-        }
-        ph_mma ^= 1;
-        ph_ab ^= (has_next && has_ab) ? 1 : 0;
-        tc::fence_before_sync();
-        __syncthreads();
+            tc::fence_before_sync();
+            signal(R_P5);
 
-        // ================= P6: X += [T - I; 0] R (rows 0-63 become E)
-        if (tid == 0) {
-            tc::fence_after_sync();
-            const uint32_t idKM = tc::idesc_bf16(128, 128, 0, 1);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_Z3, 8192, kk),
-                             tc::desc_mnmajor(sbase + OFF_LQ, 8192, kk), idKM, true);
-            tc::mma_commit(bar_mma);
-        }
-        wait_then_sync(bar_mma, ph_mma, tid, abort_s);
-        ph_mma ^= 1;
-        // U and LQ are free: fetch the next chunk's v and vector w
-        if (tid == 0 && has_next) issue_vw(maps, sbase, t0 + C, hi, bi, vw, bar_vw);
+            // ================= P6: X += [T - I; 0] R (rows 0-63 become E)
+            wait_then_sync(bar(B_E), ph, tid, abort_s);
 
-        // ================= P7: E -> bf16; X += [0; -A_qb] E; S~ -= B"^T E
-        if (quarter < 2) {
-            float vals[32];
-            tc::tmem_ld32(tmem + lane_off + TM_X + 32 * cb, vals);
-            tc::tmem_wait_ld();
-            tc::store_row32_bf16(sm + OFF_EB + (cb >> 1) * 8192, lane_t, cb & 1, vals);
+            // ================= P7: E -> bf16; X += [0; -A_qb] E and S~ -= B"^T E run
+            // under the next chunk's decay products
+            if (quarter < 2) {
+                float vals[32];
+                tc::tmem_ld32(tmem + lane_off + TM_X + 32 * cb, vals);
+                tc::tmem_wait_ld();
+                tc::store_row32_bf16(sm + OFF_EB + (cb >> 1) * 8192, lane_t, cb & 1, vals);
+            }
+            tc::fence_async_smem();
+            tc::fence_before_sync();
+            signal(R_E);
+            if (*abort_s) break;
         }
-        tc::fence_async_smem();
-        tc::fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
-            tc::fence_after_sync();
-            const uint32_t idKM = tc::idesc_bf16(128, 128, 0, 1);
-            const uint32_t idMMn = tc::idesc_bf16(128, 128, 1, 1) | IDESC_NEG_B;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_Z3 + 8192, 8192, kk),
-                             tc::desc_mnmajor(sbase + OFF_EB, 8192, kk), idKM, true);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_bf16(tmem + TM_S, tc::desc_mnmajor(sbase + OFF_X2 + 8192, 16384, kk),
-                             tc::desc_mnmajor(sbase + OFF_EB, 8192, kk), idMMn, true);
-            tc::mma_commit(bar_mma);
+        if (T > 0 && *abort_s == 0) {
+            // the last chunk's O
+            wait_then_sync(bar(B_ST), ph ^ 1, tid, abort_s);
+            read_o();
+            tc::fence_async_smem();
+            signal(R_O);
         }
-        wait_then_sync(bar_mma, ph_mma, tid, abort_s);
-        ph_mma ^= 1;
-
-        // ================= P8: O (rows 64-127 of X) -> staging tile -> TMA store
-        if (quarter >= 2) {
-            float vals[32];
-            tc::tmem_ld32(tmem + lane_off + TM_X + 32 * cb, vals);
-            tc::tmem_wait_ld();
-            tc::store_row32_bf16(sm + OFF_OST + (cb >> 1) * 8192, lane_t - 64, cb & 1, vals);
-        }
-        tc::fence_async_smem();
-        tc::fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
-            tc::tma_store_4d(&maps.o, sbase + OFF_OST, 0, hi, t0, bi);
-            tc::tma_store_4d(&maps.o, sbase + OFF_OST + 8192, 64, hi, t0, bi);
-            tc::bulk_commit();
-        }
-        if (*abort_s) break;
     }
 
-    if (tid == 0) tc::bulk_wait_all();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
     if (*abort_s) {
         atomicOr(err_word, kErrTimeout);
-        // let products and copies still in flight land before memory is freed
-        if (tid == 0) {
-            tc::mbar_wait_bounded(bar_mma, ph_mma, WAIT_NS);
-            tc::mbar_wait_bounded(bar_kq, ph_kq, WAIT_NS);
-            if (has_ab) tc::mbar_wait_bounded(bar_ab, ph_ab, WAIT_NS);
-            tc::mbar_wait_bounded(bar_vw, ph_vw, WAIT_NS);
-        }
-        __syncthreads();
-    } else if (s_final) {
-        tc::fence_after_sync();
+    } else if (s_final && tid < NTC) {
         const int c0 = 32 * cb;
         const float f = fprev[lane_t];
         float vals[32];

@@ -73,6 +73,23 @@ __device__ __forceinline__ void store_row32_bf16(uint8_t* panel_base, int row, i
     }
 }
 
+// Same for 16 columns starting at column 16*q of the panel (16-byte chunks
+// 2q, 2q+1).
+__device__ __forceinline__ void store_row16_bf16(uint8_t* panel_base, int row, int q,
+                                                 const float* v) {
+    uint8_t* rp = panel_base + row * 128;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int c16 = 2 * q + h;
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * h + 0], v[8 * h + 1]);
+        w.y = pack_bf16x2(v[8 * h + 2], v[8 * h + 3]);
+        w.z = pack_bf16x2(v[8 * h + 4], v[8 * h + 5]);
+        w.w = pack_bf16x2(v[8 * h + 6], v[8 * h + 7]);
+        *reinterpret_cast<uint4*>(rp + ((c16 ^ (row & 7)) << 4)) = w;
+    }
+}
+
 // ------------------------------------------------------------- descriptors
 
 // Shared-memory matrix descriptor (tcgen05 form): start address, leading and
@@ -125,6 +142,20 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
         :
         : "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc));
+}
+
+// Same with A read from tensor memory: M rows in lanes, K packed two bf16 per
+// 32-bit column (the lower half holds the even k), one K = 16 step spanning 8
+// columns from `a_tmem`.  A is K-major there.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, bool accumulate) {
+    const uint32_t acc = accumulate ? 1u : 0u;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+        :
+        : "r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc));
 }
 
 // Make `bar` track completion of every tcgen05.mma this thread issued so far.
@@ -198,6 +229,30 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
         : "memory");
 }
 
+// 32 lanes x 16 consecutive columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -247,6 +302,11 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar_saddr, uint32_t p
             if (mbar_try_wait(bar_saddr, parity)) return true;
         if (global_timer_ns() - t0 > limit_ns) return false;
     }
+}
+
+// One plain arrival (release semantics) on a barrier initialised with count 1.
+__device__ __forceinline__ void mbar_arrive(uint32_t bar_saddr) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar_saddr) : "memory");
 }
 
 // ------------------------------------------------------------- TMA loads
