@@ -495,9 +495,8 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             for (; t0 < T; t0 += C, ph ^= 1) {
                 const bool has_next = t0 + C < T;
                 if (t0 > 0 && !store_o(t0 - C, ph ^ 1)) break;
-                // operands of the chunk are in place; raw k, q, w are consumed
+                // operands of the chunk are in place
                 if (!wait_ready(R_OP)) break;
-                if (has_next) { issue_kqw(maps, sbase, t0 + C, hi, bi, vw, bar(B_KQW)); ++n_kqw; }
                 // gram [K';Q'] [K";B"]^T
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -523,7 +522,11 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                                     tc::desc_mnmajor(sbase + OFF_U, 8192, kk), idKM, true);
                 tc::mma_commit(bar(B_XAU));
                 if (has_next) {
-                    // X1 and U are free once these products are done
+                    // the next chunk's raw tiles, issued under the UT solve (TMA issue
+                    // is slow enough to keep off the products' path): RAW and W were
+                    // consumed by the operand pass, X1 and U are free once these
+                    // products are done
+                    issue_kqw(maps, sbase, t0 + C, hi, bi, vw, bar(B_KQW)); ++n_kqw;
                     if (!tc::mbar_wait_bounded(bar(B_XAU), ph, WAIT_NS)) { *abort_s = 1; break; }
                     if (has_ab) { issue_ab(maps, sbase, t0 + C, hi, bi, va, vb, bar(B_AB)); ++n_ab; }
                     issue_v(maps, sbase, t0 + C, hi, bi, bar(B_V)); ++n_v;
