@@ -397,7 +397,8 @@ __device__ __forceinline__ void wait_then_sync(uint32_t bar, uint32_t parity, in
 // Barriers (8 bytes each from OFF_BAR).  TMA arrivals and tensor-core
 // commits complete the first group; the compute threads tell the issuing
 // warp that an operand set is in place through the second (thread 0 arrives
-// after a compute barrier).
+// after a compute barrier; for R_O each of the 8 warps that write the o
+// staging tile arrives once).
 enum : uint32_t {
     B_KQW, B_AB, B_V,              // raw k, q, w / a, b / v landed
     B_G, B_XAU, B_E, B_ST, B_FIN,  // products done: gram / X, S~, A U / E / O, S~ / all
@@ -441,7 +442,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
 
     if (tid == 0) {
 #pragma unroll 1
-        for (int i = 0; i < NBAR; ++i) tc::mbar_init(bar(i), 1);
+        for (int i = 0; i < NBAR; ++i) tc::mbar_init(bar(i), i == R_O ? 8 : 1);
         tc::mbar_fence_init();
         *abort_s = 0;
     }
@@ -598,6 +599,8 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
         }
         uint32_t ph = 0;  // phase of the per-chunk barriers
         // O (rows 64-127 of X) -> bf16 staging tile, by the warps of lanes 64-127
+        // (each such warp then signals R_O: the issuing warp stores o as soon as
+        // all 8 have written)
         auto read_o = [&] {
             if (quarter >= 2) {
 #pragma unroll
@@ -608,6 +611,9 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                     tc::store_row16_bf16(sm + OFF_OST + (cb >> 1) * 8192, lane_t - 64,
                                          2 * (cb & 1) + hh, vals);
                 }
+                tc::fence_async_smem();
+                __syncwarp();
+                if ((tid & 31) == 0) tc::mbar_arrive(bar(R_O));
             }
         };
         // after the compute barrier that follows, thread 0 signals `id`
@@ -641,11 +647,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                              read_o();
                          });
             tc::fence_async_smem();
-            compute_sync();
-            if (tid == 0) {
-                if (t0 > 0) tc::mbar_arrive(bar(R_O));
-                tc::mbar_arrive(bar(R_OP));
-            }
+            signal(R_OP);
 
             // ================= P2: S~ <- f_i S~ (lane i), bf16 copy to smem
             {
@@ -759,8 +761,6 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             // the last chunk's O
             wait_then_sync(bar(B_ST), ph ^ 1, tid, abort_s);
             read_o();
-            tc::fence_async_smem();
-            signal(R_O);
         }
     }
 
