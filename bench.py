@@ -159,7 +159,7 @@ class ClockSampler:
 
 # --------------------------------------------------------------- the oracle arm
 
-def oracle_throughput(wl, seed: int, target_s: float = 10.0):
+def oracle_throughput(wl, seed: int, target_s: float = 15.0):
     """float64 oracle on a bounded sample of the prefill workload: every
     (b, h) of the batch over the first T_s tokens, T_s sized for about
     `target_s` seconds.  Returns (tokens/s, cores, sample description)."""
@@ -167,7 +167,9 @@ def oracle_throughput(wl, seed: int, target_s: float = 10.0):
     from gated_delta_rule_154_b200 import workload as W
 
     cores = oracle.max_threads()
-    cal = wl.replace(T=64)
+    # calibrate on 512 tokens: shorter runs are dominated by thread start-up
+    # and overestimate the rate
+    cal = wl.replace(T=min(512, wl.T))
     x = W.make_prefill(cal, seed=seed)
     f = lambda k: W.as_f32(x[k], wl.dtype)
     t = time.perf_counter()
