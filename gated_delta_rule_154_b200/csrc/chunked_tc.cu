@@ -712,21 +712,25 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                     tc::store_row32_bf16(sm + OFF_Z3, 128 + r, cb & 1, vals);  // -A_qb
                 }
             }
-            tc::fence_async_smem();
-            tc::fence_before_sync();
-            signal(R_P4);
-
-            // ================= P5: warps 0-7: UT transform T = (I + A_kb)^{-1};
-            //                       warps 8-15: R -> bf16
-            if (warp < 8) {
-                ut_solve(NS, TS, PS, sm + OFF_Z3, tid);
+            // ================= P5: the two column halves of the gram go their own ways.
+            //   warps 8-15 (A_kb, A_qb): UT transform T = (I + A_kb)^{-1};
+            //   warps 0-7 ([A_kk; A_qk] in tensor memory): X += [A_kk; A_qk] U, R -> bf16
+            if (warp >= 8) {
+                tc::fence_async_smem();
+                half_sync(2);
+                ut_solve(NS, TS, PS, sm + OFF_Z3, tid - 256);
                 tc::fence_async_smem();
             } else {
-                if (tid == 256 && !tc::mbar_wait_bounded(bar(B_XAU), ph, WAIT_NS)) *abort_s = 1;
+                tc::fence_before_sync();
+                half_sync(3);
+                if (tid == 0) {
+                    tc::mbar_arrive(bar(R_P4));
+                    if (!tc::mbar_wait_bounded(bar(B_XAU), ph, WAIT_NS)) *abort_s = 1;
+                }
                 half_sync(3);
                 tc::fence_after_sync();
                 if (quarter < 2) {   // lanes 0-63 of X hold R; each warp takes 64 columns
-                    const int c0 = 64 * (cb - 2);
+                    const int c0 = 64 * cb;
                     float vals[32];
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
