@@ -69,12 +69,14 @@ constexpr uint32_t OFF_W = 114688;      // raw vector w 64 x 128
 constexpr uint32_t OFF_Z3 = 131072;     // [T - I; 0; -A_qb] 192 x 64
 constexpr uint32_t OFF_S0 = 155648;     // S~ [i][j] bf16 128 x 128
 constexpr uint32_t OFF_R = 188416;      // scratch region:
-constexpr uint32_t OFF_QT = OFF_R;              //  P1: float [8][128], 8-token products
 constexpr uint32_t OFF_NS = OFF_R;              //  P4-P5: A_kb, float [64][68]
 constexpr uint32_t OFF_TS = OFF_R + 17408;      //  P5: T, float [64][68]
 constexpr uint32_t OFF_PS = OFF_R + 34816;      //  P5: float [2][16][16]
-constexpr uint32_t OFF_EB = OFF_R;              //  P7: E bf16 [s][j] 64 x 128
-constexpr uint32_t OFF_OST = OFF_R + 16384;     //  P8: o staging [r][j] 64 x 128
+constexpr uint32_t OFF_EB = OFF_R;              //  P7 -> next P1: E bf16 [s][j] 64 x 128
+constexpr uint32_t OFF_OST = OFF_R + 16384;     //  next P1 -> o store: staging [r][j] 64 x 128
+constexpr uint32_t OFF_QT = OFF_R + 32768;      //  P1: float [8][128], 8-token products
+                                                //  (clear of EB, which the previous chunk's
+                                                //  state update still reads, and of OST)
 constexpr uint32_t OFF_SMALL = OFF_R + 37888;   // 226304
 constexpr uint32_t OFF_FCUR = OFF_SMALL;        // float[128]: state scale this chunk
 constexpr uint32_t OFF_FPREV = OFF_SMALL + 512; // float[128]: gamma_C/g_m of last chunk
@@ -87,6 +89,7 @@ constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
 constexpr size_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory");
 static_assert(OFF_PS + 2 * 256 * 4 <= OFF_SMALL, "solve scratch");
+static_assert(OFF_QT >= OFF_OST + 16384 && OFF_QT + 8 * 128 * 4 <= OFF_SMALL, "QT placement");
 
 constexpr int NSP = 68;  // row stride (floats) of the solve's float tiles (16-byte rows)
 

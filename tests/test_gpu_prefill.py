@@ -177,6 +177,27 @@ def test_full_size_sampled_heads(name, n_heads):
     assert np.isfinite(to_host(o)).all() and np.isfinite(to_host(s)).all()
 
 
+@pytest.mark.parametrize("name", ["kda_bf16", "gdn2_bf16"])
+def test_full_size_repeatable_bit_for_bit(name):
+    """The kernels fix every reduction order, so repeated launches on the same
+    inputs must agree bit for bit; a shared-memory or tensor-memory race
+    between a chunk's steps shows up here as a difference (or a non-finite
+    value) somewhere in the full output, not only in sampled heads."""
+    wl = W.WORKLOADS[name]
+    inp = W.make_prefill(wl, seed=1)
+    d = inputs_to_dev(inp, wl)
+    runs = []
+    for _ in range(4):
+        o, s = api.forward_chunked(d["q"], d["k"], d["v"], d["a"], d["b"], d["w"], d["s0"],
+                                   chunk=wl.chunk)
+        torch.cuda.synchronize()
+        runs.append((o.clone(), s.clone()))
+    o0, s0 = runs[0]
+    assert torch.isfinite(o0.float()).all() and torch.isfinite(s0).all()
+    for o, s in runs[1:]:
+        assert torch.equal(o, o0) and torch.equal(s, s0)
+
+
 # ------------------------------------------- tensor-core kernel specific checks
 
 @pytest.mark.parametrize("name", ["kda_bf16", "gdn2_bf16"])
