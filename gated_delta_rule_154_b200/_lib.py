@@ -20,7 +20,7 @@ F32, BF16 = 0, 1
 GATE_ONE, GATE_SCALAR, GATE_VECTOR = 0, 1, 2
 
 EXPORTS = ("gdr_workspace_size", "gdr_forward_chunked", "gdr_decode_step",
-           "gdr_last_device_error", "gdr_status_string", "gdr_version")
+           "gdr_last_device_error", "gdr_status_string", "gdr_version", "gdr_test_skip_signal")
 
 
 class GdrDesc(ctypes.Structure):
@@ -62,6 +62,8 @@ def load(path: str = LIB_PATH):
     lib.gdr_status_string.argtypes = [i]
     lib.gdr_version.restype = i
     lib.gdr_version.argtypes = []
+    lib.gdr_test_skip_signal.restype = None
+    lib.gdr_test_skip_signal.argtypes = [i]
     _lib = lib
     return lib
 

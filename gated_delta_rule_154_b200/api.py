@@ -147,4 +147,11 @@ def last_device_error(stream=None) -> int:
     return _lib.last_device_error(_stream_handle(stream))
 
 
+def test_skip_signal(enable: bool = True) -> None:
+    """Test hook (gdr_test_skip_signal): the next bf16 tensor-core prefill
+    launch leaves out one completion signal, so its bounded wait runs out and
+    the launch ends with GDR_ERR_TIMEOUT in the device error word."""
+    _lib.load().gdr_test_skip_signal(1 if enable else 0)
+
+
 Desc = _lib.GdrDesc

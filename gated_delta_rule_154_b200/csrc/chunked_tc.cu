@@ -392,7 +392,7 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
 // the other compute threads.
 __device__ __forceinline__ void wait_then_sync(uint32_t bar, uint32_t parity, int tid,
                                                volatile int* abort_s) {
-    if (tid == 0 && !tc::mbar_wait_bounded(bar, parity, WAIT_NS)) *abort_s = 1;
+    if (tid == 0 && !*abort_s && !tc::mbar_wait_bounded(bar, parity, WAIT_NS)) *abort_s = 1;
     compute_sync();
     tc::fence_after_sync();
 }
@@ -414,7 +414,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                   const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                   const __nv_bfloat16* __restrict__ w, int a_kind, int b_kind, int w_kind,
                   const float* __restrict__ s0, float* __restrict__ s_final,
-                  int* __restrict__ err_word) {
+                  int* __restrict__ err_word, int skip_signal) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -507,7 +507,9 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                     tc::mma_bf16(tmem + TM_G, tc::desc_kmajor(sbase + OFF_X1, 16384, kk),
                                  tc::desc_kmajor(sbase + OFF_X2, 16384, kk), idKK, kk > 0);
                 tc::bulk_wait_read();  // the o store has left its staging tile (NS reuses it)
-                tc::mma_commit(bar(B_G));
+                // (test hook: the first gram's signal left out; the compute threads'
+                // bounded wait for it runs out)
+                if (!(skip_signal && t0 == 0)) tc::mma_commit(bar(B_G));
                 // X = [K';Q'] S~, S~ += K"^T U
                 if (!wait_ready(R_P2)) break;
 #pragma unroll
@@ -728,7 +730,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                 half_sync(3);
                 if (tid == 0) {
                     tc::mbar_arrive(bar(R_P4));
-                    if (!tc::mbar_wait_bounded(bar(B_XAU), ph, WAIT_NS)) *abort_s = 1;
+                    if (!*abort_s && !tc::mbar_wait_bounded(bar(B_XAU), ph, WAIT_NS)) *abort_s = 1;
                 }
                 half_sync(3);
                 tc::fence_after_sync();
@@ -836,7 +838,8 @@ bool chunked_tc_supports(const gdr_desc& d) {
 
 cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, const void* v,
                               const void* a, const void* b, const void* w, const float* s0,
-                              void* o, float* s_final, int* err_word, cudaStream_t st) {
+                              void* o, float* s_final, int* err_word, bool skip_signal,
+                              cudaStream_t st) {
     TcMaps maps;
     memset(&maps, 0, sizeof(maps));
     if (d.T > 0) {
@@ -854,7 +857,7 @@ cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, c
     chunked_tc_kernel<<<(unsigned)(d.B * d.H), NT, SMEM_BYTES, st>>>(
         maps, d.B, d.T, d.H, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b,
         (const __nv_bfloat16*)w, (int)d.decay, (int)d.erase, (int)d.write, s0, s_final,
-        err_word);
+        err_word, skip_signal ? 1 : 0);
     return cudaGetLastError();
 }
 

@@ -1,5 +1,6 @@
 // gdr_api.cu -- the C ABI of libgdr.so: argument checks, kernel choice,
 // device error word.  Declarations and contracts are in include/gdr.h.
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -14,7 +15,8 @@ cudaError_t launch_chunked_simt(const gdr_desc& d, const void* q, const void* k,
 bool chunked_tc_supports(const gdr_desc& d);
 cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, const void* v,
                               const void* a, const void* b, const void* w, const float* s0,
-                              void* o, float* s_final, int* err_word, cudaStream_t st);
+                              void* o, float* s_final, int* err_word, bool skip_signal,
+                              cudaStream_t st);
 }  // namespace gdr
 
 // One error word per device (each device holds its own copy of the symbol).
@@ -24,6 +26,7 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
+std::atomic<int> g_test_skip_signal{0};  // gdr_test_skip_signal, consumed by one launch
 int* g_err_ptr[kMaxDevices];
 
 // Device address of this device's error word (looked up once per device).
@@ -130,7 +133,8 @@ gdr_status gdr_forward_chunked(const gdr_desc* d, const void* q, const void* k, 
     if (gdr::chunked_tc_supports(*d)) {
         int* err = nullptr;
         if ((e = error_word(&err)) != cudaSuccess) return GDR_ERR_CUDA;
-        e = gdr::launch_chunked_tc(*d, q, k, v, a, b, w, s0, o, s_final, err, st);
+        const bool skip = g_test_skip_signal.exchange(0) != 0;
+        e = gdr::launch_chunked_tc(*d, q, k, v, a, b, w, s0, o, s_final, err, skip, st);
     } else if (simt_supports(*d)) {
         e = gdr::launch_chunked_simt(*d, q, k, v, a, b, w, s0, o, s_final, st);
     } else {
@@ -151,6 +155,8 @@ gdr_status gdr_decode_step(const gdr_desc* d, const void* q, const void* k, cons
                                        reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
+
+void gdr_test_skip_signal(int enable) { g_test_skip_signal.store(enable ? 1 : 0); }
 
 gdr_status gdr_last_device_error(gdr_stream_t stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)

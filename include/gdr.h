@@ -135,6 +135,20 @@ gdr_status gdr_decode_step(const gdr_desc *desc, const void *q, const void *k,
  * synchronisation itself failed. */
 gdr_status gdr_last_device_error(gdr_stream_t stream);
 
+/*
+ * Test hook for the bounded-wait path (fault injection without a fault).
+ * After gdr_test_skip_signal(1), the next launch of the bf16 tensor-core
+ * prefill leaves out the completion signal of its first chunk's gram
+ * product, a signal that nothing else will set: the compute threads' wait
+ * on it runs out after its limit (about 2 s), the kernel drains every copy
+ * and product it has in flight, frees its tensor memory and returns, and
+ * gdr_last_device_error() reports GDR_ERR_TIMEOUT.  The outputs of that
+ * launch are undefined.  The request is consumed by that launch (or cleared
+ * by gdr_test_skip_signal(0)); no other path reads it.  Host-only, no CUDA
+ * call.
+ */
+void gdr_test_skip_signal(int enable);
+
 /* Static, human-readable name of a status. */
 const char *gdr_status_string(gdr_status status);
 

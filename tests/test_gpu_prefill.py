@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 import torch
 
-from gated_delta_rule_154_b200 import api
+from gated_delta_rule_154_b200 import _lib, api
 from gated_delta_rule_154_b200 import workload as W
 from gpu_helpers import (TOL, gpu_prefill, inputs_to_dev, oracle_prefill, rel_err, to_dev,
                          to_host)
@@ -149,6 +149,24 @@ def test_matches_decode_kernel_token_by_token():
 def test_no_device_error_recorded():
     wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=64)
     gpu_prefill(wl, W.make_prefill(wl))
+    assert api.last_device_error() == 0
+
+
+def test_bounded_wait_runs_out_and_reports_timeout():
+    """A completion signal that nothing sets (test hook): the kernel's bounded
+    wait gives up, everything in flight is drained, the launch ends with
+    GDR_ERR_TIMEOUT, and the context stays usable: the next launch is exact
+    and records no error."""
+    import time
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=200)
+    inp = W.make_prefill(wl, seed=5)
+    assert api.last_device_error() == 0
+    api.test_skip_signal(True)
+    t = time.perf_counter()
+    gpu_prefill(wl, inp)
+    assert api.last_device_error() == _lib.ERR_TIMEOUT
+    assert time.perf_counter() - t < 60.0
+    _check_full(wl, inp)            # the hook was consumed by one launch
     assert api.last_device_error() == 0
 
 
