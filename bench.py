@@ -370,6 +370,45 @@ def run_gpu(args):
     e2e_ms = max_over_ranks(a0.elapsed_time(a1)) / e2e_steps
     del scratch, host
 
+    # ---- the same q, k, v, a under other gate forms: KDA (one scalar beta per
+    # token for erase and write, here b[..., 0]) and FG^2-GDN / FG^2-GDN+
+    # (vector learning rates entering through their square roots); context for
+    # the FG^2-GDN page's "<5 % prefill overhead over KDA" (section 4)
+    variants = None
+    if not args.no_variants and wl.dtype == "bf16":
+        beta_s = d["b"][..., 0].contiguous()
+        kw = dict(chunk=wl.chunk, out=o, s_final=sT, stream=stream)
+        runs = {
+            "kda": lambda: api.forward_chunked(d["q"], d["k"], d["v"], d["a"], beta_s, beta_s,
+                                               d["s0"], **kw),
+            "fg2": lambda: api.forward_fg2(d["q"], d["k"], d["v"], d["a"], d["b"], None,
+                                           d["s0"], **kw),
+            "fg2_plus": lambda: api.forward_fg2(d["q"], d["k"], d["v"], d["a"], d["b"], d["w"],
+                                                d["s0"], **kw),
+        }
+        variants = {}
+        for name, fn in runs.items():
+            with torch.cuda.stream(stream):
+                for _ in range(2):
+                    fn()
+                torch.cuda.synchronize()
+                barrier()
+                v0, v1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                v0.record(stream)
+                for _ in range(5):
+                    fn()
+                v1.record(stream)
+                torch.cuda.synchronize()
+                barrier()
+            vms = max_over_ranks(v0.elapsed_time(v1)) / 5
+            variants[name] = {"ms_per_step": vms, "tokens/s": tokens_step / (vms * 1e-3)}
+        if api.last_device_error(stream) != 0:
+            raise RuntimeError("device error during the gate-form variants")
+        variants["fg2_over_kda"] = variants["fg2"]["ms_per_step"] / variants["kda"]["ms_per_step"] - 1.0
+        variants["note"] = ("5 launches each on the main step's q, k, v, a; kda: scalar beta = "
+                            "b[..., 0] for erase and write; fg2: beta = b as sqrt(beta) on k "
+                            "and v; fg2_plus: beta^k = b, beta^v = w")
+
     # ---- decode: batch 256, H = 32, d = 128, float32 state in place
     dec = None
     if not args.no_decode:
@@ -443,6 +482,7 @@ def run_gpu(args):
                      "t_tensor_min_us": t_tc * 1e6,
                      "t_hbm_min_us": alg_bytes / (hbm_peak * 1e9) * 1e6},
         "decode": dec,
+        "variants": variants,
         "e2e": {"value": tokens_step / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "cpu_baseline": cpu,
@@ -464,6 +504,8 @@ def main():
     ap.add_argument("--decode-pool", type=int, default=2)
     ap.add_argument("--decode-batch", type=int, default=0, help="override the decode batch")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the KDA / FG^2-GDN gate-form timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     args = ap.parse_args()

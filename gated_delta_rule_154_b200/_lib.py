@@ -17,7 +17,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_
 # gdr_dtype
 F32, BF16 = 0, 1
 # gdr_gate
-GATE_ONE, GATE_SCALAR, GATE_VECTOR = 0, 1, 2
+GATE_ONE, GATE_SCALAR, GATE_VECTOR, GATE_FG2 = 0, 1, 2, 3
 
 EXPORTS = ("gdr_workspace_size", "gdr_forward_chunked", "gdr_decode_step",
            "gdr_last_device_error", "gdr_status_string", "gdr_version", "gdr_test_skip_signal")

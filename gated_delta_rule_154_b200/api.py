@@ -10,6 +10,11 @@ Shapes (row-major, contiguous, on one CUDA device):
     decode   the same without the T axis; state [B, H, dk, dv] float32,
              updated in place
 q, k, v, the gates and o share one dtype (torch.float32 or torch.bfloat16).
+
+FG^2-GDN / FG^2-GDN+ (forward_fg2, decode_step_fg2): per-channel learning
+rates beta^k [.., dk] and beta^v [.., dv] (one tensor for both in FG^2-GDN),
+entering through their square roots inside the kernels: key sqrt(beta^k) k,
+erase gate 1, write gate sqrt(beta^v).
 """
 
 from __future__ import annotations
@@ -58,7 +63,8 @@ def make_desc(B, T, H, dk, dv, chunk, dtype, a_kind, b_kind, w_kind) -> _lib.Gdr
     return _lib.GdrDesc(B, T, H, dk, dv, chunk, dtype, a_kind, b_kind, w_kind)
 
 
-def desc_for(q, v, a, b, w, chunk: int = 64, decode: bool = False) -> _lib.GdrDesc:
+def desc_for(q, v, a, b, w, chunk: int = 64, decode: bool = False,
+             fg2: bool = False) -> _lib.GdrDesc:
     if decode:
         B, H, dk = q.shape
         T = 1
@@ -67,6 +73,9 @@ def desc_for(q, v, a, b, w, chunk: int = 64, decode: bool = False) -> _lib.GdrDe
         B, T, H, dk = q.shape
         nd = 4
     dv = v.shape[-1]
+    if fg2:
+        return make_desc(B, T, H, dk, dv, chunk, _DT[q.dtype], _gate_kind(a, nd),
+                         _lib.GATE_FG2, _lib.GATE_FG2)
     return make_desc(B, T, H, dk, dv, chunk, _DT[q.dtype], _gate_kind(a, nd),
                      _gate_kind(b, nd), _gate_kind(w, nd))
 
@@ -80,9 +89,10 @@ def forward_chunked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                     w: Optional[torch.Tensor] = None, s0: Optional[torch.Tensor] = None,
                     *, chunk: int = 64, out: Optional[torch.Tensor] = None,
                     s_final: Optional[torch.Tensor] = None, return_final: bool = True,
-                    workspace: Optional[torch.Tensor] = None,
-                    stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Causal chunked prefill.  Returns (o [B, T, H, dv], S_T [B, H, dk, dv] or None)."""
+                    workspace: Optional[torch.Tensor] = None, stream=None,
+                    fg2: bool = False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Causal chunked prefill.  Returns (o [B, T, H, dv], S_T [B, H, dk, dv] or None).
+    With fg2=True, b and w hold the vector learning rates beta^k, beta^v."""
     if q.dtype not in _DT:
         raise ValueError("q must be float32 or bfloat16")
     B, T, H, dk = q.shape
@@ -95,13 +105,15 @@ def forward_chunked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     _check(b, "b", dt, dev, [(B, T, H, dk), (B, T, H)])
     _check(w, "w", dt, dev, [(B, T, H, dv), (B, T, H)])
     _check(s0, "s0", torch.float32, dev, [(B, H, dk, dv)])
+    if fg2 and (b is None or w is None or b.dim() != 4 or w.dim() != 4):
+        raise ValueError("fg2 needs vector beta^k [B, T, H, dk] and beta^v [B, T, H, dv]")
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=dt, device=dev)
     _check(out, "out", dt, dev, [(B, T, H, dv)])
     if s_final is None and return_final:
         s_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
     _check(s_final, "s_final", torch.float32, dev, [(B, H, dk, dv)])
-    desc = desc_for(q, v, a, b, w, chunk)
+    desc = desc_for(q, v, a, b, w, chunk, fg2=fg2)
     need = _lib.workspace_size(desc)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -117,8 +129,10 @@ def forward_chunked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                 a: Optional[torch.Tensor], b: Optional[torch.Tensor],
                 w: Optional[torch.Tensor], state: torch.Tensor, *,
-                out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """One decode step; `state` is updated in place.  Returns o [B, H, dv]."""
+                out: Optional[torch.Tensor] = None, stream=None,
+                fg2: bool = False) -> torch.Tensor:
+    """One decode step; `state` is updated in place.  Returns o [B, H, dv].
+    With fg2=True, b and w hold the vector learning rates beta^k, beta^v."""
     if q.dtype not in _DT:
         raise ValueError("q must be float32 or bfloat16")
     B, H, dk = q.shape
@@ -131,15 +145,35 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     _check(b, "b", dt, dev, [(B, H, dk), (B, H)])
     _check(w, "w", dt, dev, [(B, H, dv), (B, H)])
     _check(state, "state", torch.float32, dev, [(B, H, dk, dv)])
+    if fg2 and (b is None or w is None or b.dim() != 3 or w.dim() != 3):
+        raise ValueError("fg2 needs vector beta^k [B, H, dk] and beta^v [B, H, dv]")
     if out is None:
         out = torch.empty((B, H, dv), dtype=dt, device=dev)
     _check(out, "out", dt, dev, [(B, H, dv)])
-    desc = desc_for(q, v, a, b, w, decode=True)
+    desc = desc_for(q, v, a, b, w, decode=True, fg2=fg2)
     st = _lib.decode_step(desc, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(w),
                           _ptr(state), _ptr(out), _stream_handle(stream))
     if st != _lib.OK:
         raise _lib.GdrError(st, "gdr_decode_step")
     return out
+
+
+def forward_fg2(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,
+                beta_k: torch.Tensor, beta_v: Optional[torch.Tensor] = None,
+                s0: Optional[torch.Tensor] = None, **kw):
+    """FG^2-GDN prefill (beta_v None: one beta for both, the symmetric form)
+    or FG^2-GDN+ (separate beta_k, beta_v); alpha the per-channel (or scalar)
+    decay.  Same kernels as forward_chunked."""
+    return forward_chunked(q, k, v, alpha, beta_k, beta_k if beta_v is None else beta_v, s0,
+                           fg2=True, **kw)
+
+
+def decode_step_fg2(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,
+                    beta_k: torch.Tensor, beta_v: Optional[torch.Tensor],
+                    state: torch.Tensor, **kw) -> torch.Tensor:
+    """One FG^2-GDN(+) decode step; `state` updated in place."""
+    return decode_step(q, k, v, alpha, beta_k, beta_k if beta_v is None else beta_v, state,
+                       fg2=True, **kw)
 
 
 def last_device_error(stream=None) -> int:

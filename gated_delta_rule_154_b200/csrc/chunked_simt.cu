@@ -105,6 +105,10 @@ chunked_simt_kernel(int B, int T, int H,
                 qv = to_f32(q[base + c]);
                 kv = to_f32(k[base + c]);
                 bv = gate_value(b, b_kind, tok, base, c);
+                if (b_kind == GDR_GATE_FG2) {  // key sqrt(beta^k) k, erase gate 1
+                    kv *= bv;
+                    bv = 1.f;
+                }
                 gv = a_kind == GDR_GATE_ONE ? 0.f
                                             : safe_log_decay(gate_value(a, a_kind, tok, base, c));
             }

@@ -113,6 +113,18 @@ __device__ __forceinline__ uint32_t mul2(uint32_t x, uint32_t y) {
                                *reinterpret_cast<__nv_bfloat162*>(&y));
     return *reinterpret_cast<uint32_t*>(&r);
 }
+// Square root to about 1 ulp (one SFU op); its results are rounded to bf16.
+__device__ __forceinline__ float sqrt_approx(float x) {
+    float y;
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// Square roots of two packed bf16 (non-negative by contract; a negative
+// input gives 0), each rounded to bf16.
+__device__ __forceinline__ uint32_t sqrt2(uint32_t x) {
+    return tc::pack_bf16x2(sqrt_approx(fmaxf(__uint_as_float(x << 16), 0.f)),
+                           sqrt_approx(fmaxf(__uint_as_float(x & 0xFFFF0000u), 0.f)));
+}
 // Reciprocal to about 1 ulp (one SFU op); its results are rounded to bf16.
 __device__ __forceinline__ float rcp_approx(float x) {
     float y;
@@ -314,7 +326,8 @@ __device__ __forceinline__ void issue_v(const TcMaps& m, uint32_t sbase, int t0,
 // the exchange barrier), before anything is written to X2.
 template <typename Mid>
 __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool vb, bool vw,
-                                             int a_kind, int n, const float* sca, float* QT,
+                                             bool fb, bool fw, int a_kind, int n,
+                                             const float* sca, float* QT,
                                              float* fcur, float* fprev, int* err_word,
                                              Mid&& mid) {
     const int p2 = tid & 63, q8 = tid >> 6;
@@ -369,12 +382,17 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
         const uint32_t v2 = *reinterpret_cast<const uint32_t*>(sm + OFF_U + o64);
         const uint32_t w2 = vw ? *reinterpret_cast<const uint32_t*>(sm + OFF_W + o64)
                                : tc::pack_bf16x2(sca[128 + r], sca[128 + r]);
-        const uint32_t kk2 = mul2(k2, ei);                                       // K"
-        *reinterpret_cast<uint32_t*>(sm + OFF_X1 + o128) = mul2(k2, e);          // K'
+        // FG^2-GDN learning rates: key sqrt(beta^k) k with erase gate 1, write
+        // gate sqrt(beta^v)
+        const uint32_t kt2 = fb ? mul2(k2, sqrt2(b2)) : k2;
+        const uint32_t kk2 = mul2(kt2, ei);                                      // K"
+        *reinterpret_cast<uint32_t*>(sm + OFF_X1 + o128) = mul2(kt2, e);         // K'
         *reinterpret_cast<uint32_t*>(sm + OFF_X1 + o128 + 8192u) = mul2(q2, e);  // Q'
         *reinterpret_cast<uint32_t*>(sm + OFF_X2 + o128) = kk2;
-        *reinterpret_cast<uint32_t*>(sm + OFF_X2 + o128 + 8192u) = mul2(b2, kk2);  // B"
-        *reinterpret_cast<uint32_t*>(sm + OFF_U + o64) = mul2(w2, v2);             // U
+        *reinterpret_cast<uint32_t*>(sm + OFF_X2 + o128 + 8192u) =
+            fb ? kk2 : mul2(b2, kk2);                                            // B"
+        *reinterpret_cast<uint32_t*>(sm + OFF_U + o64) =
+            mul2(fw ? sqrt2(w2) : w2, v2);                                       // U
     }
     if (q8 == 0) {
         const int i = 2 * p2;
@@ -439,8 +457,9 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
     const int bh = blockIdx.x;
     const int bi = bh / H, hi = bh % H;
     const size_t soff = (size_t)bh * D * D;
-    const bool va = a_kind == GDR_GATE_VECTOR, vb = b_kind == GDR_GATE_VECTOR,
-               vw = w_kind == GDR_GATE_VECTOR;
+    const bool fb = b_kind == GDR_GATE_FG2, fw = w_kind == GDR_GATE_FG2;
+    const bool va = a_kind == GDR_GATE_VECTOR, vb = b_kind == GDR_GATE_VECTOR || fb,
+               vw = w_kind == GDR_GATE_VECTOR || fw;
     const bool has_ab = va || vb;
 
     if (tid == 0) {
@@ -643,7 +662,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             compute_sync();
             if (*abort_s) break;
             // ================= P1c:
-            operand_pass(sm, tid, va, vb, vw, a_kind, min(C, T - t0), sca, QT, fcur, fprev,
+            operand_pass(sm, tid, va, vb, vw, fb, fw, a_kind, min(C, T - t0), sca, QT, fcur, fprev,
                          err_word, [&] {
                              if (t0 == 0) return;
                              // the last chunk's state update has read X2 and EB and
@@ -673,7 +692,6 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             signal(R_P2);
 
             // ================= P3: the X and S~ products run under the gram readout
-            if (has_next) load_scalars(t0 + C, cur ^ 1);
             wait_then_sync(bar(B_G), ph, tid, abort_s);
 
             // ================= P4: read the gram; masked blocks out
@@ -746,6 +764,9 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                     }
                 }
                 tc::fence_async_smem();
+                // the next chunk's scalar gates: these warps wait out the global
+                // loads' latency under the solve
+                if (has_next) load_scalars(t0 + C, cur ^ 1);
             }
             tc::fence_before_sync();
             signal(R_P5);
@@ -846,8 +867,10 @@ cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, c
         bool ok = make_map(&maps.q, q, d.B, d.T, d.H) && make_map(&maps.k, k, d.B, d.T, d.H) &&
                   make_map(&maps.v, v, d.B, d.T, d.H) && make_map(&maps.o, o, d.B, d.T, d.H);
         if (ok && d.decay == GDR_GATE_VECTOR) ok = make_map(&maps.a, a, d.B, d.T, d.H);
-        if (ok && d.erase == GDR_GATE_VECTOR) ok = make_map(&maps.b, b, d.B, d.T, d.H);
-        if (ok && d.write == GDR_GATE_VECTOR) ok = make_map(&maps.w, w, d.B, d.T, d.H);
+        if (ok && (d.erase == GDR_GATE_VECTOR || d.erase == GDR_GATE_FG2))
+            ok = make_map(&maps.b, b, d.B, d.T, d.H);
+        if (ok && (d.write == GDR_GATE_VECTOR || d.write == GDR_GATE_FG2))
+            ok = make_map(&maps.w, w, d.B, d.T, d.H);
         if (!ok) return cudaErrorInvalidValue;
     }
     cudaError_t e = cudaFuncSetAttribute(chunked_tc_kernel,

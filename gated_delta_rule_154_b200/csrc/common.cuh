@@ -29,6 +29,7 @@ __device__ __forceinline__ float gate_value(const T* g, int kind, long long sidx
                                             long long vbase, int c) {
     if (kind == GDR_GATE_ONE) return 1.0f;
     if (kind == GDR_GATE_SCALAR) return to_f32(g[sidx]);
+    if (kind == GDR_GATE_FG2) return sqrtf(fmaxf(to_f32(g[vbase + c]), 0.0f));  // sqrt(beta)
     return to_f32(g[vbase + c]);
 }
 

@@ -52,11 +52,16 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
 
     for (int i = tid; i < DK; i += NT) {
         const long long vb = bh * DK;
-        const float kv = to_f32(k[vb + i]);
+        float kv = to_f32(k[vb + i]);
+        float bv = gate_value(b, b_kind, bh, vb, i);
+        if (b_kind == GDR_GATE_FG2) {  // key sqrt(beta^k) k, erase gate 1
+            kv *= bv;
+            bv = 1.f;
+        }
         qs[i] = to_f32(q[vb + i]);
         ks[i] = kv;
         as_[i] = gate_value(a, a_kind, bh, vb, i);
-        bks[i] = gate_value(b, b_kind, bh, vb, i) * kv;
+        bks[i] = bv * kv;
     }
     for (int j = tid; j < DV; j += NT) {
         const long long vb = bh * DV;

@@ -49,6 +49,7 @@ cudaError_t error_word(int** out) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool valid_gate(int g) { return g == GDR_GATE_ONE || g == GDR_GATE_SCALAR || g == GDR_GATE_VECTOR; }
+bool valid_gate_beta(int g) { return valid_gate(g) || g == GDR_GATE_FG2; }  // erase, write
 
 // Checks shared by both entry points; `T_axis` tells whether T is part of the
 // tensor shapes (prefill) or fixed to 1 (decode).
@@ -61,7 +62,7 @@ gdr_status check_desc(const gdr_desc* d) {
         return GDR_ERR_INVALID_ARG;
     if (!(d->chunk == 16 || d->chunk == 32 || d->chunk == 64)) return GDR_ERR_INVALID_ARG;
     if (!(d->in_dtype == GDR_F32 || d->in_dtype == GDR_BF16)) return GDR_ERR_INVALID_ARG;
-    if (!valid_gate(d->decay) || !valid_gate(d->erase) || !valid_gate(d->write))
+    if (!valid_gate(d->decay) || !valid_gate_beta(d->erase) || !valid_gate_beta(d->write))
         return GDR_ERR_INVALID_ARG;
     return GDR_OK;
 }

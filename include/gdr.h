@@ -71,8 +71,24 @@ typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
 /* How a gate is given.  ONE: the gate is identically 1 and its pointer is
  * ignored (may be NULL).  SCALAR: one value per (b, t, h), [B, T, H].
  * VECTOR: one value per channel, [B, T, H, dk] for a and b, [B, T, H, dv]
- * for w. */
-typedef enum { GDR_GATE_ONE = 0, GDR_GATE_SCALAR = 1, GDR_GATE_VECTOR = 2 } gdr_gate;
+ * for w.
+ * FG2 (erase and write only): the tensor holds FG^2-GDN's per-channel
+ * learning rate beta >= 0, laid out as VECTOR, and enters through its square
+ * root.  erase = FG2: the key used everywhere is sqrt(beta^k) * k and the
+ * erase gate is 1.  write = FG2: the write gate is sqrt(beta^v).  With both
+ * FG2 and one tensor for b and w this is FG^2-GDN's symmetric update
+ *     S_t = (I - k~ k~^T) Diag(a_t) S_{t-1} + k~ v~^T,  k~ = sqrt(beta) k,
+ *     v~ = sqrt(beta) v
+ * (FG^2-GDN page, section 2 "Methodology", FG2-GDN update rule); with
+ * separate beta^k and beta^v tensors it is the reading taken for FG^2-GDN+
+ * (same page, the FG2-GDN+ variant, which prints no formula).  The square
+ * roots are taken inside the kernels; no scaled copy of k, v is written. */
+typedef enum {
+    GDR_GATE_ONE = 0,
+    GDR_GATE_SCALAR = 1,
+    GDR_GATE_VECTOR = 2,
+    GDR_GATE_FG2 = 3
+} gdr_gate;
 
 typedef struct {
     int B, T, H;          /* batch, tokens, heads; B, H >= 1, T >= 0        */

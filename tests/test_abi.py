@@ -104,3 +104,18 @@ def test_gate_one_needs_no_pointer_and_empty_is_a_no_op(lib):
 def test_null_descriptor(lib):
     assert lib.gdr_forward_chunked(None, *([None] * 9), None, 0, None) == _lib.ERR_INVALID_ARG
     assert lib.gdr_decode_step(None, *([None] * 9)) == _lib.ERR_INVALID_ARG
+
+
+def test_fg2_gate_kind_accepted_for_erase_and_write_only(lib):
+    # accepted (T = 0 and no final state: validated, nothing launched)
+    d = _desc(T=0, erase=_lib.GATE_FG2, write=_lib.GATE_FG2)
+    assert _lib.forward_chunked(d, P, P, P, P, P, P, 0, P, 0, 0, 0, 0) == _lib.OK
+    # FG2 is no decay form, and its learning-rate pointers are required
+    assert _lib.forward_chunked(_desc(decay=_lib.GATE_FG2), P, P, P, P, P, P, 0, P, 0, 0, 0,
+                                0) == _lib.ERR_INVALID_ARG
+    d = _desc(erase=_lib.GATE_FG2, write=_lib.GATE_FG2)
+    assert _lib.forward_chunked(d, P, P, P, P, 0, P, 0, P, 0, 0, 0, 0) == _lib.ERR_INVALID_ARG
+    assert _lib.forward_chunked(d, P, P, P, P, P, 0, 0, P, 0, 0, 0, 0) == _lib.ERR_INVALID_ARG
+    for bad in (4, 99):
+        assert _lib.forward_chunked(_desc(erase=bad), P, P, P, P, P, P, 0, P, 0, 0, 0,
+                                    0) == _lib.ERR_INVALID_ARG
