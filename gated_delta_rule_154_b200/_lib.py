@@ -20,7 +20,8 @@ F32, BF16 = 0, 1
 GATE_ONE, GATE_SCALAR, GATE_VECTOR, GATE_FG2 = 0, 1, 2, 3
 
 EXPORTS = ("gdr_workspace_size", "gdr_forward_chunked", "gdr_decode_step",
-           "gdr_last_device_error", "gdr_status_string", "gdr_version", "gdr_test_skip_signal")
+           "gdr_last_device_error", "gdr_status_string", "gdr_version", "gdr_test_skip_signal",
+           "gdr_decode_step_paged")
 
 
 class GdrDesc(ctypes.Structure):
@@ -62,6 +63,8 @@ def load(path: str = LIB_PATH):
     lib.gdr_status_string.argtypes = [i]
     lib.gdr_version.restype = i
     lib.gdr_version.argtypes = []
+    lib.gdr_decode_step_paged.restype = i
+    lib.gdr_decode_step_paged.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp]
     lib.gdr_test_skip_signal.restype = None
     lib.gdr_test_skip_signal.argtypes = [i]
     _lib = lib
@@ -86,6 +89,12 @@ def forward_chunked(desc: GdrDesc, q, k, v, a, b, w, s0, o, s_final, workspace, 
 def decode_step(desc: GdrDesc, q, k, v, a, b, w, state, o, stream) -> int:
     """Raw call: every pointer an int (0 = NULL).  Returns the gdr_status."""
     return int(load().gdr_decode_step(ctypes.byref(desc), q, k, v, a, b, w, state, o, stream))
+
+
+def decode_step_paged(desc: GdrDesc, q, k, v, a, b, w, pool, slot, n_slots, o, stream) -> int:
+    """Raw call: every pointer an int (0 = NULL).  Returns the gdr_status."""
+    return int(load().gdr_decode_step_paged(ctypes.byref(desc), q, k, v, a, b, w, pool, slot,
+                                            int(n_slots), o, stream))
 
 
 def last_device_error(stream) -> int:

@@ -158,6 +158,42 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return out
 
 
+def decode_step_paged(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                      a: Optional[torch.Tensor], b: Optional[torch.Tensor],
+                      w: Optional[torch.Tensor], pool: torch.Tensor, slot: torch.Tensor, *,
+                      out: Optional[torch.Tensor] = None, stream=None,
+                      fg2: bool = False) -> torch.Tensor:
+    """One decode step over a state pool [n_slots, H, dk, dv] float32: batch
+    entry b updates pool[slot[b]] in place (slot int32 [B], distinct entries).
+    Returns o [B, H, dv]; an out-of-range slot is skipped and reported by
+    last_device_error() as ERR_INVALID_ARG."""
+    if q.dtype not in _DT:
+        raise ValueError("q must be float32 or bfloat16")
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    _check(q, "q", dt, dev, [(B, H, dk)])
+    _check(k, "k", dt, dev, [(B, H, dk)])
+    _check(v, "v", dt, dev, [(B, H, dv)])
+    _check(a, "a", dt, dev, [(B, H, dk), (B, H)])
+    _check(b, "b", dt, dev, [(B, H, dk), (B, H)])
+    _check(w, "w", dt, dev, [(B, H, dv), (B, H)])
+    if pool.dim() != 4 or tuple(pool.shape[1:]) != (H, dk, dv):
+        raise ValueError("pool must be [n_slots, %d, %d, %d]" % (H, dk, dv))
+    _check(pool, "pool", torch.float32, dev, [tuple(pool.shape)])
+    _check(slot, "slot", torch.int32, dev, [(B,)])
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=dt, device=dev)
+    _check(out, "out", dt, dev, [(B, H, dv)])
+    desc = desc_for(q, v, a, b, w, decode=True, fg2=fg2)
+    st = _lib.decode_step_paged(desc, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(w),
+                                _ptr(pool), _ptr(slot), pool.shape[0], _ptr(out),
+                                _stream_handle(stream))
+    if st != _lib.OK:
+        raise _lib.GdrError(st, "gdr_decode_step_paged")
+    return out
+
+
 def forward_fg2(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,
                 beta_k: torch.Tensor, beta_v: Optional[torch.Tensor] = None,
                 s0: Optional[torch.Tensor] = None, **kw):

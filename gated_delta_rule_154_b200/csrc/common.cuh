@@ -11,7 +11,7 @@ namespace gdr {
 
 // Device error word bits.  A kernel that detects a problem ORs its bit into
 // the word it was given; gdr_last_device_error() turns the bits into a status.
-enum : int { kErrTimeout = 1, kErrRange = 2 };
+enum : int { kErrTimeout = 1, kErrRange = 2, kErrIndex = 4 };
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }

@@ -15,6 +15,10 @@
 // (each warp reads whole 512-byte rows), reduce e over the key axis (in
 // registers, then across warps through shared memory), update in registers,
 // store the new state with 16-byte stores, and reduce o the same way.
+//
+// Paged form (many sequences, one state pool): batch entry b reads and
+// writes pool slot slot[b] instead of state b; an out-of-range slot is
+// skipped and flagged in the device error word.
 #include "common.cuh"
 
 namespace gdr {
@@ -25,7 +29,8 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                    const Tin* __restrict__ v, const Tin* __restrict__ a,
                    const Tin* __restrict__ b, const Tin* __restrict__ w,
                    int a_kind, int b_kind, int w_kind,
-                   float* __restrict__ state, Tin* __restrict__ o) {
+                   float* __restrict__ state, Tin* __restrict__ o, int H,
+                   const int* __restrict__ slot, int n_slots, int* __restrict__ err_word) {
     constexpr int NT = 256;
     constexpr int TPR = DV / 4;     // threads per state row (one float4 each)
     constexpr int RS = NT / TPR;    // rows handled side by side
@@ -41,7 +46,17 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     const int cg = tid % TPR;         // column group: columns 4cg .. 4cg+3
     const int rs = tid / TPR;         // row set: rows rs, rs + RS, ...
 
-    float* S = state + bh * (long long)DK * DV;
+    long long sidx = bh;  // state of this (batch, head)
+    if (slot) {
+        const long long bi = bh / H;
+        const int sl = slot[bi];
+        if (sl < 0 || sl >= n_slots) {  // whole CTA agrees: skip, flag once
+            if (tid == 0 && bh % H == 0) atomicOr(err_word, kErrIndex);
+            return;
+        }
+        sidx = (long long)sl * H + bh % H;
+    }
+    float* S = state + sidx * (long long)DK * DV;
 
     // Issue the state loads first so they are in flight while the small
     // inputs are staged.
@@ -124,38 +139,40 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     }
 }
 
+struct DecodeArgs {
+    const void *q, *k, *v, *a, *b, *w;
+    float* state;
+    void* o;
+    const int* slot;  // nullptr: state b for batch entry b
+    int n_slots;
+    int* err_word;
+};
+
 template <typename Tin, int DK, int DV>
-static cudaError_t launch_decode_t(const gdr_desc& d, const void* q, const void* k,
-                                   const void* v, const void* a, const void* b,
-                                   const void* w, float* state, void* o,
-                                   cudaStream_t stream) {
+static cudaError_t launch_decode_t(const gdr_desc& d, const DecodeArgs& x, cudaStream_t stream) {
     const unsigned grid = (unsigned)((long long)d.B * d.H);
     decode_step_kernel<Tin, DK, DV><<<grid, 256, 0, stream>>>(
-        (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)a, (const Tin*)b,
-        (const Tin*)w, (int)d.decay, (int)d.erase, (int)d.write, state, (Tin*)o);
+        (const Tin*)x.q, (const Tin*)x.k, (const Tin*)x.v, (const Tin*)x.a, (const Tin*)x.b,
+        (const Tin*)x.w, (int)d.decay, (int)d.erase, (int)d.write, x.state, (Tin*)x.o, d.H,
+        x.slot, x.n_slots, x.err_word);
     return cudaGetLastError();
 }
 
 template <typename Tin>
-static cudaError_t launch_decode_d(const gdr_desc& d, const void* q, const void* k,
-                                   const void* v, const void* a, const void* b,
-                                   const void* w, float* state, void* o,
-                                   cudaStream_t stream) {
-    if (d.dk == 128 && d.dv == 128)
-        return launch_decode_t<Tin, 128, 128>(d, q, k, v, a, b, w, state, o, stream);
-    if (d.dk == 128 && d.dv == 64)
-        return launch_decode_t<Tin, 128, 64>(d, q, k, v, a, b, w, state, o, stream);
-    if (d.dk == 64 && d.dv == 128)
-        return launch_decode_t<Tin, 64, 128>(d, q, k, v, a, b, w, state, o, stream);
-    return launch_decode_t<Tin, 64, 64>(d, q, k, v, a, b, w, state, o, stream);
+static cudaError_t launch_decode_d(const gdr_desc& d, const DecodeArgs& x, cudaStream_t stream) {
+    if (d.dk == 128 && d.dv == 128) return launch_decode_t<Tin, 128, 128>(d, x, stream);
+    if (d.dk == 128 && d.dv == 64) return launch_decode_t<Tin, 128, 64>(d, x, stream);
+    if (d.dk == 64 && d.dv == 128) return launch_decode_t<Tin, 64, 128>(d, x, stream);
+    return launch_decode_t<Tin, 64, 64>(d, x, stream);
 }
 
 cudaError_t launch_decode(const gdr_desc& d, const void* q, const void* k, const void* v,
                           const void* a, const void* b, const void* w, float* state,
-                          void* o, cudaStream_t stream) {
-    if (d.in_dtype == GDR_BF16)
-        return launch_decode_d<__nv_bfloat16>(d, q, k, v, a, b, w, state, o, stream);
-    return launch_decode_d<float>(d, q, k, v, a, b, w, state, o, stream);
+                          void* o, const int* slot, int n_slots, int* err_word,
+                          cudaStream_t stream) {
+    const DecodeArgs x{q, k, v, a, b, w, state, o, slot, n_slots, err_word};
+    if (d.in_dtype == GDR_BF16) return launch_decode_d<__nv_bfloat16>(d, x, stream);
+    return launch_decode_d<float>(d, x, stream);
 }
 
 }  // namespace gdr

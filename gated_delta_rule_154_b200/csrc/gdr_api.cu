@@ -8,7 +8,8 @@
 namespace gdr {
 cudaError_t launch_decode(const gdr_desc& d, const void* q, const void* k, const void* v,
                           const void* a, const void* b, const void* w, float* state,
-                          void* o, cudaStream_t stream);
+                          void* o, const int* slot, int n_slots, int* err_word,
+                          cudaStream_t stream);
 cudaError_t launch_chunked_simt(const gdr_desc& d, const void* q, const void* k,
                                 const void* v, const void* a, const void* b, const void* w,
                                 const float* s0, void* o, float* s_final, cudaStream_t st);
@@ -152,7 +153,23 @@ gdr_status gdr_decode_step(const gdr_desc* d, const void* q, const void* k, cons
     if (d->T != 1) return GDR_ERR_INVALID_ARG;
     if ((s = check_inputs(d, true, q, k, v, a, b, w, o)) != GDR_OK) return s;
     if ((s = check_ptr(state, true)) != GDR_OK) return s;
-    cudaError_t e = gdr::launch_decode(*d, q, k, v, a, b, w, state, o,
+    cudaError_t e = gdr::launch_decode(*d, q, k, v, a, b, w, state, o, nullptr, 0, nullptr,
+                                       reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+gdr_status gdr_decode_step_paged(const gdr_desc* d, const void* q, const void* k, const void* v,
+                                 const void* a, const void* b, const void* w, float* state_pool,
+                                 const int* slot, int n_slots, void* o, gdr_stream_t stream) {
+    gdr_status s = check_desc(d);
+    if (s != GDR_OK) return s;
+    if (d->T != 1 || n_slots < 1) return GDR_ERR_INVALID_ARG;
+    if ((s = check_inputs(d, true, q, k, v, a, b, w, o)) != GDR_OK) return s;
+    if ((s = check_ptr(state_pool, true)) != GDR_OK) return s;
+    if (slot == nullptr || reinterpret_cast<uintptr_t>(slot) % 4 != 0) return GDR_ERR_INVALID_ARG;
+    int* err = nullptr;
+    if (error_word(&err) != cudaSuccess) return GDR_ERR_CUDA;
+    cudaError_t e = gdr::launch_decode(*d, q, k, v, a, b, w, state_pool, o, slot, n_slots, err,
                                        reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
@@ -170,6 +187,7 @@ gdr_status gdr_last_device_error(gdr_stream_t stream) {
     if (cudaMemcpyToSymbol(g_gdr_error_word, &zero, sizeof(int)) != cudaSuccess)
         return GDR_ERR_CUDA;
     if (word & gdr::kErrTimeout) return GDR_ERR_TIMEOUT;
+    if (word & gdr::kErrIndex) return GDR_ERR_INVALID_ARG;
     return GDR_ERR_RANGE;
 }
 

@@ -146,9 +146,26 @@ gdr_status gdr_decode_step(const gdr_desc *desc, const void *q, const void *k,
                            const void *w, float *state, void *o,
                            gdr_stream_t stream);
 
+/*
+ * The same step over a pool of states (many sequences, one state pool):
+ * batch entry b reads and rewrites state_pool[slot[b]], each pool slot being
+ * [H, dk, dv] float32; the pool holds n_slots >= 1 of them, other slots are
+ * not touched.  slot: int32 [B] in device memory, 4-byte aligned.  Entries
+ * must be distinct (two entries on one slot race).  An entry outside
+ * [0, n_slots) is skipped (its o is not written) and recorded in the device
+ * error word, read as GDR_ERR_INVALID_ARG by gdr_last_device_error().
+ * Everything else as gdr_decode_step.
+ */
+gdr_status gdr_decode_step_paged(const gdr_desc *desc, const void *q, const void *k,
+                                 const void *v, const void *a, const void *b,
+                                 const void *w, float *state_pool, const int *slot,
+                                 int n_slots, void *o, gdr_stream_t stream);
+
 /* Synchronises `stream`, returns the status recorded on the device since the
- * previous call (GDR_OK if none) and clears it.  GDR_ERR_CUDA if the
- * synchronisation itself failed. */
+ * previous call (GDR_OK if none) and clears it: GDR_ERR_TIMEOUT (a bounded
+ * wait ran out), GDR_ERR_INVALID_ARG (a paged decode slot out of range) or
+ * GDR_ERR_RANGE (decay range), in that order of precedence.  GDR_ERR_CUDA if
+ * the synchronisation itself failed. */
 gdr_status gdr_last_device_error(gdr_stream_t stream);
 
 /*

@@ -119,3 +119,21 @@ def test_fg2_gate_kind_accepted_for_erase_and_write_only(lib):
     for bad in (4, 99):
         assert _lib.forward_chunked(_desc(erase=bad), P, P, P, P, P, P, 0, P, 0, 0, 0,
                                     0) == _lib.ERR_INVALID_ARG
+
+
+def test_paged_decode_argument_checks(lib):
+    d = _desc(T=1)
+    ok = dict(q=P, k=P, v=P, a=P, b=P, w=P, pool=P, slot=P, n=4, o=P)
+
+    def call(**kw):
+        x = dict(ok)
+        x.update(kw)
+        return _lib.decode_step_paged(d, x["q"], x["k"], x["v"], x["a"], x["b"], x["w"],
+                                      x["pool"], x["slot"], x["n"], x["o"], 0)
+    assert call(slot=0) == _lib.ERR_INVALID_ARG        # slot array required
+    assert call(slot=P + 2) == _lib.ERR_INVALID_ARG    # int32 alignment
+    assert call(pool=0) == _lib.ERR_INVALID_ARG
+    assert call(pool=P + 4) == _lib.ERR_INVALID_ARG
+    assert call(n=0) == _lib.ERR_INVALID_ARG
+    d.T = 2
+    assert call() == _lib.ERR_INVALID_ARG
