@@ -21,7 +21,7 @@ GATE_ONE, GATE_SCALAR, GATE_VECTOR, GATE_FG2 = 0, 1, 2, 3
 
 EXPORTS = ("gdr_workspace_size", "gdr_forward_chunked", "gdr_decode_step",
            "gdr_last_device_error", "gdr_status_string", "gdr_version", "gdr_test_skip_signal",
-           "gdr_decode_step_paged")
+           "gdr_decode_step_paged", "gdr_forward_varlen")
 
 
 class GdrDesc(ctypes.Structure):
@@ -63,6 +63,8 @@ def load(path: str = LIB_PATH):
     lib.gdr_status_string.argtypes = [i]
     lib.gdr_version.restype = i
     lib.gdr_version.argtypes = []
+    lib.gdr_forward_varlen.restype = i
+    lib.gdr_forward_varlen.argtypes = [dp, vp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.gdr_decode_step_paged.restype = i
     lib.gdr_decode_step_paged.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp]
     lib.gdr_test_skip_signal.restype = None
@@ -89,6 +91,13 @@ def forward_chunked(desc: GdrDesc, q, k, v, a, b, w, s0, o, s_final, workspace, 
 def decode_step(desc: GdrDesc, q, k, v, a, b, w, state, o, stream) -> int:
     """Raw call: every pointer an int (0 = NULL).  Returns the gdr_status."""
     return int(load().gdr_decode_step(ctypes.byref(desc), q, k, v, a, b, w, state, o, stream))
+
+
+def forward_varlen(desc: GdrDesc, cu_seqlens, n_seqs, q, k, v, a, b, w, s0, o, s_final,
+                   workspace, ws_bytes, stream) -> int:
+    """Raw call: every pointer an int (0 = NULL).  Returns the gdr_status."""
+    return int(load().gdr_forward_varlen(ctypes.byref(desc), cu_seqlens, int(n_seqs), q, k, v,
+                                         a, b, w, s0, o, s_final, workspace, ws_bytes, stream))
 
 
 def decode_step_paged(desc: GdrDesc, q, k, v, a, b, w, pool, slot, n_slots, o, stream) -> int:

@@ -158,6 +158,49 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return out
 
 
+def forward_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                   a: Optional[torch.Tensor], b: Optional[torch.Tensor],
+                   w: Optional[torch.Tensor], cu_seqlens: torch.Tensor,
+                   s0: Optional[torch.Tensor] = None, *, chunk: int = 64,
+                   out: Optional[torch.Tensor] = None, s_final: Optional[torch.Tensor] = None,
+                   return_final: bool = True, stream=None,
+                   fg2: bool = False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Prefill of packed sequences: q, k, v, gates, o are [1, T, H, *]; sequence
+    n is tokens [cu_seqlens[n], cu_seqlens[n + 1]) (int32 [N + 1] on the
+    device); s0 and the returned final states are [N, H, dk, dv]."""
+    if q.dtype not in _DT:
+        raise ValueError("q must be float32 or bfloat16")
+    B, T, H, dk = q.shape
+    if B != 1:
+        raise ValueError("packed sequences take q as [1, T, H, dk]")
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev, [tuple(cu_seqlens.shape)])
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ValueError("cu_seqlens must be int32 [N + 1], N >= 1")
+    N = cu_seqlens.numel() - 1
+    _check(q, "q", dt, dev, [(B, T, H, dk)])
+    _check(k, "k", dt, dev, [(B, T, H, dk)])
+    _check(v, "v", dt, dev, [(B, T, H, dv)])
+    _check(a, "a", dt, dev, [(B, T, H, dk), (B, T, H)])
+    _check(b, "b", dt, dev, [(B, T, H, dk), (B, T, H)])
+    _check(w, "w", dt, dev, [(B, T, H, dv), (B, T, H)])
+    _check(s0, "s0", torch.float32, dev, [(N, H, dk, dv)])
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    _check(out, "out", dt, dev, [(B, T, H, dv)])
+    if s_final is None and return_final:
+        s_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    _check(s_final, "s_final", torch.float32, dev, [(N, H, dk, dv)])
+    desc = desc_for(q, v, a, b, w, chunk, fg2=fg2)
+    st = _lib.forward_varlen(desc, _ptr(cu_seqlens), N, _ptr(q), _ptr(k), _ptr(v), _ptr(a),
+                             _ptr(b), _ptr(w), _ptr(s0), _ptr(out), _ptr(s_final), 0, 0,
+                             _stream_handle(stream))
+    if st != _lib.OK:
+        raise _lib.GdrError(st, "gdr_forward_varlen")
+    return out, s_final
+
+
 def decode_step_paged(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                       a: Optional[torch.Tensor], b: Optional[torch.Tensor],
                       w: Optional[torch.Tensor], pool: torch.Tensor, slot: torch.Tensor, *,

@@ -59,7 +59,8 @@ chunked_simt_kernel(int B, int T, int H,
                     const Tin* __restrict__ b, const Tin* __restrict__ w,
                     int a_kind, int b_kind, int w_kind,
                     const float* __restrict__ s0, Tin* __restrict__ o,
-                    float* __restrict__ s_final) {
+                    float* __restrict__ s_final, const int* __restrict__ cu_seqlens,
+                    int* __restrict__ err_word) {
     constexpr int NT = 256;
     constexpr int SL = NT / DVB;  // s-slices per column in the triangular solve
     static_assert(SL == 8 || SL == 16, "DVB must be 32 or 16");
@@ -82,7 +83,14 @@ chunked_simt_kernel(int B, int T, int H,
 
     const int tid = threadIdx.x;
     const int bh = blockIdx.x;
-    const int bi = bh / H, hi = bh % H;
+    const int hi = bh % H;
+    // this CTA's tokens: [tb, tb + len) of batch row bi (packed sequences: one
+    // batch row; a range outside the tensor is reported and skipped)
+    int bi, tb, len;
+    if (!seq_range(cu_seqlens, bh / H, T, bi, tb, len)) {
+        if (tid == 0 && blockIdx.y == 0) atomicOr(err_word, kErrIndex);
+        return;
+    }
     const int j0 = blockIdx.y * DVB;
 
     const size_t soff = (size_t)bh * DK * DV;
@@ -91,8 +99,8 @@ chunked_simt_kernel(int B, int T, int H,
         Ss[x] = s0 ? s0[soff + (size_t)c * DV + j0 + j] : 0.0f;
     }
 
-    for (int t0 = 0; t0 < T; t0 += C) {
-        const int n = min(C, T - t0);
+    for (int t0 = 0; t0 < len; t0 += C) {
+        const int n = min(C, len - t0);
         __syncthreads();  // previous chunk finished with every buffer
 
         // ---- load the chunk; padded tokens act as a = 1, k = q = v = 0
@@ -100,7 +108,7 @@ chunked_simt_kernel(int B, int T, int H,
             const int r = x / DK, c = x % DK;
             float qv = 0.f, kv = 0.f, bv = 0.f, gv = 0.f;
             if (r < n) {
-                const long long tok = ((long long)bi * T + t0 + r) * H + hi;
+                const long long tok = ((long long)bi * T + tb + t0 + r) * H + hi;
                 const long long base = tok * DK;
                 qv = to_f32(q[base + c]);
                 kv = to_f32(k[base + c]);
@@ -121,7 +129,7 @@ chunked_simt_kernel(int B, int T, int H,
             const int r = x / DVB, j = x % DVB;
             float u = 0.f;
             if (r < n) {
-                const long long tok = ((long long)bi * T + t0 + r) * H + hi;
+                const long long tok = ((long long)bi * T + tb + t0 + r) * H + hi;
                 const long long base = tok * DV;
                 u = gate_value(w, w_kind, tok, base, j0 + j) * to_f32(v[base + j0 + j]);
             }
@@ -215,7 +223,7 @@ chunked_simt_kernel(int B, int T, int H,
             for (int s = 0; s <= r; ++s)
                 acc = fmaf(Aqk[r * CP + s], Us[s * DVB + j],
                            fmaf(-Aqb[r * CP + s], Es[s * DVB + j], acc));
-            const long long tok = ((long long)bi * T + t0 + r) * H + hi;
+            const long long tok = ((long long)bi * T + tb + t0 + r) * H + hi;
             o[tok * DV + j0 + j] = from_f32<Tin>(acc);
         }
         __syncthreads();
@@ -239,55 +247,59 @@ chunked_simt_kernel(int B, int T, int H,
     }
 }
 
+struct SimtArgs {
+    const void *q, *k, *v, *a, *b, *w;
+    const float* s0;
+    void* o;
+    float* s_final;
+    const int* cu_seqlens;  // nullptr: batch rows as sequences
+    int n_seqs;
+    int* err_word;
+};
+
 template <typename Tin, int DK, int DV, int C, int DVB>
-static cudaError_t launch_simt_t(const gdr_desc& d, const void* q, const void* k,
-                                 const void* v, const void* a, const void* b, const void* w,
-                                 const float* s0, void* o, float* s_final, cudaStream_t st) {
+static cudaError_t launch_simt_t(const gdr_desc& d, const SimtArgs& x, cudaStream_t st) {
     auto kern = chunked_simt_kernel<Tin, DK, DV, C, DVB>;
     const size_t smem = SimtSmem<DK, DVB, C>::bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)(d.B * d.H), DV / DVB);
-    kern<<<grid, 256, smem, st>>>(d.B, d.T, d.H, (const Tin*)q, (const Tin*)k, (const Tin*)v,
-                                  (const Tin*)a, (const Tin*)b, (const Tin*)w, (int)d.decay,
-                                  (int)d.erase, (int)d.write, s0, (Tin*)o, s_final);
+    const long long nseq = x.cu_seqlens ? x.n_seqs : d.B;
+    dim3 grid((unsigned)(nseq * d.H), DV / DVB);
+    kern<<<grid, 256, smem, st>>>(d.B, d.T, d.H, (const Tin*)x.q, (const Tin*)x.k,
+                                  (const Tin*)x.v, (const Tin*)x.a, (const Tin*)x.b,
+                                  (const Tin*)x.w, (int)d.decay, (int)d.erase, (int)d.write,
+                                  x.s0, (Tin*)x.o, x.s_final, x.cu_seqlens, x.err_word);
     return cudaGetLastError();
 }
 
 template <typename Tin, int DK, int DV>
-static cudaError_t launch_simt_c(const gdr_desc& d, const void* q, const void* k,
-                                 const void* v, const void* a, const void* b, const void* w,
-                                 const float* s0, void* o, float* s_final, cudaStream_t st) {
+static cudaError_t launch_simt_c(const gdr_desc& d, const SimtArgs& x, cudaStream_t st) {
     switch (d.chunk) {
-        case 16: return launch_simt_t<Tin, DK, DV, 16, 32>(d, q, k, v, a, b, w, s0, o, s_final, st);
-        case 32: return launch_simt_t<Tin, DK, DV, 32, 32>(d, q, k, v, a, b, w, s0, o, s_final, st);
+        case 16: return launch_simt_t<Tin, DK, DV, 16, 32>(d, x, st);
+        case 32: return launch_simt_t<Tin, DK, DV, 32, 32>(d, x, st);
         default:
-            if (DK == 128)
-                return launch_simt_t<Tin, DK, DV, 64, 16>(d, q, k, v, a, b, w, s0, o, s_final, st);
-            return launch_simt_t<Tin, DK, DV, 64, 32>(d, q, k, v, a, b, w, s0, o, s_final, st);
+            if (DK == 128) return launch_simt_t<Tin, DK, DV, 64, 16>(d, x, st);
+            return launch_simt_t<Tin, DK, DV, 64, 32>(d, x, st);
     }
 }
 
 template <typename Tin>
-static cudaError_t launch_simt_d(const gdr_desc& d, const void* q, const void* k,
-                                 const void* v, const void* a, const void* b, const void* w,
-                                 const float* s0, void* o, float* s_final, cudaStream_t st) {
-    if (d.dk == 128 && d.dv == 128)
-        return launch_simt_c<Tin, 128, 128>(d, q, k, v, a, b, w, s0, o, s_final, st);
-    if (d.dk == 128 && d.dv == 64)
-        return launch_simt_c<Tin, 128, 64>(d, q, k, v, a, b, w, s0, o, s_final, st);
-    if (d.dk == 64 && d.dv == 128)
-        return launch_simt_c<Tin, 64, 128>(d, q, k, v, a, b, w, s0, o, s_final, st);
-    return launch_simt_c<Tin, 64, 64>(d, q, k, v, a, b, w, s0, o, s_final, st);
+static cudaError_t launch_simt_d(const gdr_desc& d, const SimtArgs& x, cudaStream_t st) {
+    if (d.dk == 128 && d.dv == 128) return launch_simt_c<Tin, 128, 128>(d, x, st);
+    if (d.dk == 128 && d.dv == 64) return launch_simt_c<Tin, 128, 64>(d, x, st);
+    if (d.dk == 64 && d.dv == 128) return launch_simt_c<Tin, 64, 128>(d, x, st);
+    return launch_simt_c<Tin, 64, 64>(d, x, st);
 }
 
 cudaError_t launch_chunked_simt(const gdr_desc& d, const void* q, const void* k,
                                 const void* v, const void* a, const void* b, const void* w,
-                                const float* s0, void* o, float* s_final, cudaStream_t st) {
-    if (d.in_dtype == GDR_BF16)
-        return launch_simt_d<__nv_bfloat16>(d, q, k, v, a, b, w, s0, o, s_final, st);
-    return launch_simt_d<float>(d, q, k, v, a, b, w, s0, o, s_final, st);
+                                const float* s0, void* o, float* s_final,
+                                const int* cu_seqlens, int n_seqs, int* err_word,
+                                cudaStream_t st) {
+    const SimtArgs x{q, k, v, a, b, w, s0, o, s_final, cu_seqlens, n_seqs, err_word};
+    if (d.in_dtype == GDR_BF16) return launch_simt_d<__nv_bfloat16>(d, x, st);
+    return launch_simt_d<float>(d, x, st);
 }
 
 }  // namespace gdr

@@ -375,13 +375,18 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
         const uint32_t ei = tc::pack_bf16x2(h0 * rev0, h1 * rev1);
         rev0 *= __uint_as_float(apr[x] << 16);
         rev1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
-        const uint32_t k2 = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW + o128);
-        const uint32_t q2 = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW + o128 + 8192u);
+        uint32_t k2 = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW + o128);
+        uint32_t q2 = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW + o128 + 8192u);
         const uint32_t b2 = vb ? *reinterpret_cast<const uint32_t*>(sm + OFF_X1 + o128 + 8192u)
                                : tc::pack_bf16x2(sca[64 + r], sca[64 + r]);
-        const uint32_t v2 = *reinterpret_cast<const uint32_t*>(sm + OFF_U + o64);
+        uint32_t v2 = *reinterpret_cast<const uint32_t*>(sm + OFF_U + o64);
         const uint32_t w2 = vw ? *reinterpret_cast<const uint32_t*>(sm + OFF_W + o64)
                                : tc::pack_bf16x2(sca[128 + r], sca[128 + r]);
+        if (r >= n) {  // past the sequence (a packed neighbour's tokens): k = q = v = 0
+            k2 = 0u;
+            q2 = 0u;
+            v2 = 0u;
+        }
         // FG^2-GDN learning rates: key sqrt(beta^k) k with erase gate 1, write
         // gate sqrt(beta^v)
         const uint32_t kt2 = fb ? mul2(k2, sqrt2(b2)) : k2;
@@ -432,7 +437,8 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                   const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                   const __nv_bfloat16* __restrict__ w, int a_kind, int b_kind, int w_kind,
                   const float* __restrict__ s0, float* __restrict__ s_final,
-                  int* __restrict__ err_word, int skip_signal) {
+                  int* __restrict__ err_word, int skip_signal,
+                  const int* __restrict__ cu_seqlens, __nv_bfloat16* __restrict__ o_raw) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -455,7 +461,14 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
 
     const int bh = blockIdx.x;
-    const int bi = bh / H, hi = bh % H;
+    const int hi = bh % H;
+    // this CTA's tokens: [tb, tb + L) of batch row bi (packed sequences: one
+    // batch row; a range outside the tensor is reported and skipped)
+    int bi, tb, L;
+    if (!seq_range(cu_seqlens, bh / H, T, bi, tb, L)) {
+        if (threadIdx.x == 0) atomicOr(err_word, kErrIndex);
+        return;
+    }
     const size_t soff = (size_t)bh * D * D;
     const bool fb = b_kind == GDR_GATE_FG2, fw = w_kind == GDR_GATE_FG2;
     const bool va = a_kind == GDR_GATE_VECTOR, vb = b_kind == GDR_GATE_VECTOR || fb,
@@ -487,16 +500,16 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
 
     if (warp == NTC / 32) {
         // ======================= issuing warp (one thread)
-        if ((tid & 31) == 0 && T > 0) {
+        if ((tid & 31) == 0 && L > 0) {
             tc::tma_prefetch_desc(&maps.q);
             tc::tma_prefetch_desc(&maps.k);
             tc::tma_prefetch_desc(&maps.v);
             tc::tma_prefetch_desc(&maps.o);
             uint32_t ph = 0;               // phase of the per-chunk barriers
             uint32_t n_kqw = 0, n_ab = 0, n_v = 0;
-            issue_kqw(maps, sbase, 0, hi, bi, vw, bar(B_KQW)); ++n_kqw;
-            if (has_ab) { issue_ab(maps, sbase, 0, hi, bi, va, vb, bar(B_AB)); ++n_ab; }
-            issue_v(maps, sbase, 0, hi, bi, bar(B_V)); ++n_v;
+            issue_kqw(maps, sbase, tb, hi, bi, vw, bar(B_KQW)); ++n_kqw;
+            if (has_ab) { issue_ab(maps, sbase, tb, hi, bi, va, vb, bar(B_AB)); ++n_ab; }
+            issue_v(maps, sbase, tb, hi, bi, bar(B_V)); ++n_v;
             auto wait_ready = [&](uint32_t id) {
                 if (!tc::mbar_wait_bounded(bar(id), ph, WAIT_NS)) { *abort_s = 1; return false; }
                 tc::fence_after_sync();
@@ -508,15 +521,15 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             // o of the chunk before t0 leaves by TMA once its staging tile is written
             auto store_o = [&](int t0o, uint32_t parity) {
                 if (!tc::mbar_wait_bounded(bar(R_O), parity, WAIT_NS)) { *abort_s = 1; return false; }
-                tc::tma_store_4d(&maps.o, sbase + OFF_OST, 0, hi, t0o, bi);
-                tc::tma_store_4d(&maps.o, sbase + OFF_OST + 8192, 64, hi, t0o, bi);
+                tc::tma_store_4d(&maps.o, sbase + OFF_OST, 0, hi, tb + t0o, bi);
+                tc::tma_store_4d(&maps.o, sbase + OFF_OST + 8192, 64, hi, tb + t0o, bi);
                 tc::bulk_commit();
                 return true;
             };
             int t0 = 0;
 #pragma unroll 1
-            for (; t0 < T; t0 += C, ph ^= 1) {
-                const bool has_next = t0 + C < T;
+            for (; t0 < L; t0 += C, ph ^= 1) {
+                const bool has_next = t0 + C < L;
                 if (t0 > 0 && !store_o(t0 - C, ph ^ 1)) break;
                 // operands of the chunk are in place
                 if (!wait_ready(R_OP)) break;
@@ -551,10 +564,10 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                     // is slow enough to keep off the products' path): RAW and W were
                     // consumed by the operand pass, X1 and U are free once these
                     // products are done
-                    issue_kqw(maps, sbase, t0 + C, hi, bi, vw, bar(B_KQW)); ++n_kqw;
+                    issue_kqw(maps, sbase, tb + t0 + C, hi, bi, vw, bar(B_KQW)); ++n_kqw;
                     if (!tc::mbar_wait_bounded(bar(B_XAU), ph, WAIT_NS)) { *abort_s = 1; break; }
-                    if (has_ab) { issue_ab(maps, sbase, t0 + C, hi, bi, va, vb, bar(B_AB)); ++n_ab; }
-                    issue_v(maps, sbase, t0 + C, hi, bi, bar(B_V)); ++n_v;
+                    if (has_ab) { issue_ab(maps, sbase, tb + t0 + C, hi, bi, va, vb, bar(B_AB)); ++n_ab; }
+                    issue_v(maps, sbase, tb + t0 + C, hi, bi, bar(B_V)); ++n_v;
                 }
                 // X += [T - I; 0] R (rows 0-63 become E)
                 if (!wait_ready(R_P5)) break;
@@ -576,7 +589,9 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                                  idMM | IDESC_NEG_B, true);
                 tc::mma_commit(bar(B_ST));
             }
-            if (t0 >= T && *abort_s == 0) store_o(t0 - C, ph ^ 1);  // the last chunk's o
+            // the last chunk's o (packed sequences: written directly, the TMA box
+            // would reach into the next sequence)
+            if (t0 >= L && *abort_s == 0 && !cu_seqlens) store_o(t0 - C, ph ^ 1);
             // nothing of this CTA may still be in flight when it exits
             tc::mma_commit(bar(B_FIN));
             tc::mbar_wait_bounded(bar(B_FIN), 0, WAIT_NS);
@@ -590,8 +605,8 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
         // scalar gates of chunk starting at t0n into buffer `buf` (1.0 past T)
         auto load_scalars = [&](int t0n, int buf) {
             if (tid < C) {
-                const int nn = min(C, T - t0n);
-                const long long tok = ((long long)bi * T + t0n + tid) * H + hi;
+                const int nn = min(C, L - t0n);
+                const long long tok = ((long long)bi * T + tb + t0n + tid) * H + hi;
                 const bool in = tid < nn;
                 float* sc = sca_all + buf * 192;
                 sc[tid] = (a_kind == GDR_GATE_SCALAR && in) ? to_f32(a[tok]) : 1.f;
@@ -599,7 +614,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                 sc[128 + tid] = (w_kind == GDR_GATE_SCALAR && in) ? to_f32(w[tok]) : 1.f;
             }
         };
-        if (T > 0) load_scalars(0, 0);
+        if (L > 0) load_scalars(0, 0);
 
         // ---- initial state S0 (unscaled) into tensor memory: lane i, columns j
         {
@@ -647,8 +662,8 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
         };
 
 #pragma unroll 1
-        for (int t0 = 0; t0 < T; t0 += C, ph ^= 1) {
-            const bool has_next = t0 + C < T;
+        for (int t0 = 0; t0 < L; t0 += C, ph ^= 1) {
+            const bool has_next = t0 + C < L;
             const int cur = (t0 / C) & 1;
             const float* sca = sca_all + cur * 192;
 
@@ -662,7 +677,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             compute_sync();
             if (*abort_s) break;
             // ================= P1c:
-            operand_pass(sm, tid, va, vb, vw, fb, fw, a_kind, min(C, T - t0), sca, QT, fcur, fprev,
+            operand_pass(sm, tid, va, vb, vw, fb, fw, a_kind, min(C, L - t0), sca, QT, fcur, fprev,
                          err_word, [&] {
                              if (t0 == 0) return;
                              // the last chunk's state update has read X2 and EB and
@@ -787,10 +802,31 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             signal(R_E);
             if (*abort_s) break;
         }
-        if (T > 0 && *abort_s == 0) {
+        if (L > 0 && *abort_s == 0) {
             // the last chunk's O
             wait_then_sync(bar(B_ST), ph ^ 1, tid, abort_s);
-            read_o();
+            if (!cu_seqlens) {
+                read_o();
+            } else if (quarter >= 2) {
+                // straight to global memory, only the sequence's own rows
+                const int t0l = ((L - 1) / C) * C, r = lane_t - 64;
+                float vals[32];
+                tc::tmem_ld32(tmem + lane_off + TM_X + 32 * cb, vals);
+                tc::tmem_wait_ld();
+                if (r < L - t0l) {
+                    uint4* dst = reinterpret_cast<uint4*>(
+                        o_raw + (((long long)bi * T + tb + t0l + r) * H + hi) * D + 32 * cb);
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        uint4 u;
+                        u.x = tc::pack_bf16x2(vals[8 * x], vals[8 * x + 1]);
+                        u.y = tc::pack_bf16x2(vals[8 * x + 2], vals[8 * x + 3]);
+                        u.z = tc::pack_bf16x2(vals[8 * x + 4], vals[8 * x + 5]);
+                        u.w = tc::pack_bf16x2(vals[8 * x + 6], vals[8 * x + 7]);
+                        dst[x] = u;
+                    }
+                }
+            }
         }
     }
 
@@ -860,7 +896,7 @@ bool chunked_tc_supports(const gdr_desc& d) {
 cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, const void* v,
                               const void* a, const void* b, const void* w, const float* s0,
                               void* o, float* s_final, int* err_word, bool skip_signal,
-                              cudaStream_t st) {
+                              const int* cu_seqlens, int n_seqs, cudaStream_t st) {
     TcMaps maps;
     memset(&maps, 0, sizeof(maps));
     if (d.T > 0) {
@@ -877,10 +913,11 @@ cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, c
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    chunked_tc_kernel<<<(unsigned)(d.B * d.H), NT, SMEM_BYTES, st>>>(
+    const long long nseq = cu_seqlens ? n_seqs : d.B;
+    chunked_tc_kernel<<<(unsigned)(nseq * d.H), NT, SMEM_BYTES, st>>>(
         maps, d.B, d.T, d.H, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b,
         (const __nv_bfloat16*)w, (int)d.decay, (int)d.erase, (int)d.write, s0, s_final,
-        err_word, skip_signal ? 1 : 0);
+        err_word, skip_signal ? 1 : 0, cu_seqlens, (__nv_bfloat16*)o);
     return cudaGetLastError();
 }
 

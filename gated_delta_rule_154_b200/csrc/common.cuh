@@ -33,6 +33,26 @@ __device__ __forceinline__ float gate_value(const T* g, int kind, long long sidx
     return to_f32(g[vbase + c]);
 }
 
+// Token range of one CTA's sequence: tokens [tb, tb + len) of batch row bi.
+// Without cu_seqlens, sequence `seq` is batch row `seq` (all T tokens);
+// with it (packed sequences in one batch row), sequence `seq` spans
+// [cu[seq], cu[seq + 1]).  Returns false for a range outside [0, T], which
+// the caller reports and skips.
+__device__ __forceinline__ bool seq_range(const int* cu, int seq, int T, int& bi, int& tb,
+                                          int& len) {
+    if (!cu) {
+        bi = seq;
+        tb = 0;
+        len = T;
+        return true;
+    }
+    bi = 0;
+    tb = cu[seq];
+    const int te = cu[seq + 1];
+    len = te - tb;
+    return tb >= 0 && te >= tb && te <= T;
+}
+
 // Natural log of a decay value with a floor at log(FLT_MIN) so that a = 0
 // (or a denormal) behaves as a full reset instead of producing -inf.
 __device__ __forceinline__ float safe_log_decay(float a) {

@@ -12,12 +12,14 @@ cudaError_t launch_decode(const gdr_desc& d, const void* q, const void* k, const
                           cudaStream_t stream);
 cudaError_t launch_chunked_simt(const gdr_desc& d, const void* q, const void* k,
                                 const void* v, const void* a, const void* b, const void* w,
-                                const float* s0, void* o, float* s_final, cudaStream_t st);
+                                const float* s0, void* o, float* s_final,
+                                const int* cu_seqlens, int n_seqs, int* err_word,
+                                cudaStream_t st);
 bool chunked_tc_supports(const gdr_desc& d);
 cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, const void* v,
                               const void* a, const void* b, const void* w, const float* s0,
                               void* o, float* s_final, int* err_word, bool skip_signal,
-                              cudaStream_t st);
+                              const int* cu_seqlens, int n_seqs, cudaStream_t st);
 }  // namespace gdr
 
 // One error word per device (each device holds its own copy of the symbol).
@@ -114,10 +116,11 @@ size_t gdr_workspace_size(const gdr_desc* d) {
     return 0;  // every kernel keeps its intermediates on chip
 }
 
-gdr_status gdr_forward_chunked(const gdr_desc* d, const void* q, const void* k, const void* v,
-                               const void* a, const void* b, const void* w, const float* s0,
-                               void* o, float* s_final, void* workspace, size_t ws_bytes,
-                               gdr_stream_t stream) {
+namespace {
+gdr_status forward_impl(const gdr_desc* d, const int* cu_seqlens, int n_seqs, const void* q,
+                        const void* k, const void* v, const void* a, const void* b,
+                        const void* w, const float* s0, void* o, float* s_final,
+                        void* workspace, size_t ws_bytes, gdr_stream_t stream) {
     gdr_status s = check_desc(d);
     if (s != GDR_OK) return s;
     const bool have_tokens = d->T > 0;
@@ -131,18 +134,46 @@ gdr_status gdr_forward_chunked(const gdr_desc* d, const void* q, const void* k, 
     if (d->T == 0 && s_final == nullptr) return GDR_OK;  // nothing to compute or write
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int* err = nullptr;
+    if (error_word(&err) != cudaSuccess) return GDR_ERR_CUDA;
     cudaError_t e;
     if (gdr::chunked_tc_supports(*d)) {
-        int* err = nullptr;
-        if ((e = error_word(&err)) != cudaSuccess) return GDR_ERR_CUDA;
         const bool skip = g_test_skip_signal.exchange(0) != 0;
-        e = gdr::launch_chunked_tc(*d, q, k, v, a, b, w, s0, o, s_final, err, skip, st);
+        e = gdr::launch_chunked_tc(*d, q, k, v, a, b, w, s0, o, s_final, err, skip, cu_seqlens,
+                                   n_seqs, st);
     } else if (simt_supports(*d)) {
-        e = gdr::launch_chunked_simt(*d, q, k, v, a, b, w, s0, o, s_final, st);
+        e = gdr::launch_chunked_simt(*d, q, k, v, a, b, w, s0, o, s_final, cu_seqlens, n_seqs,
+                                     err, st);
     } else {
         return GDR_ERR_UNSUPPORTED;
     }
     return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+}  // namespace
+
+gdr_status gdr_forward_chunked(const gdr_desc* d, const void* q, const void* k, const void* v,
+                               const void* a, const void* b, const void* w, const float* s0,
+                               void* o, float* s_final, void* workspace, size_t ws_bytes,
+                               gdr_stream_t stream) {
+    return forward_impl(d, nullptr, 0, q, k, v, a, b, w, s0, o, s_final, workspace, ws_bytes,
+                        stream);
+}
+
+gdr_status gdr_forward_varlen(const gdr_desc* d, const int* cu_seqlens, int n_seqs,
+                              const void* q, const void* k, const void* v, const void* a,
+                              const void* b, const void* w, const float* s0, void* o,
+                              float* s_final, void* workspace, size_t ws_bytes,
+                              gdr_stream_t stream) {
+    if (!d || d->B != 1 || n_seqs < 1) return GDR_ERR_INVALID_ARG;
+    if (cu_seqlens == nullptr || reinterpret_cast<uintptr_t>(cu_seqlens) % 4 != 0)
+        return GDR_ERR_INVALID_ARG;
+    if ((long long)n_seqs * d->H > 0x7fffffffLL) return GDR_ERR_INVALID_ARG;
+    if (d->T == 0 && s_final == nullptr) {
+        gdr_status s = check_desc(d);
+        return s;
+    }
+    return forward_impl(d, cu_seqlens, n_seqs, q, k, v, a, b, w, s0, o, s_final, workspace,
+                        ws_bytes, stream);
 }
 
 gdr_status gdr_decode_step(const gdr_desc* d, const void* q, const void* k, const void* v,

@@ -136,6 +136,25 @@ gdr_status gdr_forward_chunked(const gdr_desc *desc, const void *q, const void *
                                gdr_stream_t stream);
 
 /*
+ * The same prefill over packed sequences of different lengths (varlen):
+ * desc->B must be 1 and desc->T is the total token count; q, k, v, the gates
+ * and o are [1, T, H, *] with sequence n occupying tokens
+ * [cu_seqlens[n], cu_seqlens[n + 1]).  cu_seqlens: int32 [n_seqs + 1] in
+ * device memory, 4-byte aligned, non-decreasing, cu_seqlens[0] = 0 and
+ * cu_seqlens[n_seqs] <= T; every sequence starts from its own state and no
+ * token of one sequence affects another.  s0 and s_final are
+ * [n_seqs, H, dk, dv] float32 (s0 may be NULL for zeros).  A sequence whose
+ * range falls outside [0, T] is skipped (its o and s_final are not written)
+ * and recorded in the device error word, read as GDR_ERR_INVALID_ARG by
+ * gdr_last_device_error().  Everything else as gdr_forward_chunked.
+ */
+gdr_status gdr_forward_varlen(const gdr_desc *desc, const int *cu_seqlens, int n_seqs,
+                              const void *q, const void *k, const void *v, const void *a,
+                              const void *b, const void *w, const float *s0, void *o,
+                              float *s_final, void *workspace, size_t ws_bytes,
+                              gdr_stream_t stream);
+
+/*
  * One decode step (desc->T must be 1): reads and rewrites `state` in place.
  * Shapes drop the T axis: q, k, a, b [B, H, dk] (scalar gates [B, H]);
  * v, w [B, H, dv]; state [B, H, dk, dv] float32; o [B, H, dv] in_dtype.
@@ -163,7 +182,8 @@ gdr_status gdr_decode_step_paged(const gdr_desc *desc, const void *q, const void
 
 /* Synchronises `stream`, returns the status recorded on the device since the
  * previous call (GDR_OK if none) and clears it: GDR_ERR_TIMEOUT (a bounded
- * wait ran out), GDR_ERR_INVALID_ARG (a paged decode slot out of range) or
+ * wait ran out), GDR_ERR_INVALID_ARG (a paged decode slot or a packed
+ * sequence range out of bounds) or
  * GDR_ERR_RANGE (decay range), in that order of precedence.  GDR_ERR_CUDA if
  * the synchronisation itself failed. */
 gdr_status gdr_last_device_error(gdr_stream_t stream);

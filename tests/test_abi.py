@@ -137,3 +137,17 @@ def test_paged_decode_argument_checks(lib):
     assert call(n=0) == _lib.ERR_INVALID_ARG
     d.T = 2
     assert call() == _lib.ERR_INVALID_ARG
+
+
+def test_varlen_argument_checks(lib):
+    cu = P
+    d = _desc(B=1)
+    assert _lib.forward_varlen(d, 0, 2, P, P, P, P, P, P, 0, P, 0, 0, 0, 0) == _lib.ERR_INVALID_ARG
+    assert _lib.forward_varlen(d, P + 2, 2, P, P, P, P, P, P, 0, P, 0, 0, 0, 0) == _lib.ERR_INVALID_ARG
+    assert _lib.forward_varlen(d, cu, 0, P, P, P, P, P, P, 0, P, 0, 0, 0, 0) == _lib.ERR_INVALID_ARG
+    assert _lib.forward_varlen(_desc(B=2), cu, 2, P, P, P, P, P, P, 0, P, 0, 0, 0,
+                               0) == _lib.ERR_INVALID_ARG
+    assert _lib.forward_varlen(d, cu, 2, 0, P, P, P, P, P, 0, P, 0, 0, 0, 0) == _lib.ERR_INVALID_ARG
+    # nothing to do: no tokens and no final state
+    d0 = _desc(B=1, T=0)
+    assert _lib.forward_varlen(d0, cu, 2, P, P, P, P, P, P, 0, P, 0, 0, 0, 0) == _lib.OK
