@@ -22,6 +22,15 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// Square root to about 1 ulp in one SFU op (non-negative input; ftz).  The
+// IEEE-rounded sqrtf brings a slow-path routine into the kernel that
+// measurably slowed the decode step even where it never runs.
+__device__ __forceinline__ float sqrt_fast(float x) {
+    float y;
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Value of gate `g` of kind `kind` for channel c of the token/head whose
 // scalar index is `sidx` and whose vector row starts at `vbase`.
 template <typename T>
@@ -29,7 +38,7 @@ __device__ __forceinline__ float gate_value(const T* g, int kind, long long sidx
                                             long long vbase, int c) {
     if (kind == GDR_GATE_ONE) return 1.0f;
     if (kind == GDR_GATE_SCALAR) return to_f32(g[sidx]);
-    if (kind == GDR_GATE_FG2) return sqrtf(fmaxf(to_f32(g[vbase + c]), 0.0f));  // sqrt(beta)
+    if (kind == GDR_GATE_FG2) return sqrt_fast(fmaxf(to_f32(g[vbase + c]), 0.0f));  // sqrt(beta)
     return to_f32(g[vbase + c]);
 }
 

@@ -23,7 +23,20 @@
 
 namespace gdr {
 
-template <typename Tin, int DK, int DV>
+// Gate value without the FG2 form (the common instantiations keep exactly
+// the plain staging code).
+template <typename T>
+__device__ __forceinline__ float plain_gate(const T* g, int kind, long long sidx,
+                                            long long vbase, int c) {
+    if (kind == GDR_GATE_ONE) return 1.0f;
+    if (kind == GDR_GATE_SCALAR) return to_f32(g[sidx]);
+    return to_f32(g[vbase + c]);
+}
+
+// PAGED: states come from a pool through slot[]; FG2: erase and/or write
+// given as FG^2-GDN learning rates.  Both are compile-time so the plain
+// step compiles to the plain code.
+template <typename Tin, int DK, int DV, bool PAGED, bool FG2>
 __global__ void __launch_bounds__(256, 2)
 decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                    const Tin* __restrict__ v, const Tin* __restrict__ a,
@@ -47,7 +60,7 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     const int rs = tid / TPR;         // row set: rows rs, rs + RS, ...
 
     long long sidx = bh;  // state of this (batch, head)
-    if (slot) {
+    if (PAGED) {
         const long long bi = bh / H;
         const int sl = slot[bi];
         if (sl < 0 || sl >= n_slots) {  // whole CTA agrees: skip, flag once
@@ -68,19 +81,23 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     for (int i = tid; i < DK; i += NT) {
         const long long vb = bh * DK;
         float kv = to_f32(k[vb + i]);
-        float bv = gate_value(b, b_kind, bh, vb, i);
-        if (b_kind == GDR_GATE_FG2) {  // key sqrt(beta^k) k, erase gate 1
-            kv *= bv;
+        float bv;
+        if (FG2 && b_kind == GDR_GATE_FG2) {  // key sqrt(beta^k) k, erase gate 1
+            kv *= sqrt_fast(fmaxf(to_f32(b[vb + i]), 0.f));
             bv = 1.f;
+        } else {
+            bv = plain_gate(b, b_kind, bh, vb, i);
         }
         qs[i] = to_f32(q[vb + i]);
         ks[i] = kv;
-        as_[i] = gate_value(a, a_kind, bh, vb, i);
+        as_[i] = plain_gate(a, a_kind, bh, vb, i);
         bks[i] = bv * kv;
     }
     for (int j = tid; j < DV; j += NT) {
         const long long vb = bh * DV;
-        us[j] = gate_value(w, w_kind, bh, vb, j) * to_f32(v[vb + j]);
+        const float wv = (FG2 && w_kind == GDR_GATE_FG2) ? sqrt_fast(fmaxf(to_f32(w[vb + j]), 0.f))
+                                                          : plain_gate(w, w_kind, bh, vb, j);
+        us[j] = wv * to_f32(v[vb + j]);
     }
     __syncthreads();
 
@@ -148,14 +165,24 @@ struct DecodeArgs {
     int* err_word;
 };
 
-template <typename Tin, int DK, int DV>
-static cudaError_t launch_decode_t(const gdr_desc& d, const DecodeArgs& x, cudaStream_t stream) {
+template <typename Tin, int DK, int DV, bool PAGED, bool FG2>
+static cudaError_t launch_decode_k(const gdr_desc& d, const DecodeArgs& x, cudaStream_t stream) {
     const unsigned grid = (unsigned)((long long)d.B * d.H);
-    decode_step_kernel<Tin, DK, DV><<<grid, 256, 0, stream>>>(
+    decode_step_kernel<Tin, DK, DV, PAGED, FG2><<<grid, 256, 0, stream>>>(
         (const Tin*)x.q, (const Tin*)x.k, (const Tin*)x.v, (const Tin*)x.a, (const Tin*)x.b,
         (const Tin*)x.w, (int)d.decay, (int)d.erase, (int)d.write, x.state, (Tin*)x.o, d.H,
         x.slot, x.n_slots, x.err_word);
     return cudaGetLastError();
+}
+
+template <typename Tin, int DK, int DV>
+static cudaError_t launch_decode_t(const gdr_desc& d, const DecodeArgs& x, cudaStream_t stream) {
+    const bool fg2 = d.erase == GDR_GATE_FG2 || d.write == GDR_GATE_FG2;
+    if (x.slot)
+        return fg2 ? launch_decode_k<Tin, DK, DV, true, true>(d, x, stream)
+                   : launch_decode_k<Tin, DK, DV, true, false>(d, x, stream);
+    return fg2 ? launch_decode_k<Tin, DK, DV, false, true>(d, x, stream)
+               : launch_decode_k<Tin, DK, DV, false, false>(d, x, stream);
 }
 
 template <typename Tin>
