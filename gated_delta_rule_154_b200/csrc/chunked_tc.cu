@@ -324,7 +324,7 @@ __device__ __forceinline__ void issue_v(const TcMaps& m, uint32_t sbase, int t0,
 // fprev = gamma_63/g_m, and check that the largest factors, gamma_0/g_m and
 // g_m/gamma_63, stay in float range.  `mid` runs between the two halves (after
 // the exchange barrier), before anything is written to X2.
-template <typename Mid>
+template <bool PACKED, bool FG2, typename Mid>
 __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool vb, bool vw,
                                              bool fb, bool fw, int a_kind, int n,
                                              const float* sca, float* QT,
@@ -382,22 +382,22 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
         uint32_t v2 = *reinterpret_cast<const uint32_t*>(sm + OFF_U + o64);
         const uint32_t w2 = vw ? *reinterpret_cast<const uint32_t*>(sm + OFF_W + o64)
                                : tc::pack_bf16x2(sca[128 + r], sca[128 + r]);
-        if (r >= n) {  // past the sequence (a packed neighbour's tokens): k = q = v = 0
+        if (PACKED && r >= n) {  // past the sequence (a packed neighbour's tokens): k = q = v = 0
             k2 = 0u;
             q2 = 0u;
             v2 = 0u;
         }
         // FG^2-GDN learning rates: key sqrt(beta^k) k with erase gate 1, write
         // gate sqrt(beta^v)
-        const uint32_t kt2 = fb ? mul2(k2, sqrt2(b2)) : k2;
+        const uint32_t kt2 = (FG2 && fb) ? mul2(k2, sqrt2(b2)) : k2;
         const uint32_t kk2 = mul2(kt2, ei);                                      // K"
         *reinterpret_cast<uint32_t*>(sm + OFF_X1 + o128) = mul2(kt2, e);         // K'
         *reinterpret_cast<uint32_t*>(sm + OFF_X1 + o128 + 8192u) = mul2(q2, e);  // Q'
         *reinterpret_cast<uint32_t*>(sm + OFF_X2 + o128) = kk2;
         *reinterpret_cast<uint32_t*>(sm + OFF_X2 + o128 + 8192u) =
-            fb ? kk2 : mul2(b2, kk2);                                            // B"
+            (FG2 && fb) ? kk2 : mul2(b2, kk2);                                 // B"
         *reinterpret_cast<uint32_t*>(sm + OFF_U + o64) =
-            mul2(fw ? sqrt2(w2) : w2, v2);                                       // U
+            mul2((FG2 && fw) ? sqrt2(w2) : w2, v2);                            // U
     }
     if (q8 == 0) {
         const int i = 2 * p2;
@@ -432,6 +432,11 @@ enum : uint32_t {
 };
 static_assert(R_O + 1 == NBAR, "barrier count");
 
+// PACKED: packed sequences (rows past a sequence's end are zeroed rather than
+// left to the TMA fill).  FG2: FG^2-GDN learning rates among the gates.  Both
+// compile-time, so the plain instantiation carries neither test in its
+// operand pass.
+template <bool PACKED, bool FG2>
 __global__ void __launch_bounds__(NT, 1)
 chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                   const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
@@ -677,7 +682,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             compute_sync();
             if (*abort_s) break;
             // ================= P1c:
-            operand_pass(sm, tid, va, vb, vw, fb, fw, a_kind, min(C, L - t0), sca, QT, fcur, fprev,
+            operand_pass<PACKED, FG2>(sm, tid, va, vb, vw, fb, fw, a_kind, min(C, L - t0), sca, QT, fcur, fprev,
                          err_word, [&] {
                              if (t0 == 0) return;
                              // the last chunk's state update has read X2 and EB and
@@ -909,12 +914,15 @@ cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, c
             ok = make_map(&maps.w, w, d.B, d.T, d.H);
         if (!ok) return cudaErrorInvalidValue;
     }
-    cudaError_t e = cudaFuncSetAttribute(chunked_tc_kernel,
+    const bool fg2 = d.erase == GDR_GATE_FG2 || d.write == GDR_GATE_FG2;
+    auto kern = cu_seqlens ? (fg2 ? chunked_tc_kernel<true, true> : chunked_tc_kernel<true, false>)
+                           : (fg2 ? chunked_tc_kernel<false, true> : chunked_tc_kernel<false, false>);
+    cudaError_t e = cudaFuncSetAttribute(kern,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const long long nseq = cu_seqlens ? n_seqs : d.B;
-    chunked_tc_kernel<<<(unsigned)(nseq * d.H), NT, SMEM_BYTES, st>>>(
+    kern<<<(unsigned)(nseq * d.H), NT, SMEM_BYTES, st>>>(
         maps, d.B, d.T, d.H, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b,
         (const __nv_bfloat16*)w, (int)d.decay, (int)d.erase, (int)d.write, s0, s_final,
         err_word, skip_signal ? 1 : 0, cu_seqlens, (__nv_bfloat16*)o);
