@@ -65,6 +65,11 @@ class Oracle:
         lib.oracle_decode_step.argtypes = [i, i, i, i, i, i, i,
                                            f32p, f32p, f32p, f32p, f32p, f32p,
                                            f64p, f64p, i]
+        lib.oracle_backward.restype = i
+        lib.oracle_backward.argtypes = [i, i, i, i, i, i, i, i,
+                                        f32p, f32p, f32p, f32p, f32p, f32p,
+                                        f64p, f64p, f64p,
+                                        f64p, f64p, f64p, f64p, f64p, f64p, f64p, i]
         lib.oracle_max_threads.restype = i
         lib.oracle_max_threads.argtypes = []
         self.lib = lib
@@ -79,6 +84,9 @@ class Oracle:
 
     def decode_step(self, q, k, v, a, b, w, state, *, nthreads: int = 0):
         return _decode_step(self.lib, q, k, v, a, b, w, state, nthreads)
+
+    def backward(self, q, k, v, a, b, w, s0, do, dsT=None, *, nthreads: int = 0):
+        return _backward(self.lib, q, k, v, a, b, w, s0, do, dsT, nthreads)
 
 
 def default() -> Oracle:
@@ -145,6 +153,40 @@ def _forward(lib, q, k, v, a, b, w, s0, want_o, nthreads):
     return o, sT
 
 
+def _backward(lib, q, k, v, a, b, w, s0, do, dsT, nthreads):
+    q = np.asarray(q)
+    B, T, H, dk = q.shape
+    dv = np.asarray(v).shape[-1]
+    ak = _kind(a, (B, T, H, dk), (B, T, H))
+    bk = _kind(b, (B, T, H, dk), (B, T, H))
+    wk = _kind(w, (B, T, H, dv), (B, T, H))
+    keep = []
+    ptrs = []
+    for x in (q, k, v, a, b, w):
+        arr, p = _f32(x)
+        keep.append(arr)
+        ptrs.append(p)
+    for x in (s0, do, dsT):
+        arr, p = _f64(x)
+        keep.append(arr)
+        ptrs.append(p)
+    f64 = lambda shape: np.zeros(shape, np.float64)
+    gate_shape = lambda kind, d: None if kind == GATE_ONE else (
+        (B, T, H) if kind == GATE_SCALAR else (B, T, H, d))
+    out = {"dq": f64((B, T, H, dk)), "dk": f64((B, T, H, dk)), "dv": f64((B, T, H, dv)),
+           "da": None, "db": None, "dw": None, "ds0": f64((B, H, dk, dv))}
+    for name, kind, d in (("da", ak, dk), ("db", bk, dk), ("dw", wk, dv)):
+        shp = gate_shape(kind, d)
+        out[name] = f64(shp) if shp is not None else None
+    optr = [None if out[n] is None else out[n].ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+            for n in ("dq", "dk", "dv", "da", "db", "dw", "ds0")]
+    rc = lib.oracle_backward(B, T, H, dk, dv, ak, bk, wk, *ptrs, *optr, int(nthreads))
+    if rc != 0:
+        raise RuntimeError("oracle_backward failed (%d)" % rc)
+    del keep
+    return out
+
+
 def _decode_step(lib, q, k, v, a, b, w, state, nthreads):
     q = np.asarray(q)
     B, H, dk = q.shape
@@ -191,3 +233,16 @@ def decode_step(q, k, v, a, b, w, state, *, nthreads: int = 0):
     w: [B, H, dv] or [B, H] or None; state: [B, H, dk, dv] (not modified).
     """
     return default().decode_step(q, k, v, a, b, w, state, nthreads=nthreads)
+
+
+def backward(q, k, v, a=None, b=None, w=None, s0=None, do=None, dsT=None, *,
+             nthreads: int = 0):
+    """Gradients of  L = sum_t <o_t, do_t> + <S_T, dsT>  with respect to every
+    input of :func:`forward` (reverse-mode differentiation of the recurrence,
+    step by step; see ``oracle_backward`` in gdr_oracle.c).
+
+    do: [B, T, H, dv]; dsT: [B, H, dk, dv] or None (zero).  Returns a dict of
+    float64 arrays: dq, dk [B, T, H, dk]; dv [B, T, H, dv]; da, db, dw in the
+    shape of a, b, w (None where the gate is None); ds0 [B, H, dk, dv].
+    """
+    return default().backward(q, k, v, a, b, w, s0, do, dsT, nthreads=nthreads)
