@@ -21,7 +21,8 @@ GATE_ONE, GATE_SCALAR, GATE_VECTOR, GATE_FG2 = 0, 1, 2, 3
 
 EXPORTS = ("gdr_workspace_size", "gdr_forward_chunked", "gdr_decode_step",
            "gdr_last_device_error", "gdr_status_string", "gdr_version", "gdr_test_skip_signal",
-           "gdr_decode_step_paged", "gdr_forward_varlen")
+           "gdr_decode_step_paged", "gdr_forward_varlen", "gdr_backward_workspace_size",
+           "gdr_backward_chunked")
 
 
 class GdrDesc(ctypes.Structure):
@@ -67,6 +68,10 @@ def load(path: str = LIB_PATH):
     lib.gdr_forward_varlen.argtypes = [dp, vp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.gdr_decode_step_paged.restype = i
     lib.gdr_decode_step_paged.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp]
+    lib.gdr_backward_workspace_size.restype = sz
+    lib.gdr_backward_workspace_size.argtypes = [dp]
+    lib.gdr_backward_chunked.restype = i
+    lib.gdr_backward_chunked.argtypes = [dp] + [vp] * 17 + [sz, vp]
     lib.gdr_test_skip_signal.restype = None
     lib.gdr_test_skip_signal.argtypes = [i]
     _lib = lib
@@ -104,6 +109,18 @@ def decode_step_paged(desc: GdrDesc, q, k, v, a, b, w, pool, slot, n_slots, o, s
     """Raw call: every pointer an int (0 = NULL).  Returns the gdr_status."""
     return int(load().gdr_decode_step_paged(ctypes.byref(desc), q, k, v, a, b, w, pool, slot,
                                             int(n_slots), o, stream))
+
+
+def backward_workspace_size(desc: GdrDesc) -> int:
+    return int(load().gdr_backward_workspace_size(ctypes.byref(desc)))
+
+
+def backward_chunked(desc: GdrDesc, q, k, v, a, b, w, s0, d_o, ds_final, dq, dk, dv, da, db,
+                     dw, ds0, workspace, ws_bytes, stream) -> int:
+    """Raw call: every pointer an int (0 = NULL).  Returns the gdr_status."""
+    return int(load().gdr_backward_chunked(ctypes.byref(desc), q, k, v, a, b, w, s0, d_o,
+                                           ds_final, dq, dk, dv, da, db, dw, ds0, workspace,
+                                           ws_bytes, stream))
 
 
 def last_device_error(stream) -> int:

@@ -126,6 +126,52 @@ def forward_chunked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return out, s_final
 
 
+def backward_workspace_size(desc: _lib.GdrDesc) -> int:
+    return _lib.backward_workspace_size(desc)
+
+
+def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+             a: Optional[torch.Tensor], b: Optional[torch.Tensor], w: Optional[torch.Tensor],
+             s0: Optional[torch.Tensor], d_o: torch.Tensor,
+             ds_final: Optional[torch.Tensor] = None, *, want_ds0: bool = True,
+             workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Gradients of  L = sum_t <o_t, d_o_t> + <S_T, ds_final>  for the prefill
+    of (q, k, v, a, b, w, s0).  Returns a dict with dq, dk, dv (input dtype),
+    da, db, dw (shape and dtype of a, b, w; None for an absent gate) and ds0
+    (float32 [B, H, dk, dv], or None with want_ds0=False).  With b and w the
+    same tensor (shared beta) its gradient is db + dw."""
+    if q.dtype not in _DT:
+        raise ValueError("q must be float32 or bfloat16")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    _check(q, "q", dt, dev, [(B, T, H, dk)])
+    _check(k, "k", dt, dev, [(B, T, H, dk)])
+    _check(v, "v", dt, dev, [(B, T, H, dv)])
+    _check(a, "a", dt, dev, [(B, T, H, dk), (B, T, H)])
+    _check(b, "b", dt, dev, [(B, T, H, dk), (B, T, H)])
+    _check(w, "w", dt, dev, [(B, T, H, dv), (B, T, H)])
+    _check(s0, "s0", torch.float32, dev, [(B, H, dk, dv)])
+    _check(d_o, "d_o", dt, dev, [(B, T, H, dv)])
+    _check(ds_final, "ds_final", torch.float32, dev, [(B, H, dk, dv)])
+    like = lambda t: None if t is None else torch.empty_like(t)
+    g = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+         "da": like(a), "db": like(b), "dw": like(w),
+         "ds0": torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if want_ds0 else None}
+    desc = desc_for(q, v, a, b, w, 32)
+    need = _lib.backward_workspace_size(desc)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _lib.backward_chunked(desc, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(w),
+                               _ptr(s0), _ptr(d_o), _ptr(ds_final), _ptr(g["dq"]), _ptr(g["dk"]),
+                               _ptr(g["dv"]), _ptr(g["da"]), _ptr(g["db"]), _ptr(g["dw"]),
+                               _ptr(g["ds0"]), _ptr(workspace), ws_bytes, _stream_handle(stream))
+    if st != _lib.OK:
+        raise _lib.GdrError(st, "gdr_backward_chunked")
+    return g
+
+
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                 a: Optional[torch.Tensor], b: Optional[torch.Tensor],
                 w: Optional[torch.Tensor], state: torch.Tensor, *,

@@ -13,9 +13,13 @@ cudaError_t launch_decode(const gdr_desc& d, const void* q, const void* k, const
 cudaError_t launch_chunked_simt(const gdr_desc& d, const void* q, const void* k,
                                 const void* v, const void* a, const void* b, const void* w,
                                 const float* s0, void* o, float* s_final,
-                                const int* cu_seqlens, int n_seqs, int* err_word,
-                                cudaStream_t st);
+                                const int* cu_seqlens, int n_seqs, float* h_out,
+                                int* err_word, cudaStream_t st);
 bool chunked_tc_supports(const gdr_desc& d);
+size_t backward_workspace_bytes(const gdr_desc& d);
+cudaError_t launch_backward(const gdr_desc& d, const void* const* in, const float* s0,
+                            const void* dout, const float* ds_final, void* const* grads,
+                            float* ds0, void* workspace, int* err_word, cudaStream_t st);
 cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, const void* v,
                               const void* a, const void* b, const void* w, const float* s0,
                               void* o, float* s_final, int* err_word, bool skip_signal,
@@ -143,7 +147,7 @@ gdr_status forward_impl(const gdr_desc* d, const int* cu_seqlens, int n_seqs, co
                                    n_seqs, st);
     } else if (simt_supports(*d)) {
         e = gdr::launch_chunked_simt(*d, q, k, v, a, b, w, s0, o, s_final, cu_seqlens, n_seqs,
-                                     err, st);
+                                     nullptr, err, st);
     } else {
         return GDR_ERR_UNSUPPORTED;
     }
@@ -202,6 +206,39 @@ gdr_status gdr_decode_step_paged(const gdr_desc* d, const void* q, const void* k
     if (error_word(&err) != cudaSuccess) return GDR_ERR_CUDA;
     cudaError_t e = gdr::launch_decode(*d, q, k, v, a, b, w, state_pool, o, slot, n_slots, err,
                                        reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+size_t gdr_backward_workspace_size(const gdr_desc* d) {
+    if (check_desc(d) != GDR_OK) return 0;
+    return gdr::backward_workspace_bytes(*d);
+}
+
+gdr_status gdr_backward_chunked(const gdr_desc* d, const void* q, const void* k, const void* v,
+                                const void* a, const void* b, const void* w, const float* s0,
+                                const void* d_o, const float* ds_final, void* dq, void* dk,
+                                void* dv, void* da, void* db, void* dw, float* ds0,
+                                void* workspace, size_t ws_bytes, gdr_stream_t stream) {
+    gdr_status s = check_desc(d);
+    if (s != GDR_OK) return s;
+    if (d->erase == GDR_GATE_FG2 || d->write == GDR_GATE_FG2) return GDR_ERR_UNSUPPORTED;
+    const bool have_tokens = d->T > 0;
+    if ((s = check_inputs(d, have_tokens, q, k, v, a, b, w, d_o)) != GDR_OK) return s;
+    if ((s = check_inputs(d, have_tokens, dq, dk, dv, da, db, dw, d_o)) != GDR_OK) return s;
+    if ((s = check_ptr(s0, false)) != GDR_OK) return s;
+    if ((s = check_ptr(ds_final, false)) != GDR_OK) return s;
+    if ((s = check_ptr(ds0, false)) != GDR_OK) return s;
+    const size_t need = gdr::backward_workspace_bytes(*d);
+    if (workspace == nullptr || ws_bytes < need) return GDR_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GDR_ERR_INVALID_ARG;
+    if (ds0 == nullptr && !have_tokens) return GDR_OK;  // nothing to write
+
+    int* err = nullptr;
+    if (error_word(&err) != cudaSuccess) return GDR_ERR_CUDA;
+    const void* in[6] = {q, k, v, a, b, w};
+    void* grads[6] = {dq, dk, dv, da, db, dw};
+    cudaError_t e = gdr::launch_backward(*d, in, s0, d_o, ds_final, grads, ds0, workspace, err,
+                                         reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

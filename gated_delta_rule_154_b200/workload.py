@@ -250,3 +250,31 @@ def as_f32(x: Optional[np.ndarray], dtype: str) -> Optional[np.ndarray]:
     if x is None:
         return None
     return x if dtype == "f32" else bf16_bits_to_f32(x)
+
+
+def make_upstream(wl: Workload, seed: int = 0,
+                  heads: Optional[Sequence[Tuple[int, int]]] = None,
+                  threads: int = 8) -> Dict[str, np.ndarray]:
+    """Upstream gradients for the backward pass of a prefill workload: do
+    [B, T, H, dv] ~ N(0, 1) in the workload's dtype (bf16 bits or float32) and
+    dsT [B, H, dk, dv] ~ N(0, 0.1) float32, from streams of their own
+    (spawn key (b, h, 2^20)), so they are independent of the inputs.  With
+    ``heads`` only those (b, h) slices are drawn (the rest stay zero)."""
+    B, T, H, dk, dv = wl.B, wl.T, wl.H, wl.dk, wl.dv
+    st = np.float32 if wl.dtype == "f32" else np.uint16
+    out = {"do": np.zeros((B, T, H, dv), st), "dsT": np.zeros((B, H, dk, dv), np.float32)}
+    todo = list(heads) if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+
+    def one(bh):
+        b, h = bh
+        g = _stream(seed, b, h, 1 << 20)
+        out["do"][b, :, h] = _store(g.standard_normal((T, dv)), wl.dtype)
+        out["dsT"][b, h] = g.normal(0.0, 0.1, (dk, dv)).astype(np.float32)
+
+    if threads > 1 and len(todo) > 1:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(one, todo))
+    else:
+        for bh in todo:
+            one(bh)
+    return out

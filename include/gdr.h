@@ -180,6 +180,51 @@ gdr_status gdr_decode_step_paged(const gdr_desc *desc, const void *q, const void
                                  const void *w, float *state_pool, const int *slot,
                                  int n_slots, void *o, gdr_stream_t stream);
 
+/* Bytes of device workspace gdr_backward_chunked needs for `desc`: the state
+ * at the start of every 32-token chunk plus one running state gradient, i.e.
+ * B * H * dk * dv * 4 * (ceil(T / 32) + 1); 0 if desc is invalid.  Pure host
+ * function, no CUDA call. */
+size_t gdr_backward_workspace_size(const gdr_desc *desc);
+
+/*
+ * Gradients of the prefill (training).  With the loss
+ *     L = sum_t <o_t, do_t> + <S_T, ds_final>,
+ * where o and S_T are what gdr_forward_chunked returns for the same inputs,
+ * the call writes dL/dq, dL/dk, dL/dv, dL/da, dL/db, dL/dw and dL/ds0.  The
+ * pages train this recurrence through its chunkwise (WY) form (FG^2-GDN
+ * page, section 2 "Methodology"); the call differentiates that form: a
+ * forward pass stores the state at the start of every 32-token chunk in the
+ * workspace, then one CTA per (batch, head) walks the chunks backwards
+ * carrying dS.  Float32 arithmetic on the CUDA cores; equal, up to rounding,
+ * to differentiating the token-by-token recurrence.
+ *
+ *   q .. w, s0  the forward's inputs (s0 NULL for zeros); desc->chunk is not
+ *            used (the pass always takes chunks of 32 tokens)
+ *   d_o      [B, T, H, dv] in_dtype, the gradient on o
+ *   ds_final [B, H, dk, dv] float32, the gradient on S_T, or NULL for zero
+ *   dq, dk   [B, T, H, dk] in_dtype, written
+ *   dv       [B, T, H, dv] in_dtype, written
+ *   da, db, dw  in the shape and dtype of a, b, w (scalar gates: one value
+ *            per token and head, the sum over channels); required when the
+ *            gate is not ONE, ignored when it is.  With b and w the same
+ *            tensor (shared beta) its gradient is db + dw.
+ *   ds0      [B, H, dk, dv] float32, or NULL (not written); may equal
+ *            ds_final
+ *   workspace, ws_bytes  device scratch of gdr_backward_workspace_size(desc)
+ *
+ * Outputs must not overlap the inputs.  Supported: dk, dv in {64, 128},
+ * float32 or bf16 inputs, gates ONE / SCALAR / VECTOR; GDR_GATE_FG2 returns
+ * GDR_ERR_UNSUPPORTED.  Decay range: every channel's decay, multiplied over
+ * each 32-token chunk, must stay at or above exp(-80); otherwise the device
+ * error word reports GDR_ERR_RANGE and the gradients are undefined.
+ */
+gdr_status gdr_backward_chunked(const gdr_desc *desc, const void *q, const void *k,
+                                const void *v, const void *a, const void *b,
+                                const void *w, const float *s0, const void *d_o,
+                                const float *ds_final, void *dq, void *dk, void *dv,
+                                void *da, void *db, void *dw, float *ds0, void *workspace,
+                                size_t ws_bytes, gdr_stream_t stream);
+
 /* Synchronises `stream`, returns the status recorded on the device since the
  * previous call (GDR_OK if none) and clears it: GDR_ERR_TIMEOUT (a bounded
  * wait ran out), GDR_ERR_INVALID_ARG (a paged decode slot or a packed

@@ -151,3 +151,42 @@ def test_varlen_argument_checks(lib):
     # nothing to do: no tokens and no final state
     d0 = _desc(B=1, T=0)
     assert _lib.forward_varlen(d0, cu, 2, P, P, P, P, P, P, 0, P, 0, 0, 0, 0) == _lib.OK
+
+
+def _bwd(d, **kw):
+    """gdr_backward_chunked with every pointer a valid fake address unless given."""
+    names = ("q", "k", "v", "a", "b", "w", "s0", "d_o", "ds_final", "dq", "dk", "dv", "da",
+             "db", "dw", "ds0", "ws")
+    p = {n: P for n in names}
+    p["s0"] = p["ds_final"] = p["ds0"] = 0
+    p.update(kw)
+    ws_bytes = kw.pop("ws_bytes", None)
+    if ws_bytes is None:
+        ws_bytes = _lib.backward_workspace_size(d)
+    return _lib.backward_chunked(d, *(p[n] for n in names), ws_bytes, 0)
+
+
+def test_backward_workspace_size(lib):
+    d = _desc(B=2, T=100, H=4, dk=128, dv=64)
+    # chunk-start states on a 32-token grid plus one running state gradient
+    assert _lib.backward_workspace_size(d) == 2 * 4 * 128 * 64 * 4 * (4 + 1)
+    assert _lib.backward_workspace_size(_desc(T=0)) == 2 * 4 * 128 * 128 * 4
+    assert _lib.backward_workspace_size(_desc(dk=96)) == 0
+    assert lib.gdr_backward_workspace_size(None) == 0
+
+
+def test_backward_argument_checks(lib):
+    d = _desc()
+    assert _bwd(_desc(dk=96)) == _lib.ERR_INVALID_ARG
+    for name in ("q", "k", "v", "a", "b", "w", "d_o", "dq", "dk", "dv", "da", "db", "dw"):
+        assert _bwd(d, **{name: 0}) == _lib.ERR_INVALID_ARG, name
+        assert _bwd(d, **{name: P + 8}) == _lib.ERR_INVALID_ARG, name
+    for name in ("s0", "ds_final", "ds0"):
+        assert _bwd(d, **{name: P + 4}) == _lib.ERR_INVALID_ARG, name
+    assert _bwd(d, ws=0) == _lib.ERR_WORKSPACE
+    assert _bwd(d, ws_bytes=_lib.backward_workspace_size(d) - 1) == _lib.ERR_WORKSPACE
+    assert _bwd(d, ws=P + 8) == _lib.ERR_INVALID_ARG
+    assert _bwd(_desc(erase=_lib.GATE_FG2, write=_lib.GATE_FG2)) == _lib.ERR_UNSUPPORTED
+    # absent gates need neither the gate nor its gradient
+    one = _desc(T=0, decay=_lib.GATE_ONE, erase=_lib.GATE_ONE, write=_lib.GATE_ONE)
+    assert _bwd(one, a=0, b=0, w=0, da=0, db=0, dw=0) == _lib.OK  # nothing to write

@@ -1,0 +1,166 @@
+"""GPU parity of the backward pass (gdr_backward_chunked) against the float64
+oracle's reverse-mode gradients (oracle.backward, itself pinned by finite
+differences of the forward), through the C ABI.  Loss
+L = sum_t <o_t, do_t> + <S_T, dsT> with seeded upstream gradients
+(workload.make_upstream).  The pages train the recurrence in its chunked WY
+form (FG^2-GDN page, gist.science 2604.19021, section 2 "Methodology").
+
+Tolerances as for the forward (max |x - ref| / max |ref| per gradient
+tensor): 1e-4 for float32 inputs, 2e-2 for bf16 inputs (gradients are
+returned in the input dtype; dS0 in float32)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_154_b200 import api
+from gated_delta_rule_154_b200 import workload as W
+from gpu_helpers import TOL, inputs_to_dev, rel_err, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+GRADS = ("dq", "dk", "dv", "da", "db", "dw", "ds0")
+
+
+def _gpu(wl, inp, up, with_dsT=True, s0=True):
+    d = inputs_to_dev(inp, wl)
+    do = to_dev(up["do"], wl.dtype)
+    dsT = to_dev(up["dsT"], "f32") if with_dsT else None
+    g = api.backward(d["q"], d["k"], d["v"], d["a"], d["b"], d["w"], d["s0"] if s0 else None,
+                     do, dsT)
+    torch.cuda.synchronize()
+    return g
+
+
+def _oracle(wl, inp, up, with_dsT=True, s0=True, heads=None):
+    f = lambda key: W.as_f32(inp[key], wl.dtype)
+    q, k, v, a, b = f("q"), f("k"), f("v"), f("a"), f("b")
+    w = f("w") if inp.get("w") is not None else b
+    do = W.as_f32(up["do"], wl.dtype)
+    s0v = inp.get("s0") if s0 else None
+    dsT = up["dsT"] if with_dsT else None
+    if heads is None:
+        return oracle.backward(q, k, v, a, b, w, s0v, do, dsT)
+    # sampled heads stacked along H of one batch row
+    cat = lambda x: None if x is None else np.concatenate(
+        [x[bi:bi + 1, :, hi:hi + 1] for bi, hi in heads], axis=2)
+    st = lambda x: None if x is None else np.stack([x[bi, hi] for bi, hi in heads])[None]
+    return oracle.backward(cat(q), cat(k), cat(v), cat(a), cat(b), cat(w), st(s0v), cat(do),
+                           st(dsT))
+
+
+def _compare(g, ref, tol, where=""):
+    errs = {}
+    for name in GRADS:
+        if ref[name] is None:
+            assert g[name] is None, name
+            continue
+        errs[name] = rel_err(to_host(g[name]), ref[name])
+    bad = {k: e for k, e in errs.items() if not e <= tol}
+    assert not bad, (where, errs)
+    return errs
+
+
+@pytest.mark.parametrize("name", ["gdn_fp32", "kda_bf16", "gdn2_bf16", "long_bf16"])
+@pytest.mark.parametrize("T", [1, 32, 97, 200])
+def test_small_shapes_every_gate_kind(name, T):
+    """Reduced B/H/T of each prefill workload (scalar gates, shared beta,
+    decoupled vector gates, zero s0), ragged chunk tails included."""
+    wl = W.WORKLOADS[name].replace(B=2, H=2, T=T)
+    inp = W.make_prefill(wl, seed=T)
+    up = W.make_upstream(wl, seed=T)
+    g = _gpu(wl, inp, up)
+    assert api.last_device_error() == 0
+    _compare(g, _oracle(wl, inp, up), TOL[wl.dtype], (name, T))
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 64), (64, 128), (128, 128)])
+def test_head_dims_fp32(dk, dv):
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=70, dk=dk, dv=dv, dtype="f32")
+    inp = W.make_prefill(wl, seed=dk + dv)
+    up = W.make_upstream(wl, seed=dk + dv)
+    _compare(_gpu(wl, inp, up), _oracle(wl, inp, up), TOL["f32"], (dk, dv))
+
+
+def test_scalar_gates_bf16():
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=3, T=100, decay="scalar", erase="scalar",
+                                          write="scalar")
+    inp = W.make_prefill(wl, seed=5)
+    up = W.make_upstream(wl, seed=5)
+    _compare(_gpu(wl, inp, up), _oracle(wl, inp, up), TOL["bf16"])
+
+
+def test_gate_one_everywhere():
+    """No gate tensors (a = b = w = 1): plain DeltaNet; no gate gradients."""
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=75, dtype="f32")
+    inp = W.make_prefill(wl, seed=3)
+    up = W.make_upstream(wl, seed=3)
+    d = inputs_to_dev(inp, wl)
+    g = api.backward(d["q"], d["k"], d["v"], None, None, None, d["s0"], to_dev(up["do"], "f32"),
+                     to_dev(up["dsT"], "f32"))
+    torch.cuda.synchronize()
+    f = lambda key: W.as_f32(inp[key], "f32")
+    ref = oracle.backward(f("q"), f("k"), f("v"), None, None, None, inp["s0"], up["do"], up["dsT"])
+    _compare(g, ref, TOL["f32"])
+
+
+def test_without_state_gradient_or_initial_state():
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=2, H=1, T=90, dtype="f32")
+    inp = W.make_prefill(wl, seed=9)
+    up = W.make_upstream(wl, seed=9)
+    g = _gpu(wl, inp, up, with_dsT=False, s0=False)
+    _compare(g, _oracle(wl, inp, up, with_dsT=False, s0=False), TOL["f32"])
+
+
+def test_zero_length_passes_the_state_gradient_through():
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=0, dtype="f32")
+    inp = W.make_prefill(wl.replace(T=1), seed=2)
+    up = W.make_upstream(wl.replace(T=1), seed=2)
+    z = lambda d: torch.zeros((1, 0, 2, d), dtype=torch.float32, device="cuda")
+    dsT = to_dev(up["dsT"], "f32")
+    g = api.backward(z(128), z(128), z(128), z(128), z(128), z(128), None, z(128), dsT)
+    torch.cuda.synchronize()
+    assert torch.equal(g["ds0"], dsT)
+
+
+def test_decay_beyond_range_is_reported():
+    """Every channel's decay over a 32-token chunk must multiply to at least
+    exp(-80); a stronger one is flagged as GDR_ERR_RANGE."""
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=64)
+    inp = W.make_prefill(wl, seed=1)
+    a = inp["a"].copy()
+    a[0, :, 1, 5] = W.f32_to_bf16_bits(np.full(64, 0.01, np.float32))  # log(0.01)*32 < -80
+    _gpu(wl, dict(inp, a=a), W.make_upstream(wl, seed=1))
+    assert api.last_device_error() == 6   # GDR_ERR_RANGE
+    assert api.last_device_error() == 0
+
+
+def test_repeatable_bit_for_bit():
+    """Every reduction order is fixed: repeated calls agree bit for bit."""
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=2, H=4, T=333)
+    inp = W.make_prefill(wl, seed=4)
+    up = W.make_upstream(wl, seed=4)
+    g0 = _gpu(wl, inp, up)
+    for _ in range(2):
+        g = _gpu(wl, inp, up)
+        for name in GRADS:
+            assert torch.equal(g[name], g0[name]), name
+
+
+def test_full_size_sampled_heads():
+    """The bench-sized workload (B=8, T=8192, H=16, d=128, bf16) on the GPU;
+    the oracle recomputes the gradients of a seeded sample of whole heads."""
+    wl = W.WORKLOADS["gdn2_bf16"]
+    heads = [(0, 3), (5, 11)]
+    inp = W.make_prefill(wl, seed=0)
+    up = W.make_upstream(wl, seed=0)
+    g = _gpu(wl, inp, up)
+    assert api.last_device_error() == 0
+    ref = _oracle(wl, inp, up, heads=heads)
+    for i, (bi, hi) in enumerate(heads):
+        for name in GRADS:
+            x = g[name][bi, hi] if name == "ds0" else g[name][bi, :, hi]
+            r = ref[name][0, i] if name == "ds0" else ref[name][0, :, i]
+            e = rel_err(to_host(x), r)
+            assert e <= TOL["bf16"], (bi, hi, name, e)
