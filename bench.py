@@ -9,8 +9,10 @@ per-channel erase and write gates, bf16 inputs, float32 state with a random
 N(0, 0.1) initial state.  `value` is tokens/s (B*T per step) over all ranks.
 The same line carries the decode step's HBM bandwidth (batch 256, H = 32,
 d = 128, float32 state read and written in place), the roofline fraction of
-the prefill kernel, the float64 oracle's throughput on this host, the
-end-to-end figure through host buffers, and the SM clocks seen while timing.
+the prefill kernel, the backward pass on the same inputs (training: the
+gradients of every input, measured against the CUDA cores' float32 FMA
+peak), the float64 oracle's throughput on this host, the end-to-end figure
+through host buffers, and the SM clocks seen while timing.
 
 Under torchrun each rank runs its own B = 8 batch (weak scaling, no
 collective on the data path); the barrier and the max-over-ranks timing use
@@ -91,6 +93,43 @@ def prefill_flops(wl) -> int:
     8 d^2 + 16 C d + C^2 with decoupled vector gates."""
     d, C = wl.dk, wl.chunk
     return wl.B * wl.T * wl.H * (8 * d * d + 16 * C * d + C * C)
+
+
+BWD_CHUNK = 32  # the backward pass always walks 32-token chunks
+
+
+def backward_flops(wl) -> int:
+    """Flops of one backward call, counted 2mnk over dense tiles, per
+    token-head: the forward sweep that stores the chunk-start states
+    (two grams, Y, E and the state update: 6 dk dv + 4 C dk + 4 C dv) plus the
+    reverse sweep (18 dk dv + 20 C dv + 24 C dk: four grams, Y and E, dE and
+    dY, dU, four dA, four [C, dk] gradient sums, dS, the grams' gradients)."""
+    dk, dv, C = wl.dk, wl.dv, BWD_CHUNK
+    fwd = 6 * dk * dv + 4 * C * dk + 4 * C * dv
+    rev = 18 * dk * dv + 20 * C * dv + 24 * C * dk
+    return wl.B * wl.T * wl.H * (fwd + rev)
+
+
+def backward_bytes(wl) -> int:
+    """Algorithmic HBM bytes of one backward call: the forward's inputs and
+    do read once, their gradients written once, s0 and dS_T read, dS0 written
+    (no intermediates: the chunk-start states are workspace traffic)."""
+    e = 2 if wl.dtype == "bf16" else 4
+    th = wl.B * wl.T * wl.H
+    per_th = e * (2 * wl.dk + wl.dv)                         # q, k, v
+    per_th += e * (wl.dk if wl.decay == "vector" else 1)       # a
+    per_th += e * (wl.dk if wl.erase == "vector" else 1)       # b
+    if wl.write != "shared":
+        per_th += e * (wl.dv if wl.write == "vector" else 1)   # w
+    per_th = 2 * per_th + 2 * e * wl.dv                        # + gradients, do
+    state = 4 * wl.B * wl.H * wl.dk * wl.dv
+    return th * per_th + state * (3 if wl.random_s0 else 2)
+
+
+def fp32_alu_peak_tflops(peaks) -> float:
+    """FP32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flop x the
+    maximum SM clock."""
+    return 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
 
 
 def decode_bytes(wl) -> int:
@@ -409,6 +448,53 @@ def run_gpu(args):
                             "b[..., 0] for erase and write; fg2: beta = b as sqrt(beta) on k "
                             "and v; fg2_plus: beta^k = b, beta^v = w")
 
+    # ---- backward (training): gradients of the main step's prefill for
+    # seeded upstream gradients; one call = one launch (a forward sweep that
+    # stores the chunk-start states, then the reverse sweep)
+    bwd = None
+    if not args.no_backward:
+        up = W.make_upstream(wl, seed=rank_seed(rank))
+        d_o = dev_t(up["do"], wl.dtype)
+        dsT = dev_t(up["dsT"], "f32")
+        del up
+        bdesc = api.desc_for(d["q"], d["v"], d["a"], d["b"], d["w"], BWD_CHUNK)
+        ws = torch.empty(api.backward_workspace_size(bdesc), dtype=torch.uint8, device=dev)
+
+        def bstep():
+            api.backward(d["q"], d["k"], d["v"], d["a"], d["b"], d["w"], d["s0"], d_o, dsT,
+                         workspace=ws, stream=stream)
+
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                bstep()
+            torch.cuda.synchronize()
+            barrier()
+            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b0.record(stream)
+            for _ in range(args.backward_steps):
+                bstep()
+            b1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+        bms = max_over_ranks(b0.elapsed_time(b1)) / args.backward_steps
+        if api.last_device_error(stream) != 0:
+            raise RuntimeError("device error during backward timing")
+        bflops, bbytes = backward_flops(wl), backward_bytes(wl)
+        alu = fp32_alu_peak_tflops(peaks)
+        bwd = {"workload": "gradients of the main step (%s), do ~ N(0,1), dS_T ~ N(0,0.1)"
+                           % wl.name,
+               "steps": args.backward_steps, "ms_per_step": bms,
+               "tokens/s": tokens_step / (bms * 1e-3), "launches_per_step": 1,
+               "roofline": {"bound": "alu", "achieved": bflops / (bms * 1e-3) / 1e12,
+                            "peak": alu, "unit": "TFLOP/s",
+                            "frac": bflops / (bms * 1e-3) / 1e12 / alu,
+                            "flops_per_step": bflops,
+                            "peak_source": "148 SMs x 128 FP32 lanes x 2 x sm_max_mhz"},
+               "hbm": {"algorithmic_bytes_per_step": bbytes,
+                       "GB/s": bbytes / (bms * 1e-3) / 1e9,
+                       "frac": bbytes / (bms * 1e-3) / 1e9 / hbm_peak}}
+        del ws, d_o, dsT
+
     # ---- decode: batch 256, H = 32, d = 128, float32 state in place
     dec = None
     if not args.no_decode:
@@ -482,11 +568,12 @@ def run_gpu(args):
                      "t_tensor_min_us": t_tc * 1e6,
                      "t_hbm_min_us": alg_bytes / (hbm_peak * 1e9) * 1e6},
         "decode": dec,
+        "backward": bwd,
         "variants": variants,
         "e2e": {"value": tokens_step / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "cpu_baseline": cpu,
-        "gpu_launches": args.steps * 1,
+        "gpu_launches": args.steps * 1,  # prefill launches in the timed region
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)
@@ -507,6 +594,8 @@ def main():
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the KDA / FG^2-GDN gate-form timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward timing")
+    ap.add_argument("--backward-steps", type=int, default=3)
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -36,137 +36,170 @@
 // a chunk multiplies to at least e^-80; a chunk below that is reported
 // (GDR_ERR_RANGE) like the tensor-core forward's range check.
 //
-// Two launches.  The float32 forward kernel (chunk 32) stores the state at the
-// start of every chunk in the workspace.  This kernel then takes one
-// (batch, head) per CTA and walks the chunks backwards, carrying dS in the
-// workspace (L2-resident, one [dk, dv] matrix per head).  Per chunk: stage A
-// forms the gated operands, the four grams and T; stage B runs the dv-side
-// products in blocks of 16 value columns, keeping dA and the C x dk gradient
-// sums in registers; stage C adds the grams' gradients; stage D maps the
-// sums back to q, k, b and the decay.
+// One launch, one CTA per (batch, head).  A forward sweep first stores the
+// state at the start of every chunk in the workspace (the chunk form above
+// without its outputs); the reverse sweep then walks the chunks backwards,
+// carrying dS in the workspace (L2-resident, one [dk, dv] matrix per head).
+// Per chunk: stage A forms the gated operands, the grams and T; stage B runs
+// the value-side products in blocks of 16 columns, keeping dA and the
+// [C, dk] gradient sums in registers; stage C adds the grams' gradients;
+// stage D maps the sums back to q, k, b and the decay.  The products are
+// register tiles fed by 16-byte shared-memory loads (rows of the [*, dk]
+// tiles are float4-aligned), the state blocks are held transposed
+// ([value column][key channel]) so both operands of the key-side sums load
+// as float4.
 #include "common.cuh"
 
 namespace gdr {
 
 constexpr int BW_C = 32;    // tokens per chunk
 constexpr int BW_DB = 16;   // value columns per stage-B block
-constexpr int BW_NT = 512;  // threads: one per (row, column) of a [C][DB] tile
+constexpr int BW_NT = 512;  // threads
 constexpr float BW_MIN_LOG_DECAY = -80.0f;
 
 template <int DK>
 struct BwdSmem {
     static constexpr int C = BW_C, DB = BW_DB;
-    static constexpr int P = DK + 1;   // row stride of [C][DK] tiles
+    static constexpr int P = DK + 4;   // row stride of [C][DK] and [DB][DK] tiles
     static constexpr int CP = C + 1;   // row stride of [C][C] tiles
-    static constexpr int SP = DB + 1;  // row stride of [DK][DB] and [C][DB] tiles
+    static constexpr int UP = DB + 4;  // row stride of [C][DB] tiles
     static constexpr int kQh = 0;
     static constexpr int kKh = kQh + C * P;
     static constexpr int kKt = kKh + C * P;
     static constexpr int kBt = kKt + C * P;
     static constexpr int kB = kBt + C * P;  // erase gate
     static constexpr int kG = kB + C * P;   // cumulative log decay
-    static constexpr int kAqk = kG + C * P;
+    static constexpr int kA = kG + C * P;   // decay a itself (for da = d log a / a)
+    static constexpr int kAqk = kA + C * P;
     static constexpr int kAqb = kAqk + C * CP;
     static constexpr int kAkk = kAqb + C * CP;
     static constexpr int kAkb = kAkk + C * CP;
     static constexpr int kT = kAkb + C * CP;
     static constexpr int kScr = kT + C * CP;
     // stage B tiles inside the scratch
-    static constexpr int sS0 = 0;
-    static constexpr int sdS = sS0 + DK * SP;
-    static constexpr int sU = sdS + DK * SP;
-    static constexpr int sdO = sU + C * SP;
-    static constexpr int sY = sdO + C * SP;
-    static constexpr int sE = sY + C * SP;
-    static constexpr int sdE = sE + C * SP;
-    static constexpr int sdY = sdE + C * SP;
-    static constexpr int scrB = sdY + C * SP;
-    // stage C: masked dA_qk, dA_qb, dA_kk, dA_kb; stage D: dG [C][P]
-    static constexpr int scrC = 4 * C * CP;
+    static constexpr int sS0 = 0;               // S0 block, [DB][DK]
+    static constexpr int sdS = sS0 + DB * P;    // dS_C block, [DB][DK]
+    static constexpr int sU = sdS + DB * P;
+    static constexpr int sdO = sU + C * UP;
+    static constexpr int sY = sdO + C * UP;
+    static constexpr int sE = sY + C * UP;
+    static constexpr int sdE = sE + C * UP;
+    static constexpr int sdY = sdE + C * UP;
+    static constexpr int scrB = sdY + C * UP;
+    // stage D: dG [C][P]
     static constexpr int scrD = C * P;
-    static constexpr int scr = scrB > scrC ? (scrB > scrD ? scrB : scrD) : (scrC > scrD ? scrC : scrD);
-    static constexpr int kGcr = kScr + scr;  // per-row shares of the G_C gradient [C][P]
-    static constexpr int kEgc = kGcr + C * P;  // e^G_C per channel
-    static constexpr int kIgc = kEgc + DK;   // e^-G_C
-    static constexpr int kDgc = kIgc + DK;   // gradient on G_C
+    static constexpr int scr = ((scrB > scrD ? scrB : scrD) + 3) / 4 * 4;
+    static constexpr int kGcr = kScr + scr;     // per-row shares of the G_C gradient [C][P]
+    static constexpr int kDA = kGcr + C * P;    // dA_qk, dA_qb, dA_kk, dA_kb [C][CP] each
+    static constexpr int kEgc = kDA + 4 * C * CP;  // e^G_C per channel
+    static constexpr int kIgc = kEgc + DK;      // e^-G_C
+    static constexpr int kDgc = kIgc + DK;      // gradient on G_C
     static constexpr int floats = kDgc + DK;
     static constexpr size_t bytes = sizeof(float) * floats;
+    static_assert(kScr % 4 == 0 && kGcr % 4 == 0 && kEgc % 4 == 0 && sU % 4 == 0 &&
+                  kDA % 4 == 0 &&
+                  C * P % 4 == 0 && C * UP % 4 == 0, "float4 alignment");
 };
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float dot4(float4 a, float4 b) {
+    return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
+}
+__device__ __forceinline__ float comp(float4 v, int e) {
+    return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
+}
+
+// Four consecutive values of a gradient row (16-byte or 8-byte store).
+__device__ __forceinline__ void store4(float* p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float a, float b, float c, float d) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&lo);
+    u.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(p) = u;
+}
 
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(BW_NT, 1)
 backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__ k,
                 const Tin* __restrict__ v, const Tin* __restrict__ a,
                 const Tin* __restrict__ b, const Tin* __restrict__ w, int a_kind, int b_kind,
-                int w_kind, const Tin* __restrict__ dout, const float* __restrict__ ds_final,
-                const float* __restrict__ hs, float* __restrict__ ds_run,
-                Tin* __restrict__ dq, Tin* __restrict__ dk, Tin* __restrict__ dv,
-                Tin* __restrict__ da, Tin* __restrict__ db, Tin* __restrict__ dw,
-                float* __restrict__ ds0, int* __restrict__ err_word) {
+                int w_kind, const Tin* __restrict__ dout, const float* __restrict__ s0,
+                const float* __restrict__ ds_final, float* __restrict__ hs,
+                float* __restrict__ ds_run, Tin* __restrict__ dq, Tin* __restrict__ dk,
+                Tin* __restrict__ dv, Tin* __restrict__ da, Tin* __restrict__ db,
+                Tin* __restrict__ dw, float* __restrict__ ds0, int* __restrict__ err_word) {
     using L = BwdSmem<DK>;
     constexpr int C = BW_C, DB = BW_DB, NT = BW_NT;
-    constexpr int P = L::P, CP = L::CP, SP = L::SP;
-    constexpr int NCI = DK / 16;  // key channels per thread in the [C][DK] sums
-    static_assert(C * DB == NT && DV % DB == 0 && DK % 16 == 0, "shape");
+    constexpr int P = L::P, CP = L::CP, UP = L::UP;
+    constexpr int NG = DK / 64;      // float4 groups of key channels per thread: 4 cl + 64 g
+    constexpr int NCI = 4 * NG;      // key channels per thread in the [C][DK] sums
+    static_assert(C * DB == NT && DV % DB == 0 && (DK == 64 || DK == 128), "shape");
 
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     float* Qh = sm + L::kQh;
     float* Kh = sm + L::kKh;
     float* Kt = sm + L::kKt;
     float* Bt = sm + L::kBt;
     float* Bs = sm + L::kB;
     float* Gs = sm + L::kG;
+    float* As = sm + L::kA;
     float* Aqk = sm + L::kAqk;
     float* Aqb = sm + L::kAqb;
     float* Akk = sm + L::kAkk;
     float* Akb = sm + L::kAkb;
     float* Tm = sm + L::kT;
     float* scr = sm + L::kScr;
-    float* S0b = scr + L::sS0;
-    float* dSb = scr + L::sdS;
+    float* S0T = scr + L::sS0;
+    float* dST = scr + L::sdS;
     float* Ub = scr + L::sU;
     float* dOb = scr + L::sdO;
     float* Yb = scr + L::sY;
     float* Eb = scr + L::sE;
     float* dEb = scr + L::sdE;
     float* dYb = scr + L::sdY;
+    float* gcr = sm + L::kGcr;
+    float* dAqk = sm + L::kDA;
+    float* dAqb = dAqk + C * CP;
+    float* dAkk = dAqk + 2 * C * CP;
+    float* dAkb = dAqk + 3 * C * CP;
     float* egc = sm + L::kEgc;
     float* igc = sm + L::kIgc;
     float* dgc = sm + L::kDgc;
-    float* gcr = sm + L::kGcr;
 
     const int tid = threadIdx.x;
     const int bh = blockIdx.x;
     const int bi = bh / H, hi = bh % H;
-    const int rr = tid >> 4;  // row of this thread in [C][*] tiles
-    const int cl = tid & 15;  // column lane: value column in stage B, key channels cl + 16 i
+    const int rr = tid >> 4;   // row in [C][*] tiles (one row per thread)
+    const int cl = tid & 15;   // lane in the row: value column, or key channels 4 cl + 64 g
+    const int task = tid >> 8; // two half-CTA tasks side by side in stage B
+    const int t2 = tid & 255;
+    const int r2 = t2 >> 4;    // rows r2 and r2 + 16 of a half-CTA task
     const int n_chunks = (T + C - 1) / C;
     const size_t soff = (size_t)bh * DK * DV;
+    float* hbase = hs + (size_t)bh * n_chunks * DK * DV;
     auto tok_of = [&](int t) { return ((long long)bi * T + t) * H + hi; };
 
-    for (int x = tid; x < DK * DV; x += NT) ds_run[soff + x] = ds_final ? ds_final[soff + x] : 0.f;
-
-    for (int ci = n_chunks - 1; ci >= 0; --ci) {
-        const int t0 = ci * C;
-        const int n = min(C, T - t0);
-        __syncthreads();  // previous chunk done with every buffer; ds_run visible
-
-        // ---------------- stage A: gated operands, grams, T
+    // ---------------- stage A: gated operands, grams (all four when with_q), T
+    auto stage_a = [&](int t0, int n, bool with_q) {
         for (int x = tid; x < C * DK; x += NT) {
             const int r = x / DK, c = x % DK;
-            float qv = 0.f, kv = 0.f, bv = 0.f, gv = 0.f;
+            float qv = 0.f, kv = 0.f, bv = 0.f, gv = 0.f, av = 1.f;
             if (r < n) {
                 const long long tok = tok_of(t0 + r), base = tok * DK;
-                qv = to_f32(q[base + c]);
+                if (with_q) qv = to_f32(q[base + c]);
                 kv = to_f32(k[base + c]);
                 bv = gate_value(b, b_kind, tok, base, c);
-                gv = a_kind == GDR_GATE_ONE ? 0.f
-                                            : safe_log_decay(gate_value(a, a_kind, tok, base, c));
+                av = gate_value(a, a_kind, tok, base, c);
+                gv = a_kind == GDR_GATE_ONE ? 0.f : safe_log_decay(av);
             }
             Qh[r * P + c] = qv;
             Kh[r * P + c] = kv;
             Bs[r * P + c] = bv;
             Gs[r * P + c] = gv;
+            As[r * P + c] = av;
         }
         __syncthreads();
         if (tid < DK) {
@@ -199,20 +232,27 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
                 float qk = 0.f, qb = 0.f, kk = 0.f, kb = 0.f;
                 if (s <= r) {
 #pragma unroll 4
-                    for (int c = 0; c < DK; ++c) {
-                        const float kbs = Kt[s * P + c] * igc[c];
-                        const float bbs = Bt[s * P + c] * igc[c];
-                        const float qr = Qh[r * P + c], kr = Kh[r * P + c];
-                        qk = fmaf(qr, kbs, qk);
-                        qb = fmaf(qr, bbs, qb);
-                        kk = fmaf(kr, kbs, kk);
-                        kb = fmaf(kr, bbs, kb);
+                    for (int c = 0; c < DK; c += 4) {
+                        const float4 ig = ld4(igc + c);
+                        float4 kb4 = ld4(Kt + s * P + c), bb4 = ld4(Bt + s * P + c);
+                        kb4.x *= ig.x; kb4.y *= ig.y; kb4.z *= ig.z; kb4.w *= ig.w;
+                        bb4.x *= ig.x; bb4.y *= ig.y; bb4.z *= ig.z; bb4.w *= ig.w;
+                        const float4 kr = ld4(Kh + r * P + c);
+                        kk += dot4(kr, kb4);
+                        kb += dot4(kr, bb4);
+                        if (with_q) {
+                            const float4 qr = ld4(Qh + r * P + c);
+                            qk += dot4(qr, kb4);
+                            qb += dot4(qr, bb4);
+                        }
                     }
                 }
-                Aqk[r * CP + s] = qk;
-                Aqb[r * CP + s] = qb;
                 Akk[r * CP + s] = s < r ? kk : 0.f;
                 Akb[r * CP + s] = s < r ? kb : 0.f;
+                if (with_q) {
+                    Aqk[r * CP + s] = qk;
+                    Aqb[r * CP + s] = qb;
+                }
             }
         }
         __syncthreads();
@@ -227,148 +267,312 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
             }
         }
         __syncthreads();
+    };
+
+    // The [DK][DB] block at column j0 of a [DK][DV] matrix, fetched into
+    // registers ahead of its use and stored transposed ([DB][DK]) after the
+    // barrier that frees the tile.
+    constexpr int NPF = DK * DB / NT;
+    auto fetch_block = [&](float (&reg)[NPF], const float* src, int j0) {
+#pragma unroll
+        for (int i = 0; i < NPF; ++i) {
+            const int x = tid + NT * i, c = x / DB, j = x % DB;
+            reg[i] = src[(size_t)c * DV + j0 + j];
+        }
+    };
+    auto put_block = [&](float* dst, const float (&reg)[NPF]) {
+#pragma unroll
+        for (int i = 0; i < NPF; ++i) {
+            const int x = tid + NT * i, c = x / DB, j = x % DB;
+            dst[j * P + c] = reg[i];
+        }
+    };
+
+    // ================= forward sweep: chunk-start states h_c into the workspace
+    for (int x = tid; x < DK * DV; x += NT) {
+        if (n_chunks > 0) hbase[x] = s0 ? s0[soff + x] : 0.f;
+        ds_run[soff + x] = ds_final ? ds_final[soff + x] : 0.f;
+    }
+    for (int ci = 0; ci + 1 < n_chunks; ++ci) {  // every chunk before the last is full
+        const int t0 = ci * C;
+        __syncthreads();  // h_ci written
+        stage_a(t0, C, false);
+        const float* hc = hbase + (size_t)ci * DK * DV;
+        float* hn = hbase + (size_t)(ci + 1) * DK * DV;
+        float pf_s[NPF];
+        fetch_block(pf_s, hc, 0);
+        for (int j0 = 0; j0 < DV; j0 += DB) {
+            put_block(S0T, pf_s);
+            {
+                const long long tok = tok_of(t0 + rr), base = tok * DV;
+                Ub[rr * UP + cl] = gate_value(w, w_kind, tok, base, j0 + cl) *
+                                   to_f32(v[base + j0 + cl]);
+            }
+            __syncthreads();
+            {  // Y = Kh S0 + A_kk U
+                const int r = rr, j = cl;
+                float y = 0.f;
+#pragma unroll 4
+                for (int c = 0; c < DK; c += 4) y += dot4(ld4(Kh + r * P + c), ld4(S0T + j * P + c));
+                for (int s = 0; s < r; ++s) y = fmaf(Akk[r * CP + s], Ub[s * UP + j], y);
+                Yb[r * UP + j] = y;
+            }
+            __syncthreads();
+            {  // E = T Y
+                const int r = rr, j = cl;
+                float e = 0.f;
+                for (int s = 0; s <= r; ++s) e = fmaf(Tm[r * CP + s], Yb[s * UP + j], e);
+                Eb[r * UP + j] = e;
+            }
+            __syncthreads();
+            if (rr < DK / 4) {  // S_C = e^G_C S0 + Kt^T U - Bt^T E, channels 4 rr .. 4 rr + 3
+                const int c = 4 * rr, j = cl;
+                const float4 g4 = ld4(egc + c), s4 = ld4(S0T + j * P + c);
+                float acc[4] = {g4.x * s4.x, g4.y * s4.y, g4.z * s4.z, g4.w * s4.w};
+#pragma unroll 4
+                for (int r = 0; r < C; ++r) {
+                    const float4 kt = ld4(Kt + r * P + c), bt = ld4(Bt + r * P + c);
+                    const float u = Ub[r * UP + j], e = Eb[r * UP + j];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)
+                        acc[x] = fmaf(comp(kt, x), u, fmaf(-comp(bt, x), e, acc[x]));
+                }
+#pragma unroll
+                for (int x = 0; x < 4; ++x) hn[(size_t)(c + x) * DV + j0 + j] = acc[x];
+            }
+            if (j0 + DB < DV) fetch_block(pf_s, hc, j0 + DB);
+            __syncthreads();  // block's tiles consumed
+        }
+    }
+
+    // ================= reverse sweep
+    for (int ci = n_chunks - 1; ci >= 0; --ci) {
+        const int t0 = ci * C;
+        const int n = min(C, T - t0);
+        __syncthreads();  // previous chunk done with every buffer; ds_run, h visible
+        stage_a(t0, n, true);
 
         // ---------------- stage B: value-column blocks
-        float aqk[2] = {0.f, 0.f}, aqb[2] = {0.f, 0.f}, akk[2] = {0.f, 0.f}, akb[2] = {0.f, 0.f};
-        float xq[NCI], xk[NCI], yk[NCI], yb[NCI];
+        // dA entries (r2 + 16 (p >> 1), cl + 16 (p & 1)), p < 4, belong to task-1
+        // thread t2: only it reads and writes them until the masking below
+        if (task == 1) {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const int o = (r2 + 16 * (p >> 1)) * CP + cl + 16 * (p & 1);
+                dAqk[o] = dAqb[o] = dAkk[o] = dAkb[o] = 0.f;
+            }
+        }
+        float xq[NCI], xk[NCI], yk[NCI], yb[NCI];  // channel 4 cl + 64 g + e at [4 g + e]
 #pragma unroll
         for (int i = 0; i < NCI; ++i) xq[i] = xk[i] = yk[i] = yb[i] = 0.f;
-        float gcp = 0.f;    // rowsum(dS_C * S0) of key channel tid (tid < DK)
-        float dw_row = 0.f; // scalar write gate: sum over value columns of v dU
-        const float* hc = hs + ((size_t)bh * n_chunks + ci) * DK * DV;
+        float gcp = 0.f;                 // rowsum(dS_C * S0) of key channel tid (tid < DK)
+        float dw_r0 = 0.f, dw_r1 = 0.f;  // scalar write gate: sums of v dU over value columns
+        const float* hc = hbase + (size_t)ci * DK * DV;
+        const float* dsc = ds_run + soff;
+        float pf_s[NPF], pf_d[NPF];
+        fetch_block(pf_s, hc, 0);
+        fetch_block(pf_d, dsc, 0);
 
         for (int j0 = 0; j0 < DV; j0 += DB) {
-            // B1: load S0, dS_C, U, dO blocks
-            for (int x = tid; x < DK * DB; x += NT) {
-                const int c = x / DB, j = x % DB;
-                S0b[c * SP + j] = hc[(size_t)c * DV + j0 + j];
-                dSb[c * SP + j] = ds_run[soff + (size_t)c * DV + j0 + j];
-            }
-            float wv = 0.f, vv = 0.f;
+            // B1: S0 and dS_C blocks (transposed), U, dO
+            put_block(S0T, pf_s);
+            put_block(dST, pf_d);
             {
                 const int r = rr, j = cl;
                 float u = 0.f, g = 0.f;
                 if (r < n) {
                     const long long tok = tok_of(t0 + r), base = tok * DV;
-                    vv = to_f32(v[base + j0 + j]);
-                    wv = gate_value(w, w_kind, tok, base, j0 + j);
-                    u = wv * vv;
+                    u = gate_value(w, w_kind, tok, base, j0 + j) * to_f32(v[base + j0 + j]);
                     g = to_f32(dout[base + j0 + j]);
                 }
-                Ub[r * SP + j] = u;
-                dOb[r * SP + j] = g;
+                Ub[r * UP + j] = u;
+                dOb[r * UP + j] = g;
             }
             __syncthreads();
-            // B2: Y = Kh S0 + A_kk U;  dE = -A_qb^T dO - Bt dS_C
+            // B2: Y = Kh S0 + A_kk U (task 0);  dE = -A_qb^T dO - Bt dS_C (task 1)
             {
-                const int r = rr, j = cl;
-                float y = 0.f, de = 0.f;
+                const int j = cl, ra = r2, rb = r2 + 16;
+                const float* X = task == 0 ? Kh : Bt;
+                const float* ST = task == 0 ? S0T : dST;
+                float o0 = 0.f, o1 = 0.f;
 #pragma unroll 4
-                for (int c = 0; c < DK; ++c) {
-                    y = fmaf(Kh[r * P + c], S0b[c * SP + j], y);
-                    de = fmaf(-Bt[r * P + c], dSb[c * SP + j], de);
+                for (int c = 0; c < DK; c += 4) {
+                    const float4 s4 = ld4(ST + j * P + c);
+                    o0 += dot4(ld4(X + ra * P + c), s4);
+                    o1 += dot4(ld4(X + rb * P + c), s4);
                 }
-                for (int s = 0; s < r; ++s) y = fmaf(Akk[r * CP + s], Ub[s * SP + j], y);
-                for (int s = r; s < C; ++s) de = fmaf(-Aqb[s * CP + r], dOb[s * SP + j], de);
-                Yb[r * SP + j] = y;
-                dEb[r * SP + j] = de;
+                if (task == 0) {
+                    for (int s = 0; s < ra; ++s) o0 = fmaf(Akk[ra * CP + s], Ub[s * UP + j], o0);
+                    for (int s = 0; s < rb; ++s) o1 = fmaf(Akk[rb * CP + s], Ub[s * UP + j], o1);
+                    Yb[ra * UP + j] = o0;
+                    Yb[rb * UP + j] = o1;
+                } else {
+                    for (int s = ra; s < C; ++s) o0 = fmaf(Aqb[s * CP + ra], dOb[s * UP + j], o0);
+                    for (int s = rb; s < C; ++s) o1 = fmaf(Aqb[s * CP + rb], dOb[s * UP + j], o1);
+                    dEb[ra * UP + j] = -o0;
+                    dEb[rb * UP + j] = -o1;
+                }
             }
             __syncthreads();
-            // B3: E = T Y;  dY = T^T dE
+            // B3: E = T Y (task 0);  dY = T^T dE (task 1)
             {
-                const int r = rr, j = cl;
-                float e = 0.f, dy = 0.f;
-                for (int s = 0; s <= r; ++s) e = fmaf(Tm[r * CP + s], Yb[s * SP + j], e);
-                for (int s = r; s < C; ++s) dy = fmaf(Tm[s * CP + r], dEb[s * SP + j], dy);
-                Eb[r * SP + j] = e;
-                dYb[r * SP + j] = dy;
+                const int j = cl, ra = r2, rb = r2 + 16;
+                float o0 = 0.f, o1 = 0.f;
+                if (task == 0) {
+                    for (int s = 0; s <= ra; ++s) o0 = fmaf(Tm[ra * CP + s], Yb[s * UP + j], o0);
+                    for (int s = 0; s <= rb; ++s) o1 = fmaf(Tm[rb * CP + s], Yb[s * UP + j], o1);
+                    Eb[ra * UP + j] = o0;
+                    Eb[rb * UP + j] = o1;
+                } else {
+                    for (int s = ra; s < C; ++s) o0 = fmaf(Tm[s * CP + ra], dEb[s * UP + j], o0);
+                    for (int s = rb; s < C; ++s) o1 = fmaf(Tm[s * CP + rb], dEb[s * UP + j], o1);
+                    dYb[ra * UP + j] = o0;
+                    dYb[rb * UP + j] = o1;
+                }
             }
             __syncthreads();
-            // B4: dU; dA; the [C][DK] sums; dG_C share; dS0 of this block
-            {
-                const int r = rr, j = cl;
-                float du = 0.f;
+            // B4a: dU -> dv, dw (task 0);  dA (task 1)
+            if (task == 0) {
+                const int j = cl, ra = r2, rb = r2 + 16;
+                float o0 = 0.f, o1 = 0.f;
 #pragma unroll 4
-                for (int c = 0; c < DK; ++c) du = fmaf(Kt[r * P + c], dSb[c * SP + j], du);
-                for (int s = r; s < C; ++s) du = fmaf(Aqk[s * CP + r], dOb[s * SP + j], du);
-                for (int s = r + 1; s < C; ++s) du = fmaf(Akk[s * CP + r], dYb[s * SP + j], du);
-                if (r < n) {
-                    const long long tok = tok_of(t0 + r), base = tok * DV;
-                    dv[base + j0 + j] = from_f32<Tin>(wv * du);
-                    if (w_kind == GDR_GATE_VECTOR) dw[base + j0 + j] = from_f32<Tin>(vv * du);
-                    dw_row = fmaf(vv, du, dw_row);
+                for (int c = 0; c < DK; c += 4) {
+                    const float4 d4 = ld4(dST + j * P + c);
+                    o0 += dot4(ld4(Kt + ra * P + c), d4);
+                    o1 += dot4(ld4(Kt + rb * P + c), d4);
+                }
+                for (int s = ra; s < C; ++s) o0 = fmaf(Aqk[s * CP + ra], dOb[s * UP + j], o0);
+                for (int s = rb; s < C; ++s) o1 = fmaf(Aqk[s * CP + rb], dOb[s * UP + j], o1);
+                for (int s = ra + 1; s < C; ++s) o0 = fmaf(Akk[s * CP + ra], dYb[s * UP + j], o0);
+                for (int s = rb + 1; s < C; ++s) o1 = fmaf(Akk[s * CP + rb], dYb[s * UP + j], o1);
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int r = h2 ? rb : ra;
+                    const float du = h2 ? o1 : o0;
+                    if (r < n) {
+                        const long long tok = tok_of(t0 + r), base = tok * DV;
+                        const float ww = gate_value(w, w_kind, tok, base, j0 + j);
+                        const float vx = to_f32(v[base + j0 + j]);
+                        dv[base + j0 + j] = from_f32<Tin>(ww * du);
+                        if (w_kind == GDR_GATE_VECTOR) dw[base + j0 + j] = from_f32<Tin>(vx * du);
+                        if (h2) dw_r1 = fmaf(vx, du, dw_r1);
+                        else dw_r0 = fmaf(vx, du, dw_r0);
+                    }
+                }
+            } else {
+                const int ra = r2, rb = r2 + 16, sa = cl, sb = cl + 16;
+                float aqk[4], aqb[4], akk[4], akb[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const int o = (r2 + 16 * (p >> 1)) * CP + cl + 16 * (p & 1);
+                    aqk[p] = dAqk[o];
+                    aqb[p] = dAqb[o];
+                    akk[p] = dAkk[o];
+                    akb[p] = dAkb[o];
+                }
+#pragma unroll
+                for (int jj = 0; jj < DB; jj += 4) {
+                    const float4 oa = ld4(dOb + ra * UP + jj), ob = ld4(dOb + rb * UP + jj);
+                    const float4 ya = ld4(dYb + ra * UP + jj), yb4 = ld4(dYb + rb * UP + jj);
+                    const float4 ua = ld4(Ub + sa * UP + jj), ub = ld4(Ub + sb * UP + jj);
+                    const float4 ea = ld4(Eb + sa * UP + jj), eb = ld4(Eb + sb * UP + jj);
+                    aqk[0] += dot4(oa, ua); aqk[1] += dot4(oa, ub);
+                    aqk[2] += dot4(ob, ua); aqk[3] += dot4(ob, ub);
+                    aqb[0] -= dot4(oa, ea); aqb[1] -= dot4(oa, eb);
+                    aqb[2] -= dot4(ob, ea); aqb[3] -= dot4(ob, eb);
+                    akk[0] += dot4(ya, ua); akk[1] += dot4(ya, ub);
+                    akk[2] += dot4(yb4, ua); akk[3] += dot4(yb4, ub);
+                    akb[0] -= dot4(ya, ea); akb[1] -= dot4(ya, eb);
+                    akb[2] -= dot4(yb4, ea); akb[3] -= dot4(yb4, eb);
+                }
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const int o = (r2 + 16 * (p >> 1)) * CP + cl + 16 * (p & 1);
+                    dAqk[o] = aqk[p];
+                    dAqb[o] = aqb[p];
+                    dAkk[o] = akk[p];
+                    dAkb[o] = akb[p];
                 }
             }
+            // B4b: the [C][DK] sums, the dG_C share, and dS0 of this block
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const int r = rr, s = cl + 16 * h2;
+            for (int jj = 0; jj < DB; jj += 4) {
+                const float4 o4 = ld4(dOb + rr * UP + jj), y4 = ld4(dYb + rr * UP + jj);
+                const float4 u4 = ld4(Ub + rr * UP + jj), e4 = ld4(Eb + rr * UP + jj);
 #pragma unroll
-                for (int j = 0; j < DB; ++j) {
-                    const float go = dOb[r * SP + j], gy = dYb[r * SP + j];
-                    const float us = Ub[s * SP + j], es = Eb[s * SP + j];
-                    aqk[h2] = fmaf(go, us, aqk[h2]);
-                    aqb[h2] = fmaf(-go, es, aqb[h2]);
-                    akk[h2] = fmaf(gy, us, akk[h2]);
-                    akb[h2] = fmaf(-gy, es, akb[h2]);
-                }
-            }
-#pragma unroll 4
-            for (int j = 0; j < DB; ++j) {
-                const int r = rr;
-                const float go = dOb[r * SP + j], gy = dYb[r * SP + j];
-                const float ur = Ub[r * SP + j], er = Eb[r * SP + j];
+                for (int e = 0; e < 4; ++e) {
+                    const int j = jj + e;
+                    const float go = comp(o4, e), gy = comp(y4, e), gu = comp(u4, e), ge = comp(e4, e);
 #pragma unroll
-                for (int i = 0; i < NCI; ++i) {
-                    const int c = cl + 16 * i;
-                    const float s0 = S0b[c * SP + j], ds = dSb[c * SP + j];
-                    xq[i] = fmaf(go, s0, xq[i]);
-                    xk[i] = fmaf(gy, s0, xk[i]);
-                    yk[i] = fmaf(ur, ds, yk[i]);
-                    yb[i] = fmaf(-er, ds, yb[i]);
+                    for (int g = 0; g < NG; ++g) {
+                        const int c = 4 * cl + 64 * g;
+                        const float4 s4 = ld4(S0T + j * P + c), d4 = ld4(dST + j * P + c);
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            xq[4 * g + x] = fmaf(go, comp(s4, x), xq[4 * g + x]);
+                            xk[4 * g + x] = fmaf(gy, comp(s4, x), xk[4 * g + x]);
+                            yk[4 * g + x] = fmaf(gu, comp(d4, x), yk[4 * g + x]);
+                            yb[4 * g + x] = fmaf(-ge, comp(d4, x), yb[4 * g + x]);
+                        }
+                    }
                 }
             }
             if (tid < DK) {
 #pragma unroll 4
-                for (int j = 0; j < DB; ++j) gcp = fmaf(dSb[tid * SP + j], S0b[tid * SP + j], gcp);
+                for (int j = 0; j < DB; ++j) gcp = fmaf(dST[j * P + tid], S0T[j * P + tid], gcp);
             }
-            for (int x = tid; x < DK * DB; x += NT) {
-                const int c = x / DB, j = x % DB;
-                float acc = egc[c] * dSb[c * SP + j];
+            if (rr < DK / 4) {  // dS0 = e^G_C dS_C + Qh^T dO + Kh^T dY, channels 4 rr ..
+                const int c = 4 * rr, j = cl;
+                const float4 g4 = ld4(egc + c), d4 = ld4(dST + j * P + c);
+                float acc[4] = {g4.x * d4.x, g4.y * d4.y, g4.z * d4.z, g4.w * d4.w};
+#pragma unroll 4
                 for (int r = 0; r < n; ++r) {
-                    acc = fmaf(Qh[r * P + c], dOb[r * SP + j], acc);
-                    acc = fmaf(Kh[r * P + c], dYb[r * SP + j], acc);
+                    const float4 qh = ld4(Qh + r * P + c), kh = ld4(Kh + r * P + c);
+                    const float go = dOb[r * UP + j], gy = dYb[r * UP + j];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)
+                        acc[x] = fmaf(comp(qh, x), go, fmaf(comp(kh, x), gy, acc[x]));
                 }
-                ds_run[soff + (size_t)c * DV + j0 + j] = acc;
+#pragma unroll
+                for (int x = 0; x < 4; ++x) ds_run[soff + (size_t)(c + x) * DV + j0 + j] = acc[x];
+            }
+            if (j0 + DB < DV) {  // next block's columns: not written by this chunk yet
+                fetch_block(pf_s, hc, j0 + DB);
+                fetch_block(pf_d, dsc, j0 + DB);
             }
             __syncthreads();  // block's tiles consumed before the next block loads
         }
 
-        // scalar write gate: one value per token
-        if (w_kind == GDR_GATE_SCALAR) {
+        // scalar write gate: one value per token (task-0 warps hold the row sums)
+        if (w_kind == GDR_GATE_SCALAR && task == 0) {
 #pragma unroll
-            for (int m = 8; m >= 1; m >>= 1) dw_row += __shfl_xor_sync(0xffffffffu, dw_row, m);
-            if (cl == 0 && rr < n) dw[tok_of(t0 + rr)] = from_f32<Tin>(dw_row);
+            for (int m = 8; m >= 1; m >>= 1) {
+                dw_r0 += __shfl_xor_sync(0xffffffffu, dw_r0, m);
+                dw_r1 += __shfl_xor_sync(0xffffffffu, dw_r1, m);
+            }
+            if (cl == 0 && r2 < n) dw[tok_of(t0 + r2)] = from_f32<Tin>(dw_r0);
+            if (cl == 0 && r2 + 16 < n) dw[tok_of(t0 + r2 + 16)] = from_f32<Tin>(dw_r1);
         }
 
         // gradient on G_C: e^G_C rowsum(dS_C S0) + colsum(Kt YK + Bt YB), taken
         // before the grams' shares join YK and YB (rows summed in a fixed order)
 #pragma unroll
-        for (int i = 0; i < NCI; ++i) {
-            const int c = cl + 16 * i;
-            gcr[rr * P + c] = Kt[rr * P + c] * yk[i] + Bt[rr * P + c] * yb[i];
+        for (int g = 0; g < NG; ++g) {
+            const int c = 4 * cl + 64 * g;
+            const float4 kt = ld4(Kt + rr * P + c), bt = ld4(Bt + rr * P + c);
+            store4(gcr + rr * P + c, kt.x * yk[4 * g] + bt.x * yb[4 * g],
+                   kt.y * yk[4 * g + 1] + bt.y * yb[4 * g + 1],
+                   kt.z * yk[4 * g + 2] + bt.z * yb[4 * g + 2],
+                   kt.w * yk[4 * g + 3] + bt.w * yb[4 * g + 3]);
         }
-        // masked dA into the scratch (stage-B tiles are consumed)
-        float* dAqk = scr;
-        float* dAqb = scr + C * CP;
-        float* dAkk = scr + 2 * C * CP;
-        float* dAkb = scr + 3 * C * CP;
+        // dA masks (their owners, as above)
+        if (task == 1) {
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            const int r = rr, s = cl + 16 * h2;
-            dAqk[r * CP + s] = s <= r ? aqk[h2] : 0.f;
-            dAqb[r * CP + s] = s <= r ? aqb[h2] : 0.f;
-            dAkk[r * CP + s] = s < r ? akk[h2] : 0.f;
-            dAkb[r * CP + s] = s < r ? akb[h2] : 0.f;
+            for (int p = 0; p < 4; ++p) {
+                const int r = r2 + 16 * (p >> 1), s = cl + 16 * (p & 1);
+                if (s > r) dAqk[r * CP + s] = dAqb[r * CP + s] = 0.f;
+                if (s >= r) dAkk[r * CP + s] = dAkb[r * CP + s] = 0.f;
+            }
         }
         __syncthreads();
         if (tid < DK) {
@@ -377,35 +581,34 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
             dgc[tid] = g;
         }
 
-        // ---------------- stage C: the grams' gradients
+        // ---------------- stage C: the grams' gradients (e^-G_C folded into the operands)
         {
             const int r = rr;
-            float pq[NCI], pk[NCI], qk_[NCI], qb_[NCI];
+            float4 ig[NG];
 #pragma unroll
-            for (int i = 0; i < NCI; ++i) pq[i] = pk[i] = qk_[i] = qb_[i] = 0.f;
+            for (int g = 0; g < NG; ++g) ig[g] = ld4(igc + 4 * cl + 64 * g);
             for (int s = 0; s < C; ++s) {
                 const float gqk = dAqk[r * CP + s], gqb = dAqb[r * CP + s];
                 const float gkk = dAkk[r * CP + s], gkb = dAkb[r * CP + s];
                 const float tqk = dAqk[s * CP + r], tqb = dAqb[s * CP + r];
                 const float tkk = dAkk[s * CP + r], tkb = dAkb[s * CP + r];
 #pragma unroll
-                for (int i = 0; i < NCI; ++i) {
-                    const int c = cl + 16 * i;
-                    const float kts = Kt[s * P + c], bts = Bt[s * P + c];
-                    const float qhs = Qh[s * P + c], khs = Kh[s * P + c];
-                    pq[i] = fmaf(gqk, kts, fmaf(gqb, bts, pq[i]));
-                    pk[i] = fmaf(gkk, kts, fmaf(gkb, bts, pk[i]));
-                    qk_[i] = fmaf(tqk, qhs, fmaf(tkk, khs, qk_[i]));
-                    qb_[i] = fmaf(tqb, qhs, fmaf(tkb, khs, qb_[i]));
-                }
-            }
+                for (int g = 0; g < NG; ++g) {
+                    const int c = 4 * cl + 64 * g;
+                    const float4 kt = ld4(Kt + s * P + c), bt = ld4(Bt + s * P + c);
+                    const float4 qh = ld4(Qh + s * P + c), kh = ld4(Kh + s * P + c);
 #pragma unroll
-            for (int i = 0; i < NCI; ++i) {
-                const float f = igc[cl + 16 * i];
-                xq[i] = fmaf(f, pq[i], xq[i]);
-                xk[i] = fmaf(f, pk[i], xk[i]);
-                yk[i] = fmaf(f, qk_[i], yk[i]);
-                yb[i] = fmaf(f, qb_[i], yb[i]);
+                    for (int x = 0; x < 4; ++x) {
+                        const float f = comp(ig[g], x);
+                        const float ktf = comp(kt, x) * f, btf = comp(bt, x) * f;
+                        const float qhf = comp(qh, x) * f, khf = comp(kh, x) * f;
+                        const int i = 4 * g + x;
+                        xq[i] = fmaf(gqk, ktf, fmaf(gqb, btf, xq[i]));
+                        xk[i] = fmaf(gkk, ktf, fmaf(gkb, btf, xk[i]));
+                        yk[i] = fmaf(tqk, qhf, fmaf(tkk, khf, yk[i]));
+                        yb[i] = fmaf(tqb, qhf, fmaf(tkb, khf, yb[i]));
+                    }
+                }
             }
         }
         __syncthreads();  // dA reads done: the scratch becomes dG
@@ -415,24 +618,32 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
         {
             const int r = rr;
             float db_row = 0.f;
+            const long long tok = tok_of(t0 + min(r, n - 1)), base = tok * DK;
 #pragma unroll
-            for (int i = 0; i < NCI; ++i) {
-                const int c = cl + 16 * i;
-                float g = 0.f;
-                if (r < n) {
-                    const float gr = Gs[r * P + c], gc = Gs[(C - 1) * P + c];
+            for (int g = 0; g < NG; ++g) {
+                const int c = 4 * cl + 64 * g;
+                float gq[4], gk[4], gb[4], gg[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int i = 4 * g + x;
+                    const float gr = Gs[r * P + c + x], gc = Gs[(C - 1) * P + c + x];
                     const float eg = __expf(gr), et = __expf(gc - gr);
-                    const float kt = Kt[r * P + c], bt = Bt[r * P + c];
-                    const long long tok = tok_of(t0 + r), base = tok * DK;
-                    dq[base + c] = from_f32<Tin>(eg * xq[i]);
-                    dk[base + c] = from_f32<Tin>(fmaf(eg, xk[i], et * (yk[i] + Bs[r * P + c] * yb[i])));
-                    const float dbv = kt * yb[i];
-                    if (b_kind == GDR_GATE_VECTOR) db[base + c] = from_f32<Tin>(dbv);
-                    db_row += dbv;
-                    g = Qh[r * P + c] * xq[i] + Kh[r * P + c] * xk[i] - kt * yk[i] - bt * yb[i];
-                    if (r == n - 1) g += dgc[c];
+                    const float kt = Kt[r * P + c + x], bt = Bt[r * P + c + x];
+                    gq[x] = eg * xq[i];
+                    gk[x] = fmaf(eg, xk[i], et * (yk[i] + Bs[r * P + c + x] * yb[i]));
+                    gb[x] = kt * yb[i];
+                    db_row += gb[x];
+                    gg[x] = Qh[r * P + c + x] * xq[i] + Kh[r * P + c + x] * xk[i] - kt * yk[i] -
+                            bt * yb[i];
+                    if (r == n - 1) gg[x] += dgc[c + x];
+                    if (r >= n) gg[x] = 0.f;
                 }
-                dG[r * P + c] = g;
+                store4(dG + r * P + c, gg[0], gg[1], gg[2], gg[3]);
+                if (r < n) {
+                    store4(dq + base + c, gq[0], gq[1], gq[2], gq[3]);
+                    store4(dk + base + c, gk[0], gk[1], gk[2], gk[3]);
+                    if (b_kind == GDR_GATE_VECTOR) store4(db + base + c, gb[0], gb[1], gb[2], gb[3]);
+                }
             }
             if (b_kind == GDR_GATE_SCALAR) {
 #pragma unroll
@@ -447,10 +658,8 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
                 float run = 0.f;
                 for (int r = n - 1; r >= 0; --r) {
                     run += dG[r * P + c];
-                    const long long tok = tok_of(t0 + r), base = tok * DK;
-                    const float av = gate_value(a, a_kind, tok, base, c);
-                    const float g = run / av;
-                    if (a_kind == GDR_GATE_VECTOR) da[base + c] = from_f32<Tin>(g);
+                    const float g = run / As[r * P + c];
+                    if (a_kind == GDR_GATE_VECTOR) da[(tok_of(t0 + r)) * DK + c] = from_f32<Tin>(g);
                     else dG[r * P + c] = g;
                 }
             }
@@ -458,7 +667,10 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
                 __syncthreads();
                 float s = 0.f;
 #pragma unroll
-                for (int i = 0; i < NCI; ++i) s += dG[rr * P + cl + 16 * i];
+                for (int g = 0; g < NG; ++g) {
+                    const float4 d4 = ld4(dG + rr * P + 4 * cl + 64 * g);
+                    s += d4.x + d4.y + d4.z + d4.w;
+                }
 #pragma unroll
                 for (int m = 8; m >= 1; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
                 if (cl == 0 && rr < n) da[tok_of(t0 + rr)] = from_f32<Tin>(s);
@@ -472,10 +684,10 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
 }
 
 template <typename Tin, int DK, int DV>
-static cudaError_t launch_backward_t(const gdr_desc& d, const void* const* in, const void* dout,
-                                     const float* ds_final, float* hs, float* ds_run,
-                                     void* const* grads, float* ds0, int* err_word,
-                                     cudaStream_t st) {
+static cudaError_t launch_backward_t(const gdr_desc& d, const void* const* in, const float* s0,
+                                     const void* dout, const float* ds_final, float* hs,
+                                     float* ds_run, void* const* grads, float* ds0,
+                                     int* err_word, cudaStream_t st) {
     auto kern = backward_kernel<Tin, DK, DV>;
     const size_t smem = BwdSmem<DK>::bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -484,20 +696,20 @@ static cudaError_t launch_backward_t(const gdr_desc& d, const void* const* in, c
     kern<<<(unsigned)((long long)d.B * d.H), BW_NT, smem, st>>>(
         d.T, d.H, (const Tin*)in[0], (const Tin*)in[1], (const Tin*)in[2], (const Tin*)in[3],
         (const Tin*)in[4], (const Tin*)in[5], (int)d.decay, (int)d.erase, (int)d.write,
-        (const Tin*)dout, ds_final, hs, ds_run, (Tin*)grads[0], (Tin*)grads[1], (Tin*)grads[2],
-        (Tin*)grads[3], (Tin*)grads[4], (Tin*)grads[5], ds0, err_word);
+        (const Tin*)dout, s0, ds_final, hs, ds_run, (Tin*)grads[0], (Tin*)grads[1],
+        (Tin*)grads[2], (Tin*)grads[3], (Tin*)grads[4], (Tin*)grads[5], ds0, err_word);
     return cudaGetLastError();
 }
 
 template <typename Tin>
-static cudaError_t launch_backward_d(const gdr_desc& d, const void* const* in, const void* dout,
-                                     const float* ds_final, float* hs, float* ds_run,
-                                     void* const* grads, float* ds0, int* err_word,
-                                     cudaStream_t st) {
-#define GDR_BWD(DK_, DV_)                                                                    \
-    if (d.dk == DK_ && d.dv == DV_)                                                          \
-        return launch_backward_t<Tin, DK_, DV_>(d, in, dout, ds_final, hs, ds_run, grads, ds0, \
-                                                err_word, st);
+static cudaError_t launch_backward_d(const gdr_desc& d, const void* const* in, const float* s0,
+                                     const void* dout, const float* ds_final, float* hs,
+                                     float* ds_run, void* const* grads, float* ds0,
+                                     int* err_word, cudaStream_t st) {
+#define GDR_BWD(DK_, DV_)                                                                  \
+    if (d.dk == DK_ && d.dv == DV_)                                                        \
+        return launch_backward_t<Tin, DK_, DV_>(d, in, s0, dout, ds_final, hs, ds_run, grads, \
+                                                ds0, err_word, st);
     GDR_BWD(128, 128)
     GDR_BWD(128, 64)
     GDR_BWD(64, 128)
@@ -513,12 +725,6 @@ size_t backward_workspace_bytes(const gdr_desc& d) {
     return heads * mat * (n_chunks + 1);  // chunk-start states, then the running dS
 }
 
-cudaError_t launch_chunked_simt(const gdr_desc& d, const void* q, const void* k,
-                                const void* v, const void* a, const void* b, const void* w,
-                                const float* s0, void* o, float* s_final,
-                                const int* cu_seqlens, int n_seqs, float* h_out,
-                                int* err_word, cudaStream_t st);
-
 // in = {q, k, v, a, b, w}; grads = {dq, dk, dv, da, db, dw}.
 cudaError_t launch_backward(const gdr_desc& d, const void* const* in, const float* s0,
                             const void* dout, const float* ds_final, void* const* grads,
@@ -527,17 +733,11 @@ cudaError_t launch_backward(const gdr_desc& d, const void* const* in, const floa
     const size_t n_chunks = ((size_t)d.T + BW_C - 1) / BW_C;
     float* hs = static_cast<float*>(workspace);
     float* ds_run = hs + heads * n_chunks * d.dk * d.dv;
-    if (d.T > 0) {
-        gdr_desc f = d;
-        f.chunk = BW_C;  // chunk-start states on the backward's chunk grid
-        cudaError_t e = launch_chunked_simt(f, in[0], in[1], in[2], in[3], in[4], in[5], s0,
-                                            nullptr, nullptr, nullptr, 0, hs, err_word, st);
-        if (e != cudaSuccess) return e;
-    }
     if (d.in_dtype == GDR_BF16)
-        return launch_backward_d<__nv_bfloat16>(d, in, dout, ds_final, hs, ds_run, grads, ds0,
-                                                err_word, st);
-    return launch_backward_d<float>(d, in, dout, ds_final, hs, ds_run, grads, ds0, err_word, st);
+        return launch_backward_d<__nv_bfloat16>(d, in, s0, dout, ds_final, hs, ds_run, grads,
+                                                ds0, err_word, st);
+    return launch_backward_d<float>(d, in, s0, dout, ds_final, hs, ds_run, grads, ds0,
+                                    err_word, st);
 }
 
 }  // namespace gdr

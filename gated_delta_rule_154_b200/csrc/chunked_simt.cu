@@ -24,9 +24,7 @@
 // the tensor-core kernel factorises instead.
 //
 // One CTA owns one (batch, head, block of DVB value columns) and walks the
-// chunks in order, keeping its [dk, DVB] slice of S in shared memory.  For the
-// backward pass it can also store the state at the start of every chunk
-// (h_out) and skip the outputs (o == nullptr).  The
+// chunks in order, keeping its [dk, DVB] slice of S in shared memory.  The
 // columns of S evolve independently (the transition multiplies from the
 // left), so value-column blocks need no communication.
 #include "common.cuh"
@@ -62,7 +60,7 @@ chunked_simt_kernel(int B, int T, int H,
                     int a_kind, int b_kind, int w_kind,
                     const float* __restrict__ s0, Tin* __restrict__ o,
                     float* __restrict__ s_final, const int* __restrict__ cu_seqlens,
-                    float* __restrict__ h_out, int* __restrict__ err_word) {
+                    int* __restrict__ err_word) {
     constexpr int NT = 256;
     constexpr int SL = NT / DVB;  // s-slices per column in the triangular solve
     static_assert(SL == 8 || SL == 16, "DVB must be 32 or 16");
@@ -101,17 +99,9 @@ chunked_simt_kernel(int B, int T, int H,
         Ss[x] = s0 ? s0[soff + (size_t)c * DV + j0 + j] : 0.0f;
     }
 
-    const int n_chunks = (len + C - 1) / C;
     for (int t0 = 0; t0 < len; t0 += C) {
         const int n = min(C, len - t0);
         __syncthreads();  // previous chunk finished with every buffer
-        if (h_out) {  // state at the chunk start: h_out[seq, h, chunk, dk, dv]
-            float* hc = h_out + ((size_t)bh * n_chunks + t0 / C) * DK * DV;
-            for (int x = tid; x < DK * DVB; x += NT) {
-                const int c = x / DVB, j = x % DVB;
-                hc[(size_t)c * DV + j0 + j] = Ss[x];
-            }
-        }
 
         // ---- load the chunk; padded tokens act as a = 1, k = q = v = 0
         for (int x = tid; x < C * DK; x += NT) {
@@ -224,7 +214,7 @@ chunked_simt_kernel(int B, int T, int H,
         __syncthreads();
 
         // ---- outputs: O = Qh S0 + A_qk U - A_qb E
-        for (int x = tid; o && x < C * DVB; x += NT) {
+        for (int x = tid; x < C * DVB; x += NT) {
             const int r = x / DVB, j = x % DVB;
             if (r >= n) continue;
             float acc = 0.f;
@@ -264,7 +254,6 @@ struct SimtArgs {
     float* s_final;
     const int* cu_seqlens;  // nullptr: batch rows as sequences
     int n_seqs;
-    float* h_out;           // nullptr: chunk-start states not stored
     int* err_word;
 };
 
@@ -280,8 +269,7 @@ static cudaError_t launch_simt_t(const gdr_desc& d, const SimtArgs& x, cudaStrea
     kern<<<grid, 256, smem, st>>>(d.B, d.T, d.H, (const Tin*)x.q, (const Tin*)x.k,
                                   (const Tin*)x.v, (const Tin*)x.a, (const Tin*)x.b,
                                   (const Tin*)x.w, (int)d.decay, (int)d.erase, (int)d.write,
-                                  x.s0, (Tin*)x.o, x.s_final, x.cu_seqlens, x.h_out,
-                                  x.err_word);
+                                  x.s0, (Tin*)x.o, x.s_final, x.cu_seqlens, x.err_word);
     return cudaGetLastError();
 }
 
@@ -307,9 +295,9 @@ static cudaError_t launch_simt_d(const gdr_desc& d, const SimtArgs& x, cudaStrea
 cudaError_t launch_chunked_simt(const gdr_desc& d, const void* q, const void* k,
                                 const void* v, const void* a, const void* b, const void* w,
                                 const float* s0, void* o, float* s_final,
-                                const int* cu_seqlens, int n_seqs, float* h_out,
-                                int* err_word, cudaStream_t st) {
-    const SimtArgs x{q, k, v, a, b, w, s0, o, s_final, cu_seqlens, n_seqs, h_out, err_word};
+                                const int* cu_seqlens, int n_seqs, int* err_word,
+                                cudaStream_t st) {
+    const SimtArgs x{q, k, v, a, b, w, s0, o, s_final, cu_seqlens, n_seqs, err_word};
     if (d.in_dtype == GDR_BF16) return launch_simt_d<__nv_bfloat16>(d, x, st);
     return launch_simt_d<float>(d, x, st);
 }

@@ -13,8 +13,8 @@ cudaError_t launch_decode(const gdr_desc& d, const void* q, const void* k, const
 cudaError_t launch_chunked_simt(const gdr_desc& d, const void* q, const void* k,
                                 const void* v, const void* a, const void* b, const void* w,
                                 const float* s0, void* o, float* s_final,
-                                const int* cu_seqlens, int n_seqs, float* h_out,
-                                int* err_word, cudaStream_t st);
+                                const int* cu_seqlens, int n_seqs, int* err_word,
+                                cudaStream_t st);
 bool chunked_tc_supports(const gdr_desc& d);
 size_t backward_workspace_bytes(const gdr_desc& d);
 cudaError_t launch_backward(const gdr_desc& d, const void* const* in, const float* s0,
@@ -147,7 +147,7 @@ gdr_status forward_impl(const gdr_desc* d, const int* cu_seqlens, int n_seqs, co
                                    n_seqs, st);
     } else if (simt_supports(*d)) {
         e = gdr::launch_chunked_simt(*d, q, k, v, a, b, w, s0, o, s_final, cu_seqlens, n_seqs,
-                                     nullptr, err, st);
+                                     err, st);
     } else {
         return GDR_ERR_UNSUPPORTED;
     }
