@@ -105,6 +105,14 @@ __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast
 __device__ __forceinline__ float dot4(float4 a, float4 b) {
     return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
 }
+// a . b added into two partial sums (even and odd components): two
+// independent FMA chains instead of one four-deep chain.
+__device__ __forceinline__ void dot4_2(float4 a, float4 b, float& e, float& o) {
+    e = fmaf(a.x, b.x, e);
+    o = fmaf(a.y, b.y, o);
+    e = fmaf(a.z, b.z, e);
+    o = fmaf(a.w, b.w, o);
+}
 __device__ __forceinline__ float comp(float4 v, int e) {
     return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
 }
@@ -230,6 +238,7 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
             for (int h2 = 0; h2 < 2; ++h2) {
                 const int s = cl + 16 * h2;
                 float qk = 0.f, qb = 0.f, kk = 0.f, kb = 0.f;
+                float qk2 = 0.f, qb2 = 0.f, kk2 = 0.f, kb2 = 0.f;
                 if (s <= r) {
 #pragma unroll 4
                     for (int c = 0; c < DK; c += 4) {
@@ -238,15 +247,19 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
                         kb4.x *= ig.x; kb4.y *= ig.y; kb4.z *= ig.z; kb4.w *= ig.w;
                         bb4.x *= ig.x; bb4.y *= ig.y; bb4.z *= ig.z; bb4.w *= ig.w;
                         const float4 kr = ld4(Kh + r * P + c);
-                        kk += dot4(kr, kb4);
-                        kb += dot4(kr, bb4);
+                        dot4_2(kr, kb4, kk, kk2);
+                        dot4_2(kr, bb4, kb, kb2);
                         if (with_q) {
                             const float4 qr = ld4(Qh + r * P + c);
-                            qk += dot4(qr, kb4);
-                            qb += dot4(qr, bb4);
+                            dot4_2(qr, kb4, qk, qk2);
+                            dot4_2(qr, bb4, qb, qb2);
                         }
                     }
                 }
+                kk += kk2;
+                kb += kb2;
+                qk += qk2;
+                qb += qb2;
                 Akk[r * CP + s] = s < r ? kk : 0.f;
                 Akb[r * CP + s] = s < r ? kb : 0.f;
                 if (with_q) {
@@ -311,9 +324,10 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
             __syncthreads();
             {  // Y = Kh S0 + A_kk U
                 const int r = rr, j = cl;
-                float y = 0.f;
+                float y = 0.f, y2 = 0.f;
 #pragma unroll 4
-                for (int c = 0; c < DK; c += 4) y += dot4(ld4(Kh + r * P + c), ld4(S0T + j * P + c));
+                for (int c = 0; c < DK; c += 4) dot4_2(ld4(Kh + r * P + c), ld4(S0T + j * P + c), y, y2);
+                y += y2;
                 for (int s = 0; s < r; ++s) y = fmaf(Akk[r * CP + s], Ub[s * UP + j], y);
                 Yb[r * UP + j] = y;
             }
@@ -394,13 +408,15 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
                 const int j = cl, ra = r2, rb = r2 + 16;
                 const float* X = task == 0 ? Kh : Bt;
                 const float* ST = task == 0 ? S0T : dST;
-                float o0 = 0.f, o1 = 0.f;
+                float o0 = 0.f, o1 = 0.f, p0 = 0.f, p1 = 0.f;
 #pragma unroll 4
                 for (int c = 0; c < DK; c += 4) {
                     const float4 s4 = ld4(ST + j * P + c);
-                    o0 += dot4(ld4(X + ra * P + c), s4);
-                    o1 += dot4(ld4(X + rb * P + c), s4);
+                    dot4_2(ld4(X + ra * P + c), s4, o0, p0);
+                    dot4_2(ld4(X + rb * P + c), s4, o1, p1);
                 }
+                o0 += p0;
+                o1 += p1;
                 if (task == 0) {
                     for (int s = 0; s < ra; ++s) o0 = fmaf(Akk[ra * CP + s], Ub[s * UP + j], o0);
                     for (int s = 0; s < rb; ++s) o1 = fmaf(Akk[rb * CP + s], Ub[s * UP + j], o1);
@@ -434,13 +450,15 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
             // B4a: dU -> dv, dw (task 0);  dA (task 1)
             if (task == 0) {
                 const int j = cl, ra = r2, rb = r2 + 16;
-                float o0 = 0.f, o1 = 0.f;
+                float o0 = 0.f, o1 = 0.f, p0 = 0.f, p1 = 0.f;
 #pragma unroll 4
                 for (int c = 0; c < DK; c += 4) {
                     const float4 d4 = ld4(dST + j * P + c);
-                    o0 += dot4(ld4(Kt + ra * P + c), d4);
-                    o1 += dot4(ld4(Kt + rb * P + c), d4);
+                    dot4_2(ld4(Kt + ra * P + c), d4, o0, p0);
+                    dot4_2(ld4(Kt + rb * P + c), d4, o1, p1);
                 }
+                o0 += p0;
+                o1 += p1;
                 for (int s = ra; s < C; ++s) o0 = fmaf(Aqk[s * CP + ra], dOb[s * UP + j], o0);
                 for (int s = rb; s < C; ++s) o1 = fmaf(Aqk[s * CP + rb], dOb[s * UP + j], o1);
                 for (int s = ra + 1; s < C; ++s) o0 = fmaf(Akk[s * CP + ra], dYb[s * UP + j], o0);
