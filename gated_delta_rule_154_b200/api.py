@@ -133,42 +133,72 @@ def backward_workspace_size(desc: _lib.GdrDesc) -> int:
 def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
              a: Optional[torch.Tensor], b: Optional[torch.Tensor], w: Optional[torch.Tensor],
              s0: Optional[torch.Tensor], d_o: torch.Tensor,
-             ds_final: Optional[torch.Tensor] = None, *, want_ds0: bool = True,
+             ds_final: Optional[torch.Tensor] = None, *,
+             cu_seqlens: Optional[torch.Tensor] = None, fg2: bool = False,
+             want_ds0: bool = True, out: Optional[dict] = None,
              workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
     """Gradients of  L = sum_t <o_t, d_o_t> + <S_T, ds_final>  for the prefill
     of (q, k, v, a, b, w, s0).  Returns a dict with dq, dk, dv (input dtype),
     da, db, dw (shape and dtype of a, b, w; None for an absent gate) and ds0
-    (float32 [B, H, dk, dv], or None with want_ds0=False).  With b and w the
-    same tensor (shared beta) its gradient is db + dw."""
+    (float32, or None with want_ds0=False).  With b and w the same tensor
+    (shared beta) its gradient is db + dw.  fg2=True: b and w are FG^2-GDN
+    learning rates beta^k, beta^v and db, dw their gradients.  cu_seqlens
+    (int32 [N + 1] on the device): packed sequences in q [1, T, H, dk] as in
+    forward_varlen; s0, ds_final and ds0 are then [N, H, dk, dv] and tokens
+    outside every sequence keep whatever `out` held.  `out` may supply any of
+    the gradient tensors."""
     if q.dtype not in _DT:
         raise ValueError("q must be float32 or bfloat16")
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dev, dt = q.device, q.dtype
+    N = B
+    if cu_seqlens is not None:
+        if B != 1:
+            raise ValueError("packed sequences take q as [1, T, H, dk]")
+        _check(cu_seqlens, "cu_seqlens", torch.int32, dev, [tuple(cu_seqlens.shape)])
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise ValueError("cu_seqlens must be int32 [N + 1], N >= 1")
+        N = cu_seqlens.numel() - 1
     _check(q, "q", dt, dev, [(B, T, H, dk)])
     _check(k, "k", dt, dev, [(B, T, H, dk)])
     _check(v, "v", dt, dev, [(B, T, H, dv)])
     _check(a, "a", dt, dev, [(B, T, H, dk), (B, T, H)])
     _check(b, "b", dt, dev, [(B, T, H, dk), (B, T, H)])
     _check(w, "w", dt, dev, [(B, T, H, dv), (B, T, H)])
-    _check(s0, "s0", torch.float32, dev, [(B, H, dk, dv)])
+    _check(s0, "s0", torch.float32, dev, [(N, H, dk, dv)])
     _check(d_o, "d_o", dt, dev, [(B, T, H, dv)])
-    _check(ds_final, "ds_final", torch.float32, dev, [(B, H, dk, dv)])
+    _check(ds_final, "ds_final", torch.float32, dev, [(N, H, dk, dv)])
+    if fg2 and (b is None or w is None or b.dim() != 4 or w.dim() != 4):
+        raise ValueError("fg2 needs vector beta^k [B, T, H, dk] and beta^v [B, T, H, dv]")
     like = lambda t: None if t is None else torch.empty_like(t)
     g = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
          "da": like(a), "db": like(b), "dw": like(w),
-         "ds0": torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if want_ds0 else None}
-    desc = desc_for(q, v, a, b, w, 32)
-    need = _lib.backward_workspace_size(desc)
+         "ds0": torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev) if want_ds0 else None}
+    for name, t in (out or {}).items():
+        if name not in g or g[name] is None:
+            raise ValueError("unexpected output %s" % name)
+        ref = g[name]
+        _check(t, name, ref.dtype, dev, [tuple(ref.shape)])
+        g[name] = t
+    desc = desc_for(q, v, a, b, w, 32, fg2=fg2)
+    need = (_lib.backward_varlen_workspace_size(desc, N) if cu_seqlens is not None
+            else _lib.backward_workspace_size(desc))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size()
-    st = _lib.backward_chunked(desc, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(w),
-                               _ptr(s0), _ptr(d_o), _ptr(ds_final), _ptr(g["dq"]), _ptr(g["dk"]),
-                               _ptr(g["dv"]), _ptr(g["da"]), _ptr(g["db"]), _ptr(g["dw"]),
-                               _ptr(g["ds0"]), _ptr(workspace), ws_bytes, _stream_handle(stream))
+    grads = [_ptr(g[n]) for n in ("dq", "dk", "dv", "da", "db", "dw", "ds0")]
+    ins = [_ptr(x) for x in (q, k, v, a, b, w, s0, d_o, ds_final)]
+    if cu_seqlens is not None:
+        st = _lib.backward_varlen(desc, _ptr(cu_seqlens), N, *ins, *grads, _ptr(workspace),
+                                  ws_bytes, _stream_handle(stream))
+        what = "gdr_backward_varlen"
+    else:
+        st = _lib.backward_chunked(desc, *ins, *grads, _ptr(workspace), ws_bytes,
+                                   _stream_handle(stream))
+        what = "gdr_backward_chunked"
     if st != _lib.OK:
-        raise _lib.GdrError(st, "gdr_backward_chunked")
+        raise _lib.GdrError(st, what)
     return g
 
 

@@ -36,6 +36,15 @@
 // a chunk multiplies to at least e^-80; a chunk below that is reported
 // (GDR_ERR_RANGE) like the tensor-core forward's range check.
 //
+// FG^2-GDN learning rates (gate kind FG2; FG^2-GDN page, section 2): the key
+// used is sqrt(beta^k) k with erase gate 1, the write gate sqrt(beta^v).  The
+// gradients above are taken for that key and write gate, then carried
+// through the square roots: dk = sqrt(beta^k) dk~, dbeta^k = k dk~ /
+// (2 sqrt(beta^k)), dbeta^v = v dU / (2 sqrt(beta^v)) (beta > 0).
+//
+// Packed sequences (cu_seqlens): CTA (sequence, head) takes its sequence's
+// tokens; its chunk-start states follow those of the sequences before it.
+//
 // One launch, one CTA per (batch, head).  A forward sweep first stores the
 // state at the start of every chunk in the workspace (the chunk form above
 // without its outputs); the reverse sweep then walks the chunks backwards,
@@ -131,7 +140,8 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float a, float b, float
 
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(BW_NT, 1)
-backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__ k,
+backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
+                const Tin* __restrict__ q, const Tin* __restrict__ k,
                 const Tin* __restrict__ v, const Tin* __restrict__ a,
                 const Tin* __restrict__ b, const Tin* __restrict__ w, int a_kind, int b_kind,
                 int w_kind, const Tin* __restrict__ dout, const float* __restrict__ s0,
@@ -179,16 +189,38 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
 
     const int tid = threadIdx.x;
     const int bh = blockIdx.x;
-    const int bi = bh / H, hi = bh % H;
+    const int seq = bh / H, hi = bh % H;
+    // this CTA's tokens: [tb, tb + len) of batch row bi.  Packed sequences must
+    // be ordered (cu non-decreasing from cu[0] >= 0 up to this one): that bounds
+    // the chunk-state offset below by the workspace size; otherwise the
+    // sequence is reported and skipped.
+    int bi, tb, len;
+    long long chunk_base = 0;  // chunk-start states of the sequences before this one
+    bool ok = seq_range(cu_seqlens, seq, T, bi, tb, len);
+    if (cu_seqlens) {
+        ok = ok && cu_seqlens[0] >= 0;
+        for (int m = 0; ok && m < seq; ++m) {
+            const int l = cu_seqlens[m + 1] - cu_seqlens[m];
+            ok = l >= 0;
+            chunk_base += (l + BW_C - 1) / BW_C;
+        }
+    } else {
+        chunk_base = (long long)seq * ((T + BW_C - 1) / BW_C);
+    }
+    if (!ok) {
+        if (tid == 0 && hi == 0) atomicOr(err_word, kErrIndex);
+        return;
+    }
     const int rr = tid >> 4;   // row in [C][*] tiles (one row per thread)
     const int cl = tid & 15;   // lane in the row: value column, or key channels 4 cl + 64 g
     const int task = tid >> 8; // two half-CTA tasks side by side in stage B
     const int t2 = tid & 255;
     const int r2 = t2 >> 4;    // rows r2 and r2 + 16 of a half-CTA task
-    const int n_chunks = (T + C - 1) / C;
+    const int n_chunks = (len + C - 1) / C;
     const size_t soff = (size_t)bh * DK * DV;
-    float* hbase = hs + (size_t)bh * n_chunks * DK * DV;
-    auto tok_of = [&](int t) { return ((long long)bi * T + t) * H + hi; };
+    float* hbase = hs + ((size_t)chunk_base * H + (size_t)hi * n_chunks) * DK * DV;
+    auto tok_of = [&](int t) { return ((long long)bi * T + tb + t) * H + hi; };
+    const bool fg2_b = b_kind == GDR_GATE_FG2;
 
     // ---------------- stage A: gated operands, grams (all four when with_q), T
     auto stage_a = [&](int t0, int n, bool with_q) {
@@ -199,7 +231,8 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
                 const long long tok = tok_of(t0 + r), base = tok * DK;
                 if (with_q) qv = to_f32(q[base + c]);
                 kv = to_f32(k[base + c]);
-                bv = gate_value(b, b_kind, tok, base, c);
+                bv = gate_value(b, b_kind, tok, base, c);  // FG2: sqrt(beta^k)
+                if (fg2_b) kv *= bv;                       // key sqrt(beta^k) k, erase gate 1
                 av = gate_value(a, a_kind, tok, base, c);
                 gv = a_kind == GDR_GATE_ONE ? 0.f : safe_log_decay(av);
             }
@@ -229,7 +262,7 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
             Qh[r * P + c] *= eg;
             Kh[r * P + c] = kv * eg;
             Kt[r * P + c] = kv * et;
-            Bt[r * P + c] = Bs[r * P + c] * kv * et;
+            Bt[r * P + c] = (fg2_b ? 1.f : Bs[r * P + c]) * kv * et;
         }
         __syncthreads();
         {
@@ -362,7 +395,7 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
     // ================= reverse sweep
     for (int ci = n_chunks - 1; ci >= 0; --ci) {
         const int t0 = ci * C;
-        const int n = min(C, T - t0);
+        const int n = min(C, len - t0);
         __syncthreads();  // previous chunk done with every buffer; ds_run, h visible
         stage_a(t0, n, true);
 
@@ -473,6 +506,8 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
                         const float vx = to_f32(v[base + j0 + j]);
                         dv[base + j0 + j] = from_f32<Tin>(ww * du);
                         if (w_kind == GDR_GATE_VECTOR) dw[base + j0 + j] = from_f32<Tin>(vx * du);
+                        if (w_kind == GDR_GATE_FG2)  // through w = sqrt(beta^v)
+                            dw[base + j0 + j] = from_f32<Tin>(vx * du / (2.f * ww));
                         if (h2) dw_r1 = fmaf(vx, du, dw_r1);
                         else dw_r0 = fmaf(vx, du, dw_r0);
                     }
@@ -648,8 +683,14 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
                     const float eg = __expf(gr), et = __expf(gc - gr);
                     const float kt = Kt[r * P + c + x], bt = Bt[r * P + c + x];
                     gq[x] = eg * xq[i];
-                    gk[x] = fmaf(eg, xk[i], et * (yk[i] + Bs[r * P + c + x] * yb[i]));
+                    const float bg = fg2_b ? 1.f : Bs[r * P + c + x];
+                    gk[x] = fmaf(eg, xk[i], et * (yk[i] + bg * yb[i]));
                     gb[x] = kt * yb[i];
+                    if (fg2_b) {  // through k~ = sqrt(beta^k) k
+                        const float sb = Bs[r * P + c + x];
+                        gb[x] = gk[x] * to_f32(k[base + c + x]) / (2.f * sb);
+                        gk[x] *= sb;
+                    }
                     db_row += gb[x];
                     gg[x] = Qh[r * P + c + x] * xq[i] + Kh[r * P + c + x] * xk[i] - kt * yk[i] -
                             bt * yb[i];
@@ -660,7 +701,8 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
                 if (r < n) {
                     store4(dq + base + c, gq[0], gq[1], gq[2], gq[3]);
                     store4(dk + base + c, gk[0], gk[1], gk[2], gk[3]);
-                    if (b_kind == GDR_GATE_VECTOR) store4(db + base + c, gb[0], gb[1], gb[2], gb[3]);
+                    if (b_kind == GDR_GATE_VECTOR || fg2_b)
+                        store4(db + base + c, gb[0], gb[1], gb[2], gb[3]);
                 }
             }
             if (b_kind == GDR_GATE_SCALAR) {
@@ -702,7 +744,8 @@ backward_kernel(int T, int H, const Tin* __restrict__ q, const Tin* __restrict__
 }
 
 template <typename Tin, int DK, int DV>
-static cudaError_t launch_backward_t(const gdr_desc& d, const void* const* in, const float* s0,
+static cudaError_t launch_backward_t(const gdr_desc& d, const int* cu_seqlens, int n_seqs,
+                                     const void* const* in, const float* s0,
                                      const void* dout, const float* ds_final, float* hs,
                                      float* ds_run, void* const* grads, float* ds0,
                                      int* err_word, cudaStream_t st) {
@@ -711,8 +754,9 @@ static cudaError_t launch_backward_t(const gdr_desc& d, const void* const* in, c
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)((long long)d.B * d.H), BW_NT, smem, st>>>(
-        d.T, d.H, (const Tin*)in[0], (const Tin*)in[1], (const Tin*)in[2], (const Tin*)in[3],
+    const long long nseq = cu_seqlens ? n_seqs : d.B;
+    kern<<<(unsigned)(nseq * d.H), BW_NT, smem, st>>>(
+        d.T, d.H, cu_seqlens, (const Tin*)in[0], (const Tin*)in[1], (const Tin*)in[2], (const Tin*)in[3],
         (const Tin*)in[4], (const Tin*)in[5], (int)d.decay, (int)d.erase, (int)d.write,
         (const Tin*)dout, s0, ds_final, hs, ds_run, (Tin*)grads[0], (Tin*)grads[1],
         (Tin*)grads[2], (Tin*)grads[3], (Tin*)grads[4], (Tin*)grads[5], ds0, err_word);
@@ -720,14 +764,15 @@ static cudaError_t launch_backward_t(const gdr_desc& d, const void* const* in, c
 }
 
 template <typename Tin>
-static cudaError_t launch_backward_d(const gdr_desc& d, const void* const* in, const float* s0,
+static cudaError_t launch_backward_d(const gdr_desc& d, const int* cu_seqlens, int n_seqs,
+                                     const void* const* in, const float* s0,
                                      const void* dout, const float* ds_final, float* hs,
                                      float* ds_run, void* const* grads, float* ds0,
                                      int* err_word, cudaStream_t st) {
 #define GDR_BWD(DK_, DV_)                                                                  \
     if (d.dk == DK_ && d.dv == DV_)                                                        \
-        return launch_backward_t<Tin, DK_, DV_>(d, in, s0, dout, ds_final, hs, ds_run, grads, \
-                                                ds0, err_word, st);
+        return launch_backward_t<Tin, DK_, DV_>(d, cu_seqlens, n_seqs, in, s0, dout, ds_final, \
+                                                hs, ds_run, grads, ds0, err_word, st);
     GDR_BWD(128, 128)
     GDR_BWD(128, 64)
     GDR_BWD(64, 128)
@@ -736,26 +781,34 @@ static cudaError_t launch_backward_d(const gdr_desc& d, const void* const* in, c
     return cudaErrorInvalidValue;
 }
 
-size_t backward_workspace_bytes(const gdr_desc& d) {
-    const size_t heads = (size_t)d.B * d.H;
+// Chunk-start states: B sequences of ceil(T / 32) chunks each, or packed
+// sequences with at most ceil(T / 32) + n_seqs chunks in all (their lengths
+// sum to at most T), for each of the H heads.
+static size_t state_matrices(const gdr_desc& d, bool packed, int n_seqs) {
+    const size_t nc = ((size_t)d.T + BW_C - 1) / BW_C;
+    return packed ? (nc + (size_t)n_seqs) * d.H : nc * d.B * d.H;
+}
+
+// n_seqs > 0: packed sequences; 0: the B batch rows.
+size_t backward_workspace_bytes(const gdr_desc& d, int n_seqs) {
     const size_t mat = (size_t)d.dk * d.dv * sizeof(float);
-    const size_t n_chunks = ((size_t)d.T + BW_C - 1) / BW_C;
-    return heads * mat * (n_chunks + 1);  // chunk-start states, then the running dS
+    const size_t nseq = n_seqs > 0 ? (size_t)n_seqs : (size_t)d.B;
+    // chunk-start states, then the running dS of every (sequence, head)
+    return mat * (state_matrices(d, n_seqs > 0, n_seqs) + nseq * d.H);
 }
 
 // in = {q, k, v, a, b, w}; grads = {dq, dk, dv, da, db, dw}.
-cudaError_t launch_backward(const gdr_desc& d, const void* const* in, const float* s0,
-                            const void* dout, const float* ds_final, void* const* grads,
-                            float* ds0, void* workspace, int* err_word, cudaStream_t st) {
-    const size_t heads = (size_t)d.B * d.H;
-    const size_t n_chunks = ((size_t)d.T + BW_C - 1) / BW_C;
+cudaError_t launch_backward(const gdr_desc& d, const int* cu_seqlens, int n_seqs,
+                            const void* const* in, const float* s0, const void* dout,
+                            const float* ds_final, void* const* grads, float* ds0,
+                            void* workspace, int* err_word, cudaStream_t st) {
     float* hs = static_cast<float*>(workspace);
-    float* ds_run = hs + heads * n_chunks * d.dk * d.dv;
+    float* ds_run = hs + state_matrices(d, cu_seqlens != nullptr, n_seqs) * d.dk * d.dv;
     if (d.in_dtype == GDR_BF16)
-        return launch_backward_d<__nv_bfloat16>(d, in, s0, dout, ds_final, hs, ds_run, grads,
-                                                ds0, err_word, st);
-    return launch_backward_d<float>(d, in, s0, dout, ds_final, hs, ds_run, grads, ds0,
-                                    err_word, st);
+        return launch_backward_d<__nv_bfloat16>(d, cu_seqlens, n_seqs, in, s0, dout, ds_final,
+                                                hs, ds_run, grads, ds0, err_word, st);
+    return launch_backward_d<float>(d, cu_seqlens, n_seqs, in, s0, dout, ds_final, hs, ds_run,
+                                    grads, ds0, err_word, st);
 }
 
 }  // namespace gdr

@@ -16,10 +16,11 @@ cudaError_t launch_chunked_simt(const gdr_desc& d, const void* q, const void* k,
                                 const int* cu_seqlens, int n_seqs, int* err_word,
                                 cudaStream_t st);
 bool chunked_tc_supports(const gdr_desc& d);
-size_t backward_workspace_bytes(const gdr_desc& d);
-cudaError_t launch_backward(const gdr_desc& d, const void* const* in, const float* s0,
-                            const void* dout, const float* ds_final, void* const* grads,
-                            float* ds0, void* workspace, int* err_word, cudaStream_t st);
+size_t backward_workspace_bytes(const gdr_desc& d, int n_seqs);
+cudaError_t launch_backward(const gdr_desc& d, const int* cu_seqlens, int n_seqs,
+                            const void* const* in, const float* s0, const void* dout,
+                            const float* ds_final, void* const* grads, float* ds0,
+                            void* workspace, int* err_word, cudaStream_t st);
 cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, const void* v,
                               const void* a, const void* b, const void* w, const float* s0,
                               void* o, float* s_final, int* err_word, bool skip_signal,
@@ -211,24 +212,30 @@ gdr_status gdr_decode_step_paged(const gdr_desc* d, const void* q, const void* k
 
 size_t gdr_backward_workspace_size(const gdr_desc* d) {
     if (check_desc(d) != GDR_OK) return 0;
-    return gdr::backward_workspace_bytes(*d);
+    return gdr::backward_workspace_bytes(*d, 0);
 }
 
-gdr_status gdr_backward_chunked(const gdr_desc* d, const void* q, const void* k, const void* v,
-                                const void* a, const void* b, const void* w, const float* s0,
-                                const void* d_o, const float* ds_final, void* dq, void* dk,
-                                void* dv, void* da, void* db, void* dw, float* ds0,
-                                void* workspace, size_t ws_bytes, gdr_stream_t stream) {
+size_t gdr_backward_varlen_workspace_size(const gdr_desc* d, int n_seqs) {
+    if (check_desc(d) != GDR_OK || n_seqs < 1) return 0;
+    return gdr::backward_workspace_bytes(*d, n_seqs);
+}
+
+namespace {
+gdr_status backward_impl(const gdr_desc* d, const int* cu_seqlens, int n_seqs, const void* q,
+                         const void* k, const void* v, const void* a, const void* b,
+                         const void* w, const float* s0, const void* d_o,
+                         const float* ds_final, void* dq, void* dk, void* dv, void* da,
+                         void* db, void* dw, float* ds0, void* workspace, size_t ws_bytes,
+                         gdr_stream_t stream) {
     gdr_status s = check_desc(d);
     if (s != GDR_OK) return s;
-    if (d->erase == GDR_GATE_FG2 || d->write == GDR_GATE_FG2) return GDR_ERR_UNSUPPORTED;
     const bool have_tokens = d->T > 0;
     if ((s = check_inputs(d, have_tokens, q, k, v, a, b, w, d_o)) != GDR_OK) return s;
     if ((s = check_inputs(d, have_tokens, dq, dk, dv, da, db, dw, d_o)) != GDR_OK) return s;
     if ((s = check_ptr(s0, false)) != GDR_OK) return s;
     if ((s = check_ptr(ds_final, false)) != GDR_OK) return s;
     if ((s = check_ptr(ds0, false)) != GDR_OK) return s;
-    const size_t need = gdr::backward_workspace_bytes(*d);
+    const size_t need = gdr::backward_workspace_bytes(*d, cu_seqlens ? n_seqs : 0);
     if (workspace == nullptr || ws_bytes < need) return GDR_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GDR_ERR_INVALID_ARG;
     if (ds0 == nullptr && !have_tokens) return GDR_OK;  // nothing to write
@@ -237,9 +244,34 @@ gdr_status gdr_backward_chunked(const gdr_desc* d, const void* q, const void* k,
     if (error_word(&err) != cudaSuccess) return GDR_ERR_CUDA;
     const void* in[6] = {q, k, v, a, b, w};
     void* grads[6] = {dq, dk, dv, da, db, dw};
-    cudaError_t e = gdr::launch_backward(*d, in, s0, d_o, ds_final, grads, ds0, workspace, err,
+    cudaError_t e = gdr::launch_backward(*d, cu_seqlens, n_seqs, in, s0, d_o, ds_final, grads,
+                                         ds0, workspace, err,
                                          reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+}  // namespace
+
+gdr_status gdr_backward_chunked(const gdr_desc* d, const void* q, const void* k, const void* v,
+                                const void* a, const void* b, const void* w, const float* s0,
+                                const void* d_o, const float* ds_final, void* dq, void* dk,
+                                void* dv, void* da, void* db, void* dw, float* ds0,
+                                void* workspace, size_t ws_bytes, gdr_stream_t stream) {
+    return backward_impl(d, nullptr, 0, q, k, v, a, b, w, s0, d_o, ds_final, dq, dk, dv, da, db,
+                         dw, ds0, workspace, ws_bytes, stream);
+}
+
+gdr_status gdr_backward_varlen(const gdr_desc* d, const int* cu_seqlens, int n_seqs,
+                               const void* q, const void* k, const void* v, const void* a,
+                               const void* b, const void* w, const float* s0, const void* d_o,
+                               const float* ds_final, void* dq, void* dk, void* dv, void* da,
+                               void* db, void* dw, float* ds0, void* workspace,
+                               size_t ws_bytes, gdr_stream_t stream) {
+    if (!d || d->B != 1 || n_seqs < 1) return GDR_ERR_INVALID_ARG;
+    if (cu_seqlens == nullptr || reinterpret_cast<uintptr_t>(cu_seqlens) % 4 != 0)
+        return GDR_ERR_INVALID_ARG;
+    if ((long long)n_seqs * d->H > 0x7fffffffLL) return GDR_ERR_INVALID_ARG;
+    return backward_impl(d, cu_seqlens, n_seqs, q, k, v, a, b, w, s0, d_o, ds_final, dq, dk, dv,
+                         da, db, dw, ds0, workspace, ws_bytes, stream);
 }
 
 void gdr_test_skip_signal(int enable) { g_test_skip_signal.store(enable ? 1 : 0); }

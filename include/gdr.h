@@ -207,14 +207,16 @@ size_t gdr_backward_workspace_size(const gdr_desc *desc);
  *   da, db, dw  in the shape and dtype of a, b, w (scalar gates: one value
  *            per token and head, the sum over channels); required when the
  *            gate is not ONE, ignored when it is.  With b and w the same
- *            tensor (shared beta) its gradient is db + dw.
+ *            tensor (shared beta) its gradient is db + dw.  With
+ *            GDR_GATE_FG2 (FG^2-GDN learning rates, beta > 0) db and dw are
+ *            the gradients on beta^k and beta^v, carried through the square
+ *            roots the forward takes.
  *   ds0      [B, H, dk, dv] float32, or NULL (not written); may equal
  *            ds_final
  *   workspace, ws_bytes  device scratch of gdr_backward_workspace_size(desc)
  *
  * Outputs must not overlap the inputs.  Supported: dk, dv in {64, 128},
- * float32 or bf16 inputs, gates ONE / SCALAR / VECTOR; GDR_GATE_FG2 returns
- * GDR_ERR_UNSUPPORTED.  Decay range: every channel's decay, multiplied over
+ * float32 or bf16 inputs, every gate kind.  Decay range: every channel's decay, multiplied over
  * each 32-token chunk, must stay at or above exp(-80); otherwise the device
  * error word reports GDR_ERR_RANGE and the gradients are undefined.
  */
@@ -225,10 +227,35 @@ gdr_status gdr_backward_chunked(const gdr_desc *desc, const void *q, const void 
                                 void *da, void *db, void *dw, float *ds0, void *workspace,
                                 size_t ws_bytes, gdr_stream_t stream);
 
+/* Bytes of device workspace gdr_backward_varlen needs for `desc` and n_seqs
+ * packed sequences: H * dk * dv * 4 * (ceil(T / 32) + 2 * n_seqs); 0 if desc
+ * is invalid or n_seqs < 1.  Pure host function, no CUDA call. */
+size_t gdr_backward_varlen_workspace_size(const gdr_desc *desc, int n_seqs);
+
+/*
+ * The backward over packed sequences, as gdr_forward_varlen packs them:
+ * desc->B must be 1, sequence n occupies tokens [cu_seqlens[n],
+ * cu_seqlens[n + 1]) of the [1, T, H, *] tensors, and s0, ds_final and ds0
+ * are [n_seqs, H, dk, dv].  cu_seqlens must be non-decreasing from
+ * cu_seqlens[0] >= 0 with cu_seqlens[n_seqs] <= T; a sequence for which that
+ * does not hold up to its own end is skipped (its gradients are not written)
+ * and recorded in the device error word (GDR_ERR_INVALID_ARG from
+ * gdr_last_device_error).  Gradients of tokens outside every sequence are not
+ * written.  workspace: gdr_backward_varlen_workspace_size(desc, n_seqs)
+ * bytes.  Everything else as gdr_backward_chunked.
+ */
+gdr_status gdr_backward_varlen(const gdr_desc *desc, const int *cu_seqlens, int n_seqs,
+                               const void *q, const void *k, const void *v, const void *a,
+                               const void *b, const void *w, const float *s0,
+                               const void *d_o, const float *ds_final, void *dq, void *dk,
+                               void *dv, void *da, void *db, void *dw, float *ds0,
+                               void *workspace, size_t ws_bytes, gdr_stream_t stream);
+
 /* Synchronises `stream`, returns the status recorded on the device since the
  * previous call (GDR_OK if none) and clears it: GDR_ERR_TIMEOUT (a bounded
  * wait ran out), GDR_ERR_INVALID_ARG (a paged decode slot or a packed
- * sequence range out of bounds) or
+ * sequence range out of bounds, or unordered packed sequences in the
+ * backward) or
  * GDR_ERR_RANGE (decay range), in that order of precedence.  GDR_ERR_CUDA if
  * the synchronisation itself failed. */
 gdr_status gdr_last_device_error(gdr_stream_t stream);

@@ -186,7 +186,35 @@ def test_backward_argument_checks(lib):
     assert _bwd(d, ws=0) == _lib.ERR_WORKSPACE
     assert _bwd(d, ws_bytes=_lib.backward_workspace_size(d) - 1) == _lib.ERR_WORKSPACE
     assert _bwd(d, ws=P + 8) == _lib.ERR_INVALID_ARG
-    assert _bwd(_desc(erase=_lib.GATE_FG2, write=_lib.GATE_FG2)) == _lib.ERR_UNSUPPORTED
+    # FG^2-GDN learning rates are accepted (no tokens, no dS0: validated, nothing launched)
+    fg2 = _desc(T=0, erase=_lib.GATE_FG2, write=_lib.GATE_FG2)
+    assert _bwd(fg2) == _lib.OK
     # absent gates need neither the gate nor its gradient
     one = _desc(T=0, decay=_lib.GATE_ONE, erase=_lib.GATE_ONE, write=_lib.GATE_ONE)
     assert _bwd(one, a=0, b=0, w=0, da=0, db=0, dw=0) == _lib.OK  # nothing to write
+
+
+def test_backward_varlen_workspace_and_checks(lib):
+    d = _desc(B=1, T=100, H=4, dk=128, dv=64)
+    mat = 128 * 64 * 4
+    # at most ceil(T / 32) + n_seqs chunk-start states per head, then n_seqs running dS
+    assert _lib.backward_varlen_workspace_size(d, 3) == 4 * mat * (4 + 3 + 3)
+    assert _lib.backward_varlen_workspace_size(d, 0) == 0
+    assert _lib.backward_varlen_workspace_size(_desc(dk=96), 2) == 0
+    need = _lib.backward_varlen_workspace_size(d, 3)
+    args = lambda **kw: dict(dict(q=P, k=P, v=P, a=P, b=P, w=P, s0=0, d_o=P, ds_final=0, dq=P,
+                                  dk=P, dv=P, da=P, db=P, dw=P, ds0=0, ws=P, ws_bytes=need), **kw)
+    def call(desc, cu, n, **kw):
+        x = args(**kw)
+        return _lib.backward_varlen(desc, cu, n, x["q"], x["k"], x["v"], x["a"], x["b"], x["w"],
+                                    x["s0"], x["d_o"], x["ds_final"], x["dq"], x["dk"], x["dv"],
+                                    x["da"], x["db"], x["dw"], x["ds0"], x["ws"], x["ws_bytes"], 0)
+    assert call(d, 0, 3) == _lib.ERR_INVALID_ARG            # no cu_seqlens
+    assert call(d, P + 2, 3) == _lib.ERR_INVALID_ARG        # misaligned cu_seqlens
+    assert call(d, P, 0) == _lib.ERR_INVALID_ARG            # no sequence
+    assert call(_desc(B=2), P, 3) == _lib.ERR_INVALID_ARG   # packed sequences need B = 1
+    assert call(d, P, 3, ws_bytes=need - 1) == _lib.ERR_WORKSPACE
+    assert call(d, P, 3, dq=0) == _lib.ERR_INVALID_ARG
+    # no tokens and no dS0: validated, nothing launched
+    assert call(_desc(B=1, T=0), P, 2, ws_bytes=_lib.backward_varlen_workspace_size(
+        _desc(B=1, T=0), 2)) == _lib.OK

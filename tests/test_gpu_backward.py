@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import oracle
-from gated_delta_rule_154_b200 import api
+from gated_delta_rule_154_b200 import _lib, api
 from gated_delta_rule_154_b200 import workload as W
 from gpu_helpers import TOL, inputs_to_dev, rel_err, to_dev, to_host
 
@@ -164,3 +164,96 @@ def test_full_size_sampled_heads():
             r = ref[name][0, i] if name == "ds0" else ref[name][0, :, i]
             e = rel_err(to_host(x), r)
             assert e <= TOL["bf16"], (bi, hi, name, e)
+
+
+@pytest.mark.parametrize("plus", [False, True])
+@pytest.mark.parametrize("dtype,d,T", [("bf16", 128, 97), ("f32", 64, 70)])
+def test_fg2_learning_rates(dtype, d, T, plus):
+    """FG^2-GDN (one beta for key and value) and FG^2-GDN+ (beta^k, beta^v):
+    the oracle runs the mapped rule (key sqrt(beta^k) k, erase gate 1, write
+    gate sqrt(beta^v); FG^2-GDN page, section 2) and its gradients are
+    carried back through the square roots by the chain rule."""
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=2, H=2, T=T, dk=d, dv=d, dtype=dtype)
+    inp = W.make_prefill(wl, seed=T + d)
+    up = W.make_upstream(wl, seed=T + d)
+    dev = {x: to_dev(inp[x], dtype) for x in ("q", "k", "v", "a", "b", "w")}
+    beta_v_dev = dev["w"] if plus else dev["b"]
+    g = api.backward(dev["q"], dev["k"], dev["v"], dev["a"], dev["b"], beta_v_dev,
+                     to_dev(inp["s0"], "f32"), to_dev(up["do"], dtype), to_dev(up["dsT"], "f32"),
+                     fg2=True)
+    torch.cuda.synchronize()
+    assert api.last_device_error() == 0
+    f = lambda key: W.as_f32(inp[key], dtype).astype(np.float64)
+    kk, beta_k = f("k"), f("b")
+    beta_v = f("w") if plus else beta_k
+    sk, sv = np.sqrt(beta_k), np.sqrt(beta_v)
+    m = oracle.backward(W.as_f32(inp["q"], dtype), (sk * kk).astype(np.float32),
+                        W.as_f32(inp["v"], dtype), W.as_f32(inp["a"], dtype),
+                        np.ones(beta_k.shape, np.float32), sv.astype(np.float32), inp["s0"],
+                        W.as_f32(up["do"], dtype), up["dsT"])
+    ref = {"dq": m["dq"], "dk": sk * m["dk"], "dv": m["dv"], "da": m["da"],
+           "db": m["dk"] * kk / (2 * sk), "dw": m["dw"] / (2 * sv), "ds0": m["ds0"]}
+    _compare(g, ref, TOL[dtype], (dtype, d, T, plus))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_packed_sequences(dtype):
+    """Sequences of different lengths (0 to 100 tokens) packed in one row:
+    each sequence's gradients equal the oracle's for that sequence alone, and
+    the tokens after the last sequence are never written."""
+    lens = [0, 5, 32, 33, 100, 1, 64]
+    H = 2
+    T = sum(lens) + 5
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=H, T=T, dtype=dtype)
+    inp = W.make_prefill(wl, seed=21)
+    up = W.make_upstream(wl, seed=21)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    N = len(lens)
+    rng = np.random.default_rng(5)
+    s0 = (0.1 * rng.standard_normal((N, H, 128, 128))).astype(np.float32)
+    dsT = (0.1 * rng.standard_normal((N, H, 128, 128))).astype(np.float32)
+    dev = {x: to_dev(inp[x], dtype) for x in ("q", "k", "v", "a", "b", "w")}
+    src = {"dq": "q", "dk": "k", "dv": "v", "da": "a", "db": "b", "dw": "w"}
+    out = {n: torch.full_like(dev[x], 7.0) for n, x in src.items()}
+    g = api.backward(dev["q"], dev["k"], dev["v"], dev["a"], dev["b"], dev["w"],
+                     to_dev(s0, "f32"), to_dev(up["do"], dtype), to_dev(dsT, "f32"),
+                     cu_seqlens=torch.from_numpy(cu).cuda(), out=out)
+    torch.cuda.synchronize()
+    assert api.last_device_error() == 0
+    f = lambda key: W.as_f32(inp[key], dtype)
+    do = W.as_f32(up["do"], dtype)
+    for n, (t0, t1) in enumerate(zip(cu[:-1], cu[1:])):
+        sl = lambda x: x[:, t0:t1]
+        ref = oracle.backward(sl(f("q")), sl(f("k")), sl(f("v")), sl(f("a")), sl(f("b")),
+                              sl(f("w")), s0[n:n + 1].astype(np.float64), sl(do),
+                              dsT[n:n + 1].astype(np.float64))
+        for name in src:
+            e = rel_err(to_host(g[name][:, t0:t1]), ref[name])
+            assert e <= TOL[dtype], (n, name, e)
+        assert rel_err(to_host(g["ds0"][n:n + 1]), ref["ds0"]) <= TOL[dtype], n
+    for name in src:
+        assert torch.all(g[name][:, cu[-1]:] == 7.0), name
+
+
+def test_unordered_packed_sequences_are_reported():
+    """A decreasing offset makes the sequences after it unordered: they are
+    skipped and reported (GDR_ERR_INVALID_ARG); the ordered ones before it are
+    computed."""
+    H = 1
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=H, T=96, dtype="f32")
+    inp = W.make_prefill(wl, seed=2)
+    up = W.make_upstream(wl, seed=2)
+    cu = np.array([0, 40, 20, 96], np.int32)
+    dev = {x: to_dev(inp[x], "f32") for x in ("q", "k", "v", "a", "b", "w")}
+    out = {"dq": torch.full_like(dev["q"], 7.0)}
+    g = api.backward(dev["q"], dev["k"], dev["v"], dev["a"], dev["b"], dev["w"], None,
+                     to_dev(up["do"], "f32"), None, cu_seqlens=torch.from_numpy(cu).cuda(),
+                     out=out)
+    torch.cuda.synchronize()
+    assert api.last_device_error() == _lib.ERR_INVALID_ARG
+    f = lambda key: W.as_f32(inp[key], "f32")
+    sl = lambda x: x[:, 0:40]
+    ref = oracle.backward(sl(f("q")), sl(f("k")), sl(f("v")), sl(f("a")), sl(f("b")), sl(f("w")),
+                          None, sl(up["do"]), None)
+    assert rel_err(to_host(g["dq"][:, 0:40]), ref["dq"]) <= TOL["f32"]
+    assert torch.all(g["dq"][:, 40:] == 7.0)
