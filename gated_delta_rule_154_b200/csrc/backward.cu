@@ -103,7 +103,8 @@ struct BwdSmem {
     static constexpr int kEgc = kDA + 4 * C * CP;  // e^G_C per channel
     static constexpr int kIgc = kEgc + DK;      // e^-G_C
     static constexpr int kDgc = kIgc + DK;      // gradient on G_C
-    static constexpr int floats = kDgc + DK;
+    static constexpr int kDwp = kDgc + DK;     // scalar write gate: row sums per column half [2][C]
+    static constexpr int floats = kDwp + 2 * C;
     static constexpr size_t bytes = sizeof(float) * floats;
     static_assert(kScr % 4 == 0 && kGcr % 4 == 0 && kEgc % 4 == 0 && sU % 4 == 0 &&
                   kDA % 4 == 0 &&
@@ -122,6 +123,58 @@ __device__ __forceinline__ void dot4_2(float4 a, float4 b, float& e, float& o) {
     e = fmaf(a.z, b.z, e);
     o = fmaf(a.w, b.w, o);
 }
+// Tensor-core products of the bf16 path: mma.sync m16n8k8 with tf32 operands
+// (round to nearest) and float32 accumulation, operands read straight from the
+// float32 tiles in shared memory.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// One warp: acc (the 16 x 8 tile at rows m0, columns n0) += sum over k in
+// [k0, k0 + K) of A(m, k) B(k, n).  A(m, k) = A[m * lda + k], or A[k * lda + m]
+// when AT; B(k, n) = B[k * ldb + n] when BK (stored [K][N]), else B[n * ldb + k].
+// Lane (g = lane / 4, t = lane % 4) holds D(m0 + g, n0 + 2t), D(m0 + g, n0 + 2t + 1),
+// D(m0 + g + 8, n0 + 2t), D(m0 + g + 8, n0 + 2t + 1) in acc[0..3]; K is a multiple of 8.
+template <bool AT, bool BK>
+__device__ __forceinline__ void mma_tile(float (&acc)[4], const float* A, int lda, const float* B,
+                                         int ldb, int m0, int n0, int k0, int K) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    auto ea = [&](int m, int kk) { return AT ? A[kk * lda + m] : A[m * lda + kk]; };
+    auto eb = [&](int kk, int nn) { return BK ? B[kk * ldb + nn] : B[nn * ldb + kk]; };
+#pragma unroll 4
+    for (int k = k0; k < k0 + K; k += 8) {
+        uint32_t a[4];
+        a[0] = to_tf32(ea(m0 + g, k + t));
+        a[1] = to_tf32(ea(m0 + g + 8, k + t));
+        a[2] = to_tf32(ea(m0 + g, k + t + 4));
+        a[3] = to_tf32(ea(m0 + g + 8, k + t + 4));
+        mma_tf32(acc, a, to_tf32(eb(k + t, n0 + g)), to_tf32(eb(k + t + 4, n0 + g)));
+    }
+}
+// Element x of a lane's tile: row m0 + g + 8 (x >> 1), column n0 + 2t + (x & 1).
+__device__ __forceinline__ int tile_row(int m0, int x) { return m0 + ((threadIdx.x & 31) >> 2) + 8 * (x >> 1); }
+__device__ __forceinline__ int tile_col(int n0, int x) { return n0 + 2 * (threadIdx.x & 3) + (x & 1); }
+__device__ __forceinline__ void store_tile(float* dst, int ld, int m0, int n0, const float (&acc)[4],
+                                           float sign = 1.f) {
+#pragma unroll
+    for (int x = 0; x < 4; ++x) dst[tile_row(m0, x) * ld + tile_col(n0, x)] = sign * acc[x];
+}
+__device__ __forceinline__ void store2(__nv_bfloat16* p, float a, float b) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+}
+__device__ __forceinline__ void store2(float* p, float a, float b) {
+    *reinterpret_cast<float2*>(p) = make_float2(a, b);
+}
+
 __device__ __forceinline__ float comp(float4 v, int e) {
     return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
 }
@@ -138,7 +191,9 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float a, float b, float
     *reinterpret_cast<uint2*>(p) = u;
 }
 
-template <typename Tin, int DK, int DV>
+// MMA: the products on the tensor cores (tf32, bf16 inputs); otherwise on the
+// CUDA cores in float32 (float32 inputs and their 1e-4 budget).
+template <typename Tin, int DK, int DV, bool MMA>
 __global__ void __launch_bounds__(BW_NT, 1)
 backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
                 const Tin* __restrict__ q, const Tin* __restrict__ k,
@@ -186,6 +241,7 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
     float* egc = sm + L::kEgc;
     float* igc = sm + L::kIgc;
     float* dgc = sm + L::kDgc;
+    float* dwp = sm + L::kDwp;
 
     const int tid = threadIdx.x;
     const int bh = blockIdx.x;
@@ -345,6 +401,7 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
         stage_a(t0, C, false);
         const float* hc = hbase + (size_t)ci * DK * DV;
         float* hn = hbase + (size_t)(ci + 1) * DK * DV;
+        if constexpr (!MMA) {
         float pf_s[NPF];
         fetch_block(pf_s, hc, 0);
         for (int j0 = 0; j0 < DV; j0 += DB) {
@@ -390,6 +447,48 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
             if (j0 + DB < DV) fetch_block(pf_s, hc, j0 + DB);
             __syncthreads();  // block's tiles consumed
         }
+        } else {
+        float pf_s[NPF];
+        fetch_block(pf_s, hc, 0);
+        const int wid = tid >> 5;
+        for (int j0 = 0; j0 < DV; j0 += DB) {
+            put_block(S0T, pf_s);
+            {
+                const long long tok = tok_of(t0 + rr), base = tok * DV;
+                Ub[rr * UP + cl] = gate_value(w, w_kind, tok, base, j0 + cl) *
+                                   to_f32(v[base + j0 + cl]);
+            }
+            __syncthreads();
+            if (wid < 4) {  // Y = Kh S0 + A_kk U: four 16 x 8 tiles
+                const int m0 = 16 * (wid >> 1), n0 = 8 * (wid & 1);
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_tile<false, false>(acc, Kh, P, S0T, P, m0, n0, 0, DK);
+                mma_tile<false, true>(acc, Akk, CP, Ub, UP, m0, n0, 0, C);
+                store_tile(Yb, UP, m0, n0, acc);
+            }
+            __syncthreads();
+            if (wid < 4) {  // E = T Y
+                const int m0 = 16 * (wid >> 1), n0 = 8 * (wid & 1);
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_tile<false, true>(acc, Tm, CP, Yb, UP, m0, n0, 0, C);
+                store_tile(Eb, UP, m0, n0, acc);
+            }
+            __syncthreads();
+            if (wid < DK / 8) {  // S_C = e^G_C S0 + Kt^T U - Bt^T E: [DK][DB] in 16 x 8 tiles
+                const int m0 = 16 * (wid >> 1), n0 = 8 * (wid & 1);
+                float au[4] = {0.f, 0.f, 0.f, 0.f}, ae[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_tile<true, true>(au, Kt, P, Ub, UP, m0, n0, 0, C);
+                mma_tile<true, true>(ae, Bt, P, Eb, UP, m0, n0, 0, C);
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int c = tile_row(m0, x), j = tile_col(n0, x);
+                    hn[(size_t)c * DV + j0 + j] = fmaf(egc[c], S0T[j * P + c], au[x] - ae[x]);
+                }
+            }
+            if (j0 + DB < DV) fetch_block(pf_s, hc, j0 + DB);
+            __syncthreads();  // block's tiles consumed
+        }
+        }
     }
 
     // ================= reverse sweep
@@ -399,6 +498,8 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
         __syncthreads();  // previous chunk done with every buffer; ds_run, h visible
         stage_a(t0, n, true);
 
+        float* dG = scr;
+        if constexpr (!MMA) {
         // ---------------- stage B: value-column blocks
         // dA entries (r2 + 16 (p >> 1), cl + 16 (p & 1)), p < 4, belong to task-1
         // thread t2: only it reads and writes them until the masking below
@@ -667,7 +768,6 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
         __syncthreads();  // dA reads done: the scratch becomes dG
 
         // ---------------- stage D: back to q, k, b and the decay
-        float* dG = scr;
         {
             const int r = rr;
             float db_row = 0.f;
@@ -711,6 +811,263 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
                 if (cl == 0 && r < n) db[tok_of(t0 + r)] = from_f32<Tin>(db_row);
             }
         }
+        } else {
+        // ---------------- stages B-D on the tensor cores
+        {
+            const int wid = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+            constexpr int NTN = DK / 8;   // 8-wide column tiles across DK
+            constexpr int NTW = DK / 64;  // [C][DK] tiles per warp, of each of the four sums
+            float xq[NTW][4], xk[NTW][4], yk[NTW][4], yb[NTW][4];  // yb holds +E dS^T until negated
+            float dacc[2][4];  // this warp's dA tiles: ids 2 wid, 2 wid + 1 (matrix id >> 3)
+#pragma unroll
+            for (int u = 0; u < NTW; ++u)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) xq[u][x] = xk[u][x] = yk[u][x] = yb[u][x] = 0.f;
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) dacc[u][x] = 0.f;
+            if (tid < 2 * C) dwp[tid] = 0.f;
+            float gcp = 0.f;  // rowsum(dS_C * S0) of key channel tid (tid < DK)
+            const float* hc = hbase + (size_t)ci * DK * DV;
+            const float* dsc = ds_run + soff;
+            float pf_s[NPF], pf_d[NPF];
+            fetch_block(pf_s, hc, 0);
+            fetch_block(pf_d, dsc, 0);
+
+            for (int j0 = 0; j0 < DV; j0 += DB) {
+                put_block(S0T, pf_s);
+                put_block(dST, pf_d);
+                {
+                    const int r = rr, j = cl;
+                    float u = 0.f, gg = 0.f;
+                    if (r < n) {
+                        const long long tok = tok_of(t0 + r), base = tok * DV;
+                        u = gate_value(w, w_kind, tok, base, j0 + j) * to_f32(v[base + j0 + j]);
+                        gg = to_f32(dout[base + j0 + j]);
+                    }
+                    Ub[r * UP + j] = u;
+                    dOb[r * UP + j] = gg;
+                }
+                __syncthreads();
+                // B2: Y = Kh S0 + A_kk U (warps 0-3);  dE = -(Bt dS_C + A_qb^T dO) (warps 4-7)
+                if (wid < 8) {
+                    const int q4 = wid & 3, m0 = 16 * (q4 >> 1), n0 = 8 * (q4 & 1);
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (wid < 4) {
+                        mma_tile<false, false>(acc, Kh, P, S0T, P, m0, n0, 0, DK);
+                        mma_tile<false, true>(acc, Akk, CP, Ub, UP, m0, n0, 0, C);
+                        store_tile(Yb, UP, m0, n0, acc);
+                    } else {
+                        mma_tile<false, false>(acc, Bt, P, dST, P, m0, n0, 0, DK);
+                        mma_tile<true, true>(acc, Aqb, CP, dOb, UP, m0, n0, 0, C);
+                        store_tile(dEb, UP, m0, n0, acc, -1.f);
+                    }
+                }
+                __syncthreads();
+                // B3: E = T Y (warps 0-3);  dY = T^T dE (warps 4-7)
+                if (wid < 8) {
+                    const int q4 = wid & 3, m0 = 16 * (q4 >> 1), n0 = 8 * (q4 & 1);
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (wid < 4) {
+                        mma_tile<false, true>(acc, Tm, CP, Yb, UP, m0, n0, 0, C);
+                        store_tile(Eb, UP, m0, n0, acc);
+                    } else {
+                        mma_tile<true, true>(acc, Tm, CP, dEb, UP, m0, n0, 0, C);
+                        store_tile(dYb, UP, m0, n0, acc);
+                    }
+                }
+                __syncthreads();
+                // B4a: dU -> dv, dw (warps 0-3)
+                if (wid < 4) {
+                    const int m0 = 16 * (wid >> 1), n0 = 8 * (wid & 1);
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma_tile<false, false>(acc, Kt, P, dST, P, m0, n0, 0, DK);
+                    mma_tile<true, true>(acc, Aqk, CP, dOb, UP, m0, n0, 0, C);
+                    mma_tile<true, true>(acc, Akk, CP, dYb, UP, m0, n0, 0, C);
+                    float rs[2] = {0.f, 0.f};  // v dU over this tile's columns, rows m0 + g (+ 8)
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const int r = tile_row(m0, x), j = tile_col(n0, x);
+                        if (r < n) {
+                            const long long tok = tok_of(t0 + r), base = tok * DV;
+                            const float ww = gate_value(w, w_kind, tok, base, j0 + j);
+                            const float vx = to_f32(v[base + j0 + j]);
+                            dv[base + j0 + j] = from_f32<Tin>(ww * acc[x]);
+                            if (w_kind == GDR_GATE_VECTOR) dw[base + j0 + j] = from_f32<Tin>(vx * acc[x]);
+                            if (w_kind == GDR_GATE_FG2)  // through w = sqrt(beta^v)
+                                dw[base + j0 + j] = from_f32<Tin>(vx * acc[x] / (2.f * ww));
+                            rs[x >> 1] = fmaf(vx, acc[x], rs[x >> 1]);
+                        }
+                    }
+                    if (w_kind == GDR_GATE_SCALAR) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            rs[h] += __shfl_xor_sync(0xffffffffu, rs[h], 1);
+                            rs[h] += __shfl_xor_sync(0xffffffffu, rs[h], 2);
+                        }
+                        if (t == 0) {  // this warp alone owns these entries
+                            dwp[(wid & 1) * C + m0 + g] += rs[0];
+                            dwp[(wid & 1) * C + m0 + g + 8] += rs[1];
+                        }
+                    }
+                }
+                // dA: dO U^T, dO E^T, dY U^T, dY E^T (the E ones negated at the masking)
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int id = 2 * wid + u, mat = id >> 3, rem = id & 7;
+                    const int m0 = 16 * (rem >> 2), n0 = 8 * (rem & 3);
+                    mma_tile<false, false>(dacc[u], (mat & 2) ? dYb : dOb, UP, (mat & 1) ? Eb : Ub,
+                                           UP, m0, n0, 0, DB);
+                }
+                // B4b: XQ += dO S0^T, XK += dY S0^T, YK += U dS_C^T, YB += E dS_C^T
+#pragma unroll
+                for (int u = 0; u < NTW; ++u) {
+                    const int id = NTW * wid + u, m0 = 16 * (id / NTN), n0 = 8 * (id % NTN);
+                    mma_tile<false, true>(xq[u], dOb, UP, S0T, P, m0, n0, 0, DB);
+                    mma_tile<false, true>(xk[u], dYb, UP, S0T, P, m0, n0, 0, DB);
+                    mma_tile<false, true>(yk[u], Ub, UP, dST, P, m0, n0, 0, DB);
+                    mma_tile<false, true>(yb[u], Eb, UP, dST, P, m0, n0, 0, DB);
+                }
+                if (tid < DK) {
+#pragma unroll 4
+                    for (int j = 0; j < DB; ++j) gcp = fmaf(dST[j * P + tid], S0T[j * P + tid], gcp);
+                }
+                if (wid < DK / 8) {  // dS0 = e^G_C dS_C + Qh^T dO + Kh^T dY
+                    const int m0 = 16 * (wid >> 1), n0 = 8 * (wid & 1);
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma_tile<true, true>(acc, Qh, P, dOb, UP, m0, n0, 0, C);
+                    mma_tile<true, true>(acc, Kh, P, dYb, UP, m0, n0, 0, C);
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const int c = tile_row(m0, x), j = tile_col(n0, x);
+                        ds_run[soff + (size_t)c * DV + j0 + j] = fmaf(egc[c], dST[j * P + c], acc[x]);
+                    }
+                }
+                if (j0 + DB < DV) {  // next block's columns: not written by this chunk yet
+                    fetch_block(pf_s, hc, j0 + DB);
+                    fetch_block(pf_d, dsc, j0 + DB);
+                }
+                __syncthreads();  // block's tiles consumed before the next block loads
+            }
+
+            // scalar write gate: one value per token
+            if (w_kind == GDR_GATE_SCALAR && tid < n)
+                dw[tok_of(t0 + tid)] = from_f32<Tin>(dwp[tid] + dwp[C + tid]);
+
+            // YB's stage-B share is -E dS_C^T; gradient on G_C: e^G_C rowsum(dS_C S0) +
+            // colsum(Kt YK + Bt YB) before the grams' shares join, per row half in gcr
+#pragma unroll
+            for (int u = 0; u < NTW; ++u) {
+                const int id = NTW * wid + u, mt = id / NTN, m0 = 16 * mt, n0 = 8 * (id % NTN);
+                float cs[2] = {0.f, 0.f};
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    yb[u][x] = -yb[u][x];
+                    const int r = tile_row(m0, x), c = tile_col(n0, x);
+                    cs[x & 1] += Kt[r * P + c] * yk[u][x] + Bt[r * P + c] * yb[u][x];
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    cs[h] += __shfl_xor_sync(0xffffffffu, cs[h], 4);
+                    cs[h] += __shfl_xor_sync(0xffffffffu, cs[h], 8);
+                    cs[h] += __shfl_xor_sync(0xffffffffu, cs[h], 16);
+                }
+                if (g == 0) {
+                    gcr[mt * P + n0 + 2 * t] = cs[0];
+                    gcr[mt * P + n0 + 2 * t + 1] = cs[1];
+                }
+            }
+            // masked dA into shared memory
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int id = 2 * wid + u, mat = id >> 3, rem = id & 7;
+                const int m0 = 16 * (rem >> 2), n0 = 8 * (rem & 3);
+                float* dst = dAqk + mat * C * CP;
+                const float sgn = (mat & 1) ? -1.f : 1.f;
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int r = tile_row(m0, x), sc = tile_col(n0, x);
+                    const bool keep = (mat >= 2) ? (sc < r) : (sc <= r);
+                    dst[r * CP + sc] = keep ? sgn * dacc[u][x] : 0.f;
+                }
+            }
+            __syncthreads();
+            if (tid < DK) dgc[tid] = egc[tid] * gcp + gcr[tid] + gcr[P + tid];
+
+            // ---------------- stage C: the grams' gradients, e^-G_C per key channel
+#pragma unroll
+            for (int u = 0; u < NTW; ++u) {
+                const int id = NTW * wid + u, m0 = 16 * (id / NTN), n0 = 8 * (id % NTN);
+                float tq[4] = {0.f, 0.f, 0.f, 0.f}, tk[4] = {0.f, 0.f, 0.f, 0.f};
+                float ty[4] = {0.f, 0.f, 0.f, 0.f}, tb[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_tile<false, true>(tq, dAqk, CP, Kt, P, m0, n0, 0, C);
+                mma_tile<false, true>(tq, dAqb, CP, Bt, P, m0, n0, 0, C);
+                mma_tile<false, true>(tk, dAkk, CP, Kt, P, m0, n0, 0, C);
+                mma_tile<false, true>(tk, dAkb, CP, Bt, P, m0, n0, 0, C);
+                mma_tile<true, true>(ty, dAqk, CP, Qh, P, m0, n0, 0, C);
+                mma_tile<true, true>(ty, dAkk, CP, Kh, P, m0, n0, 0, C);
+                mma_tile<true, true>(tb, dAqb, CP, Qh, P, m0, n0, 0, C);
+                mma_tile<true, true>(tb, dAkb, CP, Kh, P, m0, n0, 0, C);
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const float f = igc[tile_col(n0, x)];
+                    xq[u][x] = fmaf(f, tq[x], xq[u][x]);
+                    xk[u][x] = fmaf(f, tk[x], xk[u][x]);
+                    yk[u][x] = fmaf(f, ty[x], yk[u][x]);
+                    yb[u][x] = fmaf(f, tb[x], yb[u][x]);
+                }
+            }
+            __syncthreads();  // dA and gcr reads done: the scratch becomes dG, gcr the db rows
+
+            // ---------------- stage D: back to q, k, b and the decay
+#pragma unroll
+            for (int u = 0; u < NTW; ++u) {
+                const int id = NTW * wid + u, m0 = 16 * (id / NTN), n0 = 8 * (id % NTN);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {  // rows m0 + g + 8 h, columns c0, c0 + 1
+                    const int r = m0 + g + 8 * h, c0 = n0 + 2 * t;
+                    float gq[2], gk[2], gb[2], gg[2];
+                    const long long tok = tok_of(t0 + min(r, n - 1)), base = tok * DK;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int x = 2 * h + e, c = c0 + e;
+                        const float gr = Gs[r * P + c], gc = Gs[(C - 1) * P + c];
+                        const float eg = __expf(gr), et = __expf(gc - gr);
+                        const float kt = Kt[r * P + c], bt = Bt[r * P + c];
+                        const float bgate = fg2_b ? 1.f : Bs[r * P + c];
+                        gq[e] = eg * xq[u][x];
+                        gk[e] = fmaf(eg, xk[u][x], et * (yk[u][x] + bgate * yb[u][x]));
+                        gb[e] = kt * yb[u][x];
+                        if (fg2_b) {  // through k~ = sqrt(beta^k) k
+                            const float sb = Bs[r * P + c];
+                            gb[e] = gk[e] * to_f32(k[base + c]) / (2.f * sb);
+                            gk[e] *= sb;
+                        }
+                        gg[e] = Qh[r * P + c] * xq[u][x] + Kh[r * P + c] * xk[u][x] -
+                                kt * yk[u][x] - bt * yb[u][x];
+                        if (r == n - 1) gg[e] += dgc[c];
+                        if (r >= n) gg[e] = 0.f;
+                        gcr[r * P + c] = r < n ? gb[e] : 0.f;
+                    }
+                    store2(dG + r * P + c0, gg[0], gg[1]);
+                    if (r < n) {
+                        store2(dq + base + c0, gq[0], gq[1]);
+                        store2(dk + base + c0, gk[0], gk[1]);
+                        if (b_kind == GDR_GATE_VECTOR || fg2_b) store2(db + base + c0, gb[0], gb[1]);
+                    }
+                }
+            }
+            if (b_kind == GDR_GATE_SCALAR) {
+                __syncthreads();
+                if (tid < n) {
+                    float sum = 0.f;
+                    for (int c = 0; c < DK; ++c) sum += gcr[tid * P + c];
+                    db[tok_of(t0 + tid)] = from_f32<Tin>(sum);
+                }
+            }
+        }
+        }
         __syncthreads();
         if (a_kind != GDR_GATE_ONE) {
             if (tid < DK) {  // d log a_r = sum_{r' >= r} dG_r';  da = d log a / a
@@ -749,7 +1106,7 @@ static cudaError_t launch_backward_t(const gdr_desc& d, const int* cu_seqlens, i
                                      const void* dout, const float* ds_final, float* hs,
                                      float* ds_run, void* const* grads, float* ds0,
                                      int* err_word, cudaStream_t st) {
-    auto kern = backward_kernel<Tin, DK, DV>;
+    auto kern = backward_kernel<Tin, DK, DV, sizeof(Tin) == 2>;  // bf16: tensor cores
     const size_t smem = BwdSmem<DK>::bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
