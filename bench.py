@@ -126,6 +126,9 @@ def backward_bytes(wl) -> int:
     return th * per_th + state * (3 if wl.random_s0 else 2)
 
 
+TF32_OVER_BF16 = 1.1 / 2.25  # nominal dense tensor rates of the B200
+
+
 def fp32_alu_peak_tflops(peaks) -> float:
     """FP32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flop x the
     maximum SM clock."""
@@ -480,16 +483,23 @@ def run_gpu(args):
         if api.last_device_error(stream) != 0:
             raise RuntimeError("device error during backward timing")
         bflops, bbytes = backward_flops(wl), backward_bytes(wl)
-        alu = fp32_alu_peak_tflops(peaks)
+        achieved_tf = bflops / (bms * 1e-3) / 1e12
+        if wl.dtype == "bf16":  # products on tf32 mma.sync: tf32 tensor peak
+            broof = {"bound": "tensor", "achieved": achieved_tf,
+                     "peak": float(peaks["bf16_tflops"]) * TF32_OVER_BF16, "unit": "TFLOP/s",
+                     "peak_source": "%s bf16_tflops x %.4f (nominal dense tf32 : bf16, "
+                                    "1.1 : 2.25 PFLOP/s)" % (peak_src, TF32_OVER_BF16)}
+        else:  # float32 inputs: CUDA-core FMA
+            broof = {"bound": "alu", "achieved": achieved_tf, "peak": fp32_alu_peak_tflops(peaks),
+                     "unit": "TFLOP/s",
+                     "peak_source": "148 SMs x 128 FP32 lanes x 2 x sm_max_mhz"}
+        broof["frac"] = achieved_tf / broof["peak"]
+        broof["flops_per_step"] = bflops
         bwd = {"workload": "gradients of the main step (%s), do ~ N(0,1), dS_T ~ N(0,0.1)"
                            % wl.name,
                "steps": args.backward_steps, "ms_per_step": bms,
                "tokens/s": tokens_step / (bms * 1e-3), "launches_per_step": 1,
-               "roofline": {"bound": "alu", "achieved": bflops / (bms * 1e-3) / 1e12,
-                            "peak": alu, "unit": "TFLOP/s",
-                            "frac": bflops / (bms * 1e-3) / 1e12 / alu,
-                            "flops_per_step": bflops,
-                            "peak_source": "148 SMs x 128 FP32 lanes x 2 x sm_max_mhz"},
+               "roofline": broof,
                "hbm": {"algorithmic_bytes_per_step": bbytes,
                        "GB/s": bbytes / (bms * 1e-3) / 1e9,
                        "frac": bbytes / (bms * 1e-3) / 1e9 / hbm_peak}}

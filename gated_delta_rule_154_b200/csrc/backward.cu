@@ -144,12 +144,17 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 // when AT; B(k, n) = B[k * ldb + n] when BK (stored [K][N]), else B[n * ldb + k].
 // Lane (g = lane / 4, t = lane % 4) holds D(m0 + g, n0 + 2t), D(m0 + g, n0 + 2t + 1),
 // D(m0 + g + 8, n0 + 2t), D(m0 + g + 8, n0 + 2t + 1) in acc[0..3]; K is a multiple of 8.
+// With ks, B(k, n) is also multiplied by ks[k].
 template <bool AT, bool BK>
 __device__ __forceinline__ void mma_tile(float (&acc)[4], const float* A, int lda, const float* B,
-                                         int ldb, int m0, int n0, int k0, int K) {
+                                         int ldb, int m0, int n0, int k0, int K,
+                                         const float* ks = nullptr) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     auto ea = [&](int m, int kk) { return AT ? A[kk * lda + m] : A[m * lda + kk]; };
-    auto eb = [&](int kk, int nn) { return BK ? B[kk * ldb + nn] : B[nn * ldb + kk]; };
+    auto eb = [&](int kk, int nn) {
+        const float x = BK ? B[kk * ldb + nn] : B[nn * ldb + kk];
+        return ks ? x * ks[kk] : x;
+    };
 #pragma unroll 4
     for (int k = k0; k < k0 + K; k += 8) {
         uint32_t a[4];
@@ -321,7 +326,26 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
             Bt[r * P + c] = (fg2_b ? 1.f : Bs[r * P + c]) * kv * et;
         }
         __syncthreads();
-        {
+        if constexpr (MMA) {  // grams on the tensor cores: 4 x (2 x 4) tiles, two per warp
+            const int wid = tid >> 5;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int id = 2 * wid + u, mat = id >> 3, rem = id & 7;  // qk, qb, kk, kb
+                if (!with_q && mat < 2) continue;
+                const int m0 = 16 * (rem >> 2), n0 = 8 * (rem & 3);
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                // A(r, c) = Qh or Kh; B(c, s) = e^-G_C[c] Kt[s][c] or e^-G_C[c] Bt[s][c]
+                mma_tile<false, false>(acc, mat < 2 ? Qh : Kh, P, (mat & 1) ? Bt : Kt, P, m0, n0,
+                                       0, DK, igc);
+                float* dst = mat == 0 ? Aqk : mat == 1 ? Aqb : mat == 2 ? Akk : Akb;
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int r = tile_row(m0, x), sc = tile_col(n0, x);
+                    const bool keep = mat < 2 ? sc <= r : sc < r;
+                    dst[r * CP + sc] = keep ? acc[x] : 0.f;
+                }
+            }
+        } else {
             const int r = rr;
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
