@@ -1,5 +1,6 @@
-// backward.cu -- gradients of the chunked gated delta rule, float32 on the
-// CUDA cores.
+// backward.cu -- gradients of the chunked gated delta rule: the products on
+// the tensor cores (mma.sync, tf32 operands, float32 accumulation) for bf16
+// inputs, on the CUDA cores in float32 for float32 inputs.
 //
 // Loss L = sum_t <o_t, do_t> + <S_T, dS_T>; the kernel returns dL/dq, dk, dv,
 // the three gates and dS_0.  The pages train the recurrence in its chunked
@@ -52,11 +53,12 @@
 // Per chunk: stage A forms the gated operands, the grams and T; stage B runs
 // the value-side products in blocks of 16 columns, keeping dA and the
 // [C, dk] gradient sums in registers; stage C adds the grams' gradients;
-// stage D maps the sums back to q, k, b and the decay.  The products are
-// register tiles fed by 16-byte shared-memory loads (rows of the [*, dk]
-// tiles are float4-aligned), the state blocks are held transposed
+// stage D maps the sums back to q, k, b and the decay.  On the CUDA cores the
+// products are register tiles fed by 16-byte shared-memory loads (rows of the
+// [*, dk] tiles are float4-aligned), with the state blocks held transposed
 // ([value column][key channel]) so both operands of the key-side sums load
-// as float4.
+// as float4.  On the tensor cores each warp owns 16 x 8 output tiles and reads
+// its fragments from the same float32 tiles.
 #include "common.cuh"
 
 namespace gdr {

@@ -195,7 +195,9 @@ size_t gdr_backward_workspace_size(const gdr_desc *desc);
  * page, section 2 "Methodology"); the call differentiates that form: a
  * forward pass stores the state at the start of every 32-token chunk in the
  * workspace, then one CTA per (batch, head) walks the chunks backwards
- * carrying dS.  Float32 arithmetic on the CUDA cores; equal, up to rounding,
+ * carrying dS.  bf16 inputs: products on the tensor cores with tf32
+ * operands and float32 accumulation; float32 inputs: float32 arithmetic on
+ * the CUDA cores.  Equal, up to rounding,
  * to differentiating the token-by-token recurrence.
  *
  *   q .. w, s0  the forward's inputs (s0 NULL for zeros); desc->chunk is not
