@@ -61,3 +61,21 @@ def test_decode_steps_differ_and_subset_consistent():
     assert np.array_equal(sub["v"][1, 1], s2["v"][1, 1])
     st = wlmod.make_decode_state(wl)
     assert st.shape == (2, 3, 128, 128) and abs(np.std(st) - 0.1) < 0.01
+
+
+def test_upstream_gradients_seeded_and_independent_of_inputs():
+    wl = wlmod.WORKLOADS["gdn2_bf16"].replace(B=2, T=40, H=3)
+    up = wlmod.make_upstream(wl, seed=0)
+    again = wlmod.make_upstream(wl, seed=0, threads=1)
+    sub = wlmod.make_upstream(wl, seed=0, heads=[(1, 2)])
+    assert up["do"].shape == (2, 40, 3, 128) and up["do"].dtype == np.uint16
+    assert up["dsT"].shape == (2, 3, 128, 128) and up["dsT"].dtype == np.float32
+    for key in ("do", "dsT"):
+        assert np.array_equal(up[key], again[key])
+    assert np.array_equal(sub["do"][1, :, 2], up["do"][1, :, 2])
+    assert np.array_equal(sub["dsT"][1, 2], up["dsT"][1, 2])
+    assert not sub["do"][0].any() and not sub["dsT"][0].any()      # undrawn heads stay zero
+    inp = wlmod.make_prefill(wl, seed=0)                             # a stream of its own
+    assert not np.array_equal(inp["v"], up["do"])
+    do = wlmod.as_f32(up["do"], wl.dtype)
+    assert abs(np.std(do) - 1.0) < 0.05 and abs(np.std(up["dsT"]) - 0.1) < 0.01
