@@ -335,10 +335,13 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
     const int ch = (p2 & 31) >> 2;                 // 16-byte chunk of the pair in its panel
     const uint32_t cofs = 4u * (uint32_t)(p2 & 3);  // byte of the pair in its chunk
     // the pair of a per token as two bf16 (1.0 past the chunk or for GATE_ONE;
-    // scalar gates came from bf16, so the pair is exact)
+    // scalar gates came from bf16, so the pair is exact).  loc = running
+    // product over the octet; lop = the same without the chunk's first token
+    // (it differs from loc only in octet 0), so that no divisor below holds
+    // a_0.
     uint32_t apr[8];
-    float loc0[8], loc1[8];
-    float run0 = 1.f, run1 = 1.f;
+    float loc0[8], loc1[8], lop0[8], lop1[8];
+    float run0 = 1.f, run1 = 1.f, rop0 = 1.f, rop1 = 1.f;
 #pragma unroll
     for (int x = 0; x < 8; ++x) {
         const int r = 8 * q8 + x;
@@ -347,32 +350,51 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
                                ((uint32_t)(ch ^ (r & 7)) << 4) + cofs)
                          : tc::pack_bf16x2(sca[r], sca[r]);
         apr[x] = (a_kind != GDR_GATE_ONE && r < n) ? pr : 0x3F803F80u;
-        run0 *= __uint_as_float(apr[x] << 16);
-        run1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
+        const float a0 = __uint_as_float(apr[x] << 16), a1 = __uint_as_float(apr[x] & 0xFFFF0000u);
+        run0 *= a0;
+        run1 *= a1;
+        if (r > 0) { rop0 *= a0; rop1 *= a1; }
         loc0[x] = run0;
         loc1[x] = run1;
+        lop0[x] = rop0;
+        lop1[x] = rop1;
     }
     *reinterpret_cast<float2*>(QT + q8 * D + 2 * p2) = make_float2(run0, run1);
     compute_sync();
     mid();
-    float pre0 = 1.f, pre1 = 1.f, gm0 = 1.f, gm1 = 1.f, gc0 = 1.f, gc1 = 1.f;
+    // Octet totals: gm = gamma_31 (octets 0-3), gc = prod over octets 4-7
+    // (= gamma_63/g_m); sp = prod over the octets after this one up to the
+    // middle (q8 < 4); mp = prod over the octets from the middle up to this
+    // one (q8 >= 4).
+    float gm0 = 1.f, gm1 = 1.f, gc0 = 1.f, gc1 = 1.f, sp0 = 1.f, sp1 = 1.f, mp0 = 1.f,
+          mp1 = 1.f;
 #pragma unroll
     for (int gg = 0; gg < 8; ++gg) {
         const float2 qv = *reinterpret_cast<const float2*>(QT + gg * D + 2 * p2);
-        if (gg < q8) { pre0 *= qv.x; pre1 *= qv.y; }
         if (gg < 4) { gm0 *= qv.x; gm1 *= qv.y; } else { gc0 *= qv.x; gc1 *= qv.y; }
+        if (gg > q8 && gg < 4) { sp0 *= qv.x; sp1 *= qv.y; }
+        if (gg >= 4 && gg < q8) { mp0 *= qv.x; mp1 *= qv.y; }
     }
-    // gamma_r/g_m = loc_x * f;  g_m/gamma_r = h * prod_{i > x} a_i  (within the octet)
-    const float f0 = pre0 * rcp_approx(gm0), f1 = pre1 * rcp_approx(gm1);
-    const float h0 = gm0 * rcp_approx(pre0 * run0), h1 = gm1 * rcp_approx(pre1 * run1);
+    // Token r = 8 q8 + x, rev = product of a over the octet's tokens after x:
+    //   r <= 31: g_m/gamma_r = rev * sp, gamma_r/g_m = lop_x / (rop * sp)
+    //   r >= 32: gamma_r/g_m = mp * loc_x, g_m/gamma_r = rev / (mp * run)
+    // Every divisor is a product of a over tokens 1..31 or 32..63 of the chunk
+    // (or a part of one), which the range check below bounds from below, so
+    // the factors never pass through gamma_r itself (which may be far
+    // smaller than either factor).
+    const bool lo = q8 < 4;
+    const float d0 = lo ? rcp_approx(rop0 * sp0) : rcp_approx(mp0 * run0);
+    const float d1 = lo ? rcp_approx(rop1 * sp1) : rcp_approx(mp1 * run1);
     float rev0 = 1.f, rev1 = 1.f;
 #pragma unroll
     for (int x = 7; x >= 0; --x) {
         const int r = 8 * q8 + x;
         const uint32_t sw = (uint32_t)r * 128u + ((uint32_t)(ch ^ (r & 7)) << 4) + cofs;
         const uint32_t o128 = pnl * 16384u + sw, o64 = pnl * 8192u + sw;
-        const uint32_t e = tc::pack_bf16x2(loc0[x] * f0, loc1[x] * f1);
-        const uint32_t ei = tc::pack_bf16x2(h0 * rev0, h1 * rev1);
+        const uint32_t e = lo ? tc::pack_bf16x2(lop0[x] * d0, lop1[x] * d1)
+                              : tc::pack_bf16x2(mp0 * loc0[x], mp1 * loc1[x]);
+        const uint32_t ei = lo ? tc::pack_bf16x2(rev0 * sp0, rev1 * sp1)
+                               : tc::pack_bf16x2(rev0 * d0, rev1 * d1);
         rev0 *= __uint_as_float(apr[x] << 16);
         rev1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
         uint32_t k2 = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW + o128);
@@ -405,8 +427,10 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
         fcur[i + 1] = fprev[i + 1] * gm1;
         fprev[i] = gc0;
         fprev[i + 1] = gc1;
-        const bool ok0 = gm0 > 0.f && loc0[0] <= gm0 * 1e35f && gc0 >= 1e-35f;
-        const bool ok1 = gm1 > 0.f && loc1[0] <= gm1 * 1e35f && gc1 >= 1e-35f;
+        // the divisors above: prod of a over tokens 1..31 (octet 0 holds it as
+        // rop * sp) and over tokens 32..63 (gc)
+        const bool ok0 = rop0 * sp0 >= 1e-35f && gc0 >= 1e-35f;
+        const bool ok1 = rop1 * sp1 >= 1e-35f && gc1 >= 1e-35f;
         if (a_kind != GDR_GATE_ONE && !(ok0 && ok1)) atomicOr(err_word, kErrRange);
     }
 }
