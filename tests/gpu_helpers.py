@@ -24,6 +24,27 @@ def rel_err(x, ref) -> float:
     return float(np.max(np.abs(x - ref)) / den)
 
 
+def elem_err(x, ref, floor: float = 1e-6) -> float:
+    """Largest element-wise relative error |x - ref| / max(|ref|, floor); logged
+    next to rel_err, which is the metric the tolerances apply to."""
+    x = np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    if not ref.size:
+        return 0.0
+    return float(np.max(np.abs(x - ref) / np.maximum(np.abs(ref), floor)))
+
+
+def report(tag: str, x, ref, tol: float) -> str:
+    """One line with the per-tensor error, its margin to the tolerance and the
+    element-wise error (floor 1e-6); printed so that runs with -s log it."""
+    e = rel_err(x, ref)
+    line = "%s: max|x-ref|/max|ref| = %.3e (tolerance %.0e, margin x%.1f); " \
+           "element-wise max (floor 1e-6) = %.3e" % (tag, e, tol, tol / max(e, 1e-30),
+                                                      elem_err(x, ref))
+    print(line, flush=True)
+    return line
+
+
 def to_dev(x, dtype: str, device="cuda"):
     if x is None:
         return None

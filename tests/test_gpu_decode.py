@@ -1,8 +1,8 @@
 """GPU parity of the single-token decode step against the float64 oracle.
 
 Full decode workload (batch 256, H = 32, d = 128, bf16 inputs, float32 state
-~ N(0, 0.1)) checked on every head for the first steps; a 64-head slice is
-carried through 1000 consecutive steps with fresh inputs each step.
+~ N(0, 0.1)) checked on every head for 100 consecutive steps; a 64-head slice
+is carried through 1000 consecutive steps with fresh inputs each step.
 Tolerance 2e-2 for bf16 inputs, 1e-4 for float32 (max |x - ref| / max |ref|)."""
 
 import numpy as np
@@ -12,7 +12,7 @@ import torch
 import oracle
 from gated_delta_rule_154_b200 import api
 from gated_delta_rule_154_b200 import workload as W
-from gpu_helpers import TOL, rel_err, to_dev, to_host
+from gpu_helpers import TOL, rel_err, report, to_dev, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -52,20 +52,30 @@ def test_decode_small(dtype, dk, dv, gates):
         assert rel_err(to_host(state), ref_state) <= TOL[dtype]
 
 
-def test_decode_full_batch_first_steps():
+def test_decode_full_batch_hundred_steps():
+    """The whole decode batch (256 x 32 heads) through 100 consecutive steps
+    with fresh inputs each step, every head compared with the oracle at every
+    step (o) and the carried state at steps 1, 10, 50 and 100."""
     wl = W.WORKLOADS["decode_bf16"]
-    state_np = W.make_decode_state(wl)
+    state_np = W.make_decode_state(wl, threads=16)
     state = to_dev(state_np, "f32")
     ref_state = state_np.astype(np.float64)
-    for step in range(1, 6):
-        inp = W.make_decode_step(wl, step)
+    worst_o = 0.0
+    for step in range(1, 101):
+        inp = W.make_decode_step(wl, step, threads=16)
         d, f = _step_dev(inp, wl), _step_f32(inp, wl)
         o = api.decode_step(d["q"], d["k"], d["v"], d["a"], d["b"], d["w"], state)
         o_ref, ref_state = oracle.decode_step(f["q"], f["k"], f["v"], f["a"], f["b"], f["w"],
                                               ref_state)
         torch.cuda.synchronize()
-        eo, es = rel_err(to_host(o), o_ref), rel_err(to_host(state), ref_state)
-        assert eo <= TOL["bf16"] and es <= TOL["bf16"], (step, eo, es)
+        eo = rel_err(to_host(o), o_ref)
+        worst_o = max(worst_o, eo)
+        assert eo <= TOL["bf16"], (step, eo)
+        if step in (1, 10, 50, 100):
+            msg = report("decode step %d state" % step, to_host(state), ref_state, TOL["bf16"])
+            assert rel_err(to_host(state), ref_state) <= TOL["bf16"], msg
+    report("decode step 100 o", to_host(o), o_ref, TOL["bf16"])
+    print("decode worst o over 100 steps: %.3e" % worst_o, flush=True)
 
 
 def test_decode_thousand_steps_head_slice():
