@@ -49,28 +49,21 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def measured_traffic():
-    """DRAM bytes per prefill launch from the committed ncu summary, or None
-    when the kernel sources changed since that capture."""
+def measured_traffic(name: str = "chunked_tc_gdn2_bf16_T1024.json"):
+    """DRAM bytes per launch of the bench's prefill workload from the committed
+    ncu counters (a JSON data file under profiles/), or None when the kernel
+    sources it names changed since that capture."""
     import hashlib
-    prof = os.path.join(ROOT, "profiles", "chunked_tc_gdn2_bf16_T1024.md")
-    if not os.path.exists(prof):
-        return None
-    fields = {}
-    for line in open(prof):
-        if ":" in line and not line.startswith(("|", "#", " ")):
-            k, v = line.split(":", 1)
-            fields[k.strip()] = v.strip()
-    csrc = os.path.join(ROOT, "gated_delta_rule_154_b200", "csrc")
+    path = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(path):
+        return None, None
+    rec = json.load(open(path))
     h = hashlib.sha256()
-    for name in ("chunked_tc.cu", "tc_common.cuh"):
-        h.update(open(os.path.join(csrc, name), "rb").read())
-    if fields.get("source_sha256") != h.hexdigest():
-        return None
-    try:
-        return int(fields["traffic_bytes_per_launch_scaled"])
-    except (KeyError, ValueError):
-        return None
+    for rel in rec.get("sources", []):
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
+    if rec.get("source_sha256") != h.hexdigest():
+        return None, rec.get("note")
+    return int(rec["traffic_bytes_per_launch"]), rec.get("note")
 
 
 def prefill_bytes(wl) -> int:
@@ -199,6 +192,16 @@ class ClockSampler:
                 "samples_under_load": len(loaded), "reasons": reasons}
 
 
+def config_dict(wl, world: int) -> dict:
+    """The `config` object of the JSON line, the same in both arms."""
+    return {"workload": "%s: B=%d T=%d H=%d dk=dv=%d chunk=%d, per-channel decay, "
+                        "decoupled vector erase/write gates, s0~N(0,0.1)"
+                        % (wl.name, wl.B, wl.T, wl.H, wl.dk, wl.chunk),
+            "global_batch": wl.B * world, "seq_len": wl.T, "heads": wl.H,
+            "parallelism": "dp%d (independent sequences per rank)" % world,
+            "l2": "inputs (%.2f GB per rank) larger than L2" % (prefill_bytes(wl) / 1e9)}
+
+
 # --------------------------------------------------------------- the oracle arm
 
 def oracle_throughput(wl, seed: int, target_s: float = 15.0):
@@ -251,8 +254,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "%s: B=%d T=%d H=%d dk=dv=%d chunk=%d, bf16 inputs (exact in f64)"
-                   % (wl.name, wl.B, wl.T, wl.H, wl.dk, wl.chunk)},
+        "config": config_dict(wl, args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -371,6 +373,7 @@ def run_gpu(args):
 
     tokens_step = wl.B * wl.T * world
     value = tokens_step / (ms_step * 1e-3)
+    traffic, traffic_note = measured_traffic() if wl.T == 8192 else (None, None)
     alg_bytes = prefill_bytes(wl)
     avg_launch_s = statistics.mean(launch_ms) * 1e-3
     achieved = alg_bytes / avg_launch_s / 1e9
@@ -451,6 +454,54 @@ def run_gpu(args):
                             "b[..., 0] for erase and write; fg2: beta = b as sqrt(beta) on k "
                             "and v; fg2_plus: beta^k = b, beta^v = w")
 
+    # ---- the other prefill workloads: KDA (per-channel decay, scalar beta),
+    # long-context (B=1 H=32 T=65536) and the float32 Gated DeltaNet case,
+    # each timed on its own with its HBM roofline (inputs drawn on the device)
+    others = None
+    if not args.no_other_configs:
+        others = {}
+        for name in ("kda_bf16", "long_bf16", "gdn_fp32"):
+            owl = W.WORKLOADS[name]
+            x = W.make_prefill_device(owl, seed=rank_seed(rank), device=dev)
+            xw = x["w"] if x["w"] is not None else x["b"]
+            oo = torch.empty((owl.B, owl.T, owl.H, owl.dv), dtype=x["q"].dtype, device=dev)
+            ss = torch.empty((owl.B, owl.H, owl.dk, owl.dv), dtype=torch.float32, device=dev)
+
+            def ostep():
+                api.forward_chunked(x["q"], x["k"], x["v"], x["a"], x["b"], xw, x["s0"],
+                                    chunk=owl.chunk, out=oo, s_final=ss, stream=stream)
+
+            n_t = args.steps if name != "gdn_fp32" else 100
+            with torch.cuda.stream(stream):
+                for _ in range(3):
+                    ostep()
+                torch.cuda.synchronize()
+                barrier()
+                c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                c0.record(stream)
+                for _ in range(n_t):
+                    ostep()
+                c1.record(stream)
+                torch.cuda.synchronize()
+                barrier()
+            oms = max_over_ranks(c0.elapsed_time(c1)) / n_t
+            if api.last_device_error(stream) != 0:
+                raise RuntimeError("device error during the %s timing" % name)
+            ob = prefill_bytes(owl)
+            ogbs = ob / (oms * 1e-3) / 1e9
+            others[name] = {
+                "workload": "%s: B=%d T=%d H=%d dk=dv=%d chunk=%d %s, decay %s, erase %s, "
+                            "write %s, s0 %s" % (name, owl.B, owl.T, owl.H, owl.dk, owl.chunk,
+                                                 owl.dtype, owl.decay, owl.erase, owl.write,
+                                                 "N(0,0.1)" if owl.random_s0 else "0"),
+                "steps": n_t, "ms_per_step": oms,
+                "tokens/s": owl.B * owl.T * world / (oms * 1e-3),
+                "roofline": {"bound": "hbm", "achieved": ogbs, "peak": hbm_peak, "unit": "GB/s",
+                             "frac": ogbs / hbm_peak, "algorithmic_bytes_per_launch": ob,
+                             "t_hbm_min_us": ob / (hbm_peak * 1e9) * 1e6}}
+            del x, xw, oo, ss
+        torch.cuda.empty_cache()
+
     # ---- backward (training): gradients of the main step's prefill for
     # seeded upstream gradients; one call = one launch (a forward sweep that
     # stores the chunk-start states, then the reverse sweep)
@@ -512,16 +563,15 @@ def run_gpu(args):
         if args.decode_batch:
             dwl = dwl.replace(B=args.decode_batch)
         state = torch.from_numpy(W.make_decode_state(dwl, seed=rank_seed(rank))).to(dev)
-        pool = []
-        for s in range(1, args.decode_pool + 1):
-            x = W.make_decode_step(dwl, s, seed=rank_seed(rank))
-            pool.append({k: dev_t(x[k], dwl.dtype) for k in ("q", "k", "v", "a", "b", "w")})
+        # fresh inputs for every step (warm-up and timed), drawn on the device:
+        # [steps, B, H, d] per tensor, 12.6 MB per step at the decode workload
+        n_in = args.decode_steps + 10
+        seq = W.make_decode_steps_device(dwl, n_in, seed=1000 + rank_seed(rank), device=dev)
         od = torch.empty((dwl.B, dwl.H, dwl.dv), dtype=torch.bfloat16, device=dev)
 
         def dstep(i):
-            p = pool[i % len(pool)]
-            api.decode_step(p["q"], p["k"], p["v"], p["a"], p["b"], p["w"], state, out=od,
-                            stream=stream)
+            api.decode_step(seq["q"][i], seq["k"][i], seq["v"][i], seq["a"][i], seq["b"][i],
+                            seq["w"][i], state, out=od, stream=stream)
 
         with torch.cuda.stream(stream):
             for i in range(10):
@@ -531,7 +581,7 @@ def run_gpu(args):
             d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             d0.record(stream)
             for i in range(args.decode_steps):
-                dstep(i)
+                dstep(10 + i)
             d1.record(stream)
             torch.cuda.synchronize()
             barrier()
@@ -542,6 +592,7 @@ def run_gpu(args):
         dec = {"workload": "%s: batch %d, H=%d, dk=dv=%d, bf16 inputs, f32 state in place"
                            % (dwl.name, dwl.B, dwl.H, dwl.dk),
                "steps": args.decode_steps, "us_per_step": dms * 1e3,
+               "inputs": "fresh every step (drawn on the device before timing)",
                "GB/s": gbs, "frac_of_hbm": gbs / hbm_peak,
                "bytes_per_step": decode_bytes(dwl),
                "tokens/s": dwl.B * world / (dms * 1e-3)}
@@ -561,23 +612,18 @@ def run_gpu(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "%s: B=%d T=%d H=%d dk=dv=%d chunk=%d, per-channel decay, "
-                               "decoupled vector erase/write gates, s0~N(0,0.1)"
-                               % (wl.name, wl.B, wl.T, wl.H, wl.dk, wl.chunk),
-                   "global_batch": wl.B * world, "seq_len": wl.T, "heads": wl.H,
-                   "parallelism": "dp%d (independent sequences per rank)" % world,
-                   "l2": "inputs (%.2f GB per rank) larger than L2" % (alg_bytes / 1e9)},
+        "config": config_dict(wl, world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak,
-                     "traffic": measured_traffic() if (wl.T == 8192 and world >= 1) else None,
-                     "traffic_source": "ncu dram__bytes_read+write at T=1024 scaled x8 "
-                                       "(profiles/chunked_tc_gdn2_bf16_T1024.md)",
+                     "traffic": traffic,
+                     "traffic_source": traffic_note,
                      "peak_source": "%s hbm_gbs" % peak_src,
                      "algorithmic_bytes_per_launch": alg_bytes,
                      "tensor_flops_per_launch": flops,
                      "t_tensor_min_us": t_tc * 1e6,
                      "t_hbm_min_us": alg_bytes / (hbm_peak * 1e9) * 1e6},
         "decode": dec,
+        "prefill_configs": others,
         "backward": bwd,
         "variants": variants,
         "e2e": {"value": tokens_step / (e2e_ms * 1e-3), "unit": "tokens/s",
@@ -598,12 +644,13 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--T", type=int, default=0, help="override the sequence length")
     ap.add_argument("--decode-steps", type=int, default=1000)
-    ap.add_argument("--decode-pool", type=int, default=2)
     ap.add_argument("--decode-batch", type=int, default=0, help="override the decode batch")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the KDA / FG^2-GDN gate-form timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the KDA / long-context / float32 prefill timings")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward timing")
     ap.add_argument("--backward-steps", type=int, default=3)
     ap.add_argument("--ref-seconds", type=float, default=10.0)

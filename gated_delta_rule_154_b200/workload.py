@@ -278,3 +278,55 @@ def make_upstream(wl: Workload, seed: int = 0,
         for bh in todo:
             one(bh)
     return out
+
+
+# ------------------------------------------------- device-side draws (timing)
+
+def _torch_draws(wl: Workload, lead: Tuple[int, ...], seed: int, device):
+    """The same distributions as _draw_head, drawn by torch's generator on
+    ``device`` for leading shape ``lead`` (a different random stream from the
+    numpy one: used where host-side drawing would dominate a timing run)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    dk, dv = wl.dk, wl.dv
+    dt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+
+    def normal(shape, mean=0.0, std=1.0):
+        return torch.randn(shape, generator=g, device=device, dtype=torch.float32) * std + mean
+
+    def unit(shape):
+        x = normal(shape)
+        return x / x.norm(dim=-1, keepdim=True)
+
+    cast = lambda x: x.to(dt).contiguous()   # each tensor leaves float32 at once
+    out = {"q": cast(unit(lead + (dk,))), "k": cast(unit(lead + (dk,))),
+           "v": cast(normal(lead + (dv,)))}
+    xa = normal(lead + ((dk,) if wl.decay == "vector" else ()), -4.0, 1.0)
+    out["a"] = cast(torch.exp(-torch.nn.functional.softplus(xa)))
+    del xa
+    out["b"] = cast(torch.sigmoid(normal(lead + ((dk,) if wl.erase == "vector" else ()))))
+    out["w"] = None
+    if wl.write != "shared":
+        out["w"] = cast(torch.sigmoid(normal(lead + ((dv,) if wl.write == "vector" else ()))))
+    return out
+
+
+def make_prefill_device(wl: Workload, seed: int = 0, device="cuda"):
+    """Prefill inputs of ``wl`` drawn on the device (torch tensors in the
+    workload's dtype, [B, T, H, ...]); s0 ~ N(0, 0.1) float32 when the
+    workload has a random initial state.  ``w`` is None for a shared gate."""
+    import torch
+    x = _torch_draws(wl, (wl.B, wl.T, wl.H), seed, device)
+    x["s0"] = None
+    if wl.random_s0:
+        g = torch.Generator(device=device)
+        g.manual_seed(seed + 7919)
+        x["s0"] = torch.randn((wl.B, wl.H, wl.dk, wl.dv), generator=g, device=device) * 0.1
+    return x
+
+
+def make_decode_steps_device(wl: Workload, steps: int, seed: int = 0, device="cuda"):
+    """Fresh inputs for ``steps`` consecutive decode steps, drawn on the
+    device: tensors [steps, B, H, ...] in the workload's dtype."""
+    return _torch_draws(wl, (steps, wl.B, wl.H), seed, device)
