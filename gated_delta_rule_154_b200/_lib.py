@@ -22,7 +22,11 @@ GATE_ONE, GATE_SCALAR, GATE_VECTOR, GATE_FG2 = 0, 1, 2, 3
 EXPORTS = ("gdr_workspace_size", "gdr_forward_chunked", "gdr_decode_step",
            "gdr_last_device_error", "gdr_status_string", "gdr_version", "gdr_test_skip_signal",
            "gdr_decode_step_paged", "gdr_forward_varlen", "gdr_backward_workspace_size",
-           "gdr_backward_chunked", "gdr_backward_varlen", "gdr_backward_varlen_workspace_size")
+           "gdr_backward_chunked", "gdr_backward_varlen", "gdr_backward_varlen_workspace_size",
+           "gdr_backward_chunked_noalloc")
+
+# bytes of the library-owned scratch of gdr_backward_chunked_noalloc
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class GdrDesc(ctypes.Structure):
@@ -76,6 +80,8 @@ def load(path: str = LIB_PATH):
     lib.gdr_backward_varlen_workspace_size.argtypes = [dp, i]
     lib.gdr_backward_varlen.restype = i
     lib.gdr_backward_varlen.argtypes = [dp, vp, i] + [vp] * 17 + [sz, vp]
+    lib.gdr_backward_chunked_noalloc.restype = i
+    lib.gdr_backward_chunked_noalloc.argtypes = [dp] + [vp] * 16 + [vp]
     lib.gdr_test_skip_signal.restype = None
     lib.gdr_test_skip_signal.argtypes = [i]
     _lib = lib
@@ -125,6 +131,14 @@ def backward_chunked(desc: GdrDesc, q, k, v, a, b, w, s0, d_o, ds_final, dq, dk,
     return int(load().gdr_backward_chunked(ctypes.byref(desc), q, k, v, a, b, w, s0, d_o,
                                            ds_final, dq, dk, dv, da, db, dw, ds0, workspace,
                                            ws_bytes, stream))
+
+
+def backward_chunked_noalloc(desc: GdrDesc, q, k, v, a, b, w, s0, d_o, ds_final, dq, dk, dv,
+                             da, db, dw, ds0, stream) -> int:
+    """Raw call: every pointer an int (0 = NULL).  Returns the gdr_status."""
+    return int(load().gdr_backward_chunked_noalloc(ctypes.byref(desc), q, k, v, a, b, w, s0,
+                                                   d_o, ds_final, dq, dk, dv, da, db, dw, ds0,
+                                                   stream))
 
 
 def backward_varlen_workspace_size(desc: GdrDesc, n_seqs: int) -> int:

@@ -274,6 +274,64 @@ gdr_status gdr_backward_varlen(const gdr_desc* d, const int* cu_seqlens, int n_s
                          da, db, dw, ds0, workspace, ws_bytes, stream);
 }
 
+// ---- backward with library-owned scratch (gdr_backward_chunked_noalloc)
+//
+// Some callers cannot allocate device memory at all: a plugin running inside
+// a host runtime that owns every byte of device memory and hands the library
+// no allocator, or code on a latency-critical path where cudaMalloc is ruled
+// out because it may synchronise the device.  For them the backward pass can
+// use this file-scope scratch instead of a caller-supplied workspace.  It is
+// a __device__ array: every GPU on which the library's module is loaded holds
+// GDR_NOALLOC_SCRATCH_BYTES of it until the process exits, and all calls on
+// that GPU share it.
+} // extern "C"
+static __device__ __align__(256) unsigned char g_gdr_noalloc_scratch[GDR_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices];  // device address of the scratch, per device (g_mu)
+
+// The scratch's device address on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up
+// once per device, with that device current, and cached.
+cudaError_t noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_gdr_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+}  // namespace
+
+extern "C" {
+
+gdr_status gdr_backward_chunked_noalloc(const gdr_desc* d, const void* q, const void* k,
+                                        const void* v, const void* a, const void* b,
+                                        const void* w, const float* s0, const void* d_o,
+                                        const float* ds_final, void* dq, void* dk, void* dv,
+                                        void* da, void* db, void* dw, float* ds0,
+                                        gdr_stream_t stream) {
+    gdr_status s = check_desc(d);
+    if (s != GDR_OK) return s;
+    // larger than the scratch: refused before any CUDA call
+    if (gdr::backward_workspace_bytes(*d, 0) > (size_t)GDR_NOALLOC_SCRATCH_BYTES)
+        return GDR_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return GDR_ERR_CUDA;
+    // The backward writes every word of its workspace before it reads it
+    // (chunk-start states from s0, the running dS from ds_final), so nothing
+    // left in the scratch by an earlier call needs clearing.
+    return backward_impl(d, nullptr, 0, q, k, v, a, b, w, s0, d_o, ds_final, dq, dk, dv, da, db,
+                         dw, ds0, scratch, (size_t)GDR_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 void gdr_test_skip_signal(int enable) { g_test_skip_signal.store(enable ? 1 : 0); }
 
 gdr_status gdr_last_device_error(gdr_stream_t stream) {

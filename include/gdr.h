@@ -253,6 +253,40 @@ gdr_status gdr_backward_varlen(const gdr_desc *desc, const int *cu_seqlens, int 
                                void *dv, void *da, void *db, void *dw, float *ds0,
                                void *workspace, size_t ws_bytes, gdr_stream_t stream);
 
+/* Bytes of the library-owned scratch that gdr_backward_chunked_noalloc uses
+ * (64 MiB, held on every GPU that loads the library until the process exits). */
+#define GDR_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * gdr_backward_chunked for callers that cannot allocate device memory: a
+ * plugin inside a host runtime that owns all device memory and gives the
+ * library no allocator, or latency-critical code that must not call
+ * cudaMalloc because it may synchronise the device.  The pages have no
+ * counterpart to this call; it only changes where the workspace lives.
+ *
+ * Arguments and results are those of gdr_backward_chunked without the
+ * workspace: the call uses a file-scope scratch array of the library
+ * instead, GDR_NOALLOC_SCRATCH_BYTES on each GPU.  It allocates nothing: no
+ * cudaMalloc, no cudaFree, no allocating library routine.
+ *   - Size limit: when gdr_backward_workspace_size(desc) exceeds
+ *     GDR_NOALLOC_SCRATCH_BYTES the call returns GDR_ERR_WORKSPACE before any
+ *     CUDA call (e.g. dk = dv = 128: B * H * (ceil(T / 32) + 1) <= 1024).
+ *   - First call on a device: it looks up the scratch's device address with
+ *     cudaGetSymbolAddress on the current device and caches it.  Make that
+ *     first call on each device before any stream capture begins.
+ *   - Every call on a device shares the one scratch and it keeps the last
+ *     call's contents; the kernel writes every word it reads, so nothing has
+ *     to be cleared between calls.  Calls whose work overlaps on the GPU
+ *     (other streams, or other threads of the process) race on the scratch:
+ *     order them, e.g. on one stream.
+ */
+gdr_status gdr_backward_chunked_noalloc(const gdr_desc *desc, const void *q, const void *k,
+                                        const void *v, const void *a, const void *b,
+                                        const void *w, const float *s0, const void *d_o,
+                                        const float *ds_final, void *dq, void *dk, void *dv,
+                                        void *da, void *db, void *dw, float *ds0,
+                                        gdr_stream_t stream);
+
 /* Synchronises `stream`, returns the status recorded on the device since the
  * previous call (GDR_OK if none) and clears it: GDR_ERR_TIMEOUT (a bounded
  * wait ran out), GDR_ERR_INVALID_ARG (a paged decode slot or a packed
