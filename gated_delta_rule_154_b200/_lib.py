@@ -23,7 +23,9 @@ EXPORTS = ("gdr_workspace_size", "gdr_forward_chunked", "gdr_decode_step",
            "gdr_last_device_error", "gdr_status_string", "gdr_version", "gdr_test_skip_signal",
            "gdr_decode_step_paged", "gdr_forward_varlen", "gdr_backward_workspace_size",
            "gdr_backward_chunked", "gdr_backward_varlen", "gdr_backward_varlen_workspace_size",
-           "gdr_backward_chunked_noalloc")
+           "gdr_backward_chunked_noalloc", "gdr_segment_maps_workspace_size",
+           "gdr_segment_maps", "gdr_segment_scan", "gdr_segmented_workspace_size",
+           "gdr_forward_segmented")
 
 # bytes of the library-owned scratch of gdr_backward_chunked_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -82,6 +84,17 @@ def load(path: str = LIB_PATH):
     lib.gdr_backward_varlen.argtypes = [dp, vp, i] + [vp] * 17 + [sz, vp]
     lib.gdr_backward_chunked_noalloc.restype = i
     lib.gdr_backward_chunked_noalloc.argtypes = [dp] + [vp] * 16 + [vp]
+    lib.gdr_segment_maps_workspace_size.restype = sz
+    lib.gdr_segment_maps_workspace_size.argtypes = [dp]
+    lib.gdr_segment_maps.restype = i
+    lib.gdr_segment_maps.argtypes = [dp] + [vp] * 9 + [sz, vp]
+    ll = ctypes.c_longlong
+    lib.gdr_segment_scan.restype = i
+    lib.gdr_segment_scan.argtypes = [i, i, i, i, i, ll, ll, vp, vp, vp, vp, vp, vp]
+    lib.gdr_segmented_workspace_size.restype = sz
+    lib.gdr_segmented_workspace_size.argtypes = [dp, i]
+    lib.gdr_forward_segmented.restype = i
+    lib.gdr_forward_segmented.argtypes = [dp, i] + [vp] * 10 + [sz, vp]
     lib.gdr_test_skip_signal.restype = None
     lib.gdr_test_skip_signal.argtypes = [i]
     _lib = lib
@@ -151,6 +164,36 @@ def backward_varlen(desc: GdrDesc, cu_seqlens, n_seqs, q, k, v, a, b, w, s0, d_o
     return int(load().gdr_backward_varlen(ctypes.byref(desc), cu_seqlens, int(n_seqs), q, k, v,
                                           a, b, w, s0, d_o, ds_final, dq, dk, dv, da, db, dw,
                                           ds0, workspace, ws_bytes, stream))
+
+
+def segment_maps_workspace_size(desc: GdrDesc) -> int:
+    return int(load().gdr_segment_maps_workspace_size(ctypes.byref(desc)))
+
+
+def segment_maps(desc: GdrDesc, q, k, v, a, b, w, m_out, n_out, workspace, ws_bytes,
+                 stream) -> int:
+    """Raw call: every pointer an int (0 = NULL).  Returns the gdr_status."""
+    return int(load().gdr_segment_maps(ctypes.byref(desc), q, k, v, a, b, w, m_out, n_out,
+                                       workspace, ws_bytes, stream))
+
+
+def segment_scan(n_segments, B, H, dk, dv, seg_stride, batch_stride, m, n, s0, s_start,
+                 s_final, stream) -> int:
+    """Raw call: every pointer an int (0 = NULL).  Returns the gdr_status."""
+    return int(load().gdr_segment_scan(int(n_segments), int(B), int(H), int(dk), int(dv),
+                                       int(seg_stride), int(batch_stride), m, n, s0, s_start,
+                                       s_final, stream))
+
+
+def segmented_workspace_size(desc: GdrDesc, n_segments: int) -> int:
+    return int(load().gdr_segmented_workspace_size(ctypes.byref(desc), int(n_segments)))
+
+
+def forward_segmented(desc: GdrDesc, n_segments, q, k, v, a, b, w, s0, o, s_final, workspace,
+                      ws_bytes, stream) -> int:
+    """Raw call: every pointer an int (0 = NULL).  Returns the gdr_status."""
+    return int(load().gdr_forward_segmented(ctypes.byref(desc), int(n_segments), q, k, v, a, b,
+                                            w, s0, o, s_final, workspace, ws_bytes, stream))
 
 
 def last_device_error(stream) -> int:

@@ -344,3 +344,87 @@ def test_skip_signal(enable: bool = True) -> None:
 
 
 Desc = _lib.GdrDesc
+
+
+# ------------------------------------------------- sequence-parallel prefill
+
+def _desc_dk128(q, v, a, b, w, fg2):
+    if q.shape[-1] != 128 or v.shape[-1] != 128:
+        raise ValueError("segmented prefill needs dk = dv = 128")
+    return desc_for(q, v, a, b, w, 64 if q.dtype == torch.bfloat16 else 32, fg2=fg2)
+
+
+def forward_segmented(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                      a: Optional[torch.Tensor] = None, b: Optional[torch.Tensor] = None,
+                      w: Optional[torch.Tensor] = None, s0: Optional[torch.Tensor] = None,
+                      *, n_segments: int, out: Optional[torch.Tensor] = None,
+                      s_final: Optional[torch.Tensor] = None, stream=None,
+                      fg2: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The prefill with every sequence split into n_segments segments that run
+    side by side on this GPU (their affine maps, a scan, a second pass).
+    Same arguments and results as forward_chunked; dk = dv = 128."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    for t, n, shp in ((q, "q", [(B, T, H, dk)]), (k, "k", [(B, T, H, dk)]),
+                      (v, "v", [(B, T, H, dv)]), (a, "a", [(B, T, H, dk), (B, T, H)]),
+                      (b, "b", [(B, T, H, dk), (B, T, H)]), (w, "w", [(B, T, H, dv), (B, T, H)])):
+        _check(t, n, dt, dev, shp)
+    _check(s0, "s0", torch.float32, dev, [(B, H, dk, dv)])
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    _check(out, "out", dt, dev, [(B, T, H, dv)])
+    if s_final is None:
+        s_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    _check(s_final, "s_final", torch.float32, dev, [(B, H, dk, dv)])
+    desc = _desc_dk128(q, v, a, b, w, fg2)
+    need = _lib.segmented_workspace_size(desc, n_segments)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    st = _lib.forward_segmented(desc, int(n_segments), _ptr(q), _ptr(k), _ptr(v), _ptr(a),
+                                _ptr(b), _ptr(w), _ptr(s0), _ptr(out), _ptr(s_final), _ptr(ws),
+                                need, _stream_handle(stream))
+    if st != _lib.OK:
+        raise _lib.GdrError(st, "gdr_forward_segmented")
+    return out, s_final
+
+
+def segment_maps(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                 a: Optional[torch.Tensor] = None, b: Optional[torch.Tensor] = None,
+                 w: Optional[torch.Tensor] = None, *, stream=None,
+                 fg2: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Affine map of one segment per (batch, head): the state after the
+    segment is M S_in + N.  Returns M [B, H, dk, dk] and N [B, H, dk, dv]
+    (float32); dk = dv = 128."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    desc = _desc_dk128(q, v, a, b, w, fg2)
+    m = torch.empty((B, H, dk, dk), dtype=torch.float32, device=q.device)
+    n = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = _lib.segment_maps_workspace_size(desc)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = _lib.segment_maps(desc, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(w), _ptr(m),
+                           _ptr(n), _ptr(ws), need, _stream_handle(stream))
+    if st != _lib.OK:
+        raise _lib.GdrError(st, "gdr_segment_maps")
+    return m, n
+
+
+def segment_scan(m: torch.Tensor, n: torch.Tensor, s0: Optional[torch.Tensor] = None, *,
+                 stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Start state of every segment and the final state from the maps of P
+    consecutive segments, m [P, B, H, dk, dk] and n [P, B, H, dk, dv] (segment
+    order first), starting from s0 [B, H, dk, dv] (None: zeros).  Returns
+    (s_start [P, B, H, dk, dv], s_final [B, H, dk, dv])."""
+    P, B, H, dk, _ = m.shape
+    dv = n.shape[-1]
+    dev = m.device
+    _check(m, "m", torch.float32, dev, [(P, B, H, dk, dk)])
+    _check(n, "n", torch.float32, dev, [(P, B, H, dk, dv)])
+    _check(s0, "s0", torch.float32, dev, [(B, H, dk, dv)])
+    s_start = torch.empty((P, B, H, dk, dv), dtype=torch.float32, device=dev)
+    s_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    st = _lib.segment_scan(P, B, H, dk, dv, B * H, H, _ptr(m), _ptr(n), _ptr(s0), _ptr(s_start),
+                           _ptr(s_final), _stream_handle(stream))
+    if st != _lib.OK:
+        raise _lib.GdrError(st, "gdr_segment_scan")
+    return s_start, s_final

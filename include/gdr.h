@@ -287,6 +287,73 @@ gdr_status gdr_backward_chunked_noalloc(const gdr_desc *desc, const void *q, con
                                         void *da, void *db, void *dw, float *ds0,
                                         gdr_stream_t stream);
 
+/*
+ * Sequence-parallel prefill.  The recurrence is affine in the state: over a
+ * segment of tokens the state at its end is S_out = M S_in + N, with
+ * M = prod_t (I - (b_t * k_t) k_t^T) Diag(a_t) (dk x dk) and N the segment
+ * run from a zero state.  Splitting a sequence into P segments, computing
+ * their (M, N) side by side, chaining them in order (the only exchange) and
+ * running every segment again from its start state gives the prefill of the
+ * whole sequence: long-sequence scaling as on the FG^2-GDN page
+ * (gist.science 2604.19021), section 4 "Experimental results" (efficiency),
+ * with the update rule of its section 2.  Supported: dk = dv = 128.
+ */
+
+/* Bytes of device workspace gdr_segment_maps needs for `desc` (the segment's
+ * own B, T, H); 0 if unsupported.  Pure host function. */
+size_t gdr_segment_maps_workspace_size(const gdr_desc *desc);
+
+/*
+ * (M, N) of one segment for every (batch, head): desc, q .. w describe the
+ * segment's tokens exactly as for gdr_forward_chunked.  m_out [B, H, dk, dk]
+ * float32: the segment run from S = I with every write switched off (a
+ * scalar write gate of 0); n_out [B, H, dk, dv] float32: the segment run from
+ * S = 0.  Two prefill launches; their outputs o go to the workspace and are
+ * discarded.  Errors as gdr_forward_chunked; GDR_ERR_UNSUPPORTED unless
+ * dk = dv = 128.
+ */
+gdr_status gdr_segment_maps(const gdr_desc *desc, const void *q, const void *k,
+                            const void *v, const void *a, const void *b, const void *w,
+                            float *m_out, float *n_out, void *workspace, size_t ws_bytes,
+                            gdr_stream_t stream);
+
+/*
+ * Exclusive scan of the maps of n_segments consecutive segments, per
+ * (batch, head): S = s0 (NULL: zeros); for p = 0 .. n_segments - 1 in order,
+ * s_start[p] = S, then S = M_p S + N_p (float32); s_final = S.  Matrix
+ * (b, p, h) of m, n and s_start is at element offset
+ * (b * batch_stride + p * seg_stride + h) * dk * dv: seg_stride = B * H,
+ * batch_stride = H for segment-major arrays [P, B, H, ...] (as an all-gather
+ * leaves them); seg_stride = H, batch_stride = P * H for [B, P, H, ...].
+ * s0 and s_final are [B, H, dk, dv]; s_start and s_final may be NULL (not
+ * written).  One CTA per (batch, head).  GDR_ERR_UNSUPPORTED unless
+ * dk = dv = 128.
+ */
+gdr_status gdr_segment_scan(int n_segments, int B, int H, int dk, int dv, long long seg_stride,
+                            long long batch_stride, const float *m, const float *n,
+                            const float *s0, float *s_start, float *s_final,
+                            gdr_stream_t stream);
+
+/* Bytes of device workspace gdr_forward_segmented needs; 0 if unsupported or
+ * n_segments < 1.  Pure host function. */
+size_t gdr_segmented_workspace_size(const gdr_desc *desc, int n_segments);
+
+/*
+ * The prefill of gdr_forward_chunked on one GPU with every sequence split into
+ * n_segments segments of ceil(T / n_segments) tokens rounded up to a multiple
+ * of 64 (the last ones shorter or empty).  The B x n_segments segments run as
+ * packed sequences side by side: their maps (two launches), the scan, then a
+ * second pass from every segment's start state that writes o.  Same
+ * arguments and results as gdr_forward_chunked (o is also used as scratch by
+ * the first two launches), plus a workspace of
+ * gdr_segmented_workspace_size(desc, n_segments) bytes.  n_segments = 1 is
+ * gdr_forward_chunked itself.
+ */
+gdr_status gdr_forward_segmented(const gdr_desc *desc, int n_segments, const void *q,
+                                 const void *k, const void *v, const void *a, const void *b,
+                                 const void *w, const float *s0, void *o, float *s_final,
+                                 void *workspace, size_t ws_bytes, gdr_stream_t stream);
+
 /* Synchronises `stream`, returns the status recorded on the device since the
  * previous call (GDR_OK if none) and clears it: GDR_ERR_TIMEOUT (a bounded
  * wait ran out), GDR_ERR_INVALID_ARG (a paged decode slot or a packed
