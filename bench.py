@@ -463,6 +463,7 @@ def run_gpu(args):
         for name in ("kda_bf16", "long_bf16", "gdn_fp32"):
             owl = W.WORKLOADS[name]
             x = W.make_prefill_device(owl, seed=rank_seed(rank), device=dev)
+            torch.cuda.synchronize()   # drawn on the default stream; timed on `stream`
             xw = x["w"] if x["w"] is not None else x["b"]
             oo = torch.empty((owl.B, owl.T, owl.H, owl.dv), dtype=x["q"].dtype, device=dev)
             ss = torch.empty((owl.B, owl.H, owl.dk, owl.dv), dtype=torch.float32, device=dev)
@@ -485,8 +486,11 @@ def run_gpu(args):
                 torch.cuda.synchronize()
                 barrier()
             oms = max_over_ranks(c0.elapsed_time(c1)) / n_t
-            if api.last_device_error(stream) != 0:
-                raise RuntimeError("device error during the %s timing" % name)
+            err = api.last_device_error(stream)
+            if err != 0:
+                from gated_delta_rule_154_b200 import _lib
+                raise RuntimeError("device error during the %s timing: %s"
+                                   % (name, _lib.status_string(err)))
             ob = prefill_bytes(owl)
             ogbs = ob / (oms * 1e-3) / 1e9
             others[name] = {
@@ -567,6 +571,7 @@ def run_gpu(args):
         # [steps, B, H, d] per tensor, 12.6 MB per step at the decode workload
         n_in = args.decode_steps + 10
         seq = W.make_decode_steps_device(dwl, n_in, seed=1000 + rank_seed(rank), device=dev)
+        torch.cuda.synchronize()   # drawn on the default stream; used on `stream`
         od = torch.empty((dwl.B, dwl.H, dwl.dv), dtype=torch.bfloat16, device=dev)
 
         def dstep(i):
