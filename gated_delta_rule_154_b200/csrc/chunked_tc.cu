@@ -336,12 +336,11 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
     const uint32_t cofs = 4u * (uint32_t)(p2 & 3);  // byte of the pair in its chunk
     // the pair of a per token as two bf16 (1.0 past the chunk or for GATE_ONE;
     // scalar gates came from bf16, so the pair is exact).  loc = running
-    // product over the octet; lop = the same without the chunk's first token
-    // (it differs from loc only in octet 0), so that no divisor below holds
-    // a_0.
+    // product over the octet, leaving out the chunk's first token in octet 0
+    // (so that no divisor below holds a_0); the octet's total (QT) keeps it.
     uint32_t apr[8];
-    float loc0[8], loc1[8], lop0[8], lop1[8];
-    float run0 = 1.f, run1 = 1.f, rop0 = 1.f, rop1 = 1.f;
+    float loc0[8], loc1[8];
+    float run0 = 1.f, run1 = 1.f;
 #pragma unroll
     for (int x = 0; x < 8; ++x) {
         const int r = 8 * q8 + x;
@@ -351,15 +350,16 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
                          : tc::pack_bf16x2(sca[r], sca[r]);
         apr[x] = (a_kind != GDR_GATE_ONE && r < n) ? pr : 0x3F803F80u;
         const float a0 = __uint_as_float(apr[x] << 16), a1 = __uint_as_float(apr[x] & 0xFFFF0000u);
-        run0 *= a0;
-        run1 *= a1;
-        if (r > 0) { rop0 *= a0; rop1 *= a1; }
+        if (r > 0) {
+            run0 *= a0;
+            run1 *= a1;
+        }
         loc0[x] = run0;
         loc1[x] = run1;
-        lop0[x] = rop0;
-        lop1[x] = rop1;
     }
-    *reinterpret_cast<float2*>(QT + q8 * D + 2 * p2) = make_float2(run0, run1);
+    const float f0 = q8 == 0 ? __uint_as_float(apr[0] << 16) : 1.f;
+    const float f1 = q8 == 0 ? __uint_as_float(apr[0] & 0xFFFF0000u) : 1.f;
+    *reinterpret_cast<float2*>(QT + q8 * D + 2 * p2) = make_float2(f0 * run0, f1 * run1);
     compute_sync();
     mid();
     // Octet totals: gm = gamma_31 (octets 0-3), gc = prod over octets 4-7
@@ -376,27 +376,18 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
         if (gg >= 4 && gg < q8) { mp0 *= qv.x; mp1 *= qv.y; }
     }
     // Token r = 8 q8 + x, rev = product of a over the octet's tokens after x:
-    //   r <= 31: g_m/gamma_r = rev * sp, gamma_r/g_m = lop_x / (rop * sp)
+    //   r <= 31: g_m/gamma_r = rev * sp, gamma_r/g_m = loc_x / (run * sp)
     //   r >= 32: gamma_r/g_m = mp * loc_x, g_m/gamma_r = rev / (mp * run)
     // Every divisor is a product of a over tokens 1..31 or 32..63 of the chunk
     // (or a part of one), which the range check below bounds from below, so
     // the factors never pass through gamma_r itself (which may be far
     // smaller than either factor).
-    const bool lo = q8 < 4;
-    const float d0 = lo ? rcp_approx(rop0 * sp0) : rcp_approx(mp0 * run0);
-    const float d1 = lo ? rcp_approx(rop1 * sp1) : rcp_approx(mp1 * run1);
-    float rev0 = 1.f, rev1 = 1.f;
-#pragma unroll
-    for (int x = 7; x >= 0; --x) {
+    // per token: e = gamma_r/g_m, ei = g_m/gamma_r as bf16 pairs; K', Q', K",
+    // B", U written in place
+    auto emit = [&](int x, uint32_t e, uint32_t ei) {
         const int r = 8 * q8 + x;
         const uint32_t sw = (uint32_t)r * 128u + ((uint32_t)(ch ^ (r & 7)) << 4) + cofs;
         const uint32_t o128 = pnl * 16384u + sw, o64 = pnl * 8192u + sw;
-        const uint32_t e = lo ? tc::pack_bf16x2(lop0[x] * d0, lop1[x] * d1)
-                              : tc::pack_bf16x2(mp0 * loc0[x], mp1 * loc1[x]);
-        const uint32_t ei = lo ? tc::pack_bf16x2(rev0 * sp0, rev1 * sp1)
-                               : tc::pack_bf16x2(rev0 * d0, rev1 * d1);
-        rev0 *= __uint_as_float(apr[x] << 16);
-        rev1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
         uint32_t k2 = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW + o128);
         uint32_t q2 = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW + o128 + 8192u);
         const uint32_t b2 = vb ? *reinterpret_cast<const uint32_t*>(sm + OFF_X1 + o128 + 8192u)
@@ -420,6 +411,26 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
             (FG2 && fb) ? kk2 : mul2(b2, kk2);                                 // B"
         *reinterpret_cast<uint32_t*>(sm + OFF_U + o64) =
             mul2((FG2 && fw) ? sqrt2(w2) : w2, v2);                            // U
+    };
+    float rev0 = 1.f, rev1 = 1.f;
+    if (q8 < 4) {   // warp-uniform
+        const float d0 = rcp_approx(sp0 * run0), d1 = rcp_approx(sp1 * run1);
+#pragma unroll
+        for (int x = 7; x >= 0; --x) {
+            emit(x, tc::pack_bf16x2(loc0[x] * d0, loc1[x] * d1),
+                 tc::pack_bf16x2(rev0 * sp0, rev1 * sp1));
+            rev0 *= __uint_as_float(apr[x] << 16);
+            rev1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
+        }
+    } else {
+        const float d0 = rcp_approx(mp0 * run0), d1 = rcp_approx(mp1 * run1);
+#pragma unroll
+        for (int x = 7; x >= 0; --x) {
+            emit(x, tc::pack_bf16x2(mp0 * loc0[x], mp1 * loc1[x]),
+                 tc::pack_bf16x2(rev0 * d0, rev1 * d1));
+            rev0 *= __uint_as_float(apr[x] << 16);
+            rev1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
+        }
     }
     if (q8 == 0) {
         const int i = 2 * p2;
@@ -428,9 +439,9 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
         fprev[i] = gc0;
         fprev[i + 1] = gc1;
         // the divisors above: prod of a over tokens 1..31 (octet 0 holds it as
-        // rop * sp) and over tokens 32..63 (gc)
-        const bool ok0 = rop0 * sp0 >= 1e-35f && gc0 >= 1e-35f;
-        const bool ok1 = rop1 * sp1 >= 1e-35f && gc1 >= 1e-35f;
+        // run * sp) and over tokens 32..63 (gc)
+        const bool ok0 = run0 * sp0 >= 1e-35f && gc0 >= 1e-35f;
+        const bool ok1 = run1 * sp1 >= 1e-35f && gc1 >= 1e-35f;
         if (a_kind != GDR_GATE_ONE && !(ok0 && ok1)) atomicOr(err_word, kErrRange);
     }
 }
