@@ -503,6 +503,38 @@ def run_gpu(args):
                 "roofline": {"bound": "hbm", "achieved": ogbs, "peak": hbm_peak, "unit": "GB/s",
                              "frac": ogbs / hbm_peak, "algorithmic_bytes_per_launch": ob,
                              "t_hbm_min_us": ob / (hbm_peak * 1e9) * 1e6}}
+            if name == "long_bf16":
+                # the same inputs through the sequence split on one GPU: P = 4
+                # segments (maps, scan, second pass) instead of one launch
+                P = 4
+                with torch.cuda.stream(stream):
+                    seg = lambda: api.forward_segmented(x["q"], x["k"], x["v"], x["a"], x["b"],
+                                                        xw, x["s0"], n_segments=P, out=oo,
+                                                        s_final=ss, stream=stream)
+                    for _ in range(2):
+                        seg()
+                    torch.cuda.synchronize()
+                    barrier()
+                    c0.record(stream)
+                    for _ in range(3):
+                        seg()
+                    c1.record(stream)
+                    torch.cuda.synchronize()
+                    barrier()
+                sms = max_over_ranks(c0.elapsed_time(c1)) / 3
+                err = api.last_device_error(stream)
+                if err != 0:
+                    from gated_delta_rule_154_b200 import _lib
+                    raise RuntimeError("device error during the segmented timing: %s"
+                                       % _lib.status_string(err))
+                others["long_bf16_segmented"] = {
+                    "workload": "long_bf16 through gdr_forward_segmented, %d segments of "
+                                "%d tokens (two map launches, scan, second pass)"
+                                % (P, owl.T // P),
+                    "steps": 3, "ms_per_step": sms,
+                    "tokens/s": owl.B * owl.T * world / (sms * 1e-3),
+                    "roofline": {"bound": "hbm", "frac": ob / (sms * 1e-3) / 1e9 / hbm_peak,
+                                 "algorithmic_bytes_per_launch": ob}}
             del x, xw, oo, ss
         torch.cuda.empty_cache()
 

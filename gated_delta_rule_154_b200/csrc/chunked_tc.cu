@@ -136,6 +136,21 @@ __device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<floa
 // Named barriers: id 1 = the 16 compute warps, id 2 = warps 0-7, id 3 =
 // warps 8-15.  (Id 0, __syncthreads, includes the issuing warp.)
 __device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
+// The compute barrier returning the OR of `x` over the 512 compute threads:
+// all of them get the same answer, so they leave the chunk loop together even
+// when the issuing warp raises the abort flag while they pass the barrier.
+__device__ __forceinline__ bool compute_sync_or(bool x) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, 512, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)x)
+        : "memory");
+    return r != 0;
+}
 __device__ __forceinline__ void half_sync(int id) {
     asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");
 }
@@ -714,8 +729,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                 ok = ok && tc::mbar_wait_bounded(bar(B_V), ph, WAIT_NS);
                 if (!ok) *abort_s = 1;
             }
-            compute_sync();
-            if (*abort_s) break;
+            if (compute_sync_or(*abort_s != 0)) break;
             // ================= P1c:
             operand_pass<PACKED, FG2>(sm, tid, va, vb, vw, fb, fw, a_kind, min(C, L - t0), sca, QT, fcur, fprev,
                          err_word, [&] {
@@ -839,10 +853,12 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             }
             tc::fence_async_smem();
             tc::fence_before_sync();
-            signal(R_E);
-            if (*abort_s) break;
+            const bool stop = compute_sync_or(*abort_s != 0);
+            if (tid == 0) tc::mbar_arrive(bar(R_E));
+            if (stop) break;
         }
-        if (L > 0 && *abort_s == 0) {
+        // (one vote, so that all compute threads agree on whether to finish)
+        if (L > 0 && !compute_sync_or(*abort_s != 0)) {
             // the last chunk's O
             wait_then_sync(bar(B_ST), ph ^ 1, tid, abort_s);
             if (!cu_seqlens) {
