@@ -467,10 +467,16 @@ def run_gpu(args):
             xw = x["w"] if x["w"] is not None else x["b"]
             oo = torch.empty((owl.B, owl.T, owl.H, owl.dv), dtype=x["q"].dtype, device=dev)
             ss = torch.empty((owl.B, owl.H, owl.dk, owl.dv), dtype=torch.float32, device=dev)
+            # the library's own choice: few heads with long sequences take the
+            # sequence split, which needs the workspace it asks for
+            need = api.workspace_size(api.desc_for(x["q"], x["v"], x["a"], x["b"], xw,
+                                                   owl.chunk))
+            ows = torch.empty(max(need, 16), dtype=torch.uint8, device=dev) if need else None
 
-            def ostep():
+            def ostep(split=True):
                 api.forward_chunked(x["q"], x["k"], x["v"], x["a"], x["b"], xw, x["s0"],
-                                    chunk=owl.chunk, out=oo, s_final=ss, stream=stream)
+                                    chunk=owl.chunk, out=oo, s_final=ss, workspace=ows,
+                                    stream=stream, split=split)
 
             n_t = args.steps if name != "gdn_fp32" else 100
             with torch.cuda.stream(stream):
@@ -503,21 +509,19 @@ def run_gpu(args):
                 "roofline": {"bound": "hbm", "achieved": ogbs, "peak": hbm_peak, "unit": "GB/s",
                              "frac": ogbs / hbm_peak, "algorithmic_bytes_per_launch": ob,
                              "t_hbm_min_us": ob / (hbm_peak * 1e9) * 1e6}}
-            if name == "long_bf16":
-                # the same inputs through the sequence split on one GPU: P = 4
-                # segments (maps, scan, second pass) instead of one launch
-                P = 4
+            others[name]["sequence_split"] = (
+                "%d segments per sequence (maps, scan, second pass)" % (148 // (owl.B * owl.H))
+                if need else "none (one launch)")
+            if need:
+                # the same inputs on the one-pass kernel, for comparison
                 with torch.cuda.stream(stream):
-                    seg = lambda: api.forward_segmented(x["q"], x["k"], x["v"], x["a"], x["b"],
-                                                        xw, x["s0"], n_segments=P, out=oo,
-                                                        s_final=ss, stream=stream)
                     for _ in range(2):
-                        seg()
+                        ostep(split=False)
                     torch.cuda.synchronize()
                     barrier()
                     c0.record(stream)
                     for _ in range(3):
-                        seg()
+                        ostep(split=False)
                     c1.record(stream)
                     torch.cuda.synchronize()
                     barrier()
@@ -525,17 +529,15 @@ def run_gpu(args):
                 err = api.last_device_error(stream)
                 if err != 0:
                     from gated_delta_rule_154_b200 import _lib
-                    raise RuntimeError("device error during the segmented timing: %s"
+                    raise RuntimeError("device error during the one-launch timing: %s"
                                        % _lib.status_string(err))
-                others["long_bf16_segmented"] = {
-                    "workload": "long_bf16 through gdr_forward_segmented, %d segments of "
-                                "%d tokens (two map launches, scan, second pass)"
-                                % (P, owl.T // P),
+                others[name + "_one_launch"] = {
+                    "workload": "%s on the one-pass kernel (no sequence split)" % name,
                     "steps": 3, "ms_per_step": sms,
                     "tokens/s": owl.B * owl.T * world / (sms * 1e-3),
                     "roofline": {"bound": "hbm", "frac": ob / (sms * 1e-3) / 1e9 / hbm_peak,
                                  "algorithmic_bytes_per_launch": ob}}
-            del x, xw, oo, ss
+            del x, xw, oo, ss, ows
         torch.cuda.empty_cache()
 
     # ---- backward (training): gradients of the main step's prefill for

@@ -90,9 +90,13 @@ def forward_chunked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                     *, chunk: int = 64, out: Optional[torch.Tensor] = None,
                     s_final: Optional[torch.Tensor] = None, return_final: bool = True,
                     workspace: Optional[torch.Tensor] = None, stream=None,
-                    fg2: bool = False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                    fg2: bool = False,
+                    split: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Causal chunked prefill.  Returns (o [B, T, H, dv], S_T [B, H, dk, dv] or None).
-    With fg2=True, b and w hold the vector learning rates beta^k, beta^v."""
+    With fg2=True, b and w hold the vector learning rates beta^k, beta^v.
+    Few heads with long sequences are split into segments that run side by
+    side (the library's choice, when a workspace is given); split=False
+    passes none and keeps the one-pass kernel."""
     if q.dtype not in _DT:
         raise ValueError("q must be float32 or bfloat16")
     B, T, H, dk = q.shape
@@ -114,8 +118,10 @@ def forward_chunked(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         s_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
     _check(s_final, "s_final", torch.float32, dev, [(B, H, dk, dv)])
     desc = desc_for(q, v, a, b, w, chunk, fg2=fg2)
-    need = _lib.workspace_size(desc)
-    if need and workspace is None:
+    need = _lib.workspace_size(desc) if split else 0
+    if not split:
+        workspace = None
+    elif need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = _lib.forward_chunked(desc, _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(w),

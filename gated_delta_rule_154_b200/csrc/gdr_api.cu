@@ -116,9 +116,30 @@ const char* gdr_status_string(gdr_status s) {
     return "GDR_UNKNOWN_STATUS";
 }
 
+}  // extern "C"
+
+namespace {
+// The automatic sequence split of gdr_forward_chunked: when B * H heads leave
+// at least three quarters of the B200's 148 SMs idle, each sequence is cut
+// into P = 148 / (B * H) segments that run side by side (their affine maps,
+// a scan, a second pass: three passes of T / P tokens instead of one of T),
+// provided every segment keeps at least 64 chunks of 64 tokens.
+constexpr int kSMs = 148;
+int auto_segments(const gdr_desc& d) {
+    if (!(d.in_dtype == GDR_BF16 && d.dk == 128 && d.dv == 128 && d.chunk == 64)) return 1;
+    const long long P = kSMs / ((long long)d.B * d.H);
+    if (P < 4 || (long long)d.T < 4096LL * P) return 1;
+    return (int)P;
+}
+}  // namespace
+
+extern "C" {
+
 size_t gdr_workspace_size(const gdr_desc* d) {
     if (check_desc(d) != GDR_OK) return 0;
-    return 0;  // every kernel keeps its intermediates on chip
+    const int P = auto_segments(*d);
+    // every kernel keeps its intermediates on chip; only the split needs room
+    return P > 1 ? gdr_segmented_workspace_size(d, P) : 0;
 }
 
 namespace {
@@ -132,11 +153,15 @@ gdr_status forward_impl(const gdr_desc* d, const int* cu_seqlens, int n_seqs, co
     if ((s = check_inputs(d, have_tokens, q, k, v, a, b, w, o)) != GDR_OK) return s;
     if ((s = check_ptr(s0, false)) != GDR_OK) return s;
     if ((s = check_ptr(s_final, false)) != GDR_OK) return s;
-    const size_t need = gdr_workspace_size(d);
-    if (need > 0 && (workspace == nullptr || ws_bytes < need)) return GDR_ERR_WORKSPACE;
+    // packed sequences never split; a NULL workspace keeps the one-pass kernel
+    const size_t need = cu_seqlens ? 0 : gdr_workspace_size(d);
+    if (need > 0 && workspace != nullptr && ws_bytes < need) return GDR_ERR_WORKSPACE;
     if (workspace && !aligned16(workspace)) return GDR_ERR_INVALID_ARG;
 
     if (d->T == 0 && s_final == nullptr) return GDR_OK;  // nothing to compute or write
+    if (need > 0 && workspace != nullptr)
+        return gdr_forward_segmented(d, auto_segments(*d), q, k, v, a, b, w, s0, o, s_final,
+                                     workspace, ws_bytes, stream);
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     int* err = nullptr;

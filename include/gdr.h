@@ -100,8 +100,11 @@ typedef struct {
     gdr_gate write;       /* w; b and w may be the same tensor (shared beta) */
 } gdr_desc;
 
-/* Bytes of device workspace gdr_forward_chunked needs for `desc` (0 if none,
- * or if desc is invalid).  Pure host function, no CUDA call. */
+/* Bytes of device workspace gdr_forward_chunked can use for `desc` (0 if none,
+ * or if desc is invalid).  Non-zero only where the call splits the sequences
+ * (see gdr_forward_chunked): bf16, dk = dv = 128, chunk 64, B * H <= 37 heads
+ * and T >= 4096 * P with P = 148 / (B * H).  Pure host function, no CUDA
+ * call. */
 size_t gdr_workspace_size(const gdr_desc *desc);
 
 /*
@@ -116,8 +119,14 @@ size_t gdr_workspace_size(const gdr_desc *desc);
  *   o        [B, T, H, dv] in_dtype, written
  *   s_final  [B, H, dk, dv] float32 final state, or NULL (not written);
  *            may equal s0 (in-place update)
- *   workspace, ws_bytes  device scratch of gdr_workspace_size(desc) bytes
- *            (NULL / 0 when that is 0)
+ *   workspace, ws_bytes  device scratch of gdr_workspace_size(desc) bytes,
+ *            or NULL / 0.  When gdr_workspace_size is non-zero (few heads,
+ *            long sequences: most SMs would idle with one CTA per head) and
+ *            the workspace is given, every sequence is split into
+ *            P = 148 / (B * H) segments run side by side through
+ *            gdr_forward_segmented; with NULL the one-pass kernel runs.  A
+ *            non-NULL workspace smaller than required: GDR_ERR_WORKSPACE.
+ *            gdr_forward_varlen takes no workspace.
  *
  * Supported: dk, dv in {64, 128}; float32 inputs with chunk in {16, 32, 64}
  * (chunk <= 32 when dk = 128); bf16 inputs with chunk 64 and dk = dv = 128 on

@@ -172,15 +172,19 @@ def test_bounded_wait_runs_out_and_reports_timeout():
 
 # ------------------------------------------------------ full-size workloads
 
-@pytest.mark.parametrize("name", ["kda_bf16", "gdn2_bf16", "long_bf16"])
-def test_full_size_every_head(name):
+@pytest.mark.parametrize("name,split", [("kda_bf16", True), ("gdn2_bf16", True),
+                                        ("long_bf16", True), ("long_bf16", False)])
+def test_full_size_every_head(name, split):
     """Full workload on the GPU in the bench's launch configuration, compared
     element by element with the oracle on every (b, h): all outputs o and
-    every final state.  The per-tensor error, its margin to the tolerance and
-    the element-wise error (floor 1e-6) are printed."""
+    every final state.  The long-context workload (32 heads) runs both ways:
+    split into segments by the library (its default with a workspace) and on
+    the one-pass kernel.  The per-tensor error, its margin to the tolerance
+    and the element-wise error (floor 1e-6) are printed."""
     wl = W.WORKLOADS[name]
     inp = W.make_prefill(wl, seed=0, threads=16)
-    o, s = gpu_prefill(wl, inp)
+    o, s = gpu_prefill(wl, inp, split=split)
+    name = name + ("" if split else " one launch")
     o_h, s_h = to_host(o), to_host(s)
     del o, s
     o_ref, s_ref = oracle_prefill(wl, inp)
