@@ -384,15 +384,42 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
             }
         }
         __syncthreads();
-        if (tid < C) {  // column j = tid of T = (I + A_kb)^-1, forward substitution
-            const int j = tid;
-            for (int i = 0; i < C; ++i) {
-                float t = (i == j) ? 1.f : 0.f;
-                if (i > j) {
-                    for (int s = j; s < i; ++s) t = fmaf(-Akb[i * CP + s], Tm[s * CP + j], t);
-                }
-                Tm[i * CP + j] = t;
+        // T = (I + N)^-1, N = A_kb strictly lower (C = 32), by 16 x 16 blocks:
+        // the diagonal blocks by substitution (thread = column of one of
+        // them: at most 120 steps instead of 496 for a column of T), then
+        // T21 = -T22 N21 T11 (two 16 x 16 products, one output per thread);
+        // T12 = 0.  The scratch region is free during stage A.
+        static_assert(C == 32 && NT >= 256, "blocked inverse shape");
+        if (tid < 32) {
+            const int o = 16 * (tid >> 4), c = tid & 15;
+#pragma unroll 1
+            for (int r = 0; r < 16; ++r) {   // column c of the diagonal block at o
+                float t = (r == c) ? 1.f : 0.f;
+#pragma unroll 1
+                for (int s2 = c; s2 < r; ++s2)   // entries above row c are zero
+                    t = fmaf(-Akb[(o + r) * CP + o + s2], Tm[(o + s2) * CP + o + c], t);
+                Tm[(o + r) * CP + o + c] = t;
+                if (o == 0) Tm[r * CP + 16 + c] = 0.f;
             }
+        }
+        __syncthreads();
+        float* ys = scr;  // Y = N21 T11, 16 x 16
+        if (tid < 256) {
+            const int r = tid >> 4, c = tid & 15;
+            float acc = 0.f;
+#pragma unroll 1
+            for (int s2 = c; s2 < 16; ++s2)  // T11 is lower triangular
+                acc = fmaf(Akb[(16 + r) * CP + s2], Tm[s2 * CP + c], acc);
+            ys[r * 16 + c] = acc;
+        }
+        __syncthreads();
+        if (tid < 256) {
+            const int r = tid >> 4, c = tid & 15;
+            float acc = 0.f;
+#pragma unroll 1
+            for (int s2 = 0; s2 <= r; ++s2)  // T22 is lower triangular
+                acc = fmaf(Tm[(16 + r) * CP + 16 + s2], ys[s2 * 16 + c], acc);
+            Tm[(16 + r) * CP + c] = -acc;
         }
         __syncthreads();
     };
