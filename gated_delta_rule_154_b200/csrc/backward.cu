@@ -210,7 +210,8 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
                 const float* __restrict__ ds_final, float* __restrict__ hs,
                 float* __restrict__ ds_run, Tin* __restrict__ dq, Tin* __restrict__ dk,
                 Tin* __restrict__ dv, Tin* __restrict__ da, Tin* __restrict__ db,
-                Tin* __restrict__ dw, float* __restrict__ ds0, int* __restrict__ err_word) {
+                Tin* __restrict__ dw, float* __restrict__ ds0, int* __restrict__ err_word,
+                int states_ready) {
     using L = BwdSmem<DK>;
     constexpr int C = BW_C, DB = BW_DB, NT = BW_NT;
     constexpr int P = L::P, CP = L::CP, UP = L::UP;
@@ -444,11 +445,15 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
     };
 
     // ================= forward sweep: chunk-start states h_c into the workspace
+    // (with states_ready the tensor-core forward kernel has already written
+    // the states at the even chunks, and the reverse sweep computes each odd
+    // one from the even one before it)
     for (int x = tid; x < DK * DV; x += NT) {
-        if (n_chunks > 0) hbase[x] = s0 ? s0[soff + x] : 0.f;
+        if (n_chunks > 0 && !states_ready) hbase[x] = s0 ? s0[soff + x] : 0.f;
         ds_run[soff + x] = ds_final ? ds_final[soff + x] : 0.f;
     }
-    for (int ci = 0; ci + 1 < n_chunks; ++ci) {  // every chunk before the last is full
+    // the state at the start of chunk ci + 1 from the one of chunk ci (a full chunk)
+    auto fwd_step = [&](int ci) {
         const int t0 = ci * C;
         __syncthreads();  // h_ci written
         stage_a(t0, C, false);
@@ -542,12 +547,15 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
             __syncthreads();  // block's tiles consumed
         }
         }
-    }
+    };
+    if (!states_ready)
+        for (int ci = 0; ci + 1 < n_chunks; ++ci) fwd_step(ci);  // every chunk before the last is full
 
     // ================= reverse sweep
     for (int ci = n_chunks - 1; ci >= 0; --ci) {
         const int t0 = ci * C;
         const int n = min(C, len - t0);
+        if (states_ready && (ci & 1)) fwd_step(ci - 1);  // this chunk's start state
         __syncthreads();  // previous chunk done with every buffer; ds_run, h visible
         stage_a(t0, n, true);
 
@@ -1158,7 +1166,7 @@ static cudaError_t launch_backward_t(const gdr_desc& d, const int* cu_seqlens, i
                                      const void* const* in, const float* s0,
                                      const void* dout, const float* ds_final, float* hs,
                                      float* ds_run, void* const* grads, float* ds0,
-                                     int* err_word, cudaStream_t st) {
+                                     int* err_word, int states_ready, cudaStream_t st) {
     auto kern = backward_kernel<Tin, DK, DV, sizeof(Tin) == 2>;  // bf16: tensor cores
     const size_t smem = BwdSmem<DK>::bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1169,7 +1177,8 @@ static cudaError_t launch_backward_t(const gdr_desc& d, const int* cu_seqlens, i
         d.T, d.H, cu_seqlens, (const Tin*)in[0], (const Tin*)in[1], (const Tin*)in[2], (const Tin*)in[3],
         (const Tin*)in[4], (const Tin*)in[5], (int)d.decay, (int)d.erase, (int)d.write,
         (const Tin*)dout, s0, ds_final, hs, ds_run, (Tin*)grads[0], (Tin*)grads[1],
-        (Tin*)grads[2], (Tin*)grads[3], (Tin*)grads[4], (Tin*)grads[5], ds0, err_word);
+        (Tin*)grads[2], (Tin*)grads[3], (Tin*)grads[4], (Tin*)grads[5], ds0, err_word,
+        states_ready);
     return cudaGetLastError();
 }
 
@@ -1178,11 +1187,12 @@ static cudaError_t launch_backward_d(const gdr_desc& d, const int* cu_seqlens, i
                                      const void* const* in, const float* s0,
                                      const void* dout, const float* ds_final, float* hs,
                                      float* ds_run, void* const* grads, float* ds0,
-                                     int* err_word, cudaStream_t st) {
+                                     int* err_word, int states_ready, cudaStream_t st) {
 #define GDR_BWD(DK_, DV_)                                                                  \
     if (d.dk == DK_ && d.dv == DV_)                                                        \
         return launch_backward_t<Tin, DK_, DV_>(d, cu_seqlens, n_seqs, in, s0, dout, ds_final, \
-                                                hs, ds_run, grads, ds0, err_word, st);
+                                                hs, ds_run, grads, ds0, err_word,            \
+                                                states_ready, st);
     GDR_BWD(128, 128)
     GDR_BWD(128, 64)
     GDR_BWD(64, 128)
@@ -1207,6 +1217,11 @@ size_t backward_workspace_bytes(const gdr_desc& d, int n_seqs) {
     return mat * (state_matrices(d, n_seqs > 0, n_seqs) + nseq * d.H);
 }
 
+cudaError_t launch_chunked_tc_states(const gdr_desc& d, const void* q, const void* k,
+                                     const void* v, const void* a, const void* b,
+                                     const void* w, const float* s0, float* states, int n32,
+                                     int* err_word, cudaStream_t st);
+
 // in = {q, k, v, a, b, w}; grads = {dq, dk, dv, da, db, dw}.
 cudaError_t launch_backward(const gdr_desc& d, const int* cu_seqlens, int n_seqs,
                             const void* const* in, const float* s0, const void* dout,
@@ -1214,11 +1229,26 @@ cudaError_t launch_backward(const gdr_desc& d, const int* cu_seqlens, int n_seqs
                             void* workspace, int* err_word, cudaStream_t st) {
     float* hs = static_cast<float*>(workspace);
     float* ds_run = hs + state_matrices(d, cu_seqlens != nullptr, n_seqs) * d.dk * d.dv;
-    if (d.in_dtype == GDR_BF16)
+    if (d.in_dtype == GDR_BF16) {
+        // bf16, dk = dv = 128, one sequence per batch row: the tensor-core
+        // forward kernel writes the states at the even 32-token chunks (its
+        // 64-token chunk starts), the backward computes each odd one itself
+        int states_ready = 0;
+        if (!cu_seqlens && d.dk == 128 && d.dv == 128 && d.T > 0) {
+            gdr_desc f = d;
+            f.chunk = 64;
+            const int n32 = (d.T + BW_C - 1) / BW_C;
+            cudaError_t e = launch_chunked_tc_states(f, in[0], in[1], in[2], in[3], in[4], in[5],
+                                                     s0, hs, n32, err_word, st);
+            if (e != cudaSuccess) return e;
+            states_ready = 1;
+        }
         return launch_backward_d<__nv_bfloat16>(d, cu_seqlens, n_seqs, in, s0, dout, ds_final,
-                                                hs, ds_run, grads, ds0, err_word, st);
+                                                hs, ds_run, grads, ds0, err_word, states_ready,
+                                                st);
+    }
     return launch_backward_d<float>(d, cu_seqlens, n_seqs, in, s0, dout, ds_final, hs, ds_run,
-                                    grads, ds0, err_word, st);
+                                    grads, ds0, err_word, 0, st);
 }
 
 }  // namespace gdr

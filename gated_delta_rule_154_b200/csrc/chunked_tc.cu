@@ -81,7 +81,8 @@ constexpr uint32_t OFF_SMALL = OFF_R + 37888;   // 226304
 constexpr uint32_t OFF_FCUR = OFF_SMALL;        // float[128]: state scale this chunk
 constexpr uint32_t OFF_FPREV = OFF_SMALL + 512; // float[128]: gamma_C/g_m of last chunk
 constexpr uint32_t OFF_SCA = OFF_SMALL + 1024;  // float[2][3][64]: scalar a, b, w (2 chunks)
-constexpr uint32_t OFF_BAR = OFF_SMALL + 2560;  // NBAR mbarriers (see the kernel)
+constexpr uint32_t OFF_FSTART = OFF_SMALL + 2560;  // float[128]: fprev before the chunk (dump)
+constexpr uint32_t OFF_BAR = OFF_SMALL + 3072;  // NBAR mbarriers (see the kernel)
 constexpr int NBAR = 14;
 constexpr uint32_t OFF_TSLOT = OFF_BAR + 8 * NBAR;
 constexpr uint32_t OFF_ABORT = OFF_TSLOT + 4;
@@ -339,12 +340,12 @@ __device__ __forceinline__ void issue_v(const TcMaps& m, uint32_t sbase, int t0,
 // fprev = gamma_63/g_m, and check that the largest factors, gamma_0/g_m and
 // g_m/gamma_63, stay in float range.  `mid` runs between the two halves (after
 // the exchange barrier), before anything is written to X2.
-template <bool PACKED, bool FG2, typename Mid>
+template <bool PACKED, bool FG2, bool DUMP, typename Mid>
 __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool vb, bool vw,
                                              bool fb, bool fw, int a_kind, int n,
                                              const float* sca, float* QT,
-                                             float* fcur, float* fprev, int* err_word,
-                                             Mid&& mid) {
+                                             float* fcur, float* fprev, float* fstart,
+                                             int* err_word, Mid&& mid) {
     const int p2 = tid & 63, q8 = tid >> 6;
     const uint32_t pnl = (uint32_t)(p2 >> 5);
     const int ch = (p2 & 31) >> 2;                 // 16-byte chunk of the pair in its panel
@@ -451,6 +452,10 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
         const int i = 2 * p2;
         fcur[i] = fprev[i] * gm0;
         fcur[i + 1] = fprev[i + 1] * gm1;
+        if (DUMP) {   // the chunk-start state is Diag(fprev) times the state held now
+            fstart[i] = fprev[i];
+            fstart[i + 1] = fprev[i + 1];
+        }
         fprev[i] = gc0;
         fprev[i + 1] = gc1;
         // the divisors above: prod of a over tokens 1..31 (octet 0 holds it as
@@ -483,17 +488,20 @@ enum : uint32_t {
 static_assert(R_O + 1 == NBAR, "barrier count");
 
 // PACKED: packed sequences (rows past a sequence's end are zeroed rather than
-// left to the TMA fill).  FG2: FG^2-GDN learning rates among the gates.  Both
-// compile-time, so the plain instantiation carries neither test in its
-// operand pass.
-template <bool PACKED, bool FG2>
+// left to the TMA fill).  FG2: FG^2-GDN learning rates among the gates.  DUMP:
+// no outputs; instead the state at the start of every chunk goes to
+// `states`, [B*H][n32][128][128] float32 at slots 0, 2, 4, ... (the
+// backward's layout of 32-token chunk-start states).  All compile-time, so
+// the plain instantiation carries none of these tests.
+template <bool PACKED, bool FG2, bool DUMP>
 __global__ void __launch_bounds__(NT, 1)
 chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                   const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                   const __nv_bfloat16* __restrict__ w, int a_kind, int b_kind, int w_kind,
                   const float* __restrict__ s0, float* __restrict__ s_final,
                   int* __restrict__ err_word, int skip_signal,
-                  const int* __restrict__ cu_seqlens, __nv_bfloat16* __restrict__ o_raw) {
+                  const int* __restrict__ cu_seqlens, __nv_bfloat16* __restrict__ o_raw,
+                  float* __restrict__ states, int n32) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -504,6 +512,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
     float* PS = reinterpret_cast<float*>(sm + OFF_PS);
     float* fcur = reinterpret_cast<float*>(sm + OFF_FCUR);
     float* fprev = reinterpret_cast<float*>(sm + OFF_FPREV);
+    float* fstart = reinterpret_cast<float*>(sm + OFF_FSTART);
     float* sca_all = reinterpret_cast<float*>(sm + OFF_SCA);  // [2][3][64]
     volatile int* abort_s = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
     auto bar = [&](uint32_t id) { return sbase + OFF_BAR + 8u * id; };
@@ -559,7 +568,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             tc::tma_prefetch_desc(&maps.q);
             tc::tma_prefetch_desc(&maps.k);
             tc::tma_prefetch_desc(&maps.v);
-            tc::tma_prefetch_desc(&maps.o);
+            if (!DUMP) tc::tma_prefetch_desc(&maps.o);
             uint32_t ph = 0;               // phase of the per-chunk barriers
             uint32_t n_kqw = 0, n_ab = 0, n_v = 0;
             issue_kqw(maps, sbase, tb, hi, bi, vw, bar(B_KQW)); ++n_kqw;
@@ -585,7 +594,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
 #pragma unroll 1
             for (; t0 < L; t0 += C, ph ^= 1) {
                 const bool has_next = t0 + C < L;
-                if (t0 > 0 && !store_o(t0 - C, ph ^ 1)) break;
+                if (!DUMP && t0 > 0 && !store_o(t0 - C, ph ^ 1)) break;
                 // operands of the chunk are in place
                 if (!wait_ready(R_OP)) break;
                 // gram [K';Q'] [K";B"]^T
@@ -646,7 +655,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             }
             // the last chunk's o (packed sequences: written directly, the TMA box
             // would reach into the next sequence)
-            if (t0 >= L && *abort_s == 0 && !cu_seqlens) store_o(t0 - C, ph ^ 1);
+            if (!DUMP && t0 >= L && *abort_s == 0 && !cu_seqlens) store_o(t0 - C, ph ^ 1);
             // nothing of this CTA may still be in flight when it exits
             tc::mma_commit(bar(B_FIN));
             tc::mbar_wait_bounded(bar(B_FIN), 0, WAIT_NS);
@@ -731,13 +740,13 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             }
             if (compute_sync_or(*abort_s != 0)) break;
             // ================= P1c:
-            operand_pass<PACKED, FG2>(sm, tid, va, vb, vw, fb, fw, a_kind, min(C, L - t0), sca, QT, fcur, fprev,
-                         err_word, [&] {
+            operand_pass<PACKED, FG2, DUMP>(sm, tid, va, vb, vw, fb, fw, a_kind, min(C, L - t0),
+                         sca, QT, fcur, fprev, fstart, err_word, [&] {
                              if (t0 == 0) return;
                              // the last chunk's state update has read X2 and EB and
                              // finished its O: O -> staging tile for the issuing warp
                              wait_then_sync(bar(B_ST), ph ^ 1, tid, abort_s);
-                             read_o();
+                             if (!DUMP) read_o();
                          });
             tc::fence_async_smem();
             signal(R_OP);
@@ -750,6 +759,16 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                 tc::fence_after_sync();
                 tc::tmem_ld32(tmem + lane_off + TM_S + c0, vals);
                 tc::tmem_wait_ld();
+                if (DUMP) {  // the true state at the chunk start, row lane_t
+                    const float fs = fstart[lane_t];
+                    float4* dst = reinterpret_cast<float4*>(
+                        states + ((size_t)bh * n32 + 2 * (t0 / C)) * D * D +
+                        (size_t)lane_t * D + c0);
+#pragma unroll
+                    for (int x = 0; x < 8; ++x)
+                        dst[x] = make_float4(vals[4 * x] * fs, vals[4 * x + 1] * fs,
+                                             vals[4 * x + 2] * fs, vals[4 * x + 3] * fs);
+                }
 #pragma unroll
                 for (int x = 0; x < 32; ++x) vals[x] *= f;
                 tc::tmem_st32(tmem + lane_off + TM_S + c0, vals);
@@ -861,7 +880,9 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
         if (L > 0 && !compute_sync_or(*abort_s != 0)) {
             // the last chunk's O
             wait_then_sync(bar(B_ST), ph ^ 1, tid, abort_s);
-            if (!cu_seqlens) {
+            if (DUMP) {
+                // no outputs
+            } else if (!cu_seqlens) {
                 read_o();
             } else if (quarter >= 2) {
                 // straight to global memory, only the sequence's own rows
@@ -949,25 +970,34 @@ bool chunked_tc_supports(const gdr_desc& d) {
     return d.in_dtype == GDR_BF16 && d.dk == D && d.dv == D && d.chunk == C;
 }
 
+namespace {
+// Tensor maps of one launch; o only when it is written.
+bool make_maps(TcMaps* maps, const gdr_desc& d, const void* q, const void* k, const void* v,
+               const void* a, const void* b, const void* w, const void* o) {
+    memset(maps, 0, sizeof(*maps));
+    if (d.T == 0) return true;
+    bool ok = make_map(&maps->q, q, d.B, d.T, d.H) && make_map(&maps->k, k, d.B, d.T, d.H) &&
+              make_map(&maps->v, v, d.B, d.T, d.H);
+    if (ok && o) ok = make_map(&maps->o, o, d.B, d.T, d.H);
+    if (ok && d.decay == GDR_GATE_VECTOR) ok = make_map(&maps->a, a, d.B, d.T, d.H);
+    if (ok && (d.erase == GDR_GATE_VECTOR || d.erase == GDR_GATE_FG2))
+        ok = make_map(&maps->b, b, d.B, d.T, d.H);
+    if (ok && (d.write == GDR_GATE_VECTOR || d.write == GDR_GATE_FG2))
+        ok = make_map(&maps->w, w, d.B, d.T, d.H);
+    return ok;
+}
+}  // namespace
+
 cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, const void* v,
                               const void* a, const void* b, const void* w, const float* s0,
                               void* o, float* s_final, int* err_word, bool skip_signal,
                               const int* cu_seqlens, int n_seqs, cudaStream_t st) {
     TcMaps maps;
-    memset(&maps, 0, sizeof(maps));
-    if (d.T > 0) {
-        bool ok = make_map(&maps.q, q, d.B, d.T, d.H) && make_map(&maps.k, k, d.B, d.T, d.H) &&
-                  make_map(&maps.v, v, d.B, d.T, d.H) && make_map(&maps.o, o, d.B, d.T, d.H);
-        if (ok && d.decay == GDR_GATE_VECTOR) ok = make_map(&maps.a, a, d.B, d.T, d.H);
-        if (ok && (d.erase == GDR_GATE_VECTOR || d.erase == GDR_GATE_FG2))
-            ok = make_map(&maps.b, b, d.B, d.T, d.H);
-        if (ok && (d.write == GDR_GATE_VECTOR || d.write == GDR_GATE_FG2))
-            ok = make_map(&maps.w, w, d.B, d.T, d.H);
-        if (!ok) return cudaErrorInvalidValue;
-    }
+    if (!make_maps(&maps, d, q, k, v, a, b, w, o)) return cudaErrorInvalidValue;
     const bool fg2 = d.erase == GDR_GATE_FG2 || d.write == GDR_GATE_FG2;
-    auto kern = cu_seqlens ? (fg2 ? chunked_tc_kernel<true, true> : chunked_tc_kernel<true, false>)
-                           : (fg2 ? chunked_tc_kernel<false, true> : chunked_tc_kernel<false, false>);
+    auto kern = cu_seqlens
+                    ? (fg2 ? chunked_tc_kernel<true, true, false> : chunked_tc_kernel<true, false, false>)
+                    : (fg2 ? chunked_tc_kernel<false, true, false> : chunked_tc_kernel<false, false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
@@ -976,7 +1006,30 @@ cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, c
     kern<<<(unsigned)(nseq * d.H), NT, SMEM_BYTES, st>>>(
         maps, d.B, d.T, d.H, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b,
         (const __nv_bfloat16*)w, (int)d.decay, (int)d.erase, (int)d.write, s0, s_final,
-        err_word, skip_signal ? 1 : 0, cu_seqlens, (__nv_bfloat16*)o);
+        err_word, skip_signal ? 1 : 0, cu_seqlens, (__nv_bfloat16*)o, nullptr, 0);
+    return cudaGetLastError();
+}
+
+// The states at the start of every 64-token chunk of the B x H sequences (no
+// outputs), into slots 0, 2, 4, ... of `states` ([B*H][n32][128][128]
+// float32, n32 = ceil(T / 32)): the backward's chunk-start states at the even
+// 32-token boundaries.
+cudaError_t launch_chunked_tc_states(const gdr_desc& d, const void* q, const void* k,
+                                     const void* v, const void* a, const void* b,
+                                     const void* w, const float* s0, float* states, int n32,
+                                     int* err_word, cudaStream_t st) {
+    TcMaps maps;
+    if (!make_maps(&maps, d, q, k, v, a, b, w, nullptr)) return cudaErrorInvalidValue;
+    const bool fg2 = d.erase == GDR_GATE_FG2 || d.write == GDR_GATE_FG2;
+    auto kern = fg2 ? chunked_tc_kernel<false, true, true> : chunked_tc_kernel<false, false, true>;
+    cudaError_t e = cudaFuncSetAttribute(kern,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)((long long)d.B * d.H), NT, SMEM_BYTES, st>>>(
+        maps, d.B, d.T, d.H, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b,
+        (const __nv_bfloat16*)w, (int)d.decay, (int)d.erase, (int)d.write, s0, nullptr,
+        err_word, 0, nullptr, nullptr, states, n32);
     return cudaGetLastError();
 }
 

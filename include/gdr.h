@@ -204,10 +204,13 @@ size_t gdr_backward_workspace_size(const gdr_desc *desc);
  * page, section 2 "Methodology"); the call differentiates that form: a
  * forward pass stores the state at the start of every 32-token chunk in the
  * workspace, then one CTA per (batch, head) walks the chunks backwards
- * carrying dS.  bf16 inputs: products on the tensor cores with tf32
+ * carrying dS.  On bf16 inputs with dk = dv = 128 that forward pass is a
+ * launch of the tensor-core prefill kernel (the states at its 64-token chunk
+ * starts) ahead of the backward kernel, which adds the states in between.
+ * bf16 inputs: the backward's products on the tensor cores with tf32
  * operands and float32 accumulation; float32 inputs: float32 arithmetic on
- * the CUDA cores.  Equal, up to rounding,
- * to differentiating the token-by-token recurrence.
+ * the CUDA cores.  Equal, up to rounding, to differentiating the
+ * token-by-token recurrence.
  *
  *   q .. w, s0  the forward's inputs (s0 NULL for zeros); desc->chunk is not
  *            used (the pass always takes chunks of 32 tokens)
