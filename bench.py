@@ -588,9 +588,11 @@ def run_gpu(args):
                            % wl.name,
                "steps": args.backward_steps, "ms_per_step": bms,
                "tokens/s": tokens_step / (bms * 1e-3),
-               # bf16, d = 128: the tensor-core forward writing the chunk-start
-               # states, then the backward kernel
-               "launches_per_step": 2 if (wl.dtype == "bf16" and wl.dk == 128 and wl.dv == 128)
+               # bf16, d = 128: three launches of the tensor-core forward writing
+               # the chunk-start states (whole rows, tokens 0..31, tokens 32..),
+               # then the backward kernel
+               "launches_per_step": (4 if wl.T > 32 else 2)
+                                    if (wl.dtype == "bf16" and wl.dk == 128 and wl.dv == 128)
                                     else 1,
                "roofline": broof,
                "hbm": {"algorithmic_bytes_per_step": bbytes,

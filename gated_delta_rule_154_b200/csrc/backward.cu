@@ -445,9 +445,9 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
     };
 
     // ================= forward sweep: chunk-start states h_c into the workspace
-    // (with states_ready the tensor-core forward kernel has already written
-    // the states at the even chunks, and the reverse sweep computes each odd
-    // one from the even one before it)
+    // (states_ready 2: the tensor-core forward kernel has written every
+    // chunk-start state; 1: the even ones, and the reverse sweep computes each
+    // odd one from the even one before it)
     for (int x = tid; x < DK * DV; x += NT) {
         if (n_chunks > 0 && !states_ready) hbase[x] = s0 ? s0[soff + x] : 0.f;
         ds_run[soff + x] = ds_final ? ds_final[soff + x] : 0.f;
@@ -555,7 +555,7 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
     for (int ci = n_chunks - 1; ci >= 0; --ci) {
         const int t0 = ci * C;
         const int n = min(C, len - t0);
-        if (states_ready && (ci & 1)) fwd_step(ci - 1);  // this chunk's start state
+        if (states_ready == 1 && (ci & 1)) fwd_step(ci - 1);  // this chunk's start state
         __syncthreads();  // previous chunk done with every buffer; ds_run, h visible
         stage_a(t0, n, true);
 
@@ -1217,10 +1217,11 @@ size_t backward_workspace_bytes(const gdr_desc& d, int n_seqs) {
     return mat * (state_matrices(d, n_seqs > 0, n_seqs) + nseq * d.H);
 }
 
-cudaError_t launch_chunked_tc_states(const gdr_desc& d, const void* q, const void* k,
+cudaError_t launch_chunked_tc_states(const gdr_desc& d, int T_row, const void* q, const void* k,
                                      const void* v, const void* a, const void* b,
-                                     const void* w, const float* s0, float* states, int n32,
-                                     int* err_word, cudaStream_t st);
+                                     const void* w, const float* s0, float* s_final,
+                                     float* states, int n32, int slot0, int* err_word,
+                                     cudaStream_t st);
 
 // in = {q, k, v, a, b, w}; grads = {dq, dk, dv, da, db, dw}.
 cudaError_t launch_backward(const gdr_desc& d, const int* cu_seqlens, int n_seqs,
@@ -1230,18 +1231,44 @@ cudaError_t launch_backward(const gdr_desc& d, const int* cu_seqlens, int n_seqs
     float* hs = static_cast<float*>(workspace);
     float* ds_run = hs + state_matrices(d, cu_seqlens != nullptr, n_seqs) * d.dk * d.dv;
     if (d.in_dtype == GDR_BF16) {
-        // bf16, dk = dv = 128, one sequence per batch row: the tensor-core
-        // forward kernel writes the states at the even 32-token chunks (its
-        // 64-token chunk starts), the backward computes each odd one itself
+        // bf16, dk = dv = 128, one sequence per batch row: the chunk-start
+        // states come from the tensor-core forward kernel.  The whole rows
+        // give the even 32-token slots (its 64-token chunk starts); a 32-token
+        // run gives the state after token 31 (into the running-dS region,
+        // which the backward kernel initialises only later), and a run over
+        // tokens 32 .. T-1 from that state gives the odd slots.
         int states_ready = 0;
         if (!cu_seqlens && d.dk == 128 && d.dv == 128 && d.T > 0) {
             gdr_desc f = d;
             f.chunk = 64;
             const int n32 = (d.T + BW_C - 1) / BW_C;
-            cudaError_t e = launch_chunked_tc_states(f, in[0], in[1], in[2], in[3], in[4], in[5],
-                                                     s0, hs, n32, err_word, st);
+            cudaError_t e = launch_chunked_tc_states(f, d.T, in[0], in[1], in[2], in[3], in[4],
+                                                     in[5], s0, nullptr, hs, n32, 0, err_word,
+                                                     st);
             if (e != cudaSuccess) return e;
             states_ready = 1;
+            if (d.T > BW_C) {
+                gdr_desc f1 = f;
+                f1.T = BW_C;
+                e = launch_chunked_tc_states(f1, d.T, in[0], in[1], in[2], in[3], in[4], in[5],
+                                             s0, ds_run, hs, n32, 0, err_word, st);
+                if (e != cudaSuccess) return e;
+                // the same tensors from token 32 on
+                const long long tv = (long long)BW_C * d.H * 128, ts = (long long)BW_C * d.H;
+                auto shift = [&](const void* p, int kind) -> const void* {
+                    if (!p || kind == GDR_GATE_ONE) return p;
+                    return static_cast<const __nv_bfloat16*>(p) +
+                           (kind == GDR_GATE_SCALAR ? ts : tv);
+                };
+                gdr_desc f2 = f;
+                f2.T = d.T - BW_C;
+                e = launch_chunked_tc_states(
+                    f2, d.T, shift(in[0], GDR_GATE_VECTOR), shift(in[1], GDR_GATE_VECTOR),
+                    shift(in[2], GDR_GATE_VECTOR), shift(in[3], d.decay), shift(in[4], d.erase),
+                    shift(in[5], d.write), ds_run, nullptr, hs, n32, 1, err_word, st);
+                if (e != cudaSuccess) return e;
+                states_ready = 2;
+            }
         }
         return launch_backward_d<__nv_bfloat16>(d, cu_seqlens, n_seqs, in, s0, dout, ds_final,
                                                 hs, ds_run, grads, ds0, err_word, states_ready,

@@ -489,10 +489,12 @@ static_assert(R_O + 1 == NBAR, "barrier count");
 
 // PACKED: packed sequences (rows past a sequence's end are zeroed rather than
 // left to the TMA fill).  FG2: FG^2-GDN learning rates among the gates.  DUMP:
-// no outputs; instead the state at the start of every chunk goes to
-// `states`, [B*H][n32][128][128] float32 at slots 0, 2, 4, ... (the
+// no o; instead the state at the start of every chunk goes to `states`,
+// [B*H][n32][128][128] float32 at slots slot0, slot0 + 2, ... (the
 // backward's layout of 32-token chunk-start states).  All compile-time, so
-// the plain instantiation carries none of these tests.
+// the plain instantiation carries none of these tests.  T_row: tokens
+// between batch rows in memory (T, or more when the launch covers a token
+// range of longer rows).
 template <bool PACKED, bool FG2, bool DUMP>
 __global__ void __launch_bounds__(NT, 1)
 chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
@@ -501,7 +503,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                   const float* __restrict__ s0, float* __restrict__ s_final,
                   int* __restrict__ err_word, int skip_signal,
                   const int* __restrict__ cu_seqlens, __nv_bfloat16* __restrict__ o_raw,
-                  float* __restrict__ states, int n32) {
+                  float* __restrict__ states, int n32, int slot0, int T_row) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -670,7 +672,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
         auto load_scalars = [&](int t0n, int buf) {
             if (tid < C) {
                 const int nn = min(C, L - t0n);
-                const long long tok = ((long long)bi * T + tb + t0n + tid) * H + hi;
+                const long long tok = ((long long)bi * T_row + tb + t0n + tid) * H + hi;
                 const bool in = tid < nn;
                 float* sc = sca_all + buf * 192;
                 sc[tid] = (a_kind == GDR_GATE_SCALAR && in) ? to_f32(a[tok]) : 1.f;
@@ -762,7 +764,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                 if (DUMP) {  // the true state at the chunk start, row lane_t
                     const float fs = fstart[lane_t];
                     float4* dst = reinterpret_cast<float4*>(
-                        states + ((size_t)bh * n32 + 2 * (t0 / C)) * D * D +
+                        states + ((size_t)bh * n32 + slot0 + 2 * (t0 / C)) * D * D +
                         (size_t)lane_t * D + c0);
 #pragma unroll
                     for (int x = 0; x < 8; ++x)
@@ -950,12 +952,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // [B, T, H, 128] bf16 tensor as a 4-D map {128, H, T, B}, box {64, 1, 64, 1},
 // 128-byte swizzle; rows past T read as zero and are not written.
-bool make_map(CUtensorMap* m, const void* ptr, int B, int T, int H) {
+bool make_map(CUtensorMap* m, const void* ptr, int B, int T, int H, int T_row) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2,
-                                   (cuuint64_t)T * H * D * 2};
+                                   (cuuint64_t)T_row * H * D * 2};
     const cuuint32_t box[4] = {64, 1, 64, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
@@ -972,18 +974,19 @@ bool chunked_tc_supports(const gdr_desc& d) {
 
 namespace {
 // Tensor maps of one launch; o only when it is written.
-bool make_maps(TcMaps* maps, const gdr_desc& d, const void* q, const void* k, const void* v,
-               const void* a, const void* b, const void* w, const void* o) {
+bool make_maps(TcMaps* maps, const gdr_desc& d, int T_row, const void* q, const void* k,
+               const void* v, const void* a, const void* b, const void* w, const void* o) {
     memset(maps, 0, sizeof(*maps));
     if (d.T == 0) return true;
-    bool ok = make_map(&maps->q, q, d.B, d.T, d.H) && make_map(&maps->k, k, d.B, d.T, d.H) &&
-              make_map(&maps->v, v, d.B, d.T, d.H);
-    if (ok && o) ok = make_map(&maps->o, o, d.B, d.T, d.H);
-    if (ok && d.decay == GDR_GATE_VECTOR) ok = make_map(&maps->a, a, d.B, d.T, d.H);
+    const int B = d.B, T = d.T, H = d.H;
+    bool ok = make_map(&maps->q, q, B, T, H, T_row) && make_map(&maps->k, k, B, T, H, T_row) &&
+              make_map(&maps->v, v, B, T, H, T_row);
+    if (ok && o) ok = make_map(&maps->o, o, B, T, H, T_row);
+    if (ok && d.decay == GDR_GATE_VECTOR) ok = make_map(&maps->a, a, B, T, H, T_row);
     if (ok && (d.erase == GDR_GATE_VECTOR || d.erase == GDR_GATE_FG2))
-        ok = make_map(&maps->b, b, d.B, d.T, d.H);
+        ok = make_map(&maps->b, b, B, T, H, T_row);
     if (ok && (d.write == GDR_GATE_VECTOR || d.write == GDR_GATE_FG2))
-        ok = make_map(&maps->w, w, d.B, d.T, d.H);
+        ok = make_map(&maps->w, w, B, T, H, T_row);
     return ok;
 }
 }  // namespace
@@ -993,7 +996,7 @@ cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, c
                               void* o, float* s_final, int* err_word, bool skip_signal,
                               const int* cu_seqlens, int n_seqs, cudaStream_t st) {
     TcMaps maps;
-    if (!make_maps(&maps, d, q, k, v, a, b, w, o)) return cudaErrorInvalidValue;
+    if (!make_maps(&maps, d, d.T, q, k, v, a, b, w, o)) return cudaErrorInvalidValue;
     const bool fg2 = d.erase == GDR_GATE_FG2 || d.write == GDR_GATE_FG2;
     auto kern = cu_seqlens
                     ? (fg2 ? chunked_tc_kernel<true, true, false> : chunked_tc_kernel<true, false, false>)
@@ -1006,20 +1009,22 @@ cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, c
     kern<<<(unsigned)(nseq * d.H), NT, SMEM_BYTES, st>>>(
         maps, d.B, d.T, d.H, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b,
         (const __nv_bfloat16*)w, (int)d.decay, (int)d.erase, (int)d.write, s0, s_final,
-        err_word, skip_signal ? 1 : 0, cu_seqlens, (__nv_bfloat16*)o, nullptr, 0);
+        err_word, skip_signal ? 1 : 0, cu_seqlens, (__nv_bfloat16*)o, nullptr, 0, 0, d.T);
     return cudaGetLastError();
 }
 
-// The states at the start of every 64-token chunk of the B x H sequences (no
-// outputs), into slots 0, 2, 4, ... of `states` ([B*H][n32][128][128]
-// float32, n32 = ceil(T / 32)): the backward's chunk-start states at the even
-// 32-token boundaries.
-cudaError_t launch_chunked_tc_states(const gdr_desc& d, const void* q, const void* k,
+// The states at the start of every 64-token chunk of the B x H sequences
+// (no o) into slots slot0, slot0 + 2, ... of `states` ([B*H][n32][128][128]
+// float32): the backward's chunk-start states.  The launch covers d.T tokens
+// of rows T_row tokens apart (the pointers already at its first token);
+// s_final, if given, receives the state after them.
+cudaError_t launch_chunked_tc_states(const gdr_desc& d, int T_row, const void* q, const void* k,
                                      const void* v, const void* a, const void* b,
-                                     const void* w, const float* s0, float* states, int n32,
-                                     int* err_word, cudaStream_t st) {
+                                     const void* w, const float* s0, float* s_final,
+                                     float* states, int n32, int slot0, int* err_word,
+                                     cudaStream_t st) {
     TcMaps maps;
-    if (!make_maps(&maps, d, q, k, v, a, b, w, nullptr)) return cudaErrorInvalidValue;
+    if (!make_maps(&maps, d, T_row, q, k, v, a, b, w, nullptr)) return cudaErrorInvalidValue;
     const bool fg2 = d.erase == GDR_GATE_FG2 || d.write == GDR_GATE_FG2;
     auto kern = fg2 ? chunked_tc_kernel<false, true, true> : chunked_tc_kernel<false, false, true>;
     cudaError_t e = cudaFuncSetAttribute(kern,
@@ -1028,8 +1033,8 @@ cudaError_t launch_chunked_tc_states(const gdr_desc& d, const void* q, const voi
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)((long long)d.B * d.H), NT, SMEM_BYTES, st>>>(
         maps, d.B, d.T, d.H, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b,
-        (const __nv_bfloat16*)w, (int)d.decay, (int)d.erase, (int)d.write, s0, nullptr,
-        err_word, 0, nullptr, nullptr, states, n32);
+        (const __nv_bfloat16*)w, (int)d.decay, (int)d.erase, (int)d.write, s0, s_final,
+        err_word, 0, nullptr, nullptr, states, n32, slot0, T_row);
     return cudaGetLastError();
 }
 
