@@ -210,8 +210,7 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
                 const float* __restrict__ ds_final, float* __restrict__ hs,
                 float* __restrict__ ds_run, Tin* __restrict__ dq, Tin* __restrict__ dk,
                 Tin* __restrict__ dv, Tin* __restrict__ da, Tin* __restrict__ db,
-                Tin* __restrict__ dw, float* __restrict__ ds0, int* __restrict__ err_word,
-                int states_ready) {
+                Tin* __restrict__ dw, float* __restrict__ ds0, int* __restrict__ err_word) {
     using L = BwdSmem<DK>;
     constexpr int C = BW_C, DB = BW_DB, NT = BW_NT;
     constexpr int P = L::P, CP = L::CP, UP = L::UP;
@@ -445,11 +444,8 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
     };
 
     // ================= forward sweep: chunk-start states h_c into the workspace
-    // (states_ready 2: the tensor-core forward kernel has written every
-    // chunk-start state; 1: the even ones, and the reverse sweep computes each
-    // odd one from the even one before it)
     for (int x = tid; x < DK * DV; x += NT) {
-        if (n_chunks > 0 && !states_ready) hbase[x] = s0 ? s0[soff + x] : 0.f;
+        if (n_chunks > 0) hbase[x] = s0 ? s0[soff + x] : 0.f;
         ds_run[soff + x] = ds_final ? ds_final[soff + x] : 0.f;
     }
     // the state at the start of chunk ci + 1 from the one of chunk ci (a full chunk)
@@ -548,14 +544,12 @@ backward_kernel(int T, int H, const int* __restrict__ cu_seqlens,
         }
         }
     };
-    if (!states_ready)
-        for (int ci = 0; ci + 1 < n_chunks; ++ci) fwd_step(ci);  // every chunk before the last is full
+    for (int ci = 0; ci + 1 < n_chunks; ++ci) fwd_step(ci);  // every chunk before the last is full
 
     // ================= reverse sweep
     for (int ci = n_chunks - 1; ci >= 0; --ci) {
         const int t0 = ci * C;
         const int n = min(C, len - t0);
-        if (states_ready == 1 && (ci & 1)) fwd_step(ci - 1);  // this chunk's start state
         __syncthreads();  // previous chunk done with every buffer; ds_run, h visible
         stage_a(t0, n, true);
 
@@ -1166,7 +1160,7 @@ static cudaError_t launch_backward_t(const gdr_desc& d, const int* cu_seqlens, i
                                      const void* const* in, const float* s0,
                                      const void* dout, const float* ds_final, float* hs,
                                      float* ds_run, void* const* grads, float* ds0,
-                                     int* err_word, int states_ready, cudaStream_t st) {
+                                     int* err_word, cudaStream_t st) {
     auto kern = backward_kernel<Tin, DK, DV, sizeof(Tin) == 2>;  // bf16: tensor cores
     const size_t smem = BwdSmem<DK>::bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1177,8 +1171,7 @@ static cudaError_t launch_backward_t(const gdr_desc& d, const int* cu_seqlens, i
         d.T, d.H, cu_seqlens, (const Tin*)in[0], (const Tin*)in[1], (const Tin*)in[2], (const Tin*)in[3],
         (const Tin*)in[4], (const Tin*)in[5], (int)d.decay, (int)d.erase, (int)d.write,
         (const Tin*)dout, s0, ds_final, hs, ds_run, (Tin*)grads[0], (Tin*)grads[1],
-        (Tin*)grads[2], (Tin*)grads[3], (Tin*)grads[4], (Tin*)grads[5], ds0, err_word,
-        states_ready);
+        (Tin*)grads[2], (Tin*)grads[3], (Tin*)grads[4], (Tin*)grads[5], ds0, err_word);
     return cudaGetLastError();
 }
 
@@ -1187,12 +1180,11 @@ static cudaError_t launch_backward_d(const gdr_desc& d, const int* cu_seqlens, i
                                      const void* const* in, const float* s0,
                                      const void* dout, const float* ds_final, float* hs,
                                      float* ds_run, void* const* grads, float* ds0,
-                                     int* err_word, int states_ready, cudaStream_t st) {
+                                     int* err_word, cudaStream_t st) {
 #define GDR_BWD(DK_, DV_)                                                                  \
     if (d.dk == DK_ && d.dv == DV_)                                                        \
         return launch_backward_t<Tin, DK_, DV_>(d, cu_seqlens, n_seqs, in, s0, dout, ds_final, \
-                                                hs, ds_run, grads, ds0, err_word,            \
-                                                states_ready, st);
+                                                hs, ds_run, grads, ds0, err_word, st);
     GDR_BWD(128, 128)
     GDR_BWD(128, 64)
     GDR_BWD(64, 128)
@@ -1209,73 +1201,37 @@ static size_t state_matrices(const gdr_desc& d, bool packed, int n_seqs) {
     return packed ? (nc + (size_t)n_seqs) * d.H : nc * d.B * d.H;
 }
 
+bool backward_tc_supports(const gdr_desc& d, bool packed);
+size_t backward_tc_workspace_bytes(const gdr_desc& d);
+cudaError_t launch_backward_tc(const gdr_desc& d, const void* const* in, const float* s0,
+                               const void* dout, const float* ds_final, void* const* grads,
+                               float* ds0, void* workspace, int* err_word, cudaStream_t st);
+
 // n_seqs > 0: packed sequences; 0: the B batch rows.
 size_t backward_workspace_bytes(const gdr_desc& d, int n_seqs) {
+    if (backward_tc_supports(d, n_seqs > 0)) return backward_tc_workspace_bytes(d);
     const size_t mat = (size_t)d.dk * d.dv * sizeof(float);
     const size_t nseq = n_seqs > 0 ? (size_t)n_seqs : (size_t)d.B;
     // chunk-start states, then the running dS of every (sequence, head)
     return mat * (state_matrices(d, n_seqs > 0, n_seqs) + nseq * d.H);
 }
 
-cudaError_t launch_chunked_tc_states(const gdr_desc& d, int T_row, const void* q, const void* k,
-                                     const void* v, const void* a, const void* b,
-                                     const void* w, const float* s0, float* s_final,
-                                     float* states, int n32, int slot0, int* err_word,
-                                     cudaStream_t st);
-
-// in = {q, k, v, a, b, w}; grads = {dq, dk, dv, da, db, dw}.
+// in = {q, k, v, a, b, w}; grads = {dq, dk, dv, da, db, dw}.  bf16 with
+// dk = dv = 128 and one sequence per batch row runs on the tensor cores
+// (bwd_tc.cu); everything else on this file's kernel.
 cudaError_t launch_backward(const gdr_desc& d, const int* cu_seqlens, int n_seqs,
                             const void* const* in, const float* s0, const void* dout,
                             const float* ds_final, void* const* grads, float* ds0,
                             void* workspace, int* err_word, cudaStream_t st) {
+    if (backward_tc_supports(d, cu_seqlens != nullptr))
+        return launch_backward_tc(d, in, s0, dout, ds_final, grads, ds0, workspace, err_word, st);
     float* hs = static_cast<float*>(workspace);
     float* ds_run = hs + state_matrices(d, cu_seqlens != nullptr, n_seqs) * d.dk * d.dv;
-    if (d.in_dtype == GDR_BF16) {
-        // bf16, dk = dv = 128, one sequence per batch row: the chunk-start
-        // states come from the tensor-core forward kernel.  The whole rows
-        // give the even 32-token slots (its 64-token chunk starts); a 32-token
-        // run gives the state after token 31 (into the running-dS region,
-        // which the backward kernel initialises only later), and a run over
-        // tokens 32 .. T-1 from that state gives the odd slots.
-        int states_ready = 0;
-        if (!cu_seqlens && d.dk == 128 && d.dv == 128 && d.T > 0) {
-            gdr_desc f = d;
-            f.chunk = 64;
-            const int n32 = (d.T + BW_C - 1) / BW_C;
-            cudaError_t e = launch_chunked_tc_states(f, d.T, in[0], in[1], in[2], in[3], in[4],
-                                                     in[5], s0, nullptr, hs, n32, 0, err_word,
-                                                     st);
-            if (e != cudaSuccess) return e;
-            states_ready = 1;
-            if (d.T > BW_C) {
-                gdr_desc f1 = f;
-                f1.T = BW_C;
-                e = launch_chunked_tc_states(f1, d.T, in[0], in[1], in[2], in[3], in[4], in[5],
-                                             s0, ds_run, hs, n32, 0, err_word, st);
-                if (e != cudaSuccess) return e;
-                // the same tensors from token 32 on
-                const long long tv = (long long)BW_C * d.H * 128, ts = (long long)BW_C * d.H;
-                auto shift = [&](const void* p, int kind) -> const void* {
-                    if (!p || kind == GDR_GATE_ONE) return p;
-                    return static_cast<const __nv_bfloat16*>(p) +
-                           (kind == GDR_GATE_SCALAR ? ts : tv);
-                };
-                gdr_desc f2 = f;
-                f2.T = d.T - BW_C;
-                e = launch_chunked_tc_states(
-                    f2, d.T, shift(in[0], GDR_GATE_VECTOR), shift(in[1], GDR_GATE_VECTOR),
-                    shift(in[2], GDR_GATE_VECTOR), shift(in[3], d.decay), shift(in[4], d.erase),
-                    shift(in[5], d.write), ds_run, nullptr, hs, n32, 1, err_word, st);
-                if (e != cudaSuccess) return e;
-                states_ready = 2;
-            }
-        }
+    if (d.in_dtype == GDR_BF16)
         return launch_backward_d<__nv_bfloat16>(d, cu_seqlens, n_seqs, in, s0, dout, ds_final,
-                                                hs, ds_run, grads, ds0, err_word, states_ready,
-                                                st);
-    }
+                                                hs, ds_run, grads, ds0, err_word, st);
     return launch_backward_d<float>(d, cu_seqlens, n_seqs, in, s0, dout, ds_final, hs, ds_run,
-                                    grads, ds0, err_word, 0, st);
+                                    grads, ds0, err_word, st);
 }
 
 }  // namespace gdr

@@ -1,0 +1,918 @@
+// bwd_tc.cu -- gradients of the chunked gated delta rule on the Blackwell
+// tensor cores (tcgen05, accumulators in tensor memory) fed by TMA: bf16
+// inputs, dk = dv = 128, chunks of C = 64 tokens, one sequence per batch row.
+//
+// The pages train the recurrence through its chunkwise WY form (FG^2-GDN
+// page, gist.science 2604.19021, section 2 "Methodology"); this file
+// differentiates that form.  Per chunk (n <= 64 tokens, state S0 at its
+// start, gamma_r = prod_{t<=r} a_t per key channel, mid token m = 31,
+// g_m = gamma_m, gc = gamma_63 / g_m, Lam = gamma / g_m), with the operands
+// of the forward kernel
+//   Q' = Lam q, K' = Lam k, K" = k / Lam, B" = b K", U = w v, S~ = g_m S0
+//   A_qk = tril(Q' K"^T), A_qb = tril(Q' B"^T)      (diagonal in)
+//   A_kk = tril(K' K"^T), A_kb = tril(K' B"^T)      (strictly lower)
+//   T = (I + A_kb)^-1,  E = T (K' S~ + A_kk U)       (the forward's key reads)
+// and dS~ = gc dS_C (dS_C the gradient on the chunk's final state), the
+// reverse of the chunk is
+//   -dE = A_qb^T dO + B" dS~,       dU_p = A_qk^T dO + K" dS~
+//   dY  = T^T dE,                   dU = dU_p + A_kk^T dY
+//   D~  = dS~ + Q'^T dO + K'^T dY,  dS_0 = g_m D~      (dS_C of the chunk before)
+//   dA  = [[dO (-E)^T, dO U^T], [dY (-E)^T, dY U^T]]  masked like the grams
+//   XQ' = dO S~^T + dA_qb B" + dA_qk K",   XK' = dY S~^T + dA_kb B" + dA_kk K"
+//   YB' = -E dS~^T + dA_qb^T Q' + dA_kb^T K',  YK' = U dS~^T + dA_qk^T Q' + dA_kk^T K'
+// and the gradients follow elementwise:
+//   dq = Lam XQ',  dk = Lam XK' + (YK' + b YB') / Lam,  db = K" YB'
+//   dv = w dU,  dw = v dU,
+//   dG = Q' XQ' + K' XK' - K" YK' - B" YB'  (+ rowsum(dS_C * S_C) at row n-1,
+//        S_C the chunk's final state),  d log a_r = sum_{r' >= r} dG_r'.
+// (The last term is the derivative of <dS_C, S_C> through gamma_63, which
+// scales S_C as a whole.)  A float64 copy of these identities matched the
+// oracle's backward to 1e-15 before this file was written.
+//
+// Three launches: the tcgen05 forward kernel in its state-writing
+// instantiation (chunk-start states in float32, S_T, and every chunk's E in
+// bf16); bwd_tc_kernel, one CTA per (batch, head) walking the chunks from the
+// last, which carries D~ in tensor memory and writes XQ', XK', YK', YB', dU
+// (float32) and the per-chunk G_C terms; and bwd_epilogue_kernel, one CTA per
+// (batch, head, chunk), which forms the six gradients from them and the raw
+// inputs (the decay factors again, the reverse cumulative sum for da).
+//
+// Every product of bwd_tc_kernel is a 128-row tcgen05.mma with bf16 operands
+// and float32 accumulation: 64-token operands are stacked in pairs ([Q'; K'],
+// [B"; K"], [dO; dY], [-E; U]) so that one product yields two results, and
+// where only one exists the other half of the A operand is a zero panel.
+// The chain from dS~ to the next chunk's dS~ is three products (-dE, dY, D~)
+// with a tensor-memory readout between them.
+//
+// Decay range as in the forward kernel: each channel's decay multiplied over
+// tokens 1..31 and over 32..63 of a chunk must stay at or above 1e-35;
+// otherwise GDR_ERR_RANGE.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+
+#include "chunk_common.cuh"
+#include "common.cuh"
+#include "tc_common.cuh"
+
+namespace gdr {
+
+bool tc_map_bf16(CUtensorMap* m, const void* ptr, int B, int T, int H, int T_row);
+cudaError_t launch_chunked_tc_states(const gdr_desc& d, int T_row, const void* q, const void* k,
+                                     const void* v, const void* a, const void* b,
+                                     const void* w, const float* s0, float* s_final,
+                                     float* states, int n_slots, int slot0, void* e_out,
+                                     int* err_word, cudaStream_t st);
+
+namespace {
+
+constexpr int C = 64;         // chunk length
+constexpr int D = 128;        // dk = dv
+constexpr int NTC = 512;      // compute threads (warps 0-15)
+constexpr int NT = NTC + 32;  // + the warp that issues every TMA copy and product
+
+// ---- shared memory (bytes from a 1024-aligned base).  Operand tiles are
+// 64-column panels of 128-byte swizzled rows (tc_common.cuh); a "128-row"
+// tile has 16 KB panels, a "64-row" tile 8 KB panels.
+constexpr uint32_t OFF_QK = 0;         // [Q'; K'] 128 rows (raw q lands in rows 0-63, k in 64-127)
+constexpr uint32_t OFF_BK = 32768;     // [B"; K"] 128 rows (raw vector b / a in rows 0-63 / 64-127)
+constexpr uint32_t OFF_DOY = 65536;    // [dO; dY] 128 rows (dO lands in rows 0-63)
+constexpr uint32_t OFF_DS = 98304;     // dS~ [i][j] 128 rows, bf16
+constexpr uint32_t OFF_GQ = 131072;    // [A_qb | A_qk] 64 rows (r)
+constexpr uint32_t OFF_TZA = 147456;   // T + I, zero, A_kk: three 64 x 64 panels, 8 KB each
+constexpr uint32_t OFF_DE = 172032;    // dE 64 rows (raw vector w lands here)
+constexpr uint32_t OFF_SCR = 188416;   // scratch, in turn:
+constexpr uint32_t OFF_EIN = OFF_SCR;            //  loads: E 64 rows
+constexpr uint32_t OFF_UIN = OFF_SCR + 16384;    //  loads: v 64 rows, replaced by U
+constexpr uint32_t OFF_QT = OFF_SCR + 32768;     //  operand pass: float [8][128]
+constexpr uint32_t OFF_NS = OFF_SCR;             //  solve: A_kb, float [64][68]
+constexpr uint32_t OFF_TS = OFF_SCR + 17408;     //  solve: T, float [64][68]
+constexpr uint32_t OFF_PS = OFF_SCR + 34816;     //  solve: float [2][16][16]
+constexpr uint32_t OFF_DAT = OFF_SCR;            //  dA^T [s][r] 128 rows, bf16
+constexpr uint32_t OFF_SMALL = OFF_SCR + 36864;
+constexpr uint32_t OFF_GM = OFF_SMALL;           // float[128]: g_m of this chunk
+constexpr uint32_t OFF_GC = OFF_SMALL + 512;     // float[128]: gc of this chunk
+constexpr uint32_t OFF_GMN = OFF_SMALL + 1024;   // float[128]: g_m of the chunk after it
+constexpr uint32_t OFF_SCA = OFF_SMALL + 1536;   // float[3][64]: scalar a, b, w
+constexpr uint32_t OFF_EXP = OFF_SMALL + 2304;   // float[4][128]: partial G_C terms
+constexpr uint32_t OFF_BAR = OFF_SMALL + 4352;
+constexpr int NBAR = 13;
+constexpr uint32_t OFF_TSLOT = OFF_BAR + 8 * NBAR;
+constexpr uint32_t OFF_ABORT = OFF_TSLOT + 4;
+constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
+constexpr size_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory");
+static_assert(OFF_PS + 2048 <= OFF_SMALL && OFF_QT + 4096 <= OFF_SMALL, "scratch");
+
+// ---- tensor-memory columns (512 allocated)
+constexpr uint32_t TM_D = 0;     // D~ (lane = key channel i), float32, the running state gradient
+constexpr uint32_t TM_G = 128;   // gram, then dA^T, then [YB'; YK']
+constexpr uint32_t TM_Z = 256;   // [-dE -> dY; dU], then [XQ' | XK']^T
+constexpr uint32_t TM_S = 384;   // S~ as a bf16 A operand (lane i, 64 columns)
+constexpr uint32_t TM_EU = 448;  // [-E; U] as a bf16 A operand (lane s, 64 columns)
+
+constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait
+constexpr uint32_t BOX_BYTES = 64 * 128;     // one 64 x 64 bf16 TMA box
+
+struct BwMaps {
+    CUtensorMap q, k, v, a, b, w, dout, e;  // a/b/w only meaningful for vector gates
+};
+
+// Barriers: TMA and tensor-core completions, then the compute threads'
+// "ready" signals to the issuing warp (thread 0 arrives after a compute
+// barrier).
+enum : uint32_t {
+    B_LD, B_G, B_Z1, B_Z3, B_A, B_XY, B_FIN,   // loads / gram / -dE / dY / D~,dU,dA / X,Y / all
+    R_LD, R_OP, R_GQ, R_DE, R_DY, R_DA          // ready for: loads / gram / -dE / dY / D~,dU,dA / X,Y
+};
+static_assert(R_DA + 1 == NBAR, "barrier count");
+
+// Decay factors and scaled operands of one chunk (the forward kernel's
+// operand pass, with the backward's tile placement).  Thread (channel pair
+// p2, token octet q8); writes, one bf16 pair per token,
+//   Q' = Lam q and K' = Lam k over raw q, k (QK rows r, 64 + r)
+//   B" = b K" and K" = k / Lam over raw b, a (BK rows r, 64 + r)
+//   U  = w v over raw v
+// and per channel g_m and gc.  Lam and 1/Lam are formed as in the forward:
+// every divisor is a product of a over tokens 1..31 or 32..63 of the chunk,
+// which the range check bounds from below.
+template <bool FG2>
+__device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool vb, bool vw,
+                                             bool fb, bool fw, int a_kind, int n,
+                                             const float* sca, float* QT, float* GM, float* GC,
+                                             int* err_word) {
+    const int p2 = tid & 63, q8 = tid >> 6;
+    const uint32_t pnl = (uint32_t)(p2 >> 5);
+    const int ch = (p2 & 31) >> 2;
+    const uint32_t cofs = 4u * (uint32_t)(p2 & 3);
+    uint32_t apr[8];
+    float loc0[8], loc1[8];
+    float run0 = 1.f, run1 = 1.f;
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+        const int r = 8 * q8 + x;
+        // raw a in rows 64-127 of BK (row 64 + r swizzles like row r)
+        uint32_t pr = va ? *reinterpret_cast<const uint32_t*>(
+                               sm + OFF_BK + pnl * 16384u + (uint32_t)(64 + r) * 128u +
+                               ((uint32_t)(ch ^ (r & 7)) << 4) + cofs)
+                         : tc::pack_bf16x2(sca[r], sca[r]);
+        apr[x] = (a_kind != GDR_GATE_ONE && r < n) ? pr : 0x3F803F80u;
+        const float a0 = __uint_as_float(apr[x] << 16), a1 = __uint_as_float(apr[x] & 0xFFFF0000u);
+        if (r > 0) {
+            run0 *= a0;
+            run1 *= a1;
+        }
+        loc0[x] = run0;
+        loc1[x] = run1;
+    }
+    const float f0 = q8 == 0 ? __uint_as_float(apr[0] << 16) : 1.f;
+    const float f1 = q8 == 0 ? __uint_as_float(apr[0] & 0xFFFF0000u) : 1.f;
+    *reinterpret_cast<float2*>(QT + q8 * D + 2 * p2) = make_float2(f0 * run0, f1 * run1);
+    compute_sync();
+    float gm0 = 1.f, gm1 = 1.f, gc0 = 1.f, gc1 = 1.f, sp0 = 1.f, sp1 = 1.f, mp0 = 1.f,
+          mp1 = 1.f;
+#pragma unroll
+    for (int gg = 0; gg < 8; ++gg) {
+        const float2 qv = *reinterpret_cast<const float2*>(QT + gg * D + 2 * p2);
+        if (gg < 4) { gm0 *= qv.x; gm1 *= qv.y; } else { gc0 *= qv.x; gc1 *= qv.y; }
+        if (gg > q8 && gg < 4) { sp0 *= qv.x; sp1 *= qv.y; }
+        if (gg >= 4 && gg < q8) { mp0 *= qv.x; mp1 *= qv.y; }
+    }
+    auto emit = [&](int x, uint32_t e, uint32_t ei) {
+        const int r = 8 * q8 + x;
+        const uint32_t sw = (uint32_t)r * 128u + ((uint32_t)(ch ^ (r & 7)) << 4) + cofs;
+        const uint32_t o128 = pnl * 16384u + sw, o64 = pnl * 8192u + sw;
+        const uint32_t q2 = *reinterpret_cast<const uint32_t*>(sm + OFF_QK + o128);
+        const uint32_t k2 = *reinterpret_cast<const uint32_t*>(sm + OFF_QK + o128 + 8192u);
+        const uint32_t b2 = vb ? *reinterpret_cast<const uint32_t*>(sm + OFF_BK + o128)
+                               : tc::pack_bf16x2(sca[64 + r], sca[64 + r]);
+        const uint32_t v2 = *reinterpret_cast<const uint32_t*>(sm + OFF_UIN + o64);
+        const uint32_t w2 = vw ? *reinterpret_cast<const uint32_t*>(sm + OFF_DE + o64)
+                               : tc::pack_bf16x2(sca[128 + r], sca[128 + r]);
+        // FG^2-GDN learning rates: key sqrt(beta^k) k with erase gate 1, write
+        // gate sqrt(beta^v)
+        const uint32_t kt2 = (FG2 && fb) ? mul2(k2, sqrt2(b2)) : k2;
+        const uint32_t kk2 = mul2(kt2, ei);
+        *reinterpret_cast<uint32_t*>(sm + OFF_QK + o128) = mul2(q2, e);            // Q'
+        *reinterpret_cast<uint32_t*>(sm + OFF_QK + o128 + 8192u) = mul2(kt2, e);   // K'
+        *reinterpret_cast<uint32_t*>(sm + OFF_BK + o128) =
+            (FG2 && fb) ? kk2 : mul2(b2, kk2);                                    // B"
+        *reinterpret_cast<uint32_t*>(sm + OFF_BK + o128 + 8192u) = kk2;           // K"
+        *reinterpret_cast<uint32_t*>(sm + OFF_UIN + o64) =
+            mul2((FG2 && fw) ? sqrt2(w2) : w2, v2);                               // U
+    };
+    float rev0 = 1.f, rev1 = 1.f;
+    if (q8 < 4) {  // warp-uniform
+        const float d0 = rcp_approx(sp0 * run0), d1 = rcp_approx(sp1 * run1);
+#pragma unroll
+        for (int x = 7; x >= 0; --x) {
+            emit(x, tc::pack_bf16x2(loc0[x] * d0, loc1[x] * d1),
+                 tc::pack_bf16x2(rev0 * sp0, rev1 * sp1));
+            rev0 *= __uint_as_float(apr[x] << 16);
+            rev1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
+        }
+    } else {
+        const float d0 = rcp_approx(mp0 * run0), d1 = rcp_approx(mp1 * run1);
+#pragma unroll
+        for (int x = 7; x >= 0; --x) {
+            emit(x, tc::pack_bf16x2(mp0 * loc0[x], mp1 * loc1[x]),
+                 tc::pack_bf16x2(rev0 * d0, rev1 * d1));
+            rev0 *= __uint_as_float(apr[x] << 16);
+            rev1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
+        }
+    }
+    if (q8 == 0) {
+        const int i = 2 * p2;
+        GM[i] = gm0;
+        GM[i + 1] = gm1;
+        GC[i] = gc0;
+        GC[i + 1] = gc1;
+        const bool ok0 = run0 * sp0 >= 1e-35f && gc0 >= 1e-35f;
+        const bool ok1 = run1 * sp1 >= 1e-35f && gc1 >= 1e-35f;
+        if (a_kind != GDR_GATE_ONE && !(ok0 && ok1)) atomicOr(err_word, kErrRange);
+    }
+}
+
+__device__ __forceinline__ void wait_then_sync(uint32_t bar, uint32_t parity, int tid,
+                                               volatile int* abort_s) {
+    if (tid == 0 && !*abort_s && !tc::mbar_wait_bounded(bar, parity, WAIT_NS)) *abort_s = 1;
+    compute_sync();
+    tc::fence_after_sync();
+}
+
+// One row of 32 floats to global memory (16-byte stores).
+__device__ __forceinline__ void store_row32_f32(float* dst, const float* v) {
+    float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int x = 0; x < 8; ++x)
+        d4[x] = make_float4(v[4 * x], v[4 * x + 1], v[4 * x + 2], v[4 * x + 3]);
+}
+
+// The reverse sweep.  states: [B*H][NC][128][128] chunk-start states; sT
+// [B*H][128][128] the final states; xq .. du: [B, T, H, 128] float32
+// outputs; gce: [B*H][NC][128] the G_C terms.
+template <bool FG2>
+__global__ void __launch_bounds__(NT, 1)
+bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
+              const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
+              const __nv_bfloat16* __restrict__ w, int a_kind, int b_kind, int w_kind,
+              const float* __restrict__ ds_final, const float* __restrict__ states,
+              const float* __restrict__ sT, float* __restrict__ xq, float* __restrict__ xk,
+              float* __restrict__ yk, float* __restrict__ yb, float* __restrict__ du,
+              float* __restrict__ gce, float* __restrict__ ds0, int* __restrict__ err_word) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = tc::smem_u32(sm);
+    float* QT = reinterpret_cast<float*>(sm + OFF_QT);
+    float* NS = reinterpret_cast<float*>(sm + OFF_NS);
+    float* TS = reinterpret_cast<float*>(sm + OFF_TS);
+    float* PS = reinterpret_cast<float*>(sm + OFF_PS);
+    float* GM = reinterpret_cast<float*>(sm + OFF_GM);
+    float* GC = reinterpret_cast<float*>(sm + OFF_GC);
+    float* GMN = reinterpret_cast<float*>(sm + OFF_GMN);
+    float* sca = reinterpret_cast<float*>(sm + OFF_SCA);
+    float* EXP = reinterpret_cast<float*>(sm + OFF_EXP);
+    volatile int* abort_s = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
+    auto bar = [&](uint32_t id) { return sbase + OFF_BAR + 8u * id; };
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int quarter = warp & 3;                  // tensor-memory lanes 32*quarter ..
+    const int cb = warp >> 2;                      // 32-column block this warp reads
+    const int lane_t = 32 * quarter + (tid & 31);  // tensor-memory lane of this thread
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+
+    const int bh = blockIdx.x;
+    const int hi = bh % H, bi = bh / H;
+    const int NC = (T + C - 1) / C;
+    const size_t soff = (size_t)bh * D * D;
+    const bool fb = b_kind == GDR_GATE_FG2, fw = w_kind == GDR_GATE_FG2;
+    const bool va = a_kind == GDR_GATE_VECTOR, vb = b_kind == GDR_GATE_VECTOR || fb,
+               vw = w_kind == GDR_GATE_VECTOR || fw;
+
+    if (tid == 0) {
+#pragma unroll 1
+        for (int i = 0; i < NBAR; ++i) tc::mbar_init(bar(i), 1);
+        tc::mbar_fence_init();
+        *abort_s = 0;
+    }
+    if (tid < D) GMN[tid] = 1.0f;
+    // the zero panel of TZA, and the 16 x 16 blocks above the diagonal of
+    // T + I (never written by the solve)
+    if (tid < NTC) {
+        const int r = tid >> 3, c16 = tid & 7;
+        if ((c16 >> 1) > (r >> 4))
+            *reinterpret_cast<uint4*>(sm + OFF_TZA + r * 128 + ((c16 ^ (r & 7)) << 4)) =
+                make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(sm + OFF_TZA + 8192 + 16 * tid) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (warp == 0) tc::tmem_alloc(sbase + OFF_TSLOT, 512);
+    tc::fence_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + OFF_TSLOT);
+
+    if (warp == NTC / 32) {
+        // ======================= issuing warp (one thread)
+        if ((tid & 31) == 0 && NC > 0) {
+            tc::tma_prefetch_desc(&maps.q);
+            tc::tma_prefetch_desc(&maps.k);
+            tc::tma_prefetch_desc(&maps.v);
+            tc::tma_prefetch_desc(&maps.dout);
+            tc::tma_prefetch_desc(&maps.e);
+            uint32_t ph = 0;
+            uint32_t n_ld = 0;
+            auto wait_ready = [&](uint32_t id, uint32_t parity) {
+                if (!tc::mbar_wait_bounded(bar(id), parity, WAIT_NS)) { *abort_s = 1; return false; }
+                tc::fence_after_sync();
+                return *abort_s == 0;
+            };
+            const uint32_t idKK = tc::idesc_bf16(128, 128, 0, 0);
+            const uint32_t idKM = tc::idesc_bf16(128, 128, 0, 1);
+            const uint32_t idMM = tc::idesc_bf16(128, 128, 1, 1);
+            const uint32_t nbox = 10u + (va ? 2u : 0u) + (vb ? 2u : 0u) + (vw ? 2u : 0u);
+            int it = 0;
+#pragma unroll 1
+            for (int c = NC - 1; c >= 0; --c, ph ^= 1, ++it) {
+                const int t0 = c * C;
+                // the previous chunk's tiles are free (its last products and
+                // readouts are done)
+                if (it > 0 && !wait_ready(R_LD, ph ^ 1)) break;
+                tc::mbar_arrive_expect_tx(bar(B_LD), nbox * BOX_BYTES);
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    const int x = 64 * p;
+                    tc::tma_load_4d(sbase + OFF_QK + p * 16384, &maps.q, x, hi, t0, bi, bar(B_LD));
+                    tc::tma_load_4d(sbase + OFF_QK + p * 16384 + 8192, &maps.k, x, hi, t0, bi,
+                                    bar(B_LD));
+                    if (vb)
+                        tc::tma_load_4d(sbase + OFF_BK + p * 16384, &maps.b, x, hi, t0, bi,
+                                        bar(B_LD));
+                    if (va)
+                        tc::tma_load_4d(sbase + OFF_BK + p * 16384 + 8192, &maps.a, x, hi, t0, bi,
+                                        bar(B_LD));
+                    tc::tma_load_4d(sbase + OFF_DOY + p * 16384, &maps.dout, x, hi, t0, bi,
+                                    bar(B_LD));
+                    tc::tma_load_4d(sbase + OFF_EIN + p * 8192, &maps.e, x, hi, t0, bi, bar(B_LD));
+                    tc::tma_load_4d(sbase + OFF_UIN + p * 8192, &maps.v, x, hi, t0, bi, bar(B_LD));
+                    if (vw)
+                        tc::tma_load_4d(sbase + OFF_DE + p * 8192, &maps.w, x, hi, t0, bi, bar(B_LD));
+                }
+                ++n_ld;
+                // gram [Q'; K'] [B"; K"]^T; Z = [B"; K"] dS~; D~ += Q'^T dO
+                if (!wait_ready(R_OP, ph)) break;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16(tmem + TM_G, tc::desc_kmajor(sbase + OFF_QK, 16384, kk),
+                                 tc::desc_kmajor(sbase + OFF_BK, 16384, kk), idKK, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16(tmem + TM_Z, tc::desc_kmajor(sbase + OFF_BK, 16384, kk),
+                                 tc::desc_mnmajor(sbase + OFF_DS, 16384, kk), idKM, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_D, tc::desc_mnmajor(sbase + OFF_QK, 16384, kk),
+                                 tc::desc_mnmajor(sbase + OFF_DOY, 16384, kk), idMM, true);
+                tc::mma_commit(bar(B_G));
+                // Z += [A_qb^T; A_qk^T] dO: rows 0-63 become -dE, rows 64-127 dU_p
+                if (!wait_ready(R_GQ, ph)) break;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_Z, tc::desc_mnmajor(sbase + OFF_GQ, 8192, kk),
+                                 tc::desc_mnmajor(sbase + OFF_DOY, 16384, kk), idMM, true);
+                tc::mma_commit(bar(B_Z1));
+                // Z += [T^T + I; 0] dE: rows 0-63 become dY
+                if (!wait_ready(R_DE, ph)) break;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_Z, tc::desc_mnmajor(sbase + OFF_TZA, 8192, kk),
+                                 tc::desc_mnmajor(sbase + OFF_DE, 8192, kk), idMM, true);
+                tc::mma_commit(bar(B_Z3));
+                // D~ += K'^T dY;  Z += [0; A_kk^T] dY (rows 64-127 become dU);
+                // dA^T = [-E; U] [dO; dY]^T
+                if (!wait_ready(R_DY, ph)) break;
+#pragma unroll
+                for (int kk = 4; kk < 8; ++kk)
+                    tc::mma_bf16(tmem + TM_D, tc::desc_mnmajor(sbase + OFF_QK, 16384, kk),
+                                 tc::desc_mnmajor(sbase + OFF_DOY, 16384, kk), idMM, true);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_bf16(tmem + TM_Z, tc::desc_mnmajor(sbase + OFF_TZA + 8192, 8192, kk),
+                                 tc::desc_mnmajor(sbase + OFF_DOY + 8192, 16384, kk), idMM, true);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16_ts(tmem + TM_G, tmem + TM_EU + 8 * kk,
+                                    tc::desc_kmajor(sbase + OFF_DOY, 16384, kk), idKK, kk > 0);
+                tc::mma_commit(bar(B_A));
+                // [XQ' | XK']^T = S~ [dO; dY]^T + [B"; K"]^T dA^T   (lane = channel)
+                // [YB'; YK']   = [-E; U] dS~^T + dA^T [Q'; K']      (lane = token)
+                if (!wait_ready(R_DA, ph)) break;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16_ts(tmem + TM_Z, tmem + TM_S + 8 * kk,
+                                    tc::desc_kmajor(sbase + OFF_DOY, 16384, kk), idKK, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16(tmem + TM_Z, tc::desc_mnmajor(sbase + OFF_BK, 16384, kk),
+                                 tc::desc_mnmajor(sbase + OFF_DAT, 16384, kk), idMM, true);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16_ts(tmem + TM_G, tmem + TM_EU + 8 * kk,
+                                    tc::desc_kmajor(sbase + OFF_DS, 16384, kk), idKK, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_bf16(tmem + TM_G, tc::desc_kmajor(sbase + OFF_DAT, 16384, kk),
+                                 tc::desc_mnmajor(sbase + OFF_QK, 16384, kk), idKM, true);
+                tc::mma_commit(bar(B_XY));
+            }
+            // nothing of this CTA may still be in flight when it exits
+            tc::mma_commit(bar(B_FIN));
+            tc::mbar_wait_bounded(bar(B_FIN), 0, WAIT_NS);
+            if (n_ld) tc::mbar_wait_bounded(bar(B_LD), (n_ld - 1) & 1, WAIT_NS);
+        }
+    } else {
+        // ======================= compute warps
+        // D~ = dS_T (unscaled: the first chunk's rescale takes it as dS_C)
+        {
+            float vals[32];
+            if (ds_final) {
+                const float4* src =
+                    reinterpret_cast<const float4*>(ds_final + soff + (size_t)lane_t * D + 32 * cb);
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const float4 v4 = src[x];
+                    vals[4 * x] = v4.x; vals[4 * x + 1] = v4.y;
+                    vals[4 * x + 2] = v4.z; vals[4 * x + 3] = v4.w;
+                }
+            } else {
+#pragma unroll
+                for (int x = 0; x < 32; ++x) vals[x] = 0.f;
+            }
+            tc::tmem_st32(tmem + lane_off + TM_D + 32 * cb, vals);
+            tc::tmem_wait_st();
+        }
+        uint32_t ph = 0;
+        auto signal_or_stop = [&](uint32_t id) {
+            const bool stop = compute_sync_or(*abort_s != 0);
+            if (tid == 0) tc::mbar_arrive(bar(id));
+            return stop;
+        };
+        auto tok_row = [&](int t) { return ((size_t)bi * T + t) * H + hi; };
+#pragma unroll 1
+        for (int c = NC - 1; c >= 0; --c, ph ^= 1) {
+            const int t0 = c * C;
+            const int n = min(C, T - t0);
+            // ================= C1: scalar gates, the chunk's tiles, the operand pass
+            if (tid < C) {
+                const long long tok = ((long long)bi * T + t0 + tid) * H + hi;
+                const bool in = tid < n;
+                sca[tid] = (a_kind == GDR_GATE_SCALAR && in) ? to_f32(a[tok]) : 1.f;
+                sca[64 + tid] = (b_kind == GDR_GATE_SCALAR && in) ? to_f32(b[tok]) : 1.f;
+                sca[128 + tid] = (w_kind == GDR_GATE_SCALAR && in) ? to_f32(w[tok]) : 1.f;
+            }
+            if (tid == 0 && !*abort_s && !tc::mbar_wait_bounded(bar(B_LD), ph, WAIT_NS))
+                *abort_s = 1;
+            if (compute_sync_or(*abort_s != 0)) break;
+            operand_pass<FG2>(sm, tid, va, vb, vw, fb, fw, a_kind, n, sca, QT, GM, GC, err_word);
+            compute_sync();
+            // ================= C1b: [-E; U] and S~ into tensor memory; the rescale
+            {
+                // [-E; U]: lane s of the stack, 32 value columns
+                const int s = lane_t & 63;
+                const uint8_t* src = sm + (lane_t < 64 ? OFF_EIN : OFF_UIN) + (cb >> 1) * 8192 + s * 128;
+                const uint32_t flip = lane_t < 64 ? 0x80008000u : 0u;
+                uint32_t words[16];
+#pragma unroll
+                for (int qd = 0; qd < 4; ++qd) {
+                    const int c16 = 4 * (cb & 1) + qd;
+                    const uint4 u = *reinterpret_cast<const uint4*>(src + ((c16 ^ (s & 7)) << 4));
+                    words[4 * qd] = u.x ^ flip;
+                    words[4 * qd + 1] = u.y ^ flip;
+                    words[4 * qd + 2] = u.z ^ flip;
+                    words[4 * qd + 3] = u.w ^ flip;
+                }
+                tc::tmem_st16(tmem + lane_off + TM_EU + 16 * cb, words);
+            }
+            {
+                // S~ = g_m S0: lane i, 32 value columns
+                const float g = GM[lane_t];
+                const float4* src = reinterpret_cast<const float4*>(
+                    states + ((size_t)bh * NC + c) * D * D + (size_t)lane_t * D + 32 * cb);
+                uint32_t words[16];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const float4 v4 = src[x];
+                    words[2 * x] = tc::pack_bf16x2(v4.x * g, v4.y * g);
+                    words[2 * x + 1] = tc::pack_bf16x2(v4.z * g, v4.w * g);
+                }
+                tc::tmem_st16(tmem + lane_off + TM_S + 16 * cb, words);
+            }
+            {
+                // dS_C = g_m(next) D~;  its share of the G_C term, rowsum(dS_C * S_C);
+                // dS~ = gc dS_C into tensor memory and, bf16, into OFF_DS
+                float vals[32];
+                tc::tmem_ld32(tmem + lane_off + TM_D + 32 * cb, vals);
+                tc::tmem_wait_ld();
+                const float fn = GMN[lane_t], fc = GC[lane_t];
+                const float* scp = (c == NC - 1 ? sT + soff
+                                                : states + ((size_t)bh * NC + c + 1) * D * D) +
+                                   (size_t)lane_t * D + 32 * cb;
+                const float4* sc4 = reinterpret_cast<const float4*>(scp);
+                float part = 0.f;
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const float4 s4 = sc4[x];
+                    vals[4 * x] *= fn; vals[4 * x + 1] *= fn;
+                    vals[4 * x + 2] *= fn; vals[4 * x + 3] *= fn;
+                    part = fmaf(vals[4 * x], s4.x, part);
+                    part = fmaf(vals[4 * x + 1], s4.y, part);
+                    part = fmaf(vals[4 * x + 2], s4.z, part);
+                    part = fmaf(vals[4 * x + 3], s4.w, part);
+                }
+#pragma unroll
+                for (int x = 0; x < 32; ++x) vals[x] *= fc;
+                EXP[cb * D + lane_t] = part;
+                tc::tmem_st32(tmem + lane_off + TM_D + 32 * cb, vals);
+                tc::store_row32_bf16(sm + OFF_DS + (cb >> 1) * 16384, lane_t, cb & 1, vals);
+            }
+            tc::tmem_wait_st();
+            tc::fence_async_smem();
+            tc::fence_before_sync();
+            if (signal_or_stop(R_OP)) break;
+
+            // ================= C2: the G_C term out; the gram's blocks
+            if (tid < D) {
+                gce[((size_t)bh * NC + c) * D + tid] =
+                    (EXP[tid] + EXP[D + tid]) + (EXP[2 * D + tid] + EXP[3 * D + tid]);
+                GMN[tid] = GM[tid];
+            }
+            wait_then_sync(bar(B_G), ph, tid, abort_s);
+            {
+                // rows r of Q' (lanes 0-63) or K' (lanes 64-127); this warp's 32 x 32
+                // block lies below (mode < 0), on (0) or above (> 0) the diagonal
+                // of its 64 x 64 gram block: warp-uniform
+                const bool top = lane_t < 64;
+                const int r = lane_t & 63;
+                const int s0c = 32 * (cb & 1);
+                const int mode = (cb & 1) - (quarter & 1);
+                float vals[32];
+                if (mode > 0) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) vals[x] = 0.f;
+                } else {
+                    tc::tmem_ld32(tmem + lane_off + TM_G + 32 * cb, vals);
+                    tc::tmem_wait_ld();
+                    if (mode == 0) {
+                        const int lim = top ? r - s0c + 1 : r - s0c;
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) vals[x] = x < lim ? vals[x] : 0.f;
+                    }
+                }
+                if (top) {           // A_qb (cb 0-1), A_qk (cb 2-3)
+                    tc::store_row32_bf16(sm + OFF_GQ + (cb >> 1) * 8192, r, cb & 1, vals);
+                } else if (cb < 2) { // A_kb, for the solve
+                    float* nrow = NS + r * NSP + s0c;
+#pragma unroll
+                    for (int x = 0; x < 32; x += 4)
+                        st4(nrow + x, make_float4(vals[x], vals[x + 1], vals[x + 2], vals[x + 3]));
+                } else {             // A_kk
+                    tc::store_row32_bf16(sm + OFF_TZA + 16384, r, cb & 1, vals);
+                }
+            }
+            tc::fence_async_smem();
+            tc::fence_before_sync();
+            if (signal_or_stop(R_GQ)) break;
+
+            // ================= C3: warps 8-15 solve T + I; warps 0-7 read -dE
+            if (warp >= 8) {
+                ut_solve<2>(NS, TS, PS, sm + OFF_TZA, tid - 256);
+                tc::fence_async_smem();
+            } else {
+                if (tid == 0 && !*abort_s && !tc::mbar_wait_bounded(bar(B_Z1), ph, WAIT_NS))
+                    *abort_s = 1;
+                half_sync(3);
+                tc::fence_after_sync();
+                if (quarter < 2) {  // warps 0, 1, 4, 5: lanes 0-63, 64 columns each
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float vals[32];
+                        tc::tmem_ld32(tmem + lane_off + TM_Z + 64 * cb + 32 * hh, vals);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) vals[x] = -vals[x];
+                        tc::store_row32_bf16(sm + OFF_DE + cb * 8192, lane_t, hh, vals);
+                    }
+                }
+                tc::fence_async_smem();
+            }
+            tc::fence_before_sync();
+            if (signal_or_stop(R_DE)) break;
+
+            // ================= C4: dY -> rows 64-127 of [dO; dY]
+            wait_then_sync(bar(B_Z3), ph, tid, abort_s);
+            if (quarter < 2) {
+                float vals[32];
+                tc::tmem_ld32(tmem + lane_off + TM_Z + 32 * cb, vals);
+                tc::tmem_wait_ld();
+                tc::store_row32_bf16(sm + OFF_DOY + (cb >> 1) * 16384, 64 + lane_t, cb & 1, vals);
+            }
+            tc::fence_async_smem();
+            tc::fence_before_sync();
+            if (signal_or_stop(R_DY)) break;
+
+            // ================= C5: dA^T masked -> bf16; dU out
+            wait_then_sync(bar(B_A), ph, tid, abort_s);
+            {
+                // lane s of [-E; U], columns r of [dO; dY]: keep r >= s against dO,
+                // r > s against dY; block relation as for the gram
+                const int s = lane_t & 63;
+                const int rb = 32 * (cb & 1);
+                const int mode = (quarter & 1) - (cb & 1);
+                float vals[32];
+                if (mode > 0) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) vals[x] = 0.f;
+                } else {
+                    tc::tmem_ld32(tmem + lane_off + TM_G + 32 * cb, vals);
+                    tc::tmem_wait_ld();
+                    if (mode == 0) {
+                        const int lim = s - rb + (cb >= 2 ? 1 : 0);  // keep x >= lim
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) vals[x] = x >= lim ? vals[x] : 0.f;
+                    }
+                }
+                tc::store_row32_bf16(sm + OFF_DAT + (cb >> 1) * 16384, lane_t, cb & 1, vals);
+            }
+            if (quarter >= 2) {
+                const int s = lane_t - 64;
+                float vals[32];
+                tc::tmem_ld32(tmem + lane_off + TM_Z + 32 * cb, vals);
+                tc::tmem_wait_ld();
+                if (s < n) store_row32_f32(du + tok_row(t0 + s) * D + 32 * cb, vals);
+            }
+            tc::fence_async_smem();
+            tc::fence_before_sync();
+            if (signal_or_stop(R_DA)) break;
+
+            // ================= C6: [XQ' | XK']^T and [YB'; YK'] out
+            wait_then_sync(bar(B_XY), ph, tid, abort_s);
+            {
+                float vals[32];
+                tc::tmem_ld32(tmem + lane_off + TM_Z + 32 * cb, vals);
+                tc::tmem_wait_ld();
+                float* dst = cb < 2 ? xq : xk;
+                const int r0 = 32 * (cb & 1);
+#pragma unroll
+                for (int x = 0; x < 32; ++x)
+                    if (r0 + x < n) dst[tok_row(t0 + r0 + x) * D + lane_t] = vals[x];
+            }
+            {
+                float vals[32];
+                tc::tmem_ld32(tmem + lane_off + TM_G + 32 * cb, vals);
+                tc::tmem_wait_ld();
+                const int s = lane_t & 63;
+                if (s < n) store_row32_f32((lane_t < 64 ? yb : yk) + tok_row(t0 + s) * D + 32 * cb,
+                                           vals);
+            }
+            tc::fence_before_sync();
+            if (signal_or_stop(R_LD)) break;
+        }
+        // dS0 = g_m(first chunk) D~
+        if (ds0 && NC > 0 && !compute_sync_or(*abort_s != 0)) {
+            float vals[32];
+            tc::tmem_ld32(tmem + lane_off + TM_D + 32 * cb, vals);
+            tc::tmem_wait_ld();
+            const float g = GMN[lane_t];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) vals[x] *= g;
+            store_row32_f32(ds0 + soff + (size_t)lane_t * D + 32 * cb, vals);
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    if (*abort_s) {
+        if (tid == 0) atomicOr(err_word, kErrTimeout);
+    }
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_free(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------- epilogue
+// One CTA per (batch, head, chunk), thread = key/value channel i.  From the
+// raw inputs and the reverse sweep's XQ', XK', YK', YB', dU and G_C terms:
+//   Lam_r = 1 / prod_{t=r+1}^{31} a_t (r <= 31),  prod_{t=32}^{r} a_t (r >= 32)
+//   dq = Lam XQ', dk = Lam XK' + (YK' + b YB') / Lam, db = K" YB',
+//   dv = w dU, dw = v dU, d log a by the reverse cumulative sum of dG,
+//   da = d log a / a.
+// Scalar gates take the sum over channels.  FG^2-GDN learning rates: the
+// gradients of the key sqrt(beta^k) k and write gate sqrt(beta^v) carried
+// through the square roots (dk = sqrt(beta^k) dk~, dbeta^k = k dk~ /
+// (2 sqrt(beta^k)), dbeta^v = v dU / (2 sqrt(beta^v))).
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
+
+__global__ void __launch_bounds__(D)
+bwd_epilogue_kernel(int T, int H, int NC, const __nv_bfloat16* __restrict__ q,
+                    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                    const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
+                    const __nv_bfloat16* __restrict__ w, int a_kind, int b_kind, int w_kind,
+                    const float* __restrict__ xq, const float* __restrict__ xk,
+                    const float* __restrict__ yk, const float* __restrict__ yb,
+                    const float* __restrict__ du, const float* __restrict__ gce,
+                    __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk,
+                    __nv_bfloat16* __restrict__ dv, __nv_bfloat16* __restrict__ da,
+                    __nv_bfloat16* __restrict__ db, __nv_bfloat16* __restrict__ dw) {
+    __shared__ float lam2[32][D];    // Lam of tokens 32..63
+    __shared__ float red[3][C][4];   // scalar gates: per-warp sums of da, db, dw
+    const int i = threadIdx.x, warp = i >> 5, lane = i & 31;
+    const int c = blockIdx.x % NC, bh = blockIdx.x / NC;
+    const int hi = bh % H, bi = bh / H;
+    const int t0 = c * C, n = min(C, T - t0);
+    const bool fb = b_kind == GDR_GATE_FG2, fw = w_kind == GDR_GATE_FG2;
+    auto tok = [&](int r) { return ((long long)bi * T + t0 + r) * H + hi; };
+    auto aval = [&](int r) -> float {
+        if (r >= n || a_kind == GDR_GATE_ONE) return 1.f;
+        return a_kind == GDR_GATE_SCALAR ? to_f32(a[tok(r)]) : to_f32(a[tok(r) * D + i]);
+    };
+    auto gval = [&](const __nv_bfloat16* g, int kind, int r) -> float {
+        if (kind == GDR_GATE_ONE) return 1.f;
+        return kind == GDR_GATE_SCALAR ? to_f32(g[tok(r)]) : to_f32(g[tok(r) * D + i]);
+    };
+    {
+        float run = 1.f;
+#pragma unroll 1
+        for (int r = 32; r < C; ++r) {
+            run *= aval(r);
+            lam2[r - 32][i] = run;
+        }
+    }
+    float P = 1.f;     // prod_{t=r+1}^{31} a_t while r <= 31
+    float cum = 0.f;   // d log a_r, channel i
+    const float gterm = gce[((size_t)bh * NC + c) * D + i];
+#pragma unroll 1
+    for (int r = C - 1; r >= 0; --r) {
+        if (r < n) {
+            const float lam = r >= 32 ? lam2[r - 32][i] : 1.f / P;
+            const float lami = r >= 32 ? 1.f / lam2[r - 32][i] : P;
+            const long long tv = tok(r) * D + i;
+            const float qv = to_f32(q[tv]), kv = to_f32(k[tv]), vv = to_f32(v[tv]);
+            const float bv = gval(b, b_kind, r), wv = gval(w, w_kind, r);
+            const float sbk = fb ? sqrt_fast(fmaxf(bv, 0.f)) : 1.f;   // sqrt(beta^k)
+            const float kt = kv * sbk;                                 // the key used
+            const float bt = fb ? 1.f : bv;                            // the erase gate used
+            const float wt = fw ? sqrt_fast(fmaxf(wv, 0.f)) : wv;      // the write gate used
+            const float XQ = xq[tv], XK = xk[tv], YK = yk[tv], YB = yb[tv], dU = du[tv];
+            const float Kpp = lami * kt;
+            float dG = lam * (qv * XQ + kt * XK) - Kpp * (YK + bt * YB);
+            if (r == n - 1) dG += gterm;
+            cum += dG;
+            const float dkt = lam * XK + lami * (YK + bt * YB);
+            dq[tv] = __float2bfloat16_rn(lam * XQ);
+            dk[tv] = __float2bfloat16_rn(dkt * sbk);
+            dv[tv] = __float2bfloat16_rn(wt * dU);
+            // erase gate
+            if (b_kind == GDR_GATE_VECTOR) {
+                db[tv] = __float2bfloat16_rn(Kpp * YB);
+            } else if (fb) {
+                db[tv] = __float2bfloat16_rn(kv * dkt / (2.f * sbk));
+            } else if (b_kind == GDR_GATE_SCALAR) {
+                const float s = warp_sum(Kpp * YB);
+                if (lane == 0) red[1][r][warp] = s;
+            }
+            // write gate
+            if (w_kind == GDR_GATE_VECTOR) {
+                dw[tv] = __float2bfloat16_rn(vv * dU);
+            } else if (fw) {
+                dw[tv] = __float2bfloat16_rn(vv * dU / (2.f * wt));
+            } else if (w_kind == GDR_GATE_SCALAR) {
+                const float s = warp_sum(vv * dU);
+                if (lane == 0) red[2][r][warp] = s;
+            }
+            // decay
+            if (a_kind == GDR_GATE_VECTOR) {
+                da[tv] = __float2bfloat16_rn(cum / aval(r));
+            } else if (a_kind == GDR_GATE_SCALAR) {
+                const float s = warp_sum(cum);
+                if (lane == 0) red[0][r][warp] = s;
+            }
+        }
+        if (r <= 31) P *= aval(r);
+    }
+    if (a_kind == GDR_GATE_SCALAR || b_kind == GDR_GATE_SCALAR || w_kind == GDR_GATE_SCALAR) {
+        __syncthreads();
+        if (i < n) {
+            const long long ts = tok(i);
+            if (a_kind == GDR_GATE_SCALAR) {
+                const float s = (red[0][i][0] + red[0][i][1]) + (red[0][i][2] + red[0][i][3]);
+                da[ts] = __float2bfloat16_rn(s / to_f32(a[ts]));
+            }
+            if (b_kind == GDR_GATE_SCALAR)
+                db[ts] = __float2bfloat16_rn((red[1][i][0] + red[1][i][1]) +
+                                             (red[1][i][2] + red[1][i][3]));
+            if (w_kind == GDR_GATE_SCALAR)
+                dw[ts] = __float2bfloat16_rn((red[2][i][0] + red[2][i][1]) +
+                                             (red[2][i][2] + red[2][i][3]));
+        }
+    }
+}
+
+inline size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct TcWorkspace {
+    float* states;   // [B*H][NC][128][128]
+    float* sT;       // [B*H][128][128]
+    void* e;         // [B, T, H, 128] bf16
+    float* pre[5];   // XQ', XK', YK', YB', dU: [B, T, H, 128] float32
+    float* gce;      // [B*H][NC][128]
+    size_t bytes;
+};
+
+TcWorkspace carve(const gdr_desc& d, void* base) {
+    const size_t bh = (size_t)d.B * d.H, nc = ((size_t)d.T + C - 1) / C;
+    const size_t tok = (size_t)d.B * d.T * d.H;
+    TcWorkspace w;
+    uint8_t* p = static_cast<uint8_t*>(base);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        uint8_t* r = p ? p + off : nullptr;
+        off += round256(bytes);
+        return r;
+    };
+    w.states = reinterpret_cast<float*>(take(bh * nc * D * D * 4));
+    w.sT = reinterpret_cast<float*>(take(bh * D * D * 4));
+    w.e = take(tok * D * 2);
+    for (int x = 0; x < 5; ++x) w.pre[x] = reinterpret_cast<float*>(take(tok * D * 4));
+    w.gce = reinterpret_cast<float*>(take(bh * nc * D * 4));
+    w.bytes = off;
+    return w;
+}
+
+}  // namespace
+
+// The tensor-core backward handles bf16, dk = dv = 128, one sequence per
+// batch row, at least one token.
+bool backward_tc_supports(const gdr_desc& d, bool packed) {
+    return !packed && d.in_dtype == GDR_BF16 && d.dk == D && d.dv == D && d.T > 0;
+}
+
+size_t backward_tc_workspace_bytes(const gdr_desc& d) { return carve(d, nullptr).bytes; }
+
+// in = {q, k, v, a, b, w}; grads = {dq, dk, dv, da, db, dw}.
+cudaError_t launch_backward_tc(const gdr_desc& d, const void* const* in, const float* s0,
+                               const void* dout, const float* ds_final, void* const* grads,
+                               float* ds0, void* workspace, int* err_word, cudaStream_t st) {
+    const TcWorkspace ws = carve(d, workspace);
+    const int NC = (d.T + C - 1) / C;
+    gdr_desc f = d;
+    f.chunk = C;
+    cudaError_t e = launch_chunked_tc_states(f, d.T, in[0], in[1], in[2], in[3], in[4], in[5], s0,
+                                             ws.sT, ws.states, NC, 0, ws.e, err_word, st);
+    if (e != cudaSuccess) return e;
+
+    BwMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    const int B = d.B, T = d.T, H = d.H;
+    bool ok = tc_map_bf16(&maps.q, in[0], B, T, H, T) && tc_map_bf16(&maps.k, in[1], B, T, H, T) &&
+              tc_map_bf16(&maps.v, in[2], B, T, H, T) &&
+              tc_map_bf16(&maps.dout, dout, B, T, H, T) && tc_map_bf16(&maps.e, ws.e, B, T, H, T);
+    if (ok && d.decay == GDR_GATE_VECTOR) ok = tc_map_bf16(&maps.a, in[3], B, T, H, T);
+    if (ok && (d.erase == GDR_GATE_VECTOR || d.erase == GDR_GATE_FG2))
+        ok = tc_map_bf16(&maps.b, in[4], B, T, H, T);
+    if (ok && (d.write == GDR_GATE_VECTOR || d.write == GDR_GATE_FG2))
+        ok = tc_map_bf16(&maps.w, in[5], B, T, H, T);
+    if (!ok) return cudaErrorInvalidValue;
+
+    const bool fg2 = d.erase == GDR_GATE_FG2 || d.write == GDR_GATE_FG2;
+    auto kern = fg2 ? bwd_tc_kernel<true> : bwd_tc_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const auto* a = static_cast<const __nv_bfloat16*>(in[3]);
+    const auto* b = static_cast<const __nv_bfloat16*>(in[4]);
+    const auto* w = static_cast<const __nv_bfloat16*>(in[5]);
+    kern<<<(unsigned)((long long)B * H), NT, SMEM_BYTES, st>>>(
+        maps, B, T, H, a, b, w, (int)d.decay, (int)d.erase, (int)d.write, ds_final, ws.states,
+        ws.sT, ws.pre[0], ws.pre[1], ws.pre[2], ws.pre[3], ws.pre[4], ws.gce, ds0, err_word);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    bwd_epilogue_kernel<<<(unsigned)((long long)B * H * NC), D, 0, st>>>(
+        T, H, NC, static_cast<const __nv_bfloat16*>(in[0]),
+        static_cast<const __nv_bfloat16*>(in[1]), static_cast<const __nv_bfloat16*>(in[2]), a, b,
+        w, (int)d.decay, (int)d.erase, (int)d.write, ws.pre[0], ws.pre[1], ws.pre[2], ws.pre[3],
+        ws.pre[4], ws.gce, static_cast<__nv_bfloat16*>(grads[0]),
+        static_cast<__nv_bfloat16*>(grads[1]), static_cast<__nv_bfloat16*>(grads[2]),
+        static_cast<__nv_bfloat16*>(grads[3]), static_cast<__nv_bfloat16*>(grads[4]),
+        static_cast<__nv_bfloat16*>(grads[5]));
+    return cudaGetLastError();
+}
+
+}  // namespace gdr

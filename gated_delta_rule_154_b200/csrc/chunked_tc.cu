@@ -46,6 +46,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "chunk_common.cuh"
 #include "common.cuh"
 #include "tc_common.cuh"
 
@@ -92,8 +93,6 @@ static_assert(SMEM_BYTES <= 232448, "shared memory");
 static_assert(OFF_PS + 2 * 256 * 4 <= OFF_SMALL, "solve scratch");
 static_assert(OFF_QT >= OFF_OST + 16384 && OFF_QT + 8 * 128 * 4 <= OFF_SMALL, "QT placement");
 
-constexpr int NSP = 68;  // row stride (floats) of the solve's float tiles (16-byte rows)
-
 // ---- tensor-memory columns (512 allocated)
 constexpr uint32_t TM_G = 0;     // gram 128 x 128
 constexpr uint32_t TM_X = 128;   // [R -> E; O] 128 x 128
@@ -107,193 +106,6 @@ constexpr uint32_t IDESC_NEG_B = 1u << 14;   // negate the B operand
 struct TcMaps {
     CUtensorMap q, k, v, a, b, w, o;  // a/b/w only meaningful for vector gates
 };
-
-// Two packed bf16 products, each rounded once to bf16
-__device__ __forceinline__ uint32_t mul2(uint32_t x, uint32_t y) {
-    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&x),
-                               *reinterpret_cast<__nv_bfloat162*>(&y));
-    return *reinterpret_cast<uint32_t*>(&r);
-}
-// Square root to about 1 ulp (one SFU op); its results are rounded to bf16.
-__device__ __forceinline__ float sqrt_approx(float x) {
-    float y;
-    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-// Square roots of two packed bf16 (non-negative by contract; a negative
-// input gives 0), each rounded to bf16.
-__device__ __forceinline__ uint32_t sqrt2(uint32_t x) {
-    return tc::pack_bf16x2(sqrt_approx(fmaxf(__uint_as_float(x << 16), 0.f)),
-                           sqrt_approx(fmaxf(__uint_as_float(x & 0xFFFF0000u), 0.f)));
-}
-// Reciprocal to about 1 ulp (one SFU op); its results are rounded to bf16.
-__device__ __forceinline__ float rcp_approx(float x) {
-    float y;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-__device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
-
-// Named barriers: id 1 = the 16 compute warps, id 2 = warps 0-7, id 3 =
-// warps 8-15.  (Id 0, __syncthreads, includes the issuing warp.)
-__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
-// The compute barrier returning the OR of `x` over the 512 compute threads:
-// all of them get the same answer, so they leave the chunk loop together even
-// when the issuing warp raises the abort flag while they pass the barrier.
-__device__ __forceinline__ bool compute_sync_or(bool x) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, 1, 512, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}\n"
-        : "=r"(r)
-        : "r"((uint32_t)x)
-        : "memory");
-    return r != 0;
-}
-__device__ __forceinline__ void half_sync(int id) {
-    asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");
-}
-
-// ---------------------------------------------------------------- UT solve
-// T = (I + N)^{-1}, N = A_kb strictly lower 64 x 64 (float, row stride NSP, in
-// NS), by the 2 x 2 block recursion of a unit lower triangular inverse,
-//   [[T1, 0], [T21, T2]] with T21 = -T2 N21 T1,
-// applied at 16 and at 32 rows: the four 16 x 16 diagonal inverses by
-// substitution, then two rounds for the 16 x 16 blocks (1,0) and (3,2), then
-// two for the 32 x 32 block below the diagonal.  Run by warps 0-7 (barrier
-// id 2).  Each finished block also goes, as bf16 T - I, into rows 0-63 of
-// the Z3 operand; the blocks above the diagonal of those rows stay zero.
-
-// One element of T - I into the 128-byte swizzled Z3 rows.
-__device__ __forceinline__ void z3_put(uint8_t* z3, int row, int col, float v) {
-    *reinterpret_cast<__nv_bfloat16*>(z3 + row * 128 + (((col >> 3) ^ (row & 7)) << 4) +
-                                      2 * (col & 7)) = __float2bfloat16_rn(v);
-}
-__device__ __forceinline__ void z3_put2(uint8_t* z3, int row, int col, float v0, float v1) {
-    *reinterpret_cast<uint32_t*>(z3 + row * 128 + (((col >> 3) ^ (row & 7)) << 4) +
-                                 2 * (col & 7)) = tc::pack_bf16x2(v0, v1);
-}
-
-__device__ __forceinline__ void ut_diag(const float* NS, float* TS, uint8_t* z3, int tid) {
-    if (tid < 64) {
-        // column c of the inverse of diagonal block I: x_r = [r == c] - sum_{s<r} N_rs x_s,
-        // each row of N read as 16-byte vectors, two partial sums per row
-        const int I = tid >> 4, c = tid & 15;
-        const float* nb = NS + (16 * I) * NSP + 16 * I;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.0f : 0.0f;
-#pragma unroll
-        for (int r = 1; r < 16; ++r) {
-            const float* row = nb + r * NSP;
-            float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-            for (int s4 = 0; 4 * s4 < r; ++s4) {
-                const float4 v = *reinterpret_cast<const float4*>(row + 4 * s4);
-                if (4 * s4 + 0 < r) acc0 = fmaf(v.x, x[4 * s4 + 0], acc0);
-                if (4 * s4 + 1 < r) acc1 = fmaf(v.y, x[4 * s4 + 1], acc1);
-                if (4 * s4 + 2 < r) acc0 = fmaf(v.z, x[4 * s4 + 2], acc0);
-                if (4 * s4 + 3 < r) acc1 = fmaf(v.w, x[4 * s4 + 3], acc1);
-            }
-            x[r] -= acc0 + acc1;
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            TS[(16 * I + r) * NSP + 16 * I + c] = x[r];
-            z3_put(z3, 16 * I + r, 16 * I + c, r > c ? x[r] : 0.f);
-        }
-    }
-    half_sync(2);
-}
-
-// tf32 operand of mma.sync (round to nearest, ties away)
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-// D(16x8) += A(16x8) B(8x8), tf32 inputs, float32 accumulate (one warp).
-__device__ __forceinline__ void mma_tf32_16x8x8(float* d, const uint32_t* a, const uint32_t* b) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-// d = A(16 x 8KS) B(8KS x 8) for float tiles in shared memory (A at its
-// (0,0) with row stride lda, B likewise with ldb).  The block products of
-// the solve are tiny and latency-bound, so they use the warp-level mma.sync
-// path in tf32 (T is rounded to bf16 afterwards); the chunk's large products
-// stay on tcgen05.  Fragments: g = lane/4, t = lane%4; A rows g, g+8 and
-// columns t, t+4; B rows t, t+4 and column g; D rows g, g+8, columns 2t, 2t+1.
-template <int KS>
-__device__ __forceinline__ void tile_16x8(float* d, const float* A, int lda, const float* Bm,
-                                          int ldb, int g, int t) {
-    d[0] = d[1] = d[2] = d[3] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-        const float* a0 = A + g * lda + 8 * ks + t;
-        const float* b0 = Bm + (8 * ks + t) * ldb + g;
-        const uint32_t af[4] = {to_tf32(a0[0]), to_tf32(a0[8 * lda]), to_tf32(a0[4]),
-                                to_tf32(a0[8 * lda + 4])};
-        const uint32_t bfr[2] = {to_tf32(b0[0]), to_tf32(b0[4 * ldb])};
-        mma_tf32_16x8x8(d, af, bfr);
-    }
-}
-
-__device__ __forceinline__ void ut_solve(float* NS, float* TS, float* PS, uint8_t* z3, int tid) {
-    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-    ut_diag(NS, TS, z3, tid);
-    // blocks (1,0) and (3,2): P = N_IJ T_JJ, then T_IJ = -T_II P (warps 0-3)
-    const int b = warp >> 1, nt = warp & 1;
-    const int I = 2 * b + 1, J = 2 * b;
-    float d[4];
-    if (warp < 4) {
-        tile_16x8<2>(d, NS + (16 * I) * NSP + 16 * J, NSP, TS + (16 * J) * NSP + 16 * J + 8 * nt,
-                     NSP, g, t);
-        float* pp = PS + b * 256 + 8 * nt + 2 * t;
-        *reinterpret_cast<float2*>(pp + g * 16) = make_float2(d[0], d[1]);
-        *reinterpret_cast<float2*>(pp + (g + 8) * 16) = make_float2(d[2], d[3]);
-    }
-    half_sync(2);
-    if (warp < 4) {
-        tile_16x8<2>(d, TS + (16 * I) * NSP + 16 * I, NSP, PS + b * 256 + 8 * nt, 16, g, t);
-        const int row = 16 * I + g, col = 16 * J + 8 * nt + 2 * t;
-        *reinterpret_cast<float2*>(TS + row * NSP + col) = make_float2(-d[0], -d[1]);
-        *reinterpret_cast<float2*>(TS + (row + 8) * NSP + col) = make_float2(-d[2], -d[3]);
-        z3_put2(z3, row, col, -d[0], -d[1]);
-        z3_put2(z3, row + 8, col, -d[2], -d[3]);
-    }
-    half_sync(2);
-    // Y = N21 T1 (rows 32-63 of N, columns 0-31), kept in the unused upper
-    // right quadrant of NS: block (i, j) sums over the blocks s = j..1 of T1.
-    const int i2 = warp >> 2, j2 = (warp >> 1) & 1;
-    {
-        const float* A = NS + (32 + 16 * i2) * NSP + 16 * j2;
-        const float* Bm = TS + (16 * j2) * NSP + 16 * j2 + 8 * nt;
-        if (j2 == 0) tile_16x8<4>(d, A, NSP, Bm, NSP, g, t);
-        else tile_16x8<2>(d, A, NSP, Bm, NSP, g, t);
-        float* yp = NS + (16 * i2 + g) * NSP + 32 + 16 * j2 + 8 * nt + 2 * t;
-        *reinterpret_cast<float2*>(yp) = make_float2(d[0], d[1]);
-        *reinterpret_cast<float2*>(yp + 8 * NSP) = make_float2(d[2], d[3]);
-    }
-    half_sync(2);
-    // T21 = -T2 Y: block (i, j) sums T2[i][s] Y[s][j] over s = 0..i
-    {
-        const float* A = TS + (32 + 16 * i2) * NSP + 32;
-        const float* Bm = NS + 32 + 16 * j2 + 8 * nt;
-        if (i2 == 0) tile_16x8<2>(d, A, NSP, Bm, NSP, g, t);
-        else tile_16x8<4>(d, A, NSP, Bm, NSP, g, t);
-        const int row = 32 + 16 * i2 + g, col = 16 * j2 + 8 * nt + 2 * t;
-        *reinterpret_cast<float2*>(TS + row * NSP + col) = make_float2(-d[0], -d[1]);
-        *reinterpret_cast<float2*>(TS + (row + 8) * NSP + col) = make_float2(-d[2], -d[3]);
-        z3_put2(z3, row, col, -d[0], -d[1]);
-        z3_put2(z3, row + 8, col, -d[2], -d[3]);
-    }
-}
 
 // ---------------------------------------------------------------- TMA issue
 // Group "kqw": raw k and q into RAW, vector w into W.  Group "ab": vector a
@@ -490,11 +302,12 @@ static_assert(R_O + 1 == NBAR, "barrier count");
 // PACKED: packed sequences (rows past a sequence's end are zeroed rather than
 // left to the TMA fill).  FG2: FG^2-GDN learning rates among the gates.  DUMP:
 // no o; instead the state at the start of every chunk goes to `states`,
-// [B*H][n32][128][128] float32 at slots slot0, slot0 + 2, ... (the
-// backward's layout of 32-token chunk-start states).  All compile-time, so
-// the plain instantiation carries none of these tests.  T_row: tokens
-// between batch rows in memory (T, or more when the launch covers a token
-// range of longer rows).
+// [B*H][n_slots][128][128] float32 at slots slot0, slot0 + 1, ..., and, when
+// o_raw is given, each chunk's E (the key reads, bf16 [B, T, H, 128]) to
+// o_raw through the o tensor map: what the backward reads back.  All
+// compile-time, so the plain instantiation carries none of these tests.
+// T_row: tokens between batch rows in memory (T, or more when the launch
+// covers a token range of longer rows).
 template <bool PACKED, bool FG2, bool DUMP>
 __global__ void __launch_bounds__(NT, 1)
 chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
@@ -503,7 +316,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                   const float* __restrict__ s0, float* __restrict__ s_final,
                   int* __restrict__ err_word, int skip_signal,
                   const int* __restrict__ cu_seqlens, __nv_bfloat16* __restrict__ o_raw,
-                  float* __restrict__ states, int n32, int slot0, int T_row) {
+                  float* __restrict__ states, int n_slots, int slot0, int T_row) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -570,7 +383,8 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             tc::tma_prefetch_desc(&maps.q);
             tc::tma_prefetch_desc(&maps.k);
             tc::tma_prefetch_desc(&maps.v);
-            if (!DUMP) tc::tma_prefetch_desc(&maps.o);
+            const bool dump_e = DUMP && o_raw != nullptr;
+            if (!DUMP || dump_e) tc::tma_prefetch_desc(&maps.o);
             uint32_t ph = 0;               // phase of the per-chunk barriers
             uint32_t n_kqw = 0, n_ab = 0, n_v = 0;
             issue_kqw(maps, sbase, tb, hi, bi, vw, bar(B_KQW)); ++n_kqw;
@@ -644,6 +458,11 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                 tc::mma_commit(bar(B_E));
                 // X += [0; -A_qb] E (rows 64-127 become O); S~ -= B"^T E
                 if (!wait_ready(R_E)) break;
+                if (dump_e) {  // E leaves by TMA (its tile is next reused after the gram)
+                    tc::tma_store_4d(&maps.o, sbase + OFF_EB, 0, hi, tb + t0, bi);
+                    tc::tma_store_4d(&maps.o, sbase + OFF_EB + 8192, 64, hi, tb + t0, bi);
+                    tc::bulk_commit();
+                }
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_Z3 + 8192, 8192, kk),
@@ -764,7 +583,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                 if (DUMP) {  // the true state at the chunk start, row lane_t
                     const float fs = fstart[lane_t];
                     float4* dst = reinterpret_cast<float4*>(
-                        states + ((size_t)bh * n32 + slot0 + 2 * (t0 / C)) * D * D +
+                        states + ((size_t)bh * n_slots + slot0 + t0 / C) * D * D +
                         (size_t)lane_t * D + c0);
 #pragma unroll
                     for (int x = 0; x < 8; ++x)
@@ -831,7 +650,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             if (warp >= 8) {
                 tc::fence_async_smem();
                 half_sync(2);
-                ut_solve(NS, TS, PS, sm + OFF_Z3, tid - 256);
+                ut_solve<0>(NS, TS, PS, sm + OFF_Z3, tid - 256);
                 tc::fence_async_smem();
             } else {
                 tc::fence_before_sync();
@@ -968,6 +787,12 @@ bool make_map(CUtensorMap* m, const void* ptr, int B, int T, int H, int T_row) {
 
 }  // namespace
 
+// [B, T, H, 128] bf16 tensor map of the kernels' operand format (used by the
+// backward's kernel too).
+bool tc_map_bf16(CUtensorMap* m, const void* ptr, int B, int T, int H, int T_row) {
+    return make_map(m, ptr, B, T, H, T_row);
+}
+
 bool chunked_tc_supports(const gdr_desc& d) {
     return d.in_dtype == GDR_BF16 && d.dk == D && d.dv == D && d.chunk == C;
 }
@@ -1014,17 +839,18 @@ cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, c
 }
 
 // The states at the start of every 64-token chunk of the B x H sequences
-// (no o) into slots slot0, slot0 + 2, ... of `states` ([B*H][n32][128][128]
-// float32): the backward's chunk-start states.  The launch covers d.T tokens
-// of rows T_row tokens apart (the pointers already at its first token);
-// s_final, if given, receives the state after them.
+// (no o) into slots slot0, slot0 + 1, ... of `states` ([B*H][n_slots][128][128]
+// float32), and, if e_out is given, every chunk's E (bf16 [B, T, H, 128]):
+// what the backward reads back.  The launch covers d.T tokens of rows T_row
+// tokens apart (the pointers already at its first token); s_final, if
+// given, receives the state after them.
 cudaError_t launch_chunked_tc_states(const gdr_desc& d, int T_row, const void* q, const void* k,
                                      const void* v, const void* a, const void* b,
                                      const void* w, const float* s0, float* s_final,
-                                     float* states, int n32, int slot0, int* err_word,
-                                     cudaStream_t st) {
+                                     float* states, int n_slots, int slot0, void* e_out,
+                                     int* err_word, cudaStream_t st) {
     TcMaps maps;
-    if (!make_maps(&maps, d, T_row, q, k, v, a, b, w, nullptr)) return cudaErrorInvalidValue;
+    if (!make_maps(&maps, d, T_row, q, k, v, a, b, w, e_out)) return cudaErrorInvalidValue;
     const bool fg2 = d.erase == GDR_GATE_FG2 || d.write == GDR_GATE_FG2;
     auto kern = fg2 ? chunked_tc_kernel<false, true, true> : chunked_tc_kernel<false, false, true>;
     cudaError_t e = cudaFuncSetAttribute(kern,
@@ -1034,7 +860,7 @@ cudaError_t launch_chunked_tc_states(const gdr_desc& d, int T_row, const void* q
     kern<<<(unsigned)((long long)d.B * d.H), NT, SMEM_BYTES, st>>>(
         maps, d.B, d.T, d.H, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b,
         (const __nv_bfloat16*)w, (int)d.decay, (int)d.erase, (int)d.write, s0, s_final,
-        err_word, 0, nullptr, nullptr, states, n32, slot0, T_row);
+        err_word, 0, nullptr, (__nv_bfloat16*)e_out, states, n_slots, slot0, T_row);
     return cudaGetLastError();
 }
 

@@ -189,10 +189,15 @@ gdr_status gdr_decode_step_paged(const gdr_desc *desc, const void *q, const void
                                  const void *w, float *state_pool, const int *slot,
                                  int n_slots, void *o, gdr_stream_t stream);
 
-/* Bytes of device workspace gdr_backward_chunked needs for `desc`: the state
- * at the start of every 32-token chunk plus one running state gradient, i.e.
- * B * H * dk * dv * 4 * (ceil(T / 32) + 1); 0 if desc is invalid.  Pure host
- * function, no CUDA call. */
+/* Bytes of device workspace gdr_backward_chunked needs for `desc`; 0 if desc
+ * is invalid.  Pure host function, no CUDA call.
+ *   - bf16 with dk = dv = 128 and T > 0 (the tensor-core path): the state at
+ *     the start of every 64-token chunk and the final state (float32), every
+ *     chunk's E (bf16), five float32 [B, T, H, 128] intermediates and one
+ *     float32 row per chunk and head:
+ *     B * H * (ceil(T / 64) * 66048 + 65536) + B * T * H * 2816 bytes.
+ *   - otherwise: the state at the start of every 32-token chunk plus one
+ *     running state gradient, B * H * dk * dv * 4 * (ceil(T / 32) + 1). */
 size_t gdr_backward_workspace_size(const gdr_desc *desc);
 
 /*
@@ -202,18 +207,21 @@ size_t gdr_backward_workspace_size(const gdr_desc *desc);
  * the call writes dL/dq, dL/dk, dL/dv, dL/da, dL/db, dL/dw and dL/ds0.  The
  * pages train this recurrence through its chunkwise (WY) form (FG^2-GDN
  * page, section 2 "Methodology"); the call differentiates that form: a
- * forward pass stores the state at the start of every 32-token chunk in the
+ * forward pass stores the state at the start of every chunk in the
  * workspace, then one CTA per (batch, head) walks the chunks backwards
- * carrying dS.  On bf16 inputs with dk = dv = 128 that forward pass is a
- * launch of the tensor-core prefill kernel (the states at its 64-token chunk
- * starts) ahead of the backward kernel, which adds the states in between.
- * bf16 inputs: the backward's products on the tensor cores with tf32
- * operands and float32 accumulation; float32 inputs: float32 arithmetic on
- * the CUDA cores.  Equal, up to rounding, to differentiating the
- * token-by-token recurrence.
+ * carrying dS.
+ *   - bf16 inputs with dk = dv = 128, T > 0: chunks of 64 tokens, three
+ *     launches.  The tensor-core prefill kernel writes the chunk-start
+ *     states, S_T and each chunk's key reads E; the reverse sweep runs every
+ *     product on the tensor cores (bf16 operands, float32 accumulation, dS
+ *     carried in float32); an elementwise kernel forms the gradients.
+ *   - otherwise (float32 inputs, d = 64): chunks of 32 tokens, one launch;
+ *     bf16 products on the tensor cores with tf32 operands, float32 inputs
+ *     in float32 on the CUDA cores.
+ * Equal, up to rounding, to differentiating the token-by-token recurrence.
  *
  *   q .. w, s0  the forward's inputs (s0 NULL for zeros); desc->chunk is not
- *            used (the pass always takes chunks of 32 tokens)
+ *            used (the pass picks its chunk length as above)
  *   d_o      [B, T, H, dv] in_dtype, the gradient on o
  *   ds_final [B, H, dk, dv] float32, the gradient on S_T, or NULL for zero
  *   dq, dk   [B, T, H, dk] in_dtype, written
@@ -230,9 +238,11 @@ size_t gdr_backward_workspace_size(const gdr_desc *desc);
  *   workspace, ws_bytes  device scratch of gdr_backward_workspace_size(desc)
  *
  * Outputs must not overlap the inputs.  Supported: dk, dv in {64, 128},
- * float32 or bf16 inputs, every gate kind.  Decay range: every channel's decay, multiplied over
- * each 32-token chunk, must stay at or above exp(-80); otherwise the device
- * error word reports GDR_ERR_RANGE and the gradients are undefined.
+ * float32 or bf16 inputs, every gate kind.  Decay range: every channel's
+ * decay, multiplied over each 32-token chunk (tensor-core path: over tokens
+ * 1-31 and 32-63 of each 64-token chunk), must stay at or above exp(-80)
+ * (1e-35); otherwise the device error word reports GDR_ERR_RANGE and the
+ * gradients are undefined.
  */
 gdr_status gdr_backward_chunked(const gdr_desc *desc, const void *q, const void *k,
                                 const void *v, const void *a, const void *b,
@@ -282,7 +292,7 @@ gdr_status gdr_backward_varlen(const gdr_desc *desc, const int *cu_seqlens, int 
  * cudaMalloc, no cudaFree, no allocating library routine.
  *   - Size limit: when gdr_backward_workspace_size(desc) exceeds
  *     GDR_NOALLOC_SCRATCH_BYTES the call returns GDR_ERR_WORKSPACE before any
- *     CUDA call (e.g. dk = dv = 128: B * H * (ceil(T / 32) + 1) <= 1024).
+ *     CUDA call (e.g. bf16, dk = dv = 128, B * H = 1: up to about 17k tokens).
  *   - First call on a device: it looks up the scratch's device address with
  *     cudaGetSymbolAddress on the current device and caches it.  Make that
  *     first call on each device before any stream capture begins.
