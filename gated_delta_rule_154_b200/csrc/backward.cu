@@ -1,6 +1,8 @@
-// backward.cu -- gradients of the chunked gated delta rule: the products on
-// the tensor cores (mma.sync, tf32 operands, float32 accumulation) for bf16
-// inputs, on the CUDA cores in float32 for float32 inputs.
+// backward.cu -- gradients of the chunked gated delta rule for the cases the
+// tcgen05 backward (bwd_tc.cu: bf16, dk = dv = 128, one sequence per batch
+// row) does not take: float32 inputs (products on the CUDA cores in
+// float32), head dimension 64 and packed sequences (bf16: products on the
+// tensor cores as mma.sync with tf32 operands, float32 accumulation).
 //
 // Loss L = sum_t <o_t, do_t> + <S_T, dS_T>; the kernel returns dL/dq, dk, dv,
 // the three gates and dS_0.  The pages train the recurrence in its chunked

@@ -30,12 +30,15 @@
 // oracle's backward to 1e-15 before this file was written.
 //
 // Three launches: the tcgen05 forward kernel in its state-writing
-// instantiation (chunk-start states in float32, S_T, and every chunk's E in
-// bf16); bwd_tc_kernel, one CTA per (batch, head) walking the chunks from the
-// last, which carries D~ in tensor memory and writes XQ', XK', YK', YB', dU
-// (float32) and the per-chunk G_C terms; and bwd_epilogue_kernel, one CTA per
-// (batch, head, chunk), which forms the six gradients from them and the raw
-// inputs (the decay factors again, the reverse cumulative sum for da).
+// instantiation (every chunk's S~ and E in bf16, exactly the tiles its own
+// products read, and S_T in float32); bwd_tc_kernel, one CTA per (batch,
+// head) walking the chunks from the last, which carries D~ in tensor memory
+// and writes XQ', XK', YK', YB', dU (float32, by TMA store) and per chunk
+// the G_C terms and gc; and bwd_epilogue_kernel, one warp per (batch, head,
+// chunk), which forms the six gradients from them and the raw inputs (the
+// reverse cumulative sum for da).  The G_C term of a chunk is rowsum(D~ S~)
+// of the chunk after it (dS_C = g_m D~ and S_C = S~ / g_m there), and
+// rowsum(dS_T S_T) for the last.
 //
 // Every product of bwd_tc_kernel is a 128-row tcgen05.mma with bf16 operands
 // and float32 accumulation: 64-token operands are stacked in pairs ([Q'; K'],
@@ -59,10 +62,12 @@
 namespace gdr {
 
 bool tc_map_bf16(CUtensorMap* m, const void* ptr, int B, int T, int H, int T_row);
+bool tc_map_f32(CUtensorMap* m, const void* ptr, int B, int T, int H);
+bool tc_map_state_bf16(CUtensorMap* m, const void* ptr, long long n_slots);
 cudaError_t launch_chunked_tc_states(const gdr_desc& d, int T_row, const void* q, const void* k,
                                      const void* v, const void* a, const void* b,
                                      const void* w, const float* s0, float* s_final,
-                                     float* states, int n_slots, int slot0, void* e_out,
+                                     void* s_tilde, int n_slots, int slot0, void* e_out,
                                      int* err_word, cudaStream_t st);
 
 namespace {
@@ -78,7 +83,7 @@ constexpr int NT = NTC + 32;  // + the warp that issues every TMA copy and produ
 constexpr uint32_t OFF_QK = 0;         // [Q'; K'] 128 rows (raw q lands in rows 0-63, k in 64-127)
 constexpr uint32_t OFF_BK = 32768;     // [B"; K"] 128 rows (raw vector b / a in rows 0-63 / 64-127)
 constexpr uint32_t OFF_DOY = 65536;    // [dO; dY] 128 rows (dO lands in rows 0-63)
-constexpr uint32_t OFF_DS = 98304;     // dS~ [i][j] 128 rows, bf16
+constexpr uint32_t OFF_DS = 98304;     // S~ lands here [i][j] 128 rows, bf16; then dS~
 constexpr uint32_t OFF_GQ = 131072;    // [A_qb | A_qk] 64 rows (r)
 constexpr uint32_t OFF_TZA = 147456;   // T + I, zero, A_kk: three 64 x 64 panels, 8 KB each
 constexpr uint32_t OFF_DE = 172032;    // dE 64 rows (raw vector w lands here)
@@ -116,8 +121,31 @@ constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait
 constexpr uint32_t BOX_BYTES = 64 * 128;     // one 64 x 64 bf16 TMA box
 
 struct BwMaps {
-    CUtensorMap q, k, v, a, b, w, dout, e;  // a/b/w only meaningful for vector gates
+    CUtensorMap q, k, v, a, b, w, dout, e;  // bf16 inputs (a/b/w only for vector gates)
+    CUtensorMap sst;                        // the forward's S~ tiles
+    CUtensorMap xq, xk, yk, yb, du;         // float32 outputs, 32-channel slabs
 };
+
+// Staging of the float32 outputs for their TMA stores: four 8 KB slabs (64
+// tokens x 32 channels, 128-byte swizzled rows) per tensor.  XQ', XK', YB',
+// YK' go where [Q'; K'], [B"; K"], [dO; dY] and dS~ were once the chunk's
+// last products are done; dU goes into the A_qb/A_qk and dE tiles, free
+// once the products that read them are done.
+__device__ __forceinline__ uint32_t slab_du(int p) {
+    return p < 2 ? OFF_GQ + 8192u * p : OFF_DE + 8192u * (p - 2);
+}
+// byte offset of float (row r, channel c) in a staged tile
+__device__ __forceinline__ uint32_t stage_off(int r, int c) {
+    return 8192u * (uint32_t)(c >> 5) + 128u * (uint32_t)r +
+           ((uint32_t)(((c & 31) >> 2) ^ (r & 7)) << 4) + 4u * (uint32_t)(c & 3);
+}
+// one row of 32 channels (slab base given) as eight 16-byte stores
+__device__ __forceinline__ void stage_row32(uint8_t* slab, int r, const float* v) {
+#pragma unroll
+    for (int c16 = 0; c16 < 8; ++c16)
+        *reinterpret_cast<float4*>(slab + 128 * r + ((c16 ^ (r & 7)) << 4)) =
+            make_float4(v[4 * c16], v[4 * c16 + 1], v[4 * c16 + 2], v[4 * c16 + 3]);
+}
 
 // Barriers: TMA and tensor-core completions, then the compute threads'
 // "ready" signals to the issuing warp (thread 0 arrives after a compute
@@ -249,18 +277,17 @@ __device__ __forceinline__ void store_row32_f32(float* dst, const float* v) {
         d4[x] = make_float4(v[4 * x], v[4 * x + 1], v[4 * x + 2], v[4 * x + 3]);
 }
 
-// The reverse sweep.  states: [B*H][NC][128][128] chunk-start states; sT
-// [B*H][128][128] the final states; xq .. du: [B, T, H, 128] float32
-// outputs; gce: [B*H][NC][128] the G_C terms.
+// The reverse sweep.  S~ of every chunk arrives through the sst map
+// ([B*H][NC][128][128] bf16); sT [B*H][128][128] the final states; XQ', XK',
+// YK', YB', dU leave through the float32 maps; gce, gcs: [B*H][NC][128] the
+// G_C terms and gc.
 template <bool FG2>
 __global__ void __launch_bounds__(NT, 1)
 bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
               const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
               const __nv_bfloat16* __restrict__ w, int a_kind, int b_kind, int w_kind,
-              const float* __restrict__ ds_final, const float* __restrict__ states,
-              const float* __restrict__ sT, float* __restrict__ xq, float* __restrict__ xk,
-              float* __restrict__ yk, float* __restrict__ yb, float* __restrict__ du,
-              float* __restrict__ gce, float* __restrict__ ds0, int* __restrict__ err_word) {
+              const float* __restrict__ ds_final, const float* __restrict__ sT, float* __restrict__ gce, float* __restrict__ gcs,
+              float* __restrict__ ds0, int* __restrict__ err_word) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -323,6 +350,7 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             tc::tma_prefetch_desc(&maps.v);
             tc::tma_prefetch_desc(&maps.dout);
             tc::tma_prefetch_desc(&maps.e);
+            tc::tma_prefetch_desc(&maps.sst);
             uint32_t ph = 0;
             uint32_t n_ld = 0;
             auto wait_ready = [&](uint32_t id, uint32_t parity) {
@@ -334,14 +362,32 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             const uint32_t idKM = tc::idesc_bf16(128, 128, 0, 1);
             const uint32_t idMM = tc::idesc_bf16(128, 128, 1, 1);
             const uint32_t nbox = 10u + (va ? 2u : 0u) + (vb ? 2u : 0u) + (vw ? 2u : 0u);
+            // the chunk's XQ', XK', YB', YK' from their staging tiles
+            auto store_xy = [&](int t0s) {
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const int x = 32 * p;
+                    tc::tma_store_4d(&maps.xq, sbase + OFF_QK + 8192 * p, x, hi, t0s, bi);
+                    tc::tma_store_4d(&maps.xk, sbase + OFF_BK + 8192 * p, x, hi, t0s, bi);
+                    tc::tma_store_4d(&maps.yb, sbase + OFF_DOY + 8192 * p, x, hi, t0s, bi);
+                    tc::tma_store_4d(&maps.yk, sbase + OFF_DS + 8192 * p, x, hi, t0s, bi);
+                }
+                tc::bulk_commit();
+            };
             int it = 0;
+            bool done = true;
 #pragma unroll 1
             for (int c = NC - 1; c >= 0; --c, ph ^= 1, ++it) {
                 const int t0 = c * C;
-                // the previous chunk's tiles are free (its last products and
-                // readouts are done)
-                if (it > 0 && !wait_ready(R_LD, ph ^ 1)) break;
-                tc::mbar_arrive_expect_tx(bar(B_LD), nbox * BOX_BYTES);
+                done = false;
+                // the previous chunk's outputs are staged: store them, and load
+                // this chunk's tiles once the stores have read their staging
+                if (it > 0) {
+                    if (!wait_ready(R_LD, ph ^ 1)) break;
+                    store_xy(t0 + C);
+                    tc::bulk_wait_read();
+                }
+                tc::mbar_arrive_expect_tx(bar(B_LD), nbox * BOX_BYTES + 2u * 16384u);
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
                     const int x = 64 * p;
@@ -360,6 +406,8 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                     tc::tma_load_4d(sbase + OFF_UIN + p * 8192, &maps.v, x, hi, t0, bi, bar(B_LD));
                     if (vw)
                         tc::tma_load_4d(sbase + OFF_DE + p * 8192, &maps.w, x, hi, t0, bi, bar(B_LD));
+                    tc::tma_load_4d(sbase + OFF_DS + p * 16384, &maps.sst, x, 0, bh * NC + c, 0,
+                                    bar(B_LD));
                 }
                 ++n_ld;
                 // gram [Q'; K'] [B"; K"]^T; Z = [B"; K"] dS~; D~ += Q'^T dO
@@ -427,11 +475,20 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                     tc::mma_bf16(tmem + TM_G, tc::desc_kmajor(sbase + OFF_DAT, 16384, kk),
                                  tc::desc_mnmajor(sbase + OFF_QK, 16384, kk), idKM, true);
                 tc::mma_commit(bar(B_XY));
+                // dU, staged before R_DA
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+                    tc::tma_store_4d(&maps.du, sbase + slab_du(p), 32 * p, hi, t0, bi);
+                tc::bulk_commit();
+                done = true;
             }
+            // the last chunk's XQ', XK', YB', YK'
+            if (done && *abort_s == 0 && wait_ready(R_LD, ph ^ 1)) store_xy(0);
             // nothing of this CTA may still be in flight when it exits
             tc::mma_commit(bar(B_FIN));
             tc::mbar_wait_bounded(bar(B_FIN), 0, WAIT_NS);
             if (n_ld) tc::mbar_wait_bounded(bar(B_LD), (n_ld - 1) & 1, WAIT_NS);
+            tc::bulk_wait_all();
         }
     } else {
         // ======================= compute warps
@@ -454,13 +511,26 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             tc::tmem_st32(tmem + lane_off + TM_D + 32 * cb, vals);
             tc::tmem_wait_st();
         }
+        // the G_C term of the last chunk: rowsum(dS_T * S_T), this thread's 32 columns
+        if (NC > 0) {
+            float part = 0.f;
+            if (ds_final) {
+                const float4* g4 = reinterpret_cast<const float4*>(ds_final + soff + (size_t)lane_t * D + 32 * cb);
+                const float4* s4 = reinterpret_cast<const float4*>(sT + soff + (size_t)lane_t * D + 32 * cb);
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const float4 g = g4[x], sv = s4[x];
+                    part = fmaf(g.x, sv.x, fmaf(g.y, sv.y, fmaf(g.z, sv.z, fmaf(g.w, sv.w, part))));
+                }
+            }
+            EXP[cb * D + lane_t] = part;
+        }
         uint32_t ph = 0;
         auto signal_or_stop = [&](uint32_t id) {
             const bool stop = compute_sync_or(*abort_s != 0);
             if (tid == 0) tc::mbar_arrive(bar(id));
             return stop;
         };
-        auto tok_row = [&](int t) { return ((size_t)bi * T + t) * H + hi; };
 #pragma unroll 1
         for (int c = NC - 1; c >= 0; --c, ph ^= 1) {
             const int t0 = c * C;
@@ -497,44 +567,31 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                 tc::tmem_st16(tmem + lane_off + TM_EU + 16 * cb, words);
             }
             {
-                // S~ = g_m S0: lane i, 32 value columns
-                const float g = GM[lane_t];
-                const float4* src = reinterpret_cast<const float4*>(
-                    states + ((size_t)bh * NC + c) * D * D + (size_t)lane_t * D + 32 * cb);
+                // S~ (the forward's tile, landed in OFF_DS) -> tensor memory: lane i,
+                // 32 value columns; this thread later overwrites exactly these bytes
+                // with dS~
+                const uint8_t* src = sm + OFF_DS + (cb >> 1) * 16384 + lane_t * 128;
                 uint32_t words[16];
 #pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    const float4 v4 = src[x];
-                    words[2 * x] = tc::pack_bf16x2(v4.x * g, v4.y * g);
-                    words[2 * x + 1] = tc::pack_bf16x2(v4.z * g, v4.w * g);
+                for (int qd = 0; qd < 4; ++qd) {
+                    const int c16 = 4 * (cb & 1) + qd;
+                    const uint4 u = *reinterpret_cast<const uint4*>(src + ((c16 ^ (lane_t & 7)) << 4));
+                    words[4 * qd] = u.x;
+                    words[4 * qd + 1] = u.y;
+                    words[4 * qd + 2] = u.z;
+                    words[4 * qd + 3] = u.w;
                 }
                 tc::tmem_st16(tmem + lane_off + TM_S + 16 * cb, words);
             }
             {
-                // dS_C = g_m(next) D~;  its share of the G_C term, rowsum(dS_C * S_C);
-                // dS~ = gc dS_C into tensor memory and, bf16, into OFF_DS
+                // dS_C = g_m(next) D~;  dS~ = gc dS_C into tensor memory and, bf16,
+                // into OFF_DS
                 float vals[32];
                 tc::tmem_ld32(tmem + lane_off + TM_D + 32 * cb, vals);
                 tc::tmem_wait_ld();
-                const float fn = GMN[lane_t], fc = GC[lane_t];
-                const float* scp = (c == NC - 1 ? sT + soff
-                                                : states + ((size_t)bh * NC + c + 1) * D * D) +
-                                   (size_t)lane_t * D + 32 * cb;
-                const float4* sc4 = reinterpret_cast<const float4*>(scp);
-                float part = 0.f;
+                const float f = GMN[lane_t] * GC[lane_t];
 #pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    const float4 s4 = sc4[x];
-                    vals[4 * x] *= fn; vals[4 * x + 1] *= fn;
-                    vals[4 * x + 2] *= fn; vals[4 * x + 3] *= fn;
-                    part = fmaf(vals[4 * x], s4.x, part);
-                    part = fmaf(vals[4 * x + 1], s4.y, part);
-                    part = fmaf(vals[4 * x + 2], s4.z, part);
-                    part = fmaf(vals[4 * x + 3], s4.w, part);
-                }
-#pragma unroll
-                for (int x = 0; x < 32; ++x) vals[x] *= fc;
-                EXP[cb * D + lane_t] = part;
+                for (int x = 0; x < 32; ++x) vals[x] *= f;
                 tc::tmem_st32(tmem + lane_off + TM_D + 32 * cb, vals);
                 tc::store_row32_bf16(sm + OFF_DS + (cb >> 1) * 16384, lane_t, cb & 1, vals);
             }
@@ -547,6 +604,7 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             if (tid < D) {
                 gce[((size_t)bh * NC + c) * D + tid] =
                     (EXP[tid] + EXP[D + tid]) + (EXP[2 * D + tid] + EXP[3 * D + tid]);
+                gcs[((size_t)bh * NC + c) * D + tid] = GC[tid];
                 GMN[tid] = GM[tid];
             }
             wait_then_sync(bar(B_G), ph, tid, abort_s);
@@ -625,6 +683,22 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
 
             // ================= C5: dA^T masked -> bf16; dU out
             wait_then_sync(bar(B_A), ph, tid, abort_s);
+            if (c > 0) {
+                // the G_C term of the chunk before: rowsum(dS_C * S_C) with dS_C =
+                // g_m D~ and S_C = S~ / g_m (this chunk's start), i.e. rowsum(D~ * S~)
+                float vals[32];
+                tc::tmem_ld32(tmem + lane_off + TM_D + 32 * cb, vals);
+                uint32_t sw[16];
+                tc::tmem_ld16u(tmem + lane_off + TM_S + 16 * cb, sw);
+                tc::tmem_wait_ld();
+                float part = 0.f;
+#pragma unroll
+                for (int x = 0; x < 16; ++x) {
+                    part = fmaf(vals[2 * x], __uint_as_float(sw[x] << 16), part);
+                    part = fmaf(vals[2 * x + 1], __uint_as_float(sw[x] & 0xFFFF0000u), part);
+                }
+                EXP[cb * D + lane_t] = part;
+            }
             {
                 // lane s of [-E; U], columns r of [dO; dY]: keep r >= s against dO,
                 // r > s against dY; block relation as for the gram
@@ -646,12 +720,11 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                 }
                 tc::store_row32_bf16(sm + OFF_DAT + (cb >> 1) * 16384, lane_t, cb & 1, vals);
             }
-            if (quarter >= 2) {
-                const int s = lane_t - 64;
+            if (quarter >= 2) {   // dU -> its staging slabs (rows past T are not stored)
                 float vals[32];
                 tc::tmem_ld32(tmem + lane_off + TM_Z + 32 * cb, vals);
                 tc::tmem_wait_ld();
-                if (s < n) store_row32_f32(du + tok_row(t0 + s) * D + 32 * cb, vals);
+                stage_row32(sm + slab_du(cb), lane_t - 64, vals);
             }
             tc::fence_async_smem();
             tc::fence_before_sync();
@@ -660,23 +733,23 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             // ================= C6: [XQ' | XK']^T and [YB'; YK'] out
             wait_then_sync(bar(B_XY), ph, tid, abort_s);
             {
+                // [XQ' | XK']^T: lane = channel, columns = tokens; into [token][channel]
                 float vals[32];
                 tc::tmem_ld32(tmem + lane_off + TM_Z + 32 * cb, vals);
                 tc::tmem_wait_ld();
-                float* dst = cb < 2 ? xq : xk;
+                uint8_t* dst = sm + (cb < 2 ? OFF_QK : OFF_BK);
                 const int r0 = 32 * (cb & 1);
 #pragma unroll
                 for (int x = 0; x < 32; ++x)
-                    if (r0 + x < n) dst[tok_row(t0 + r0 + x) * D + lane_t] = vals[x];
+                    *reinterpret_cast<float*>(dst + stage_off(r0 + x, lane_t)) = vals[x];
             }
             {
                 float vals[32];
                 tc::tmem_ld32(tmem + lane_off + TM_G + 32 * cb, vals);
                 tc::tmem_wait_ld();
-                const int s = lane_t & 63;
-                if (s < n) store_row32_f32((lane_t < 64 ? yb : yk) + tok_row(t0 + s) * D + 32 * cb,
-                                           vals);
+                stage_row32(sm + (lane_t < 64 ? OFF_DOY : OFF_DS) + 8192 * cb, lane_t & 63, vals);
             }
+            tc::fence_async_smem();
             tc::fence_before_sync();
             if (signal_or_stop(R_LD)) break;
         }
@@ -704,135 +777,148 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
 }
 
 // ---------------------------------------------------------------- epilogue
-// One CTA per (batch, head, chunk), thread = key/value channel i.  From the
-// raw inputs and the reverse sweep's XQ', XK', YK', YB', dU and G_C terms:
-//   Lam_r = 1 / prod_{t=r+1}^{31} a_t (r <= 31),  prod_{t=32}^{r} a_t (r >= 32)
+// One warp per (batch, head, chunk), lane l = channels 4l .. 4l+3, the
+// chunk's tokens from the last: from the raw inputs and the reverse sweep's
+// XQ', XK', YK', YB', dU, G_C terms and gc,
+//   Lam_63 = gc, Lam_{r-1} = Lam_r / a_r   (= gamma_{r-1} / g_m)
 //   dq = Lam XQ', dk = Lam XK' + (YK' + b YB') / Lam, db = K" YB',
-//   dv = w dU, dw = v dU, d log a by the reverse cumulative sum of dG,
-//   da = d log a / a.
-// Scalar gates take the sum over channels.  FG^2-GDN learning rates: the
-// gradients of the key sqrt(beta^k) k and write gate sqrt(beta^v) carried
-// through the square roots (dk = sqrt(beta^k) dk~, dbeta^k = k dk~ /
-// (2 sqrt(beta^k)), dbeta^v = v dU / (2 sqrt(beta^v))).
+//   dv = w dU, dw = v dU, d log a_r = sum_{r' >= r} dG_r', da = d log a / a.
+// Scalar gates take the sum over channels (a warp reduction).  FG^2-GDN
+// learning rates: the gradients of the key sqrt(beta^k) k and write gate
+// sqrt(beta^v) carried through the square roots (dk = sqrt(beta^k) dk~,
+// dbeta^k = k dk~ / (2 sqrt(beta^k)), dbeta^v = v dU / (2 sqrt(beta^v))).
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
     return x;
 }
+__device__ __forceinline__ void ld_bf16x4(const __nv_bfloat16* p, float* f) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    f[0] = __uint_as_float(u.x << 16);
+    f[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(u.y << 16);
+    f[3] = __uint_as_float(u.y & 0xFFFF0000u);
+}
+__device__ __forceinline__ void st_bf16x4(__nv_bfloat16* p, const float* f) {
+    *reinterpret_cast<uint2*>(p) =
+        make_uint2(tc::pack_bf16x2(f[0], f[1]), tc::pack_bf16x2(f[2], f[3]));
+}
+__device__ __forceinline__ void ld_f32x4(const float* p, float* f) {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+}
+// gate of kind `kind` for the four channels of this lane (1.0 for GATE_ONE)
+__device__ __forceinline__ void ld_gate4(const __nv_bfloat16* g, int kind, long long th,
+                                         long long tv, float* f) {
+    if (kind == GDR_GATE_ONE) {
+        f[0] = f[1] = f[2] = f[3] = 1.f;
+    } else if (kind == GDR_GATE_SCALAR) {
+        f[0] = f[1] = f[2] = f[3] = to_f32(g[th]);
+    } else {
+        ld_bf16x4(g + tv, f);
+    }
+}
 
-__global__ void __launch_bounds__(D)
-bwd_epilogue_kernel(int T, int H, int NC, const __nv_bfloat16* __restrict__ q,
+__global__ void __launch_bounds__(128)
+bwd_epilogue_kernel(int T, int H, int NC, long long n_units, const __nv_bfloat16* __restrict__ q,
                     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                     const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                     const __nv_bfloat16* __restrict__ w, int a_kind, int b_kind, int w_kind,
                     const float* __restrict__ xq, const float* __restrict__ xk,
                     const float* __restrict__ yk, const float* __restrict__ yb,
                     const float* __restrict__ du, const float* __restrict__ gce,
-                    __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk,
-                    __nv_bfloat16* __restrict__ dv, __nv_bfloat16* __restrict__ da,
-                    __nv_bfloat16* __restrict__ db, __nv_bfloat16* __restrict__ dw) {
-    __shared__ float lam2[32][D];    // Lam of tokens 32..63
-    __shared__ float red[3][C][4];   // scalar gates: per-warp sums of da, db, dw
-    const int i = threadIdx.x, warp = i >> 5, lane = i & 31;
-    const int c = blockIdx.x % NC, bh = blockIdx.x / NC;
-    const int hi = bh % H, bi = bh / H;
+                    const float* __restrict__ gcs, __nv_bfloat16* __restrict__ dq,
+                    __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                    __nv_bfloat16* __restrict__ da, __nv_bfloat16* __restrict__ db,
+                    __nv_bfloat16* __restrict__ dw) {
+    const int lane = threadIdx.x & 31;
+    const long long unit = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+    if (unit >= n_units) return;
+    const int c = (int)(unit % NC);
+    const long long bh = unit / NC;
+    const int hi = (int)(bh % H), bi = (int)(bh / H);
     const int t0 = c * C, n = min(C, T - t0);
+    const int i0 = 4 * lane;
     const bool fb = b_kind == GDR_GATE_FG2, fw = w_kind == GDR_GATE_FG2;
-    auto tok = [&](int r) { return ((long long)bi * T + t0 + r) * H + hi; };
-    auto aval = [&](int r) -> float {
-        if (r >= n || a_kind == GDR_GATE_ONE) return 1.f;
-        return a_kind == GDR_GATE_SCALAR ? to_f32(a[tok(r)]) : to_f32(a[tok(r) * D + i]);
-    };
-    auto gval = [&](const __nv_bfloat16* g, int kind, int r) -> float {
-        if (kind == GDR_GATE_ONE) return 1.f;
-        return kind == GDR_GATE_SCALAR ? to_f32(g[tok(r)]) : to_f32(g[tok(r) * D + i]);
-    };
-    {
-        float run = 1.f;
-#pragma unroll 1
-        for (int r = 32; r < C; ++r) {
-            run *= aval(r);
-            lam2[r - 32][i] = run;
-        }
-    }
-    float P = 1.f;     // prod_{t=r+1}^{31} a_t while r <= 31
-    float cum = 0.f;   // d log a_r, channel i
-    const float gterm = gce[((size_t)bh * NC + c) * D + i];
+    const long long tok0 = ((long long)bi * T + t0) * H + hi;   // token-head index of row 0
+    float lam[4], cum[4] = {0.f, 0.f, 0.f, 0.f}, gterm[4];
+    ld_f32x4(gcs + (bh * NC + c) * D + i0, lam);
+    ld_f32x4(gce + (bh * NC + c) * D + i0, gterm);
 #pragma unroll 1
     for (int r = C - 1; r >= 0; --r) {
+        float av[4] = {1.f, 1.f, 1.f, 1.f};
         if (r < n) {
-            const float lam = r >= 32 ? lam2[r - 32][i] : 1.f / P;
-            const float lami = r >= 32 ? 1.f / lam2[r - 32][i] : P;
-            const long long tv = tok(r) * D + i;
-            const float qv = to_f32(q[tv]), kv = to_f32(k[tv]), vv = to_f32(v[tv]);
-            const float bv = gval(b, b_kind, r), wv = gval(w, w_kind, r);
-            const float sbk = fb ? sqrt_fast(fmaxf(bv, 0.f)) : 1.f;   // sqrt(beta^k)
-            const float kt = kv * sbk;                                 // the key used
-            const float bt = fb ? 1.f : bv;                            // the erase gate used
-            const float wt = fw ? sqrt_fast(fmaxf(wv, 0.f)) : wv;      // the write gate used
-            const float XQ = xq[tv], XK = xk[tv], YK = yk[tv], YB = yb[tv], dU = du[tv];
-            const float Kpp = lami * kt;
-            float dG = lam * (qv * XQ + kt * XK) - Kpp * (YK + bt * YB);
-            if (r == n - 1) dG += gterm;
-            cum += dG;
-            const float dkt = lam * XK + lami * (YK + bt * YB);
-            dq[tv] = __float2bfloat16_rn(lam * XQ);
-            dk[tv] = __float2bfloat16_rn(dkt * sbk);
-            dv[tv] = __float2bfloat16_rn(wt * dU);
-            // erase gate
-            if (b_kind == GDR_GATE_VECTOR) {
-                db[tv] = __float2bfloat16_rn(Kpp * YB);
-            } else if (fb) {
-                db[tv] = __float2bfloat16_rn(kv * dkt / (2.f * sbk));
-            } else if (b_kind == GDR_GATE_SCALAR) {
-                const float s = warp_sum(Kpp * YB);
-                if (lane == 0) red[1][r][warp] = s;
+            const long long th = tok0 + (long long)r * H, tv = th * D + i0;
+            float qv[4], kv[4], vv[4], bv[4], wv[4], XQ[4], XK[4], YK[4], YB[4], dU[4];
+            ld_bf16x4(q + tv, qv);
+            ld_bf16x4(k + tv, kv);
+            ld_bf16x4(v + tv, vv);
+            ld_gate4(a, a_kind, th, tv, av);
+            ld_gate4(b, b_kind, th, tv, bv);
+            ld_gate4(w, w_kind, th, tv, wv);
+            ld_f32x4(xq + tv, XQ);
+            ld_f32x4(xk + tv, XK);
+            ld_f32x4(yk + tv, YK);
+            ld_f32x4(yb + tv, YB);
+            ld_f32x4(du + tv, dU);
+            float oq[4], ok[4], ov[4], oa[4], ob[4], ow[4];
+            float sb = 0.f, sw = 0.f, sa = 0.f;
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const float lm = lam[x], li = 1.f / lm;
+                const float sbk = fb ? sqrt_fast(fmaxf(bv[x], 0.f)) : 1.f;   // sqrt(beta^k)
+                const float kt = kv[x] * sbk;                                 // the key used
+                const float bt = fb ? 1.f : bv[x];                            // the erase gate used
+                const float wt = fw ? sqrt_fast(fmaxf(wv[x], 0.f)) : wv[x];   // the write gate used
+                const float Kpp = li * kt;
+                float dG = lm * (qv[x] * XQ[x] + kt * XK[x]) - Kpp * (YK[x] + bt * YB[x]);
+                if (r == n - 1) dG += gterm[x];
+                cum[x] += dG;
+                const float dkt = lm * XK[x] + li * (YK[x] + bt * YB[x]);
+                oq[x] = lm * XQ[x];
+                ok[x] = dkt * sbk;
+                ov[x] = wt * dU[x];
+                ob[x] = fb ? kv[x] * dkt / (2.f * sbk) : Kpp * YB[x];
+                ow[x] = fw ? vv[x] * dU[x] / (2.f * wt) : vv[x] * dU[x];
+                oa[x] = cum[x] / av[x];
+                sb += ob[x];
+                sw += ow[x];
+                sa += cum[x];
             }
-            // write gate
-            if (w_kind == GDR_GATE_VECTOR) {
-                dw[tv] = __float2bfloat16_rn(vv * dU);
-            } else if (fw) {
-                dw[tv] = __float2bfloat16_rn(vv * dU / (2.f * wt));
-            } else if (w_kind == GDR_GATE_SCALAR) {
-                const float s = warp_sum(vv * dU);
-                if (lane == 0) red[2][r][warp] = s;
-            }
-            // decay
-            if (a_kind == GDR_GATE_VECTOR) {
-                da[tv] = __float2bfloat16_rn(cum / aval(r));
-            } else if (a_kind == GDR_GATE_SCALAR) {
-                const float s = warp_sum(cum);
-                if (lane == 0) red[0][r][warp] = s;
-            }
-        }
-        if (r <= 31) P *= aval(r);
-    }
-    if (a_kind == GDR_GATE_SCALAR || b_kind == GDR_GATE_SCALAR || w_kind == GDR_GATE_SCALAR) {
-        __syncthreads();
-        if (i < n) {
-            const long long ts = tok(i);
+            st_bf16x4(dq + tv, oq);
+            st_bf16x4(dk + tv, ok);
+            st_bf16x4(dv + tv, ov);
+            if (a_kind == GDR_GATE_VECTOR) st_bf16x4(da + tv, oa);
+            if (b_kind == GDR_GATE_VECTOR || fb) st_bf16x4(db + tv, ob);
+            if (w_kind == GDR_GATE_VECTOR || fw) st_bf16x4(dw + tv, ow);
             if (a_kind == GDR_GATE_SCALAR) {
-                const float s = (red[0][i][0] + red[0][i][1]) + (red[0][i][2] + red[0][i][3]);
-                da[ts] = __float2bfloat16_rn(s / to_f32(a[ts]));
+                sa = warp_sum(sa);
+                if (lane == 0) da[th] = __float2bfloat16_rn(sa / av[0]);
             }
-            if (b_kind == GDR_GATE_SCALAR)
-                db[ts] = __float2bfloat16_rn((red[1][i][0] + red[1][i][1]) +
-                                             (red[1][i][2] + red[1][i][3]));
-            if (w_kind == GDR_GATE_SCALAR)
-                dw[ts] = __float2bfloat16_rn((red[2][i][0] + red[2][i][1]) +
-                                             (red[2][i][2] + red[2][i][3]));
+            if (b_kind == GDR_GATE_SCALAR) {
+                sb = warp_sum(sb);
+                if (lane == 0) db[th] = __float2bfloat16_rn(sb);
+            }
+            if (w_kind == GDR_GATE_SCALAR) {
+                sw = warp_sum(sw);
+                if (lane == 0) dw[th] = __float2bfloat16_rn(sw);
+            }
         }
+        // Lam of the token before
+#pragma unroll
+        for (int x = 0; x < 4; ++x) lam[x] /= av[x];
     }
 }
 
 inline size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct TcWorkspace {
-    float* states;   // [B*H][NC][128][128]
+    void* states;    // [B*H][NC][128][128] bf16 S~
     float* sT;       // [B*H][128][128]
     void* e;         // [B, T, H, 128] bf16
     float* pre[5];   // XQ', XK', YK', YB', dU: [B, T, H, 128] float32
-    float* gce;      // [B*H][NC][128]
+    float* gce;      // [B*H][NC][128] G_C terms
+    float* gcs;      // [B*H][NC][128] gc per chunk and channel
     size_t bytes;
 };
 
@@ -847,11 +933,12 @@ TcWorkspace carve(const gdr_desc& d, void* base) {
         off += round256(bytes);
         return r;
     };
-    w.states = reinterpret_cast<float*>(take(bh * nc * D * D * 4));
+    w.states = take(bh * nc * D * D * 2);
     w.sT = reinterpret_cast<float*>(take(bh * D * D * 4));
     w.e = take(tok * D * 2);
     for (int x = 0; x < 5; ++x) w.pre[x] = reinterpret_cast<float*>(take(tok * D * 4));
     w.gce = reinterpret_cast<float*>(take(bh * nc * D * 4));
+    w.gcs = reinterpret_cast<float*>(take(bh * nc * D * 4));
     w.bytes = off;
     return w;
 }
@@ -889,6 +976,10 @@ cudaError_t launch_backward_tc(const gdr_desc& d, const void* const* in, const f
         ok = tc_map_bf16(&maps.b, in[4], B, T, H, T);
     if (ok && (d.write == GDR_GATE_VECTOR || d.write == GDR_GATE_FG2))
         ok = tc_map_bf16(&maps.w, in[5], B, T, H, T);
+    ok = ok && tc_map_f32(&maps.xq, ws.pre[0], B, T, H) && tc_map_f32(&maps.xk, ws.pre[1], B, T, H) &&
+         tc_map_f32(&maps.yk, ws.pre[2], B, T, H) && tc_map_f32(&maps.yb, ws.pre[3], B, T, H) &&
+         tc_map_f32(&maps.du, ws.pre[4], B, T, H) &&
+         tc_map_state_bf16(&maps.sst, ws.states, (long long)B * H * NC);
     if (!ok) return cudaErrorInvalidValue;
 
     const bool fg2 = d.erase == GDR_GATE_FG2 || d.write == GDR_GATE_FG2;
@@ -899,16 +990,17 @@ cudaError_t launch_backward_tc(const gdr_desc& d, const void* const* in, const f
     const auto* b = static_cast<const __nv_bfloat16*>(in[4]);
     const auto* w = static_cast<const __nv_bfloat16*>(in[5]);
     kern<<<(unsigned)((long long)B * H), NT, SMEM_BYTES, st>>>(
-        maps, B, T, H, a, b, w, (int)d.decay, (int)d.erase, (int)d.write, ds_final, ws.states,
-        ws.sT, ws.pre[0], ws.pre[1], ws.pre[2], ws.pre[3], ws.pre[4], ws.gce, ds0, err_word);
+        maps, B, T, H, a, b, w, (int)d.decay, (int)d.erase, (int)d.write, ds_final, ws.sT,
+        ws.gce, ws.gcs, ds0, err_word);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
-    bwd_epilogue_kernel<<<(unsigned)((long long)B * H * NC), D, 0, st>>>(
-        T, H, NC, static_cast<const __nv_bfloat16*>(in[0]),
+    const long long units = (long long)B * H * NC;
+    bwd_epilogue_kernel<<<(unsigned)((units + 3) / 4), 128, 0, st>>>(
+        T, H, NC, units, static_cast<const __nv_bfloat16*>(in[0]),
         static_cast<const __nv_bfloat16*>(in[1]), static_cast<const __nv_bfloat16*>(in[2]), a, b,
         w, (int)d.decay, (int)d.erase, (int)d.write, ws.pre[0], ws.pre[1], ws.pre[2], ws.pre[3],
-        ws.pre[4], ws.gce, static_cast<__nv_bfloat16*>(grads[0]),
+        ws.pre[4], ws.gce, ws.gcs, static_cast<__nv_bfloat16*>(grads[0]),
         static_cast<__nv_bfloat16*>(grads[1]), static_cast<__nv_bfloat16*>(grads[2]),
         static_cast<__nv_bfloat16*>(grads[3]), static_cast<__nv_bfloat16*>(grads[4]),
         static_cast<__nv_bfloat16*>(grads[5]));

@@ -82,7 +82,6 @@ constexpr uint32_t OFF_SMALL = OFF_R + 37888;   // 226304
 constexpr uint32_t OFF_FCUR = OFF_SMALL;        // float[128]: state scale this chunk
 constexpr uint32_t OFF_FPREV = OFF_SMALL + 512; // float[128]: gamma_C/g_m of last chunk
 constexpr uint32_t OFF_SCA = OFF_SMALL + 1024;  // float[2][3][64]: scalar a, b, w (2 chunks)
-constexpr uint32_t OFF_FSTART = OFF_SMALL + 2560;  // float[128]: fprev before the chunk (dump)
 constexpr uint32_t OFF_BAR = OFF_SMALL + 3072;  // NBAR mbarriers (see the kernel)
 constexpr int NBAR = 14;
 constexpr uint32_t OFF_TSLOT = OFF_BAR + 8 * NBAR;
@@ -105,6 +104,7 @@ constexpr uint32_t IDESC_NEG_B = 1u << 14;   // negate the B operand
 
 struct TcMaps {
     CUtensorMap q, k, v, a, b, w, o;  // a/b/w only meaningful for vector gates
+    CUtensorMap sst;                  // state-writing instantiation: S~ tiles
 };
 
 // ---------------------------------------------------------------- TMA issue
@@ -152,11 +152,11 @@ __device__ __forceinline__ void issue_v(const TcMaps& m, uint32_t sbase, int t0,
 // fprev = gamma_63/g_m, and check that the largest factors, gamma_0/g_m and
 // g_m/gamma_63, stay in float range.  `mid` runs between the two halves (after
 // the exchange barrier), before anything is written to X2.
-template <bool PACKED, bool FG2, bool DUMP, typename Mid>
+template <bool PACKED, bool FG2, typename Mid>
 __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool vb, bool vw,
                                              bool fb, bool fw, int a_kind, int n,
                                              const float* sca, float* QT,
-                                             float* fcur, float* fprev, float* fstart,
+                                             float* fcur, float* fprev,
                                              int* err_word, Mid&& mid) {
     const int p2 = tid & 63, q8 = tid >> 6;
     const uint32_t pnl = (uint32_t)(p2 >> 5);
@@ -264,10 +264,6 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool
         const int i = 2 * p2;
         fcur[i] = fprev[i] * gm0;
         fcur[i + 1] = fprev[i + 1] * gm1;
-        if (DUMP) {   // the chunk-start state is Diag(fprev) times the state held now
-            fstart[i] = fprev[i];
-            fstart[i + 1] = fprev[i + 1];
-        }
         fprev[i] = gc0;
         fprev[i + 1] = gc1;
         // the divisors above: prod of a over tokens 1..31 (octet 0 holds it as
@@ -301,10 +297,11 @@ static_assert(R_O + 1 == NBAR, "barrier count");
 
 // PACKED: packed sequences (rows past a sequence's end are zeroed rather than
 // left to the TMA fill).  FG2: FG^2-GDN learning rates among the gates.  DUMP:
-// no o; instead the state at the start of every chunk goes to `states`,
-// [B*H][n_slots][128][128] float32 at slots slot0, slot0 + 1, ..., and, when
-// o_raw is given, each chunk's E (the key reads, bf16 [B, T, H, 128]) to
-// o_raw through the o tensor map: what the backward reads back.  All
+// no o; instead every chunk's operand S~ = Diag(g_m) S0 (bf16, the tile its
+// products read) goes through the sst map to slot bh * n_slots + slot0 +
+// chunk of a [slots][128][128] array, and, when o_raw is given, each chunk's
+// E (the key reads, bf16 [B, T, H, 128]) to o_raw through the o map: what
+// the backward reads back.  All
 // compile-time, so the plain instantiation carries none of these tests.
 // T_row: tokens between batch rows in memory (T, or more when the launch
 // covers a token range of longer rows).
@@ -316,7 +313,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                   const float* __restrict__ s0, float* __restrict__ s_final,
                   int* __restrict__ err_word, int skip_signal,
                   const int* __restrict__ cu_seqlens, __nv_bfloat16* __restrict__ o_raw,
-                  float* __restrict__ states, int n_slots, int slot0, int T_row) {
+                  int n_slots, int slot0, int T_row) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -327,7 +324,6 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
     float* PS = reinterpret_cast<float*>(sm + OFF_PS);
     float* fcur = reinterpret_cast<float*>(sm + OFF_FCUR);
     float* fprev = reinterpret_cast<float*>(sm + OFF_FPREV);
-    float* fstart = reinterpret_cast<float*>(sm + OFF_FSTART);
     float* sca_all = reinterpret_cast<float*>(sm + OFF_SCA);  // [2][3][64]
     volatile int* abort_s = reinterpret_cast<volatile int*>(sm + OFF_ABORT);
     auto bar = [&](uint32_t id) { return sbase + OFF_BAR + 8u * id; };
@@ -424,6 +420,12 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                 if (!(skip_signal && t0 == 0)) tc::mma_commit(bar(B_G));
                 // X = [K';Q'] S~, S~ += K"^T U
                 if (!wait_ready(R_P2)) break;
+                if (DUMP) {  // S~ leaves by TMA (read before this chunk's state update completes)
+                    const int slot = bh * n_slots + slot0 + t0 / C;
+                    tc::tma_store_4d(&maps.sst, sbase + OFF_S0, 0, 0, slot, 0);
+                    tc::tma_store_4d(&maps.sst, sbase + OFF_S0 + 16384, 64, 0, slot, 0);
+                    tc::bulk_commit();
+                }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_bf16(tmem + TM_X, tc::desc_kmajor(sbase + OFF_X1, 16384, kk),
@@ -458,6 +460,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                 tc::mma_commit(bar(B_E));
                 // X += [0; -A_qb] E (rows 64-127 become O); S~ -= B"^T E
                 if (!wait_ready(R_E)) break;
+                if (DUMP) tc::bulk_wait_read();  // the S~ store has read its tile
                 if (dump_e) {  // E leaves by TMA (its tile is next reused after the gram)
                     tc::tma_store_4d(&maps.o, sbase + OFF_EB, 0, hi, tb + t0, bi);
                     tc::tma_store_4d(&maps.o, sbase + OFF_EB + 8192, 64, hi, tb + t0, bi);
@@ -561,8 +564,8 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             }
             if (compute_sync_or(*abort_s != 0)) break;
             // ================= P1c:
-            operand_pass<PACKED, FG2, DUMP>(sm, tid, va, vb, vw, fb, fw, a_kind, min(C, L - t0),
-                         sca, QT, fcur, fprev, fstart, err_word, [&] {
+            operand_pass<PACKED, FG2>(sm, tid, va, vb, vw, fb, fw, a_kind, min(C, L - t0),
+                         sca, QT, fcur, fprev, err_word, [&] {
                              if (t0 == 0) return;
                              // the last chunk's state update has read X2 and EB and
                              // finished its O: O -> staging tile for the issuing warp
@@ -580,16 +583,6 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                 tc::fence_after_sync();
                 tc::tmem_ld32(tmem + lane_off + TM_S + c0, vals);
                 tc::tmem_wait_ld();
-                if (DUMP) {  // the true state at the chunk start, row lane_t
-                    const float fs = fstart[lane_t];
-                    float4* dst = reinterpret_cast<float4*>(
-                        states + ((size_t)bh * n_slots + slot0 + t0 / C) * D * D +
-                        (size_t)lane_t * D + c0);
-#pragma unroll
-                    for (int x = 0; x < 8; ++x)
-                        dst[x] = make_float4(vals[4 * x] * fs, vals[4 * x + 1] * fs,
-                                             vals[4 * x + 2] * fs, vals[4 * x + 3] * fs);
-                }
 #pragma unroll
                 for (int x = 0; x < 32; ++x) vals[x] *= f;
                 tc::tmem_st32(tmem + lane_off + TM_S + c0, vals);
@@ -793,6 +786,40 @@ bool tc_map_bf16(CUtensorMap* m, const void* ptr, int B, int T, int H, int T_row
     return make_map(m, ptr, B, T, H, T_row);
 }
 
+// [B, T, H, 128] float32 tensor as a 4-D map {128, H, T, B}, box {32, 1, 64,
+// 1} (a 32-channel slab of 64 tokens, 128-byte rows), 128-byte swizzle: the
+// backward's staging format for its float32 outputs.
+bool tc_map_f32(CUtensorMap* m, const void* ptr, int B, int T, int H) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4,
+                                   (cuuint64_t)T * H * D * 4};
+    const cuuint32_t box[4] = {32, 1, 64, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(ptr), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// [n_slots][128][128] bf16 state tiles (row = key channel) as a 4-D map
+// {128, 128, n_slots, 1}, box {64, 128, 1, 1} (one 64-column panel of a
+// tile), 128-byte swizzle: the operand layout of S~.
+bool tc_map_state_bf16(CUtensorMap* m, const void* ptr, long long n_slots) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)D, (cuuint64_t)n_slots, 1};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)D * D * 2,
+                                   (cuuint64_t)n_slots * D * D * 2};
+    const cuuint32_t box[4] = {64, 128, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 bool chunked_tc_supports(const gdr_desc& d) {
     return d.in_dtype == GDR_BF16 && d.dk == D && d.dv == D && d.chunk == C;
 }
@@ -834,23 +861,25 @@ cudaError_t launch_chunked_tc(const gdr_desc& d, const void* q, const void* k, c
     kern<<<(unsigned)(nseq * d.H), NT, SMEM_BYTES, st>>>(
         maps, d.B, d.T, d.H, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b,
         (const __nv_bfloat16*)w, (int)d.decay, (int)d.erase, (int)d.write, s0, s_final,
-        err_word, skip_signal ? 1 : 0, cu_seqlens, (__nv_bfloat16*)o, nullptr, 0, 0, d.T);
+        err_word, skip_signal ? 1 : 0, cu_seqlens, (__nv_bfloat16*)o, 0, 0, d.T);
     return cudaGetLastError();
 }
 
-// The states at the start of every 64-token chunk of the B x H sequences
-// (no o) into slots slot0, slot0 + 1, ... of `states` ([B*H][n_slots][128][128]
-// float32), and, if e_out is given, every chunk's E (bf16 [B, T, H, 128]):
-// what the backward reads back.  The launch covers d.T tokens of rows T_row
-// tokens apart (the pointers already at its first token); s_final, if
-// given, receives the state after them.
+// Every 64-token chunk's S~ = Diag(g_m) S0 of the B x H sequences (no o), as
+// bf16 into slots slot0, slot0 + 1, ... of `s_tilde` ([B*H][n_slots][128][128],
+// row = key channel), and, if e_out is given, every chunk's E (bf16
+// [B, T, H, 128]): what the backward reads back.  The launch covers d.T
+// tokens of rows T_row tokens apart (the pointers already at its first
+// token); s_final, if given, receives the state after them.
 cudaError_t launch_chunked_tc_states(const gdr_desc& d, int T_row, const void* q, const void* k,
                                      const void* v, const void* a, const void* b,
                                      const void* w, const float* s0, float* s_final,
-                                     float* states, int n_slots, int slot0, void* e_out,
+                                     void* s_tilde, int n_slots, int slot0, void* e_out,
                                      int* err_word, cudaStream_t st) {
     TcMaps maps;
     if (!make_maps(&maps, d, T_row, q, k, v, a, b, w, e_out)) return cudaErrorInvalidValue;
+    if (d.T > 0 && !tc_map_state_bf16(&maps.sst, s_tilde, (long long)d.B * d.H * n_slots))
+        return cudaErrorInvalidValue;
     const bool fg2 = d.erase == GDR_GATE_FG2 || d.write == GDR_GATE_FG2;
     auto kern = fg2 ? chunked_tc_kernel<false, true, true> : chunked_tc_kernel<false, false, true>;
     cudaError_t e = cudaFuncSetAttribute(kern,
@@ -860,7 +889,7 @@ cudaError_t launch_chunked_tc_states(const gdr_desc& d, int T_row, const void* q
     kern<<<(unsigned)((long long)d.B * d.H), NT, SMEM_BYTES, st>>>(
         maps, d.B, d.T, d.H, (const __nv_bfloat16*)a, (const __nv_bfloat16*)b,
         (const __nv_bfloat16*)w, (int)d.decay, (int)d.erase, (int)d.write, s0, s_final,
-        err_word, 0, nullptr, (__nv_bfloat16*)e_out, states, n_slots, slot0, T_row);
+        err_word, 0, nullptr, (__nv_bfloat16*)e_out, n_slots, slot0, T_row);
     return cudaGetLastError();
 }
 
