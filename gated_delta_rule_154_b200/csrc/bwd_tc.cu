@@ -102,7 +102,7 @@ constexpr uint32_t OFF_GMN = OFF_SMALL + 1024;   // float[128]: g_m of the chunk
 constexpr uint32_t OFF_SCA = OFF_SMALL + 1536;   // float[3][64]: scalar a, b, w
 constexpr uint32_t OFF_EXP = OFF_SMALL + 2304;   // float[4][128]: partial G_C terms
 constexpr uint32_t OFF_BAR = OFF_SMALL + 4352;
-constexpr int NBAR = 13;
+constexpr int NBAR = 12;
 constexpr uint32_t OFF_TSLOT = OFF_BAR + 8 * NBAR;
 constexpr uint32_t OFF_ABORT = OFF_TSLOT + 4;
 constexpr uint32_t SMEM_USED = OFF_ABORT + 4;
@@ -126,33 +126,29 @@ struct BwMaps {
     CUtensorMap xq, xk, yk, yb, du;         // float32 outputs, 32-channel slabs
 };
 
-// Staging of the float32 outputs for their TMA stores: four 8 KB slabs (64
-// tokens x 32 channels, 128-byte swizzled rows) per tensor.  XQ', XK', YB',
-// YK' go where [Q'; K'], [B"; K"], [dO; dY] and dS~ were once the chunk's
-// last products are done; dU goes into the A_qb/A_qk and dE tiles, free
-// once the products that read them are done.
-__device__ __forceinline__ uint32_t slab_du(int p) {
-    return p < 2 ? OFF_GQ + 8192u * p : OFF_DE + 8192u * (p - 2);
+// Staging of the float32 outputs for their TMA stores: 4 KB boxes of 32
+// tokens x 32 channels (128-byte swizzled rows), each written and stored by
+// one compute warp.  XQ', XK', YB', YK' go where [Q'; K'], [B"; K"], [dO; dY]
+// and dS~ were, once the chunk's last products are done (box 2p + h: channels
+// 32p.., tokens 32h..); dU goes into the A_qb/A_qk and dE tiles, free once
+// the products that read them are done.
+__device__ __forceinline__ uint32_t box_du(int bx) {
+    return bx < 4 ? OFF_GQ + 4096u * bx : OFF_DE + 4096u * (bx - 4);
 }
-// byte offset of float (row r, channel c) in a staged tile
-__device__ __forceinline__ uint32_t stage_off(int r, int c) {
-    return 8192u * (uint32_t)(c >> 5) + 128u * (uint32_t)r +
-           ((uint32_t)(((c & 31) >> 2) ^ (r & 7)) << 4) + 4u * (uint32_t)(c & 3);
-}
-// one row of 32 channels (slab base given) as eight 16-byte stores
-__device__ __forceinline__ void stage_row32(uint8_t* slab, int r, const float* v) {
+// one row of 32 channels of a box as eight 16-byte stores
+__device__ __forceinline__ void stage_row32(uint8_t* box, int r, const float* v) {
 #pragma unroll
     for (int c16 = 0; c16 < 8; ++c16)
-        *reinterpret_cast<float4*>(slab + 128 * r + ((c16 ^ (r & 7)) << 4)) =
+        *reinterpret_cast<float4*>(box + 128 * r + ((c16 ^ (r & 7)) << 4)) =
             make_float4(v[4 * c16], v[4 * c16 + 1], v[4 * c16 + 2], v[4 * c16 + 3]);
 }
 
 // Barriers: TMA and tensor-core completions, then the compute threads'
 // "ready" signals to the issuing warp (thread 0 arrives after a compute
-// barrier).
+// barrier).  The compute warps issue the TMA loads and stores themselves.
 enum : uint32_t {
     B_LD, B_G, B_Z1, B_Z3, B_A, B_XY, B_FIN,   // loads / gram / -dE / dY / D~,dU,dA / X,Y / all
-    R_LD, R_OP, R_GQ, R_DE, R_DY, R_DA          // ready for: loads / gram / -dE / dY / D~,dU,dA / X,Y
+    R_OP, R_GQ, R_DE, R_DY, R_DA                // ready for: gram / -dE / dY / D~,dU,dA / X,Y
 };
 static_assert(R_DA + 1 == NBAR, "barrier count");
 
@@ -352,7 +348,6 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             tc::tma_prefetch_desc(&maps.e);
             tc::tma_prefetch_desc(&maps.sst);
             uint32_t ph = 0;
-            uint32_t n_ld = 0;
             auto wait_ready = [&](uint32_t id, uint32_t parity) {
                 if (!tc::mbar_wait_bounded(bar(id), parity, WAIT_NS)) { *abort_s = 1; return false; }
                 tc::fence_after_sync();
@@ -361,55 +356,8 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             const uint32_t idKK = tc::idesc_bf16(128, 128, 0, 0);
             const uint32_t idKM = tc::idesc_bf16(128, 128, 0, 1);
             const uint32_t idMM = tc::idesc_bf16(128, 128, 1, 1);
-            const uint32_t nbox = 10u + (va ? 2u : 0u) + (vb ? 2u : 0u) + (vw ? 2u : 0u);
-            // the chunk's XQ', XK', YB', YK' from their staging tiles
-            auto store_xy = [&](int t0s) {
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const int x = 32 * p;
-                    tc::tma_store_4d(&maps.xq, sbase + OFF_QK + 8192 * p, x, hi, t0s, bi);
-                    tc::tma_store_4d(&maps.xk, sbase + OFF_BK + 8192 * p, x, hi, t0s, bi);
-                    tc::tma_store_4d(&maps.yb, sbase + OFF_DOY + 8192 * p, x, hi, t0s, bi);
-                    tc::tma_store_4d(&maps.yk, sbase + OFF_DS + 8192 * p, x, hi, t0s, bi);
-                }
-                tc::bulk_commit();
-            };
-            int it = 0;
-            bool done = true;
 #pragma unroll 1
-            for (int c = NC - 1; c >= 0; --c, ph ^= 1, ++it) {
-                const int t0 = c * C;
-                done = false;
-                // the previous chunk's outputs are staged: store them, and load
-                // this chunk's tiles once the stores have read their staging
-                if (it > 0) {
-                    if (!wait_ready(R_LD, ph ^ 1)) break;
-                    store_xy(t0 + C);
-                    tc::bulk_wait_read();
-                }
-                tc::mbar_arrive_expect_tx(bar(B_LD), nbox * BOX_BYTES + 2u * 16384u);
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    const int x = 64 * p;
-                    tc::tma_load_4d(sbase + OFF_QK + p * 16384, &maps.q, x, hi, t0, bi, bar(B_LD));
-                    tc::tma_load_4d(sbase + OFF_QK + p * 16384 + 8192, &maps.k, x, hi, t0, bi,
-                                    bar(B_LD));
-                    if (vb)
-                        tc::tma_load_4d(sbase + OFF_BK + p * 16384, &maps.b, x, hi, t0, bi,
-                                        bar(B_LD));
-                    if (va)
-                        tc::tma_load_4d(sbase + OFF_BK + p * 16384 + 8192, &maps.a, x, hi, t0, bi,
-                                        bar(B_LD));
-                    tc::tma_load_4d(sbase + OFF_DOY + p * 16384, &maps.dout, x, hi, t0, bi,
-                                    bar(B_LD));
-                    tc::tma_load_4d(sbase + OFF_EIN + p * 8192, &maps.e, x, hi, t0, bi, bar(B_LD));
-                    tc::tma_load_4d(sbase + OFF_UIN + p * 8192, &maps.v, x, hi, t0, bi, bar(B_LD));
-                    if (vw)
-                        tc::tma_load_4d(sbase + OFF_DE + p * 8192, &maps.w, x, hi, t0, bi, bar(B_LD));
-                    tc::tma_load_4d(sbase + OFF_DS + p * 16384, &maps.sst, x, 0, bh * NC + c, 0,
-                                    bar(B_LD));
-                }
-                ++n_ld;
+            for (int c = NC - 1; c >= 0; --c, ph ^= 1) {
                 // gram [Q'; K'] [B"; K"]^T; Z = [B"; K"] dS~; D~ += Q'^T dO
                 if (!wait_ready(R_OP, ph)) break;
 #pragma unroll
@@ -475,20 +423,10 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                     tc::mma_bf16(tmem + TM_G, tc::desc_kmajor(sbase + OFF_DAT, 16384, kk),
                                  tc::desc_mnmajor(sbase + OFF_QK, 16384, kk), idKM, true);
                 tc::mma_commit(bar(B_XY));
-                // dU, staged before R_DA
-#pragma unroll
-                for (int p = 0; p < 4; ++p)
-                    tc::tma_store_4d(&maps.du, sbase + slab_du(p), 32 * p, hi, t0, bi);
-                tc::bulk_commit();
-                done = true;
             }
-            // the last chunk's XQ', XK', YB', YK'
-            if (done && *abort_s == 0 && wait_ready(R_LD, ph ^ 1)) store_xy(0);
             // nothing of this CTA may still be in flight when it exits
             tc::mma_commit(bar(B_FIN));
             tc::mbar_wait_bounded(bar(B_FIN), 0, WAIT_NS);
-            if (n_ld) tc::mbar_wait_bounded(bar(B_LD), (n_ld - 1) & 1, WAIT_NS);
-            tc::bulk_wait_all();
         }
     } else {
         // ======================= compute warps
@@ -525,6 +463,49 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             }
             EXP[cb * D + lane_t] = part;
         }
+        // TMA loads of chunk cc's tiles, spread over the compute warps (tile j
+        // by warp j % 16); B_LD is armed by thread 0 before the compute barrier
+        // that precedes this
+        const uint32_t ld_bytes = (10u + (va ? 2u : 0u) + (vb ? 2u : 0u) + (vw ? 2u : 0u)) *
+                                      BOX_BYTES + 2u * 16384u;
+        auto issue_loads = [&](int cc) {
+            if ((tid & 31) != 0) return;
+            const int t0l = cc * C;
+            const uint32_t bl = bar(B_LD);
+#pragma unroll 1
+            for (int j = warp; j < 18; j += 16) {
+                const int p = j & 1, x = 64 * p;
+                switch (j >> 1) {
+                case 0: tc::tma_load_4d(sbase + OFF_QK + p * 16384, &maps.q, x, hi, t0l, bi, bl); break;
+                case 1: tc::tma_load_4d(sbase + OFF_QK + p * 16384 + 8192, &maps.k, x, hi, t0l, bi, bl); break;
+                case 2: tc::tma_load_4d(sbase + OFF_DOY + p * 16384, &maps.dout, x, hi, t0l, bi, bl); break;
+                case 3: tc::tma_load_4d(sbase + OFF_EIN + p * 8192, &maps.e, x, hi, t0l, bi, bl); break;
+                case 4: tc::tma_load_4d(sbase + OFF_UIN + p * 8192, &maps.v, x, hi, t0l, bi, bl); break;
+                case 5: tc::tma_load_4d(sbase + OFF_DS + p * 16384, &maps.sst, x, 0, bh * NC + cc, 0, bl); break;
+                case 6: if (vb) tc::tma_load_4d(sbase + OFF_BK + p * 16384, &maps.b, x, hi, t0l, bi, bl); break;
+                case 7: if (va) tc::tma_load_4d(sbase + OFF_BK + p * 16384 + 8192, &maps.a, x, hi, t0l, bi, bl); break;
+                default: if (vw) tc::tma_load_4d(sbase + OFF_DE + p * 8192, &maps.w, x, hi, t0l, bi, bl); break;
+                }
+            }
+        };
+        int ld_out = 0;          // (thread 0) a load round issued and not yet waited for
+        uint32_t ld_ph = 0;      // its phase parity
+        if (NC > 0) {
+            if (tid == 0) tc::mbar_arrive_expect_tx(bar(B_LD), ld_bytes);
+            compute_sync();
+            issue_loads(NC - 1);
+            ld_out = 1;
+        }
+        // this warp's 32 x 32 box of a staged output out by TMA (rows past T
+        // are not stored; a box starting past T is not issued)
+        auto store_box = [&](const CUtensorMap* m, uint32_t box, int ch0, int tok0) {
+            tc::fence_async_smem();
+            __syncwarp();
+            if ((tid & 31) == 0 && tok0 < T) {
+                tc::tma_store_4d(m, sbase + box, ch0, hi, tok0, bi);
+                tc::bulk_commit();
+            }
+        };
         uint32_t ph = 0;
         auto signal_or_stop = [&](uint32_t id) {
             const bool stop = compute_sync_or(*abort_s != 0);
@@ -543,8 +524,10 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                 sca[64 + tid] = (b_kind == GDR_GATE_SCALAR && in) ? to_f32(b[tok]) : 1.f;
                 sca[128 + tid] = (w_kind == GDR_GATE_SCALAR && in) ? to_f32(w[tok]) : 1.f;
             }
-            if (tid == 0 && !*abort_s && !tc::mbar_wait_bounded(bar(B_LD), ph, WAIT_NS))
-                *abort_s = 1;
+            if (tid == 0) {
+                if (!*abort_s && !tc::mbar_wait_bounded(bar(B_LD), ph, WAIT_NS)) *abort_s = 1;
+                else ld_out = 0;
+            }
             if (compute_sync_or(*abort_s != 0)) break;
             operand_pass<FG2>(sm, tid, va, vb, vw, fb, fw, a_kind, n, sca, QT, GM, GC, err_word);
             compute_sync();
@@ -720,11 +703,13 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                 }
                 tc::store_row32_bf16(sm + OFF_DAT + (cb >> 1) * 16384, lane_t, cb & 1, vals);
             }
-            if (quarter >= 2) {   // dU -> its staging slabs (rows past T are not stored)
+            if (quarter >= 2) {   // dU: this warp's 32 tokens x 32 channels
                 float vals[32];
                 tc::tmem_ld32(tmem + lane_off + TM_Z + 32 * cb, vals);
                 tc::tmem_wait_ld();
-                stage_row32(sm + slab_du(cb), lane_t - 64, vals);
+                const int bx = 2 * cb + (quarter & 1);
+                stage_row32(sm + box_du(bx), tid & 31, vals);
+                store_box(&maps.du, box_du(bx), 32 * cb, t0 + 32 * (quarter & 1));
             }
             tc::fence_async_smem();
             tc::fence_before_sync();
@@ -733,26 +718,44 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             // ================= C6: [XQ' | XK']^T and [YB'; YK'] out
             wait_then_sync(bar(B_XY), ph, tid, abort_s);
             {
-                // [XQ' | XK']^T: lane = channel, columns = tokens; into [token][channel]
+                // [XQ' | XK']^T: lane = channel, columns = tokens; this warp's
+                // channels 32q.. and tokens 32(cb & 1).. into a [token][channel] box
                 float vals[32];
                 tc::tmem_ld32(tmem + lane_off + TM_Z + 32 * cb, vals);
                 tc::tmem_wait_ld();
-                uint8_t* dst = sm + (cb < 2 ? OFF_QK : OFF_BK);
-                const int r0 = 32 * (cb & 1);
+                const uint32_t box = (cb < 2 ? OFF_QK : OFF_BK) + 4096u * (2 * quarter + (cb & 1));
+                const int cl = tid & 31;
+                uint8_t* dst = sm + box + 4 * (cl & 3);
 #pragma unroll
                 for (int x = 0; x < 32; ++x)
-                    *reinterpret_cast<float*>(dst + stage_off(r0 + x, lane_t)) = vals[x];
+                    *reinterpret_cast<float*>(dst + 128 * x + ((((cl >> 2) ^ (x & 7))) << 4)) = vals[x];
+                store_box(cb < 2 ? &maps.xq : &maps.xk, box, 32 * quarter, t0 + 32 * (cb & 1));
             }
             {
+                // [YB'; YK']: lane = token, this warp's 32 channels 32cb..
                 float vals[32];
                 tc::tmem_ld32(tmem + lane_off + TM_G + 32 * cb, vals);
                 tc::tmem_wait_ld();
-                stage_row32(sm + (lane_t < 64 ? OFF_DOY : OFF_DS) + 8192 * cb, lane_t & 63, vals);
+                const uint32_t box = (quarter < 2 ? OFF_DOY : OFF_DS) + 4096u * (2 * cb + (quarter & 1));
+                stage_row32(sm + box, tid & 31, vals);
+                store_box(quarter < 2 ? &maps.yb : &maps.yk, box, 32 * cb, t0 + 32 * (quarter & 1));
             }
-            tc::fence_async_smem();
+            // this warp's stores (dU, X, Y) have read their boxes
+            if ((tid & 31) == 0) tc::bulk_wait_read();
+            __syncwarp();
             tc::fence_before_sync();
-            if (signal_or_stop(R_LD)) break;
+            if (tid == 0 && c > 0) tc::mbar_arrive_expect_tx(bar(B_LD), ld_bytes);
+            if (compute_sync_or(*abort_s != 0)) break;
+            // the next chunk's tiles
+            if (c > 0) {
+                issue_loads(c - 1);
+                ld_out = 1;
+                ld_ph = ph ^ 1;
+            }
         }
+        // nothing this CTA started may still be in flight when it exits
+        if (tid == 0 && ld_out) tc::mbar_wait_bounded(bar(B_LD), ld_ph, WAIT_NS);
+        if ((tid & 31) == 0) tc::bulk_wait_all();
         // dS0 = g_m(first chunk) D~
         if (ds0 && NC > 0 && !compute_sync_or(*abort_s != 0)) {
             float vals[32];

@@ -91,26 +91,32 @@ def test_scalar_gates_bf16():
     _compare(_gpu(wl, inp, up), _oracle(wl, inp, up), TOL["bf16"])
 
 
-def test_gate_one_everywhere():
-    """No gate tensors (a = b = w = 1): plain DeltaNet; no gate gradients."""
-    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=75, dtype="f32")
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_gate_one_everywhere(dtype):
+    """No gate tensors (a = b = w = 1): plain DeltaNet; no gate gradients
+    (bf16: the tensor-core path, 75 tokens = one full chunk and a tail)."""
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=75, dtype=dtype)
     inp = W.make_prefill(wl, seed=3)
     up = W.make_upstream(wl, seed=3)
     d = inputs_to_dev(inp, wl)
-    g = api.backward(d["q"], d["k"], d["v"], None, None, None, d["s0"], to_dev(up["do"], "f32"),
+    g = api.backward(d["q"], d["k"], d["v"], None, None, None, d["s0"], to_dev(up["do"], dtype),
                      to_dev(up["dsT"], "f32"))
     torch.cuda.synchronize()
-    f = lambda key: W.as_f32(inp[key], "f32")
-    ref = oracle.backward(f("q"), f("k"), f("v"), None, None, None, inp["s0"], up["do"], up["dsT"])
-    _compare(g, ref, TOL["f32"])
+    assert api.last_device_error() == 0
+    f = lambda key: W.as_f32(inp[key], dtype)
+    ref = oracle.backward(f("q"), f("k"), f("v"), None, None, None, inp["s0"],
+                          W.as_f32(up["do"], dtype), up["dsT"])
+    _compare(g, ref, TOL[dtype])
 
 
-def test_without_state_gradient_or_initial_state():
-    wl = W.WORKLOADS["gdn2_bf16"].replace(B=2, H=1, T=90, dtype="f32")
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_without_state_gradient_or_initial_state(dtype):
+    wl = W.WORKLOADS["gdn2_bf16"].replace(B=2, H=1, T=90, dtype=dtype)
     inp = W.make_prefill(wl, seed=9)
     up = W.make_upstream(wl, seed=9)
     g = _gpu(wl, inp, up, with_dsT=False, s0=False)
-    _compare(g, _oracle(wl, inp, up, with_dsT=False, s0=False), TOL["f32"])
+    assert api.last_device_error() == 0
+    _compare(g, _oracle(wl, inp, up, with_dsT=False, s0=False), TOL[dtype])
 
 
 def test_zero_length_passes_the_state_gradient_through():
@@ -125,8 +131,9 @@ def test_zero_length_passes_the_state_gradient_through():
 
 
 def test_decay_beyond_range_is_reported():
-    """Every channel's decay over a 32-token chunk must multiply to at least
-    exp(-80); a stronger one is flagged as GDR_ERR_RANGE."""
+    """Every channel's decay must multiply to at least about exp(-80) over a
+    32-token chunk (the tensor-core path: over tokens 1-31 and 32-63 of each
+    64-token chunk); a stronger one is flagged as GDR_ERR_RANGE."""
     wl = W.WORKLOADS["gdn2_bf16"].replace(B=1, H=2, T=64)
     inp = W.make_prefill(wl, seed=1)
     a = inp["a"].copy()
