@@ -88,15 +88,28 @@ def prefill_flops(wl) -> int:
     return wl.B * wl.T * wl.H * (8 * d * d + 16 * C * d + C * C)
 
 
-BWD_CHUNK = 32  # the backward pass always walks 32-token chunks
+BWD_CHUNK = 32  # the CUDA-core / mma.sync backward walks 32-token chunks
+
+
+def backward_tc_path(wl) -> bool:
+    """bf16, d = 128: the tensor-core backward (three launches)."""
+    return wl.dtype == "bf16" and wl.dk == 128 and wl.dv == 128
 
 
 def backward_flops(wl) -> int:
-    """Flops of one backward call, counted 2mnk over dense tiles, per
-    token-head: the forward sweep that stores the chunk-start states
-    (two grams, Y, E and the state update: 6 dk dv + 4 C dk + 4 C dv) plus the
-    reverse sweep (18 dk dv + 20 C dv + 24 C dk: four grams, Y and E, dE and
-    dY, dU, four dA, four [C, dk] gradient sums, dS, the grams' gradients)."""
+    """Tensor-core flops of one backward call, per token-head.
+    Tensor-core path (bf16, d = 128): the state-writing prefill launch
+    (8 d^2 + 16 C d + C^2 as for the prefill) plus the reverse sweep's
+    products as issued, 76 K-steps of a 128 x 128 x 16 tcgen05.mma per
+    64-token chunk (zero halves of padded A operands included) = 622,592.
+    Otherwise, 2mnk over dense tiles: the forward sweep that stores the
+    chunk-start states (6 dk dv + 4 C dk + 4 C dv) plus the reverse sweep
+    (18 dk dv + 20 C dv + 24 C dk), C = 32."""
+    if backward_tc_path(wl):
+        d = wl.dk
+        fwd = 8 * d * d + 16 * 64 * d + 64 * 64
+        rev = 76 * 2 * 128 * 128 * 16 // 64
+        return wl.B * wl.T * wl.H * (fwd + rev)
     dk, dv, C = wl.dk, wl.dv, BWD_CHUNK
     fwd = 6 * dk * dv + 4 * C * dk + 4 * C * dv
     rev = 18 * dk * dv + 20 * C * dv + 24 * C * dk
@@ -573,7 +586,11 @@ def run_gpu(args):
             raise RuntimeError("device error during backward timing")
         bflops, bbytes = backward_flops(wl), backward_bytes(wl)
         achieved_tf = bflops / (bms * 1e-3) / 1e12
-        if wl.dtype == "bf16":  # products on tf32 mma.sync: tf32 tensor peak
+        if backward_tc_path(wl):  # tcgen05, bf16 operands: the bf16 tensor peak
+            broof = {"bound": "tensor", "achieved": achieved_tf,
+                     "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+                     "peak_source": "%s bf16_tflops" % peak_src}
+        elif wl.dtype == "bf16":  # products on tf32 mma.sync: tf32 tensor peak
             broof = {"bound": "tensor", "achieved": achieved_tf,
                      "peak": float(peaks["bf16_tflops"]) * TF32_OVER_BF16, "unit": "TFLOP/s",
                      "peak_source": "%s bf16_tflops x %.4f (nominal dense tf32 : bf16, "
@@ -588,12 +605,9 @@ def run_gpu(args):
                            % wl.name,
                "steps": args.backward_steps, "ms_per_step": bms,
                "tokens/s": tokens_step / (bms * 1e-3),
-               # bf16, d = 128: three launches of the tensor-core forward writing
-               # the chunk-start states (whole rows, tokens 0..31, tokens 32..),
-               # then the backward kernel
-               "launches_per_step": (4 if wl.T > 32 else 2)
-                                    if (wl.dtype == "bf16" and wl.dk == 128 and wl.dv == 128)
-                                    else 1,
+               # bf16, d = 128: the tensor-core prefill writing S~, E and S_T,
+               # the reverse sweep, the elementwise gradient kernel
+               "launches_per_step": 3 if backward_tc_path(wl) else 1,
                "roofline": broof,
                "hbm": {"algorithmic_bytes_per_step": bbytes,
                        "GB/s": bbytes / (bms * 1e-3) / 1e9,
