@@ -117,6 +117,14 @@ constexpr uint32_t TM_Z = 256;   // [-dE -> dY; dU], then [XQ' | XK']^T
 constexpr uint32_t TM_S = 384;   // S~ as a bf16 A operand (lane i, 64 columns)
 constexpr uint32_t TM_EU = 448;  // [-E; U] as a bf16 A operand (lane s, 64 columns)
 
+// The operand pass's tiles: Q', K' over raw q, k (QK); B", K" over raw b, a
+// (BK); U over raw v; w in OFF_DE
+__device__ __forceinline__ OpTiles op_tiles() {
+    return OpTiles{OFF_QK, OFF_QK + 8192, OFF_BK + 8192, OFF_BK,     // q, k, a, b
+                   OFF_QK, OFF_QK + 8192, OFF_BK + 8192, OFF_BK,     // Q', K', K", B"
+                   OFF_UIN, OFF_DE};                                 // v -> U, w
+}
+
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait
 constexpr uint32_t BOX_BYTES = 64 * 128;     // one 64 x 64 bf16 TMA box
 
@@ -151,112 +159,6 @@ enum : uint32_t {
     R_OP, R_GQ, R_DE, R_DY, R_DA                // ready for: gram / -dE / dY / D~,dU,dA / X,Y
 };
 static_assert(R_DA + 1 == NBAR, "barrier count");
-
-// Decay factors and scaled operands of one chunk (the forward kernel's
-// operand pass, with the backward's tile placement).  Thread (channel pair
-// p2, token octet q8); writes, one bf16 pair per token,
-//   Q' = Lam q and K' = Lam k over raw q, k (QK rows r, 64 + r)
-//   B" = b K" and K" = k / Lam over raw b, a (BK rows r, 64 + r)
-//   U  = w v over raw v
-// and per channel g_m and gc.  Lam and 1/Lam are formed as in the forward:
-// every divisor is a product of a over tokens 1..31 or 32..63 of the chunk,
-// which the range check bounds from below.
-template <bool FG2>
-__device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool vb, bool vw,
-                                             bool fb, bool fw, int a_kind, int n,
-                                             const float* sca, float* QT, float* GM, float* GC,
-                                             int* err_word) {
-    const int p2 = tid & 63, q8 = tid >> 6;
-    const uint32_t pnl = (uint32_t)(p2 >> 5);
-    const int ch = (p2 & 31) >> 2;
-    const uint32_t cofs = 4u * (uint32_t)(p2 & 3);
-    uint32_t apr[8];
-    float loc0[8], loc1[8];
-    float run0 = 1.f, run1 = 1.f;
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-        const int r = 8 * q8 + x;
-        // raw a in rows 64-127 of BK (row 64 + r swizzles like row r)
-        uint32_t pr = va ? *reinterpret_cast<const uint32_t*>(
-                               sm + OFF_BK + pnl * 16384u + (uint32_t)(64 + r) * 128u +
-                               ((uint32_t)(ch ^ (r & 7)) << 4) + cofs)
-                         : tc::pack_bf16x2(sca[r], sca[r]);
-        apr[x] = (a_kind != GDR_GATE_ONE && r < n) ? pr : 0x3F803F80u;
-        const float a0 = __uint_as_float(apr[x] << 16), a1 = __uint_as_float(apr[x] & 0xFFFF0000u);
-        if (r > 0) {
-            run0 *= a0;
-            run1 *= a1;
-        }
-        loc0[x] = run0;
-        loc1[x] = run1;
-    }
-    const float f0 = q8 == 0 ? __uint_as_float(apr[0] << 16) : 1.f;
-    const float f1 = q8 == 0 ? __uint_as_float(apr[0] & 0xFFFF0000u) : 1.f;
-    *reinterpret_cast<float2*>(QT + q8 * D + 2 * p2) = make_float2(f0 * run0, f1 * run1);
-    compute_sync();
-    float gm0 = 1.f, gm1 = 1.f, gc0 = 1.f, gc1 = 1.f, sp0 = 1.f, sp1 = 1.f, mp0 = 1.f,
-          mp1 = 1.f;
-#pragma unroll
-    for (int gg = 0; gg < 8; ++gg) {
-        const float2 qv = *reinterpret_cast<const float2*>(QT + gg * D + 2 * p2);
-        if (gg < 4) { gm0 *= qv.x; gm1 *= qv.y; } else { gc0 *= qv.x; gc1 *= qv.y; }
-        if (gg > q8 && gg < 4) { sp0 *= qv.x; sp1 *= qv.y; }
-        if (gg >= 4 && gg < q8) { mp0 *= qv.x; mp1 *= qv.y; }
-    }
-    auto emit = [&](int x, uint32_t e, uint32_t ei) {
-        const int r = 8 * q8 + x;
-        const uint32_t sw = (uint32_t)r * 128u + ((uint32_t)(ch ^ (r & 7)) << 4) + cofs;
-        const uint32_t o128 = pnl * 16384u + sw, o64 = pnl * 8192u + sw;
-        const uint32_t q2 = *reinterpret_cast<const uint32_t*>(sm + OFF_QK + o128);
-        const uint32_t k2 = *reinterpret_cast<const uint32_t*>(sm + OFF_QK + o128 + 8192u);
-        const uint32_t b2 = vb ? *reinterpret_cast<const uint32_t*>(sm + OFF_BK + o128)
-                               : tc::pack_bf16x2(sca[64 + r], sca[64 + r]);
-        const uint32_t v2 = *reinterpret_cast<const uint32_t*>(sm + OFF_UIN + o64);
-        const uint32_t w2 = vw ? *reinterpret_cast<const uint32_t*>(sm + OFF_DE + o64)
-                               : tc::pack_bf16x2(sca[128 + r], sca[128 + r]);
-        // FG^2-GDN learning rates: key sqrt(beta^k) k with erase gate 1, write
-        // gate sqrt(beta^v)
-        const uint32_t kt2 = (FG2 && fb) ? mul2(k2, sqrt2(b2)) : k2;
-        const uint32_t kk2 = mul2(kt2, ei);
-        *reinterpret_cast<uint32_t*>(sm + OFF_QK + o128) = mul2(q2, e);            // Q'
-        *reinterpret_cast<uint32_t*>(sm + OFF_QK + o128 + 8192u) = mul2(kt2, e);   // K'
-        *reinterpret_cast<uint32_t*>(sm + OFF_BK + o128) =
-            (FG2 && fb) ? kk2 : mul2(b2, kk2);                                    // B"
-        *reinterpret_cast<uint32_t*>(sm + OFF_BK + o128 + 8192u) = kk2;           // K"
-        *reinterpret_cast<uint32_t*>(sm + OFF_UIN + o64) =
-            mul2((FG2 && fw) ? sqrt2(w2) : w2, v2);                               // U
-    };
-    float rev0 = 1.f, rev1 = 1.f;
-    if (q8 < 4) {  // warp-uniform
-        const float d0 = rcp_approx(sp0 * run0), d1 = rcp_approx(sp1 * run1);
-#pragma unroll
-        for (int x = 7; x >= 0; --x) {
-            emit(x, tc::pack_bf16x2(loc0[x] * d0, loc1[x] * d1),
-                 tc::pack_bf16x2(rev0 * sp0, rev1 * sp1));
-            rev0 *= __uint_as_float(apr[x] << 16);
-            rev1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
-        }
-    } else {
-        const float d0 = rcp_approx(mp0 * run0), d1 = rcp_approx(mp1 * run1);
-#pragma unroll
-        for (int x = 7; x >= 0; --x) {
-            emit(x, tc::pack_bf16x2(mp0 * loc0[x], mp1 * loc1[x]),
-                 tc::pack_bf16x2(rev0 * d0, rev1 * d1));
-            rev0 *= __uint_as_float(apr[x] << 16);
-            rev1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
-        }
-    }
-    if (q8 == 0) {
-        const int i = 2 * p2;
-        GM[i] = gm0;
-        GM[i + 1] = gm1;
-        GC[i] = gc0;
-        GC[i + 1] = gc1;
-        const bool ok0 = run0 * sp0 >= 1e-35f && gc0 >= 1e-35f;
-        const bool ok1 = run1 * sp1 >= 1e-35f && gc1 >= 1e-35f;
-        if (a_kind != GDR_GATE_ONE && !(ok0 && ok1)) atomicOr(err_word, kErrRange);
-    }
-}
 
 __device__ __forceinline__ void wait_then_sync(uint32_t bar, uint32_t parity, int tid,
                                                volatile int* abort_s) {
@@ -529,7 +431,12 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                 else ld_out = 0;
             }
             if (compute_sync_or(*abort_s != 0)) break;
-            operand_pass<FG2>(sm, tid, va, vb, vw, fb, fw, a_kind, n, sca, QT, GM, GC, err_word);
+            operand_pass<false, FG2>(sm, op_tiles(), tid, va, vb, vw, fb, fw, a_kind, n, sca, QT,
+                                     err_word, [] {},
+                                     [&](int i, float g_m, float g_c) {
+                                         GM[i] = g_m;
+                                         GC[i] = g_c;
+                                     });
             compute_sync();
             // ================= C1b: [-E; U] and S~ into tensor memory; the rescale
             {

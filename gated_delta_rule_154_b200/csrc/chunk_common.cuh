@@ -8,6 +8,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "common.cuh"
 #include "tc_common.cuh"
 
 namespace gdr {
@@ -61,6 +62,205 @@ __device__ __forceinline__ bool compute_sync_or(bool x) {
 }
 __device__ __forceinline__ void half_sync(int id) {
     asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");
+}
+
+// ------------------------------------------------------------ operand pass
+
+// Tile offsets (bytes from the shared-memory base) of one operand pass: the
+// raw tiles it reads and the operand tiles it writes.  q, k, a, b and Q', K',
+// K", B" are halves of 128-row tiles (16 KB panels); v (replaced by U) and w
+// are 64-row tiles (8 KB panels).
+struct OpTiles {
+    uint32_t q, k, a, b, Qp, Kp, Kpp, Bpp, v, w;
+};
+
+// Byte offset of the 8-byte group of channels 4cq .. 4cq+3 in row r of a
+// tile with `pb`-byte panels (128-byte swizzled rows).
+__device__ __forceinline__ uint32_t quad_off(int r, int cq, uint32_t pb) {
+    return (uint32_t)(cq >> 4) * pb + (uint32_t)r * 128u +
+           ((uint32_t)(((cq & 15) >> 1) ^ (r & 7)) << 4) + 8u * (uint32_t)(cq & 1);
+}
+__device__ __forceinline__ uint2 mul4(uint2 x, uint2 y) {
+    return make_uint2(mul2(x.x, y.x), mul2(x.y, y.y));
+}
+__device__ __forceinline__ uint2 sqrt4(uint2 x) { return make_uint2(sqrt2(x.x), sqrt2(x.y)); }
+__device__ __forceinline__ uint2 ld8(const uint8_t* p) { return *reinterpret_cast<const uint2*>(p); }
+__device__ __forceinline__ void st8(uint8_t* p, uint2 v) { *reinterpret_cast<uint2*>(p) = v; }
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Decay factors and scaled operands of one 64-token chunk, all 512 compute
+// threads.  Thread (token octet q8 = warp / 2, channel quad cq = 16 (warp %
+// 2) + lane / 2, half h = lane % 2) reads the decays of its four channels
+// over its four tokens of the octet (8-byte accesses; a warp covers two
+// 64-channel row halves per access), forms their running products (leaving
+// out the chunk's first token, so that no divisor below holds a_0), takes the
+// other half's product from the neighbouring lane, and for h = 0 writes the
+// octet totals (QT, float [8][128]).  After one exchange it has gamma_r / g_m and
+// g_m / gamma_r (g_m = gamma_31) for its four tokens (8 q8 + 4 h ..) and
+// writes, one 8-byte group per token and tensor,
+//   Q' = (gamma/g_m) q, K' = (gamma/g_m) k, K" = (g_m/gamma) k, B" = b K",
+//   U = w v                                       (each rounded once to bf16)
+// in place over the raw tiles.  Every divisor is a product of a over tokens
+// 1..31 or 32..63 of the chunk (or a part of one); the octet-0 threads of
+// warp 0 check that the two whole products stay at or above 1e-35 and hand
+// each channel's g_m and gc = gamma_63/g_m to chan(i, g_m, gc).  `mid` runs
+// between the two halves (after the exchange barrier), before any operand
+// tile is written.  PACKED: rows past n are zeroed (k, q, v) instead of left
+// to the TMA fill.  FG2: key sqrt(beta^k) k with erase gate 1, write gate
+// sqrt(beta^v).
+template <bool PACKED, bool FG2, typename Mid, typename Chan>
+__device__ __forceinline__ void operand_pass(uint8_t* sm, const OpTiles tl, int tid, bool va,
+                                             bool vb, bool vw, bool fb, bool fw, int a_kind,
+                                             int n, const float* sca, float* QT, int* err_word,
+                                             Mid&& mid, Chan&& chan) {
+    // lane pair (2l, 2l + 1) = the two halves of one (channel quad, octet)
+    const int lane = tid & 31, w = tid >> 5;
+    const int q8 = w >> 1, h = lane & 1, cq = 16 * (w & 1) + (lane >> 1);
+    // this half's decays, four channels per token as packed bf16 (1.0 past
+    // the chunk or for GATE_ONE; scalar gates came from bf16, so they are exact)
+    uint2 apr[4];
+#pragma unroll
+    for (int xx = 0; xx < 4; ++xx) {
+        const int r = 8 * q8 + 4 * h + xx;
+        uint2 pr;
+        if (va) {
+            pr = ld8(sm + tl.a + quad_off(r, cq, 16384u));
+        } else {
+            const uint32_t s2 = tc::pack_bf16x2(sca[r], sca[r]);
+            pr = make_uint2(s2, s2);
+        }
+        apr[xx] = (a_kind != GDR_GATE_ONE && r < n) ? pr : make_uint2(0x3F803F80u, 0x3F803F80u);
+    }
+    // running products over this half (token 0 of the chunk left out), then
+    // over the octet with the other half's product
+    float own[4] = {1.f, 1.f, 1.f, 1.f};
+    float loc[4][4];   // [token of this half][channel]
+#pragma unroll
+    for (int xx = 0; xx < 4; ++xx) {
+        if (8 * q8 + 4 * h + xx > 0) {
+            own[0] *= bf_lo(apr[xx].x);
+            own[1] *= bf_hi(apr[xx].x);
+            own[2] *= bf_lo(apr[xx].y);
+            own[3] *= bf_hi(apr[xx].y);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) loc[xx][j] = own[j];
+    }
+    float run[4], other[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        other[j] = __shfl_xor_sync(0xffffffffu, own[j], 1);
+        run[j] = own[j] * other[j];                 // the octet's product
+        if (h) {
+#pragma unroll
+            for (int xx = 0; xx < 4; ++xx) loc[xx][j] *= other[j];
+        }
+    }
+    if (h == 0) {
+        const float f0 = q8 == 0 ? bf_lo(apr[0].x) : 1.f, f1 = q8 == 0 ? bf_hi(apr[0].x) : 1.f;
+        const float f2 = q8 == 0 ? bf_lo(apr[0].y) : 1.f, f3 = q8 == 0 ? bf_hi(apr[0].y) : 1.f;
+        *reinterpret_cast<float4*>(QT + q8 * 128 + 4 * cq) =
+            make_float4(f0 * run[0], f1 * run[1], f2 * run[2], f3 * run[3]);
+    }
+    compute_sync();
+    mid();
+    // pm: for q8 < 4 the product over the octets after this one up to the
+    // middle (sp), for q8 >= 4 over the octets from the middle up to this one
+    // (mp)
+    float pm[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+    for (int gg = 0; gg < 8; ++gg) {
+        if (q8 < 4 ? (gg > q8 && gg < 4) : (gg >= 4 && gg < q8)) {
+            const float4 qv = *reinterpret_cast<const float4*>(QT + gg * 128 + 4 * cq);
+            pm[0] *= qv.x;
+            pm[1] *= qv.y;
+            pm[2] *= qv.z;
+            pm[3] *= qv.w;
+        }
+    }
+    // this half's tokens from the last: rev = product of a over the octet's
+    // tokens after x (for the first half, starting with the second half's)
+    float rev[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) rev[j] = h ? 1.f : other[j];
+    float dd[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dd[j] = rcp_approx(pm[j] * run[j]);
+#pragma unroll
+    for (int xx = 3; xx >= 0; --xx) {
+        const int x = 4 * h + xx;          // token of the octet
+        const int r = 8 * q8 + x;
+        // e = gamma_r/g_m, ei = g_m/gamma_r for the four channels:
+        //   r <= 31: e = loc / (run sp), ei = rev sp
+        //   r >= 32: e = mp loc,         ei = rev / (mp run)
+        float e[4], ei[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (q8 < 4) {
+                e[j] = loc[xx][j] * dd[j];
+                ei[j] = rev[j] * pm[j];
+            } else {
+                e[j] = pm[j] * loc[xx][j];
+                ei[j] = rev[j] * dd[j];
+            }
+        }
+        const uint2 e4 = make_uint2(tc::pack_bf16x2(e[0], e[1]), tc::pack_bf16x2(e[2], e[3]));
+        const uint2 ei4 = make_uint2(tc::pack_bf16x2(ei[0], ei[1]), tc::pack_bf16x2(ei[2], ei[3]));
+        const uint32_t o128 = quad_off(r, cq, 16384u), o64 = quad_off(r, cq, 8192u);
+        uint2 q4 = ld8(sm + tl.q + o128), k4 = ld8(sm + tl.k + o128), v4 = ld8(sm + tl.v + o64);
+        uint2 b4, w4;
+        if (vb) {
+            b4 = ld8(sm + tl.b + o128);
+        } else {
+            const uint32_t s2 = tc::pack_bf16x2(sca[64 + r], sca[64 + r]);
+            b4 = make_uint2(s2, s2);
+        }
+        if (vw) {
+            w4 = ld8(sm + tl.w + o64);
+        } else {
+            const uint32_t s2 = tc::pack_bf16x2(sca[128 + r], sca[128 + r]);
+            w4 = make_uint2(s2, s2);
+        }
+        if (PACKED && r >= n) {  // past the sequence (a packed neighbour's tokens): k = q = v = 0
+            q4 = make_uint2(0u, 0u);
+            k4 = make_uint2(0u, 0u);
+            v4 = make_uint2(0u, 0u);
+        }
+        const uint2 kt4 = (FG2 && fb) ? mul4(k4, sqrt4(b4)) : k4;
+        const uint2 kk4 = mul4(kt4, ei4);
+        st8(sm + tl.Qp + o128, mul4(q4, e4));                               // Q'
+        st8(sm + tl.Kp + o128, mul4(kt4, e4));                              // K'
+        st8(sm + tl.Kpp + o128, kk4);                                       // K"
+        st8(sm + tl.Bpp + o128, (FG2 && fb) ? kk4 : mul4(b4, kk4));         // B"
+        st8(sm + tl.v + o64, mul4((FG2 && fw) ? sqrt4(w4) : w4, v4));       // U
+        rev[0] *= bf_lo(apr[xx].x);
+        rev[1] *= bf_hi(apr[xx].x);
+        rev[2] *= bf_lo(apr[xx].y);
+        rev[3] *= bf_hi(apr[xx].y);
+    }
+    if (q8 == 0 && h == 0) {
+        // g_m = gamma_31 (octets 0-3), gc = prod over octets 4-7 (= gamma_63/g_m);
+        // the divisors above: prod of a over tokens 1..31 (octet 0 holds it as
+        // run * sp) and over tokens 32..63 (gc)
+        float gm[4] = {1.f, 1.f, 1.f, 1.f}, gc[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+        for (int gg = 0; gg < 8; ++gg) {
+            const float4 qv = *reinterpret_cast<const float4*>(QT + gg * 128 + 4 * cq);
+            float* t = gg < 4 ? gm : gc;
+            t[0] *= qv.x;
+            t[1] *= qv.y;
+            t[2] *= qv.z;
+            t[3] *= qv.w;
+        }
+        bool ok = true;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            ok = ok && run[j] * pm[j] >= 1e-35f && gc[j] >= 1e-35f;
+            chan(4 * cq + j, gm[j], gc[j]);
+        }
+        if (a_kind != GDR_GATE_ONE && !ok) atomicOr(err_word, kErrRange);
+    }
 }
 
 // ---------------------------------------------------------------- UT solve

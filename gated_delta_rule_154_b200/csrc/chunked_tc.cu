@@ -98,6 +98,12 @@ constexpr uint32_t TM_X = 128;   // [R -> E; O] 128 x 128
 constexpr uint32_t TM_S = 256;   // S~ 128 x 128 (lane = key channel), float32 state
 constexpr uint32_t TM_AQ = 384;  // A operand [A_kk; A_qk] 128 x 64 bf16 (32 columns)
 
+__device__ __forceinline__ OpTiles op_tiles() {
+    return OpTiles{OFF_RAW + 8192, OFF_RAW, OFF_X1, OFF_X1 + 8192,   // q, k, a, b
+                   OFF_X1 + 8192, OFF_X1, OFF_X2, OFF_X2 + 8192,     // Q', K', K", B"
+                   OFF_U, OFF_W};                                     // v -> U, w
+}
+
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s per wait
 constexpr uint32_t BOX_BYTES = 64 * 128;     // one 64 x 64 bf16 TMA box
 constexpr uint32_t IDESC_NEG_B = 1u << 14;   // negate the B operand
@@ -137,141 +143,6 @@ __device__ __forceinline__ void issue_v(const TcMaps& m, uint32_t sbase, int t0,
 #pragma unroll
     for (int p = 0; p < 2; ++p)
         tc::tma_load_4d(sbase + OFF_U + p * 8192, &m.v, 64 * p, hi, t0, bi, bar);
-}
-
-// Decay factors and scaled operands of one chunk, all 512 compute threads.  Thread
-// (channel pair p2, token octet q8) forms the running products of a over its
-// 8 tokens for channels 2*p2, 2*p2 + 1; after one exchange of octet totals
-// (QT) it has gamma_r/g_m and g_m/gamma_r for its tokens (g_m = gamma_31) and
-// writes, one bf16 pair per token (4-byte accesses, a warp covering one
-// 128-byte row of a panel):
-//   K' = (gamma/g_m) k, Q' = (gamma/g_m) q   over raw a, b in X1
-//   K" = (g_m/gamma) k, B" = b K"            into X2
-//   U  = w v                                 over raw v
-// Octet-0 threads also update the state scales, fcur = fprev * g_m and
-// fprev = gamma_63/g_m, and check that the largest factors, gamma_0/g_m and
-// g_m/gamma_63, stay in float range.  `mid` runs between the two halves (after
-// the exchange barrier), before anything is written to X2.
-template <bool PACKED, bool FG2, typename Mid>
-__device__ __forceinline__ void operand_pass(uint8_t* sm, int tid, bool va, bool vb, bool vw,
-                                             bool fb, bool fw, int a_kind, int n,
-                                             const float* sca, float* QT,
-                                             float* fcur, float* fprev,
-                                             int* err_word, Mid&& mid) {
-    const int p2 = tid & 63, q8 = tid >> 6;
-    const uint32_t pnl = (uint32_t)(p2 >> 5);
-    const int ch = (p2 & 31) >> 2;                 // 16-byte chunk of the pair in its panel
-    const uint32_t cofs = 4u * (uint32_t)(p2 & 3);  // byte of the pair in its chunk
-    // the pair of a per token as two bf16 (1.0 past the chunk or for GATE_ONE;
-    // scalar gates came from bf16, so the pair is exact).  loc = running
-    // product over the octet, leaving out the chunk's first token in octet 0
-    // (so that no divisor below holds a_0); the octet's total (QT) keeps it.
-    uint32_t apr[8];
-    float loc0[8], loc1[8];
-    float run0 = 1.f, run1 = 1.f;
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-        const int r = 8 * q8 + x;
-        uint32_t pr = va ? *reinterpret_cast<const uint32_t*>(
-                               sm + OFF_X1 + pnl * 16384u + (uint32_t)r * 128u +
-                               ((uint32_t)(ch ^ (r & 7)) << 4) + cofs)
-                         : tc::pack_bf16x2(sca[r], sca[r]);
-        apr[x] = (a_kind != GDR_GATE_ONE && r < n) ? pr : 0x3F803F80u;
-        const float a0 = __uint_as_float(apr[x] << 16), a1 = __uint_as_float(apr[x] & 0xFFFF0000u);
-        if (r > 0) {
-            run0 *= a0;
-            run1 *= a1;
-        }
-        loc0[x] = run0;
-        loc1[x] = run1;
-    }
-    const float f0 = q8 == 0 ? __uint_as_float(apr[0] << 16) : 1.f;
-    const float f1 = q8 == 0 ? __uint_as_float(apr[0] & 0xFFFF0000u) : 1.f;
-    *reinterpret_cast<float2*>(QT + q8 * D + 2 * p2) = make_float2(f0 * run0, f1 * run1);
-    compute_sync();
-    mid();
-    // Octet totals: gm = gamma_31 (octets 0-3), gc = prod over octets 4-7
-    // (= gamma_63/g_m); sp = prod over the octets after this one up to the
-    // middle (q8 < 4); mp = prod over the octets from the middle up to this
-    // one (q8 >= 4).
-    float gm0 = 1.f, gm1 = 1.f, gc0 = 1.f, gc1 = 1.f, sp0 = 1.f, sp1 = 1.f, mp0 = 1.f,
-          mp1 = 1.f;
-#pragma unroll
-    for (int gg = 0; gg < 8; ++gg) {
-        const float2 qv = *reinterpret_cast<const float2*>(QT + gg * D + 2 * p2);
-        if (gg < 4) { gm0 *= qv.x; gm1 *= qv.y; } else { gc0 *= qv.x; gc1 *= qv.y; }
-        if (gg > q8 && gg < 4) { sp0 *= qv.x; sp1 *= qv.y; }
-        if (gg >= 4 && gg < q8) { mp0 *= qv.x; mp1 *= qv.y; }
-    }
-    // Token r = 8 q8 + x, rev = product of a over the octet's tokens after x:
-    //   r <= 31: g_m/gamma_r = rev * sp, gamma_r/g_m = loc_x / (run * sp)
-    //   r >= 32: gamma_r/g_m = mp * loc_x, g_m/gamma_r = rev / (mp * run)
-    // Every divisor is a product of a over tokens 1..31 or 32..63 of the chunk
-    // (or a part of one), which the range check below bounds from below, so
-    // the factors never pass through gamma_r itself (which may be far
-    // smaller than either factor).
-    // per token: e = gamma_r/g_m, ei = g_m/gamma_r as bf16 pairs; K', Q', K",
-    // B", U written in place
-    auto emit = [&](int x, uint32_t e, uint32_t ei) {
-        const int r = 8 * q8 + x;
-        const uint32_t sw = (uint32_t)r * 128u + ((uint32_t)(ch ^ (r & 7)) << 4) + cofs;
-        const uint32_t o128 = pnl * 16384u + sw, o64 = pnl * 8192u + sw;
-        uint32_t k2 = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW + o128);
-        uint32_t q2 = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW + o128 + 8192u);
-        const uint32_t b2 = vb ? *reinterpret_cast<const uint32_t*>(sm + OFF_X1 + o128 + 8192u)
-                               : tc::pack_bf16x2(sca[64 + r], sca[64 + r]);
-        uint32_t v2 = *reinterpret_cast<const uint32_t*>(sm + OFF_U + o64);
-        const uint32_t w2 = vw ? *reinterpret_cast<const uint32_t*>(sm + OFF_W + o64)
-                               : tc::pack_bf16x2(sca[128 + r], sca[128 + r]);
-        if (PACKED && r >= n) {  // past the sequence (a packed neighbour's tokens): k = q = v = 0
-            k2 = 0u;
-            q2 = 0u;
-            v2 = 0u;
-        }
-        // FG^2-GDN learning rates: key sqrt(beta^k) k with erase gate 1, write
-        // gate sqrt(beta^v)
-        const uint32_t kt2 = (FG2 && fb) ? mul2(k2, sqrt2(b2)) : k2;
-        const uint32_t kk2 = mul2(kt2, ei);                                      // K"
-        *reinterpret_cast<uint32_t*>(sm + OFF_X1 + o128) = mul2(kt2, e);         // K'
-        *reinterpret_cast<uint32_t*>(sm + OFF_X1 + o128 + 8192u) = mul2(q2, e);  // Q'
-        *reinterpret_cast<uint32_t*>(sm + OFF_X2 + o128) = kk2;
-        *reinterpret_cast<uint32_t*>(sm + OFF_X2 + o128 + 8192u) =
-            (FG2 && fb) ? kk2 : mul2(b2, kk2);                                 // B"
-        *reinterpret_cast<uint32_t*>(sm + OFF_U + o64) =
-            mul2((FG2 && fw) ? sqrt2(w2) : w2, v2);                            // U
-    };
-    float rev0 = 1.f, rev1 = 1.f;
-    if (q8 < 4) {   // warp-uniform
-        const float d0 = rcp_approx(sp0 * run0), d1 = rcp_approx(sp1 * run1);
-#pragma unroll
-        for (int x = 7; x >= 0; --x) {
-            emit(x, tc::pack_bf16x2(loc0[x] * d0, loc1[x] * d1),
-                 tc::pack_bf16x2(rev0 * sp0, rev1 * sp1));
-            rev0 *= __uint_as_float(apr[x] << 16);
-            rev1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
-        }
-    } else {
-        const float d0 = rcp_approx(mp0 * run0), d1 = rcp_approx(mp1 * run1);
-#pragma unroll
-        for (int x = 7; x >= 0; --x) {
-            emit(x, tc::pack_bf16x2(mp0 * loc0[x], mp1 * loc1[x]),
-                 tc::pack_bf16x2(rev0 * d0, rev1 * d1));
-            rev0 *= __uint_as_float(apr[x] << 16);
-            rev1 *= __uint_as_float(apr[x] & 0xFFFF0000u);
-        }
-    }
-    if (q8 == 0) {
-        const int i = 2 * p2;
-        fcur[i] = fprev[i] * gm0;
-        fcur[i + 1] = fprev[i + 1] * gm1;
-        fprev[i] = gc0;
-        fprev[i + 1] = gc1;
-        // the divisors above: prod of a over tokens 1..31 (octet 0 holds it as
-        // run * sp) and over tokens 32..63 (gc)
-        const bool ok0 = run0 * sp0 >= 1e-35f && gc0 >= 1e-35f;
-        const bool ok1 = run1 * sp1 >= 1e-35f && gc1 >= 1e-35f;
-        if (a_kind != GDR_GATE_ONE && !(ok0 && ok1)) atomicOr(err_word, kErrRange);
-    }
 }
 
 // Compute thread 0 waits on `bar`; the compute barrier that follows releases
@@ -564,13 +435,19 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             }
             if (compute_sync_or(*abort_s != 0)) break;
             // ================= P1c:
-            operand_pass<PACKED, FG2>(sm, tid, va, vb, vw, fb, fw, a_kind, min(C, L - t0),
-                         sca, QT, fcur, fprev, err_word, [&] {
+            // K' over raw a, Q' over raw b (X1), K" and B" into X2, U over raw v;
+            // the state scales: fcur = fprev g_m, fprev = gamma_63 / g_m
+            operand_pass<PACKED, FG2>(sm, op_tiles(), tid, va, vb, vw, fb, fw, a_kind,
+                         min(C, L - t0), sca, QT, err_word, [&] {
                              if (t0 == 0) return;
                              // the last chunk's state update has read X2 and EB and
                              // finished its O: O -> staging tile for the issuing warp
                              wait_then_sync(bar(B_ST), ph ^ 1, tid, abort_s);
                              if (!DUMP) read_o();
+                         },
+                         [&](int i, float g_m, float g_c) {
+                             fcur[i] = fprev[i] * g_m;
+                             fprev[i] = g_c;
                          });
             tc::fence_async_smem();
             signal(R_OP);
