@@ -33,7 +33,7 @@
 // instantiation (every chunk's S~ and E in bf16, exactly the tiles its own
 // products read, and S_T in float32); bwd_tc_kernel, one CTA per (batch,
 // head) walking the chunks from the last, which carries D~ in tensor memory
-// and writes XQ', XK', YK', YB', dU (float32, by TMA store) and per chunk
+// and writes XQ', XK', YK', YB', dU (bf16, by TMA store) and per chunk
 // the G_C terms and gc; and bwd_epilogue_kernel, one warp per (batch, head,
 // chunk), which forms the six gradients from them and the raw inputs (the
 // reverse cumulative sum for da).  The G_C term of a chunk is rowsum(D~ S~)
@@ -62,7 +62,7 @@
 namespace gdr {
 
 bool tc_map_bf16(CUtensorMap* m, const void* ptr, int B, int T, int H, int T_row);
-bool tc_map_f32(CUtensorMap* m, const void* ptr, int B, int T, int H);
+bool tc_map_bf16_box32(CUtensorMap* m, const void* ptr, int B, int T, int H);
 bool tc_map_state_bf16(CUtensorMap* m, const void* ptr, long long n_slots);
 cudaError_t launch_chunked_tc_states(const gdr_desc& d, int T_row, const void* q, const void* k,
                                      const void* v, const void* a, const void* b,
@@ -131,24 +131,29 @@ constexpr uint32_t BOX_BYTES = 64 * 128;     // one 64 x 64 bf16 TMA box
 struct BwMaps {
     CUtensorMap q, k, v, a, b, w, dout, e;  // bf16 inputs (a/b/w only for vector gates)
     CUtensorMap sst;                        // the forward's S~ tiles
-    CUtensorMap xq, xk, yk, yb, du;         // float32 outputs, 32-channel slabs
+    CUtensorMap xq, xk, yk, yb, du;         // bf16 intermediates, 32 x 32 boxes
 };
 
-// Staging of the float32 outputs for their TMA stores: 4 KB boxes of 32
-// tokens x 32 channels (128-byte swizzled rows), each written and stored by
-// one compute warp.  XQ', XK', YB', YK' go where [Q'; K'], [B"; K"], [dO; dY]
-// and dS~ were, once the chunk's last products are done (box 2p + h: channels
-// 32p.., tokens 32h..); dU goes into the A_qb/A_qk and dE tiles, free once
-// the products that read them are done.
-__device__ __forceinline__ uint32_t box_du(int bx) {
-    return bx < 4 ? OFF_GQ + 4096u * bx : OFF_DE + 4096u * (bx - 4);
-}
-// one row of 32 channels of a box as eight 16-byte stores
+// Staging of the bf16 intermediates for their TMA stores: 2 KB boxes of 32
+// tokens x 32 channels (64-byte rows, 64-byte swizzle: 16-byte chunk c of row
+// r at c ^ ((r / 2) % 4)), each written and stored by one compute warp.
+// XQ', XK', YB', YK' go where [Q'; K'], [B"; K"], [dO; dY] and dS~ were, once
+// the chunk's last products are done (box 2p + h: channels 32p.., tokens
+// 32h..); dU goes into the A_qb/A_qk tile, free once the product that reads
+// it is done.
+constexpr uint32_t SBOX = 2048;   // bytes of one staging box
+__device__ __forceinline__ uint32_t box_du(int bx) { return OFF_GQ + SBOX * bx; }
+// one row of 32 channels of a box, rounded to bf16, as four 16-byte stores
 __device__ __forceinline__ void stage_row32(uint8_t* box, int r, const float* v) {
 #pragma unroll
-    for (int c16 = 0; c16 < 8; ++c16)
-        *reinterpret_cast<float4*>(box + 128 * r + ((c16 ^ (r & 7)) << 4)) =
-            make_float4(v[4 * c16], v[4 * c16 + 1], v[4 * c16 + 2], v[4 * c16 + 3]);
+    for (int c16 = 0; c16 < 4; ++c16) {
+        uint4 u;
+        u.x = tc::pack_bf16x2(v[8 * c16], v[8 * c16 + 1]);
+        u.y = tc::pack_bf16x2(v[8 * c16 + 2], v[8 * c16 + 3]);
+        u.z = tc::pack_bf16x2(v[8 * c16 + 4], v[8 * c16 + 5]);
+        u.w = tc::pack_bf16x2(v[8 * c16 + 6], v[8 * c16 + 7]);
+        *reinterpret_cast<uint4*>(box + 64 * r + ((c16 ^ ((r >> 1) & 3)) << 4)) = u;
+    }
 }
 
 // Barriers: TMA and tensor-core completions, then the compute threads'
@@ -177,7 +182,7 @@ __device__ __forceinline__ void store_row32_f32(float* dst, const float* v) {
 
 // The reverse sweep.  S~ of every chunk arrives through the sst map
 // ([B*H][NC][128][128] bf16); sT [B*H][128][128] the final states; XQ', XK',
-// YK', YB', dU leave through the float32 maps; gce, gcs: [B*H][NC][128] the
+// YK', YB', dU leave through the bf16 maps; gce, gcs: [B*H][NC][128] the
 // G_C terms and gc.
 template <bool FG2>
 __global__ void __launch_bounds__(NT, 1)
@@ -630,12 +635,14 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                 float vals[32];
                 tc::tmem_ld32(tmem + lane_off + TM_Z + 32 * cb, vals);
                 tc::tmem_wait_ld();
-                const uint32_t box = (cb < 2 ? OFF_QK : OFF_BK) + 4096u * (2 * quarter + (cb & 1));
+                const uint32_t box = (cb < 2 ? OFF_QK : OFF_BK) + SBOX * (2 * quarter + (cb & 1));
                 const int cl = tid & 31;
-                uint8_t* dst = sm + box + 4 * (cl & 3);
+                uint8_t* dst = sm + box + 2 * (cl & 7);
 #pragma unroll
                 for (int x = 0; x < 32; ++x)
-                    *reinterpret_cast<float*>(dst + 128 * x + ((((cl >> 2) ^ (x & 7))) << 4)) = vals[x];
+                    *reinterpret_cast<__nv_bfloat16*>(dst + 64 * x +
+                                                      (((cl >> 3) ^ ((x >> 1) & 3)) << 4)) =
+                        __float2bfloat16_rn(vals[x]);
                 store_box(cb < 2 ? &maps.xq : &maps.xk, box, 32 * quarter, t0 + 32 * (cb & 1));
             }
             {
@@ -643,7 +650,7 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                 float vals[32];
                 tc::tmem_ld32(tmem + lane_off + TM_G + 32 * cb, vals);
                 tc::tmem_wait_ld();
-                const uint32_t box = (quarter < 2 ? OFF_DOY : OFF_DS) + 4096u * (2 * cb + (quarter & 1));
+                const uint32_t box = (quarter < 2 ? OFF_DOY : OFF_DS) + SBOX * (2 * cb + (quarter & 1));
                 stage_row32(sm + box, tid & 31, vals);
                 store_box(quarter < 2 ? &maps.yb : &maps.yk, box, 32 * cb, t0 + 32 * (quarter & 1));
             }
@@ -734,9 +741,9 @@ bwd_epilogue_kernel(int T, int H, int NC, long long n_units, const __nv_bfloat16
                     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                     const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
                     const __nv_bfloat16* __restrict__ w, int a_kind, int b_kind, int w_kind,
-                    const float* __restrict__ xq, const float* __restrict__ xk,
-                    const float* __restrict__ yk, const float* __restrict__ yb,
-                    const float* __restrict__ du, const float* __restrict__ gce,
+                    const __nv_bfloat16* __restrict__ xq, const __nv_bfloat16* __restrict__ xk,
+                    const __nv_bfloat16* __restrict__ yk, const __nv_bfloat16* __restrict__ yb,
+                    const __nv_bfloat16* __restrict__ du, const float* __restrict__ gce,
                     const float* __restrict__ gcs, __nv_bfloat16* __restrict__ dq,
                     __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
                     __nv_bfloat16* __restrict__ da, __nv_bfloat16* __restrict__ db,
@@ -766,11 +773,11 @@ bwd_epilogue_kernel(int T, int H, int NC, long long n_units, const __nv_bfloat16
             ld_gate4(a, a_kind, th, tv, av);
             ld_gate4(b, b_kind, th, tv, bv);
             ld_gate4(w, w_kind, th, tv, wv);
-            ld_f32x4(xq + tv, XQ);
-            ld_f32x4(xk + tv, XK);
-            ld_f32x4(yk + tv, YK);
-            ld_f32x4(yb + tv, YB);
-            ld_f32x4(du + tv, dU);
+            ld_bf16x4(xq + tv, XQ);
+            ld_bf16x4(xk + tv, XK);
+            ld_bf16x4(yk + tv, YK);
+            ld_bf16x4(yb + tv, YB);
+            ld_bf16x4(du + tv, dU);
             float oq[4], ok[4], ov[4], oa[4], ob[4], ow[4];
             float sb = 0.f, sw = 0.f, sa = 0.f;
 #pragma unroll
@@ -826,7 +833,7 @@ struct TcWorkspace {
     void* states;    // [B*H][NC][128][128] bf16 S~
     float* sT;       // [B*H][128][128]
     void* e;         // [B, T, H, 128] bf16
-    float* pre[5];   // XQ', XK', YK', YB', dU: [B, T, H, 128] float32
+    void* pre[5];    // XQ', XK', YK', YB', dU: [B, T, H, 128] bf16
     float* gce;      // [B*H][NC][128] G_C terms
     float* gcs;      // [B*H][NC][128] gc per chunk and channel
     size_t bytes;
@@ -846,7 +853,7 @@ TcWorkspace carve(const gdr_desc& d, void* base) {
     w.states = take(bh * nc * D * D * 2);
     w.sT = reinterpret_cast<float*>(take(bh * D * D * 4));
     w.e = take(tok * D * 2);
-    for (int x = 0; x < 5; ++x) w.pre[x] = reinterpret_cast<float*>(take(tok * D * 4));
+    for (int x = 0; x < 5; ++x) w.pre[x] = take(tok * D * 2);
     w.gce = reinterpret_cast<float*>(take(bh * nc * D * 4));
     w.gcs = reinterpret_cast<float*>(take(bh * nc * D * 4));
     w.bytes = off;
@@ -886,9 +893,11 @@ cudaError_t launch_backward_tc(const gdr_desc& d, const void* const* in, const f
         ok = tc_map_bf16(&maps.b, in[4], B, T, H, T);
     if (ok && (d.write == GDR_GATE_VECTOR || d.write == GDR_GATE_FG2))
         ok = tc_map_bf16(&maps.w, in[5], B, T, H, T);
-    ok = ok && tc_map_f32(&maps.xq, ws.pre[0], B, T, H) && tc_map_f32(&maps.xk, ws.pre[1], B, T, H) &&
-         tc_map_f32(&maps.yk, ws.pre[2], B, T, H) && tc_map_f32(&maps.yb, ws.pre[3], B, T, H) &&
-         tc_map_f32(&maps.du, ws.pre[4], B, T, H) &&
+    ok = ok && tc_map_bf16_box32(&maps.xq, ws.pre[0], B, T, H) &&
+         tc_map_bf16_box32(&maps.xk, ws.pre[1], B, T, H) &&
+         tc_map_bf16_box32(&maps.yk, ws.pre[2], B, T, H) &&
+         tc_map_bf16_box32(&maps.yb, ws.pre[3], B, T, H) &&
+         tc_map_bf16_box32(&maps.du, ws.pre[4], B, T, H) &&
          tc_map_state_bf16(&maps.sst, ws.states, (long long)B * H * NC);
     if (!ok) return cudaErrorInvalidValue;
 
@@ -909,8 +918,10 @@ cudaError_t launch_backward_tc(const gdr_desc& d, const void* const* in, const f
     bwd_epilogue_kernel<<<(unsigned)((units + 3) / 4), 128, 0, st>>>(
         T, H, NC, units, static_cast<const __nv_bfloat16*>(in[0]),
         static_cast<const __nv_bfloat16*>(in[1]), static_cast<const __nv_bfloat16*>(in[2]), a, b,
-        w, (int)d.decay, (int)d.erase, (int)d.write, ws.pre[0], ws.pre[1], ws.pre[2], ws.pre[3],
-        ws.pre[4], ws.gce, ws.gcs, static_cast<__nv_bfloat16*>(grads[0]),
+        w, (int)d.decay, (int)d.erase, (int)d.write,
+        static_cast<const __nv_bfloat16*>(ws.pre[0]), static_cast<const __nv_bfloat16*>(ws.pre[1]),
+        static_cast<const __nv_bfloat16*>(ws.pre[2]), static_cast<const __nv_bfloat16*>(ws.pre[3]),
+        static_cast<const __nv_bfloat16*>(ws.pre[4]), ws.gce, ws.gcs, static_cast<__nv_bfloat16*>(grads[0]),
         static_cast<__nv_bfloat16*>(grads[1]), static_cast<__nv_bfloat16*>(grads[2]),
         static_cast<__nv_bfloat16*>(grads[3]), static_cast<__nv_bfloat16*>(grads[4]),
         static_cast<__nv_bfloat16*>(grads[5]));

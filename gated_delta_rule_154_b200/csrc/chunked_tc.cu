@@ -663,19 +663,19 @@ bool tc_map_bf16(CUtensorMap* m, const void* ptr, int B, int T, int H, int T_row
     return make_map(m, ptr, B, T, H, T_row);
 }
 
-// [B, T, H, 128] float32 tensor as a 4-D map {128, H, T, B}, box {32, 1, 32,
-// 1} (32 channels of 32 tokens, 128-byte rows), 128-byte swizzle: the
-// backward's staging format for its float32 outputs.
-bool tc_map_f32(CUtensorMap* m, const void* ptr, int B, int T, int H) {
+// [B, T, H, 128] bf16 tensor as a 4-D map {128, H, T, B}, box {32, 1, 32, 1}
+// (32 channels of 32 tokens, 64-byte rows), 64-byte swizzle: the backward's
+// staging format for its intermediate outputs.
+bool tc_map_bf16_box32(CUtensorMap* m, const void* ptr, int B, int T, int H) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4,
-                                   (cuuint64_t)T * H * D * 4};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2,
+                                   (cuuint64_t)T * H * D * 2};
     const cuuint32_t box[4] = {32, 1, 32, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(ptr), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }

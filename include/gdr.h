@@ -193,9 +193,9 @@ gdr_status gdr_decode_step_paged(const gdr_desc *desc, const void *q, const void
  * is invalid.  Pure host function, no CUDA call.
  *   - bf16 with dk = dv = 128 and T > 0 (the tensor-core path): the scaled
  *     state at the start of every 64-token chunk (bf16) and the final state
- *     (float32), every chunk's E (bf16), five float32 [B, T, H, 128]
+ *     (float32), every chunk's E (bf16), five bf16 [B, T, H, 128]
  *     intermediates and two float32 rows per chunk and head:
- *     B * H * (ceil(T / 64) * 33792 + 65536) + B * T * H * 2816 bytes.
+ *     B * H * (ceil(T / 64) * 33792 + 65536) + B * T * H * 1536 bytes.
  *   - otherwise: the state at the start of every 32-token chunk plus one
  *     running state gradient, B * H * dk * dv * 4 * (ceil(T / 32) + 1). */
 size_t gdr_backward_workspace_size(const gdr_desc *desc);
@@ -292,7 +292,7 @@ gdr_status gdr_backward_varlen(const gdr_desc *desc, const int *cu_seqlens, int 
  * cudaMalloc, no cudaFree, no allocating library routine.
  *   - Size limit: when gdr_backward_workspace_size(desc) exceeds
  *     GDR_NOALLOC_SCRATCH_BYTES the call returns GDR_ERR_WORKSPACE before any
- *     CUDA call (e.g. bf16, dk = dv = 128, B * H = 1: up to about 20k tokens).
+ *     CUDA call (e.g. bf16, dk = dv = 128, B * H = 1: up to about 32k tokens).
  *   - First call on a device: it looks up the scratch's device address with
  *     cudaGetSymbolAddress on the current device and caches it.  Make that
  *     first call on each device before any stream capture begins.

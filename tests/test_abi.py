@@ -172,9 +172,9 @@ def test_backward_workspace_size(lib):
     assert _lib.backward_workspace_size(d) == 2 * 4 * 128 * 64 * 4 * (4 + 1)
     assert _lib.backward_workspace_size(_desc(T=0)) == 2 * 4 * 128 * 128 * 4
     # bf16, d = 128: bf16 states at 64-token chunk starts and S_T, E, five
-    # float32 intermediates, two rows per chunk and head
+    # bf16 intermediates, two rows per chunk and head
     tc = _desc(B=2, T=100, H=4)
-    assert _lib.backward_workspace_size(tc) == 2 * 4 * (2 * 33792 + 65536) + 2 * 100 * 4 * 2816
+    assert _lib.backward_workspace_size(tc) == 2 * 4 * (2 * 33792 + 65536) + 2 * 100 * 4 * 1536
     # packed sequences keep the 32-token layout
     assert _lib.backward_varlen_workspace_size(_desc(B=1, T=100, H=4), 3) == \
         4 * 128 * 128 * 4 * (4 + 2 * 3)

@@ -77,8 +77,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(name):
 
 
 def test_noalloc_refuses_a_problem_larger_than_its_scratch():
-    """bf16, dk = dv = 128 needs about 3.3 KiB per token and head (chunk-start
-    states, E, the float32 intermediates): 32k tokens of one head do not fit
+    """bf16, dk = dv = 128 needs about 2 KiB per token and head (chunk-start
+    states, E, the bf16 intermediates): 32k tokens of one head do not fit
     and are refused with GDR_ERR_WORKSPACE before anything is launched."""
     desc = _lib.GdrDesc(B=1, T=32 * 1024, H=1, dk=128, dv=128, chunk=32, in_dtype=_lib.BF16,
                         decay=_lib.GATE_VECTOR, erase=_lib.GATE_VECTOR, write=_lib.GATE_VECTOR)
