@@ -157,9 +157,10 @@ def test_repeatable_bit_for_bit():
 
 def test_full_size_sampled_heads():
     """The bench-sized workload (B=8, T=8192, H=16, d=128, bf16) on the GPU;
-    the oracle recomputes the gradients of a seeded sample of whole heads."""
+    the oracle recomputes the gradients of one whole head of every batch row
+    (eight heads, spread over the head index)."""
     wl = W.WORKLOADS["gdn2_bf16"]
-    heads = [(0, 3), (5, 11)]
+    heads = [(bi, (5 * bi + 3) % wl.H) for bi in range(wl.B)]
     inp = W.make_prefill(wl, seed=0)
     up = W.make_upstream(wl, seed=0)
     g = _gpu(wl, inp, up)
