@@ -761,69 +761,103 @@ bwd_epilogue_kernel(int T, int H, int NC, long long n_units, const __nv_bfloat16
     float lam[4], cum[4] = {0.f, 0.f, 0.f, 0.f}, gterm[4];
     ld_f32x4(gcs + (bh * NC + c) * D + i0, lam);
     ld_f32x4(gce + (bh * NC + c) * D + i0, gterm);
+    // one token's inputs, still packed (bf16 x 4 per tensor); the next
+    // token's are loaded while this one is processed
+    struct Tok {
+        uint2 q, k, v, a, b, w, xq, xk, yk, yb, du;
+    };
+    auto gate4 = [&](const __nv_bfloat16* g, int kind, long long th, long long tv) -> uint2 {
+        if (kind == GDR_GATE_ONE) return make_uint2(0x3F803F80u, 0x3F803F80u);
+        if (kind == GDR_GATE_SCALAR) {
+            const uint32_t s1 = *reinterpret_cast<const uint16_t*>(g + th);
+            return make_uint2(s1 | (s1 << 16), s1 | (s1 << 16));
+        }
+        return *reinterpret_cast<const uint2*>(g + tv);
+    };
+    auto load_tok = [&](int r, Tok& t) {
+        const long long th = tok0 + (long long)r * H, tv = th * D + i0;
+        t.q = *reinterpret_cast<const uint2*>(q + tv);
+        t.k = *reinterpret_cast<const uint2*>(k + tv);
+        t.v = *reinterpret_cast<const uint2*>(v + tv);
+        t.a = gate4(a, a_kind, th, tv);
+        t.b = gate4(b, b_kind, th, tv);
+        t.w = gate4(w, w_kind, th, tv);
+        t.xq = *reinterpret_cast<const uint2*>(xq + tv);
+        t.xk = *reinterpret_cast<const uint2*>(xk + tv);
+        t.yk = *reinterpret_cast<const uint2*>(yk + tv);
+        t.yb = *reinterpret_cast<const uint2*>(yb + tv);
+        t.du = *reinterpret_cast<const uint2*>(du + tv);
+    };
+    auto unpack = [](uint2 u, float* f) {
+        f[0] = __uint_as_float(u.x << 16);
+        f[1] = __uint_as_float(u.x & 0xFFFF0000u);
+        f[2] = __uint_as_float(u.y << 16);
+        f[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    };
+    Tok cur, nxt;
+    if (n > 0) load_tok(n - 1, cur);
 #pragma unroll 1
-    for (int r = C - 1; r >= 0; --r) {
-        float av[4] = {1.f, 1.f, 1.f, 1.f};
-        if (r < n) {
-            const long long th = tok0 + (long long)r * H, tv = th * D + i0;
-            float qv[4], kv[4], vv[4], bv[4], wv[4], XQ[4], XK[4], YK[4], YB[4], dU[4];
-            ld_bf16x4(q + tv, qv);
-            ld_bf16x4(k + tv, kv);
-            ld_bf16x4(v + tv, vv);
-            ld_gate4(a, a_kind, th, tv, av);
-            ld_gate4(b, b_kind, th, tv, bv);
-            ld_gate4(w, w_kind, th, tv, wv);
-            ld_bf16x4(xq + tv, XQ);
-            ld_bf16x4(xk + tv, XK);
-            ld_bf16x4(yk + tv, YK);
-            ld_bf16x4(yb + tv, YB);
-            ld_bf16x4(du + tv, dU);
-            float oq[4], ok[4], ov[4], oa[4], ob[4], ow[4];
-            float sb = 0.f, sw = 0.f, sa = 0.f;
+    for (int r = n - 1; r >= 0; --r) {
+        if (r > 0) load_tok(r - 1, nxt);
+        const long long th = tok0 + (long long)r * H, tv = th * D + i0;
+        float qv[4], kv[4], vv[4], av[4], bv[4], wv[4], XQ[4], XK[4], YK[4], YB[4], dU[4];
+        unpack(cur.q, qv);
+        unpack(cur.k, kv);
+        unpack(cur.v, vv);
+        unpack(cur.a, av);
+        unpack(cur.b, bv);
+        unpack(cur.w, wv);
+        unpack(cur.xq, XQ);
+        unpack(cur.xk, XK);
+        unpack(cur.yk, YK);
+        unpack(cur.yb, YB);
+        unpack(cur.du, dU);
+        float oq[4], ok[4], ov[4], oa[4], ob[4], ow[4];
+        float sb = 0.f, sw = 0.f, sa = 0.f;
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const float lm = lam[x], li = 1.f / lm;
-                const float sbk = fb ? sqrt_fast(fmaxf(bv[x], 0.f)) : 1.f;   // sqrt(beta^k)
-                const float kt = kv[x] * sbk;                                 // the key used
-                const float bt = fb ? 1.f : bv[x];                            // the erase gate used
-                const float wt = fw ? sqrt_fast(fmaxf(wv[x], 0.f)) : wv[x];   // the write gate used
-                const float Kpp = li * kt;
-                float dG = lm * (qv[x] * XQ[x] + kt * XK[x]) - Kpp * (YK[x] + bt * YB[x]);
-                if (r == n - 1) dG += gterm[x];
-                cum[x] += dG;
-                const float dkt = lm * XK[x] + li * (YK[x] + bt * YB[x]);
-                oq[x] = lm * XQ[x];
-                ok[x] = dkt * sbk;
-                ov[x] = wt * dU[x];
-                ob[x] = fb ? kv[x] * dkt / (2.f * sbk) : Kpp * YB[x];
-                ow[x] = fw ? vv[x] * dU[x] / (2.f * wt) : vv[x] * dU[x];
-                oa[x] = cum[x] / av[x];
-                sb += ob[x];
-                sw += ow[x];
-                sa += cum[x];
-            }
-            st_bf16x4(dq + tv, oq);
-            st_bf16x4(dk + tv, ok);
-            st_bf16x4(dv + tv, ov);
-            if (a_kind == GDR_GATE_VECTOR) st_bf16x4(da + tv, oa);
-            if (b_kind == GDR_GATE_VECTOR || fb) st_bf16x4(db + tv, ob);
-            if (w_kind == GDR_GATE_VECTOR || fw) st_bf16x4(dw + tv, ow);
-            if (a_kind == GDR_GATE_SCALAR) {
-                sa = warp_sum(sa);
-                if (lane == 0) da[th] = __float2bfloat16_rn(sa / av[0]);
-            }
-            if (b_kind == GDR_GATE_SCALAR) {
-                sb = warp_sum(sb);
-                if (lane == 0) db[th] = __float2bfloat16_rn(sb);
-            }
-            if (w_kind == GDR_GATE_SCALAR) {
-                sw = warp_sum(sw);
-                if (lane == 0) dw[th] = __float2bfloat16_rn(sw);
-            }
+        for (int x = 0; x < 4; ++x) {
+            const float lm = lam[x], li = 1.f / lm;
+            const float sbk = fb ? sqrt_fast(fmaxf(bv[x], 0.f)) : 1.f;   // sqrt(beta^k)
+            const float kt = kv[x] * sbk;                                 // the key used
+            const float bt = fb ? 1.f : bv[x];                            // the erase gate used
+            const float wt = fw ? sqrt_fast(fmaxf(wv[x], 0.f)) : wv[x];   // the write gate used
+            const float Kpp = li * kt;
+            float dG = lm * (qv[x] * XQ[x] + kt * XK[x]) - Kpp * (YK[x] + bt * YB[x]);
+            if (r == n - 1) dG += gterm[x];
+            cum[x] += dG;
+            const float dkt = lm * XK[x] + li * (YK[x] + bt * YB[x]);
+            oq[x] = lm * XQ[x];
+            ok[x] = dkt * sbk;
+            ov[x] = wt * dU[x];
+            ob[x] = fb ? kv[x] * dkt / (2.f * sbk) : Kpp * YB[x];
+            ow[x] = fw ? vv[x] * dU[x] / (2.f * wt) : vv[x] * dU[x];
+            oa[x] = cum[x] / av[x];
+            sb += ob[x];
+            sw += ow[x];
+            sa += cum[x];
+        }
+        st_bf16x4(dq + tv, oq);
+        st_bf16x4(dk + tv, ok);
+        st_bf16x4(dv + tv, ov);
+        if (a_kind == GDR_GATE_VECTOR) st_bf16x4(da + tv, oa);
+        if (b_kind == GDR_GATE_VECTOR || fb) st_bf16x4(db + tv, ob);
+        if (w_kind == GDR_GATE_VECTOR || fw) st_bf16x4(dw + tv, ow);
+        if (a_kind == GDR_GATE_SCALAR) {
+            sa = warp_sum(sa);
+            if (lane == 0) da[th] = __float2bfloat16_rn(sa / av[0]);
+        }
+        if (b_kind == GDR_GATE_SCALAR) {
+            sb = warp_sum(sb);
+            if (lane == 0) db[th] = __float2bfloat16_rn(sb);
+        }
+        if (w_kind == GDR_GATE_SCALAR) {
+            sw = warp_sum(sw);
+            if (lane == 0) dw[th] = __float2bfloat16_rn(sw);
         }
         // Lam of the token before
 #pragma unroll
         for (int x = 0; x < 4; ++x) lam[x] /= av[x];
+        cur = nxt;
     }
 }
 
