@@ -267,13 +267,14 @@ __device__ __forceinline__ void operand_pass(uint8_t* sm, const OpTiles tl, int 
 // T = (I + N)^{-1}, N = A_kb strictly lower 64 x 64 (float, row stride NSP, in
 // NS), by the 2 x 2 block recursion of a unit lower triangular inverse,
 //   [[T1, 0], [T21, T2]] with T21 = -T2 N21 T1,
-// applied at 16 and at 32 rows: the four 16 x 16 diagonal inverses by
-// substitution, then two rounds for the 16 x 16 blocks (1,0) and (3,2), then
-// two for the 32 x 32 block below the diagonal.  Run by 256 threads (tid
-// 0-255 as passed; barrier id 2).  Each finished block also goes, in bf16,
-// into a 64-row operand panel Z3 (128-byte swizzled rows): T - I + DIAG * I,
-// i.e. T - I for DIAG = 0 and T + I for DIAG = 2; the blocks above the
-// diagonal are not written (the caller keeps them zero).
+// applied at 8, 16 and 32 rows: the eight 8 x 8 diagonal inverses by
+// substitution and the 8 x 8 blocks below them, then two rounds for the
+// 16 x 16 blocks (1,0) and (3,2), then two for the 32 x 32 block below the
+// diagonal.  Run by 256 threads (tid 0-255 as passed; barrier id 2).  Each
+// finished block also goes, in bf16, into a 64-row operand panel Z3
+// (128-byte swizzled rows): T - I + DIAG * I, i.e. T - I for DIAG = 0 and
+// T + I for DIAG = 2; the 16 x 16 blocks above the diagonal are not written
+// (the caller keeps them zero).
 
 // One element into the 128-byte swizzled Z3 rows.
 __device__ __forceinline__ void z3_put(uint8_t* z3, int row, int col, float v) {
@@ -285,35 +286,68 @@ __device__ __forceinline__ void z3_put2(uint8_t* z3, int row, int col, float v0,
                                  2 * (col & 7)) = tc::pack_bf16x2(v0, v1);
 }
 
+// The four 16 x 16 diagonal inverses, themselves by the 2 x 2 recursion at 8
+// rows: the eight 8 x 8 diagonal inverses by forward substitution (thread =
+// block and column, x_r = [r == c] - sum_{s<r} N_rs x_s), then the 8 x 8
+// block below each of their diagonals, T21 = -T2 (N21 T1), one element per
+// thread in two steps.  The 8 x 8 block above each diagonal is written zero.
 template <int DIAG>
-__device__ __forceinline__ void ut_diag(const float* NS, float* TS, uint8_t* z3, int tid) {
+__device__ __forceinline__ void ut_diag(const float* NS, float* TS, float* PS, uint8_t* z3,
+                                        int tid) {
+    {
+        const int B = tid >> 6, r = (tid >> 3) & 7, c = tid & 7;
+        TS[(16 * B + r) * NSP + 16 * B + 8 + c] = 0.f;
+        z3_put(z3, 16 * B + r, 16 * B + 8 + c, 0.f);
+    }
     if (tid < 64) {
-        // column c of the inverse of diagonal block I: x_r = [r == c] - sum_{s<r} N_rs x_s,
-        // each row of N read as 16-byte vectors, two partial sums per row
-        const int I = tid >> 4, c = tid & 15;
-        const float* nb = NS + (16 * I) * NSP + 16 * I;
-        float x[16];
+        const int I = tid >> 3, c = tid & 7;
+        const float* nb = NS + (8 * I) * NSP + 8 * I;
+        float x[8];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.0f : 0.0f;
+        for (int r = 0; r < 8; ++r) {
+            float acc = (r == c) ? 1.0f : 0.0f;
+            if (r > 0) {
+                const float4 n0 = *reinterpret_cast<const float4*>(nb + r * NSP);
+                const float4 n1 = *reinterpret_cast<const float4*>(nb + r * NSP + 4);
+                const float nr[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
 #pragma unroll
-        for (int r = 1; r < 16; ++r) {
-            const float* row = nb + r * NSP;
-            float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-            for (int s4 = 0; 4 * s4 < r; ++s4) {
-                const float4 v = *reinterpret_cast<const float4*>(row + 4 * s4);
-                if (4 * s4 + 0 < r) acc0 = fmaf(v.x, x[4 * s4 + 0], acc0);
-                if (4 * s4 + 1 < r) acc1 = fmaf(v.y, x[4 * s4 + 1], acc1);
-                if (4 * s4 + 2 < r) acc0 = fmaf(v.z, x[4 * s4 + 2], acc0);
-                if (4 * s4 + 3 < r) acc1 = fmaf(v.w, x[4 * s4 + 3], acc1);
+                for (int s = 0; s < r; ++s) acc = fmaf(-nr[s], x[s], acc);
             }
-            x[r] -= acc0 + acc1;
+            x[r] = acc;
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            TS[(16 * I + r) * NSP + 16 * I + c] = x[r];
-            z3_put(z3, 16 * I + r, 16 * I + c, r > c ? x[r] : (r == c ? (float)DIAG : 0.f));
+        for (int r = 0; r < 8; ++r) {
+            TS[(8 * I + r) * NSP + 8 * I + c] = x[r];
+            z3_put(z3, 8 * I + r, 8 * I + c, r > c ? x[r] : (r == c ? (float)DIAG : 0.f));
         }
+    }
+    half_sync(2);
+    const int B = tid >> 6, i = (tid >> 3) & 7, j = tid & 7;
+    {
+        // P = N21 T1: row i of N21 against column j of T1
+        const float* nr = NS + (16 * B + 8 + i) * NSP + 16 * B;
+        const float* tc = TS + (16 * B) * NSP + 16 * B + j;
+        const float4 n0 = *reinterpret_cast<const float4*>(nr);
+        const float4 n1 = *reinterpret_cast<const float4*>(nr + 4);
+        const float nv[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
+        float p = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) p = fmaf(nv[k], tc[k * NSP], p);
+        PS[64 * B + 8 * i + j] = p;
+    }
+    half_sync(2);
+    {
+        // T21 = -T2 P: row i of T2 against column j of P
+        const float* tr = TS + (16 * B + 8 + i) * NSP + 16 * B + 8;
+        const float4 t0 = *reinterpret_cast<const float4*>(tr);
+        const float4 t1 = *reinterpret_cast<const float4*>(tr + 4);
+        const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+        const float* pc = PS + 64 * B + j;
+        float v = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v = fmaf(tv[k], pc[8 * k], v);
+        TS[(16 * B + 8 + i) * NSP + 16 * B + j] = -v;
+        z3_put(z3, 16 * B + 8 + i, 16 * B + j, -v);
     }
     half_sync(2);
 }
@@ -357,7 +391,7 @@ __device__ __forceinline__ void tile_16x8(float* d, const float* A, int lda, con
 template <int DIAG>
 __device__ __forceinline__ void ut_solve(float* NS, float* TS, float* PS, uint8_t* z3, int tid) {
     const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-    ut_diag<DIAG>(NS, TS, z3, tid);
+    ut_diag<DIAG>(NS, TS, PS, z3, tid);
     // blocks (1,0) and (3,2): P = N_IJ T_JJ, then T_IJ = -T_II P (warps 0-3)
     const int b = warp >> 1, nt = warp & 1;
     const int I = 2 * b + 1, J = 2 * b;
