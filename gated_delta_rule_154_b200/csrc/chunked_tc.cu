@@ -395,6 +395,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             tc::tmem_st32(tmem + lane_off + TM_S + c0, vals);
             tc::tmem_wait_st();
         }
+        compute_sync();   // the first chunk's scalar gates are in place
         uint32_t ph = 0;  // phase of the per-chunk barriers
         // O (rows 64-127 of X) -> bf16 staging tile, by the warps of lanes 64-127
         // (each such warp then signals R_O: the issuing warp stores o as soon as
@@ -427,13 +428,16 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             const float* sca = sca_all + cur * 192;
 
             // ================= P1: the chunk's raw tiles; decay factors, scaled operands
-            if (tid == 0) {
+            // every compute thread waits on the tile groups itself (no CTA
+            // barrier here: the previous chunk ended on one); a wait that runs
+            // out sets the abort flag, and the vote at the chunk's end stops
+            // all threads together
+            if (!*abort_s) {
                 bool ok = tc::mbar_wait_bounded(bar(B_KQW), ph, WAIT_NS);
                 ok = ok && (!has_ab || tc::mbar_wait_bounded(bar(B_AB), ph, WAIT_NS));
                 ok = ok && tc::mbar_wait_bounded(bar(B_V), ph, WAIT_NS);
                 if (!ok) *abort_s = 1;
             }
-            if (compute_sync_or(*abort_s != 0)) break;
             // ================= P1c:
             // K' over raw a, Q' over raw b (X1), K" and B" into X2, U over raw v;
             // the state scales: fcur = fprev g_m, fprev = gamma_63 / g_m
