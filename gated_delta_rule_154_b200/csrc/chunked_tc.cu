@@ -145,6 +145,12 @@ __device__ __forceinline__ void issue_v(const TcMaps& m, uint32_t sbase, int t0,
         tc::tma_load_4d(sbase + OFF_U + p * 8192, &m.v, 64 * p, hi, t0, bi, bar);
 }
 
+// Arrivals that complete a "ready" barrier: one per compute warp for the
+// operand sets whose writers only need their own warp's work in place, eight
+// for R_P4 and R_O (the warps that write them), else compute thread 0 after a
+// compute barrier.
+__host__ __device__ constexpr uint32_t ready_count(uint32_t id);
+
 // Compute thread 0 waits on `bar`; the compute barrier that follows releases
 // the other compute threads.
 __device__ __forceinline__ void wait_then_sync(uint32_t bar, uint32_t parity, int tid,
@@ -165,6 +171,9 @@ enum : uint32_t {
     R_OP, R_P2, R_P4, R_P5, R_E, R_O  // ready for: gram / X, S~ / A U / E / O, S~ / o store
 };
 static_assert(R_O + 1 == NBAR, "barrier count");
+__host__ __device__ constexpr uint32_t ready_count(uint32_t id) {
+    return (id == R_P2 || id == R_P5) ? 16u : (id == R_P4 || id == R_O) ? 8u : 1u;
+}
 
 // PACKED: packed sequences (rows past a sequence's end are zeroed rather than
 // left to the TMA fill).  FG2: FG^2-GDN learning rates among the gates.  DUMP:
@@ -223,7 +232,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
 
     if (tid == 0) {
 #pragma unroll 1
-        for (int i = 0; i < NBAR; ++i) tc::mbar_init(bar(i), i == R_O ? 8 : 1);
+        for (int i = 0; i < NBAR; ++i) tc::mbar_init(bar(i), ready_count(i));
         tc::mbar_fence_init();
         *abort_s = 0;
     }
@@ -420,6 +429,17 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             compute_sync();
             if (tid == 0) tc::mbar_arrive(bar(id));
         };
+        // each warp signals `id` once its own lanes are done (no CTA barrier)
+        auto warp_signal = [&](uint32_t id) {
+            __syncwarp();
+            if ((tid & 31) == 0) tc::mbar_arrive(bar(id));
+        };
+        // every thread waits on a product's commit itself; a wait that runs out
+        // sets the abort flag (the vote at the chunk's end stops all threads)
+        auto wait_each = [&](uint32_t id, uint32_t parity) {
+            if (!*abort_s && !tc::mbar_wait_bounded(bar(id), parity, WAIT_NS)) *abort_s = 1;
+            tc::fence_after_sync();
+        };
 
 #pragma unroll 1
         for (int t0 = 0; t0 < L; t0 += C, ph ^= 1) {
@@ -446,7 +466,7 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                              if (t0 == 0) return;
                              // the last chunk's state update has read X2 and EB and
                              // finished its O: O -> staging tile for the issuing warp
-                             wait_then_sync(bar(B_ST), ph ^ 1, tid, abort_s);
+                             wait_each(B_ST, ph ^ 1);
                              if (!DUMP) read_o();
                          },
                          [&](int i, float g_m, float g_c) {
@@ -472,10 +492,10 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             }
             tc::fence_async_smem();
             tc::fence_before_sync();
-            signal(R_P2);
+            warp_signal(R_P2);
 
             // ================= P3: the X and S~ products run under the gram readout
-            wait_then_sync(bar(B_G), ph, tid, abort_s);
+            wait_each(B_G, ph);
 
             // ================= P4: read the gram; masked blocks out
             {
@@ -528,13 +548,8 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                 tc::fence_async_smem();
             } else {
                 tc::fence_before_sync();
-                half_sync(3);
-                if (tid == 0) {
-                    tc::mbar_arrive(bar(R_P4));
-                    if (!*abort_s && !tc::mbar_wait_bounded(bar(B_XAU), ph, WAIT_NS)) *abort_s = 1;
-                }
-                half_sync(3);
-                tc::fence_after_sync();
+                warp_signal(R_P4);
+                wait_each(B_XAU, ph);
                 if (quarter < 2) {   // lanes 0-63 of X hold R; each warp takes 64 columns
                     const int c0 = 64 * cb;
                     float vals[32];
@@ -552,10 +567,10 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
                 if (has_next) load_scalars(t0 + C, cur ^ 1);
             }
             tc::fence_before_sync();
-            signal(R_P5);
+            warp_signal(R_P5);
 
             // ================= P6: X += [T - I; 0] R (rows 0-63 become E)
-            wait_then_sync(bar(B_E), ph, tid, abort_s);
+            wait_each(B_E, ph);
 
             // ================= P7: E -> bf16; X += [0; -A_qb] E and S~ -= B"^T E run
             // under the next chunk's decay products
