@@ -157,19 +157,17 @@ __device__ __forceinline__ void stage_row32(uint8_t* box, int r, const float* v)
 }
 
 // Barriers: TMA and tensor-core completions, then the compute threads'
-// "ready" signals to the issuing warp (thread 0 arrives after a compute
-// barrier).  The compute warps issue the TMA loads and stores themselves.
+// "ready" signals to the issuing warp (R_OP, R_GQ: thread 0 arrives after a
+// compute barrier; R_DE, R_DY, R_DA: every compute warp arrives once its own
+// lanes are done).  The compute warps issue the TMA loads and stores
+// themselves.
 enum : uint32_t {
     B_LD, B_G, B_Z1, B_Z3, B_A, B_XY, B_FIN,   // loads / gram / -dE / dY / D~,dU,dA / X,Y / all
     R_OP, R_GQ, R_DE, R_DY, R_DA                // ready for: gram / -dE / dY / D~,dU,dA / X,Y
 };
 static_assert(R_DA + 1 == NBAR, "barrier count");
-
-__device__ __forceinline__ void wait_then_sync(uint32_t bar, uint32_t parity, int tid,
-                                               volatile int* abort_s) {
-    if (tid == 0 && !*abort_s && !tc::mbar_wait_bounded(bar, parity, WAIT_NS)) *abort_s = 1;
-    compute_sync();
-    tc::fence_after_sync();
+__host__ __device__ constexpr uint32_t ready_count(uint32_t id) {
+    return (id == R_DE || id == R_DY || id == R_DA) ? 16u : 1u;
 }
 
 // One row of 32 floats to global memory (16-byte stores).
@@ -224,7 +222,7 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
 
     if (tid == 0) {
 #pragma unroll 1
-        for (int i = 0; i < NBAR; ++i) tc::mbar_init(bar(i), 1);
+        for (int i = 0; i < NBAR; ++i) tc::mbar_init(bar(i), ready_count(i));
         tc::mbar_fence_init();
         *abort_s = 0;
     }
@@ -419,6 +417,17 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             if (tid == 0) tc::mbar_arrive(bar(id));
             return stop;
         };
+        // each warp signals `id` once its own lanes are done (no CTA barrier)
+        auto warp_signal = [&](uint32_t id) {
+            __syncwarp();
+            if ((tid & 31) == 0) tc::mbar_arrive(bar(id));
+        };
+        // every thread waits on a product's commit itself; a wait that runs out
+        // sets the abort flag (the vote at the chunk's end stops all threads)
+        auto wait_each = [&](uint32_t id, uint32_t parity) {
+            if (!*abort_s && !tc::mbar_wait_bounded(bar(id), parity, WAIT_NS)) *abort_s = 1;
+            tc::fence_after_sync();
+        };
 #pragma unroll 1
         for (int c = NC - 1; c >= 0; --c, ph ^= 1) {
             const int t0 = c * C;
@@ -502,7 +511,7 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                 gcs[((size_t)bh * NC + c) * D + tid] = GC[tid];
                 GMN[tid] = GM[tid];
             }
-            wait_then_sync(bar(B_G), ph, tid, abort_s);
+            wait_each(B_G, ph);
             {
                 // rows r of Q' (lanes 0-63) or K' (lanes 64-127); this warp's 32 x 32
                 // block lies below (mode < 0), on (0) or above (> 0) the diagonal
@@ -544,10 +553,7 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                 ut_solve<2>(NS, TS, PS, sm + OFF_TZA, tid - 256);
                 tc::fence_async_smem();
             } else {
-                if (tid == 0 && !*abort_s && !tc::mbar_wait_bounded(bar(B_Z1), ph, WAIT_NS))
-                    *abort_s = 1;
-                half_sync(3);
-                tc::fence_after_sync();
+                wait_each(B_Z1, ph);
                 if (quarter < 2) {  // warps 0, 1, 4, 5: lanes 0-63, 64 columns each
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
@@ -562,10 +568,10 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                 tc::fence_async_smem();
             }
             tc::fence_before_sync();
-            if (signal_or_stop(R_DE)) break;
+            warp_signal(R_DE);
 
             // ================= C4: dY -> rows 64-127 of [dO; dY]
-            wait_then_sync(bar(B_Z3), ph, tid, abort_s);
+            wait_each(B_Z3, ph);
             if (quarter < 2) {
                 float vals[32];
                 tc::tmem_ld32(tmem + lane_off + TM_Z + 32 * cb, vals);
@@ -574,10 +580,10 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             }
             tc::fence_async_smem();
             tc::fence_before_sync();
-            if (signal_or_stop(R_DY)) break;
+            warp_signal(R_DY);
 
             // ================= C5: dA^T masked -> bf16; dU out
-            wait_then_sync(bar(B_A), ph, tid, abort_s);
+            wait_each(B_A, ph);
             if (c > 0) {
                 // the G_C term of the chunk before: rowsum(dS_C * S_C) with dS_C =
                 // g_m D~ and S_C = S~ / g_m (this chunk's start), i.e. rowsum(D~ * S~)
@@ -625,10 +631,10 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             }
             tc::fence_async_smem();
             tc::fence_before_sync();
-            if (signal_or_stop(R_DA)) break;
+            warp_signal(R_DA);
 
             // ================= C6: [XQ' | XK']^T and [YB'; YK'] out
-            wait_then_sync(bar(B_XY), ph, tid, abort_s);
+            wait_each(B_XY, ph);
             {
                 // [XQ' | XK']^T: lane = channel, columns = tokens; this warp's
                 // channels 32q.. and tokens 32(cb & 1).. into a [token][channel] box
@@ -724,18 +730,6 @@ __device__ __forceinline__ void ld_f32x4(const float* p, float* f) {
     const float4 v = *reinterpret_cast<const float4*>(p);
     f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
 }
-// gate of kind `kind` for the four channels of this lane (1.0 for GATE_ONE)
-__device__ __forceinline__ void ld_gate4(const __nv_bfloat16* g, int kind, long long th,
-                                         long long tv, float* f) {
-    if (kind == GDR_GATE_ONE) {
-        f[0] = f[1] = f[2] = f[3] = 1.f;
-    } else if (kind == GDR_GATE_SCALAR) {
-        f[0] = f[1] = f[2] = f[3] = to_f32(g[th]);
-    } else {
-        ld_bf16x4(g + tv, f);
-    }
-}
-
 __global__ void __launch_bounds__(128)
 bwd_epilogue_kernel(int T, int H, int NC, long long n_units, const __nv_bfloat16* __restrict__ q,
                     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
