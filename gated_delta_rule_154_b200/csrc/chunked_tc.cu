@@ -172,7 +172,7 @@ enum : uint32_t {
 };
 static_assert(R_O + 1 == NBAR, "barrier count");
 __host__ __device__ constexpr uint32_t ready_count(uint32_t id) {
-    return (id == R_P2 || id == R_P5) ? 16u : (id == R_P4 || id == R_O) ? 8u : 1u;
+    return (id == R_P2 || id == R_P5 || id == R_E) ? 16u : (id == R_P4 || id == R_O) ? 8u : 1u;
 }
 
 // PACKED: packed sequences (rows past a sequence's end are zeroed rather than
@@ -582,9 +582,8 @@ chunked_tc_kernel(const __grid_constant__ TcMaps maps, int B, int T, int H,
             }
             tc::fence_async_smem();
             tc::fence_before_sync();
-            const bool stop = compute_sync_or(*abort_s != 0);
-            if (tid == 0) tc::mbar_arrive(bar(R_E));
-            if (stop) break;
+            warp_signal(R_E);
+            if (compute_sync_or(*abort_s != 0)) break;
         }
         // (one vote, so that all compute threads agree on whether to finish)
         if (L > 0 && !compute_sync_or(*abort_s != 0)) {
