@@ -368,17 +368,15 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             }
             EXP[cb * D + lane_t] = part;
         }
-        // TMA loads of chunk cc's tiles, spread over the compute warps (tile j
-        // by warp j % 16); B_LD is armed by thread 0 before the compute barrier
-        // that precedes this
+        // TMA loads of chunk cc's tiles: box j = 2 * tile + panel (q, k, do, E,
+        // v, S~, b, a, w).  B_LD is armed by thread 0 before any box of the
+        // round can be issued.
         const uint32_t ld_bytes = (10u + (va ? 2u : 0u) + (vb ? 2u : 0u) + (vw ? 2u : 0u)) *
                                       BOX_BYTES + 2u * 16384u;
-        auto issue_loads = [&](int cc) {
-            if ((tid & 31) != 0) return;
+        auto issue_box = [&](int j, int cc) {
             const int t0l = cc * C;
             const uint32_t bl = bar(B_LD);
-#pragma unroll 1
-            for (int j = warp; j < 18; j += 16) {
+            {
                 const int p = j & 1, x = 64 * p;
                 switch (j >> 1) {
                 case 0: tc::tma_load_4d(sbase + OFF_QK + p * 16384, &maps.q, x, hi, t0l, bi, bl); break;
@@ -392,6 +390,24 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                 default: if (vw) tc::tma_load_4d(sbase + OFF_DE + p * 8192, &maps.w, x, hi, t0l, bi, bl); break;
                 }
             }
+        };
+        // all 18 boxes, box j by warp j % 16
+        auto issue_loads = [&](int cc) {
+            if ((tid & 31) != 0) return;
+#pragma unroll 1
+            for (int j = warp; j < 18; j += 16) issue_box(j, cc);
+        };
+        // The X / Y readout stages X^T in panel 0 of QK and BK (boxes 0, 2, 12
+        // and 14: q, k, b, a), Y where no box lands.  The other 14 boxes go out
+        // as soon as the X / Y products are done (warps 0-13, one each), these
+        // four after the stores have read their tiles (warps 0-3).
+        auto issue_early = [&](int cc) {
+            if ((tid & 31) != 0 || warp >= 14) return;
+            issue_box(warp < 2 ? 2 * warp + 1 : warp < 10 ? warp + 2 : warp < 12 ? 2 * warp - 7 : warp + 4, cc);
+        };
+        auto issue_late = [&](int cc) {
+            if ((tid & 31) != 0 || warp >= 4) return;
+            issue_box(warp < 2 ? 2 * warp : 8 + 2 * warp, cc);
         };
         int ld_out = 0;          // (thread 0) a load round issued and not yet waited for
         uint32_t ld_ph = 0;      // its phase parity
@@ -584,6 +600,13 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
 
             // ================= C5: dA^T masked -> bf16; dU out
             wait_each(B_A, ph);
+            // arm B_LD for the next chunk's boxes: they are issued only after the
+            // X / Y products, which wait for every warp's R_DA below
+            if (tid == 0 && c > 0) {
+                tc::mbar_arrive_expect_tx(bar(B_LD), ld_bytes);
+                ld_out = 1;
+                ld_ph = ph ^ 1;
+            }
             if (c > 0) {
                 // the G_C term of the chunk before: rowsum(dS_C * S_C) with dS_C =
                 // g_m D~ and S_C = S~ / g_m (this chunk's start), i.e. rowsum(D~ * S~)
@@ -633,8 +656,29 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             tc::fence_before_sync();
             warp_signal(R_DA);
 
-            // ================= C6: [XQ' | XK']^T and [YB'; YK'] out
+            // ================= C6: [YB'; YK'] and [XQ' | XK']^T out
             wait_each(B_XY, ph);
+            // the next chunk's boxes that no staged output uses
+            if (c > 0) issue_early(c - 1);
+            {
+                // [YB'; YK']: lane = token, this warp's 32 channels 32cb..; staged
+                // where no box of the next chunk lands: the dY rows of [dO; dY]
+                // (lanes 0-63), or this warp's own dU box once its store has read it
+                float vals[32];
+                tc::tmem_ld32(tmem + lane_off + TM_G + 32 * cb, vals);
+                tc::tmem_wait_ld();
+                const int bx = 2 * cb + (quarter & 1);
+                uint32_t box;
+                if (quarter < 2) {
+                    box = OFF_DOY + (bx >> 2) * 16384 + 8192 + (bx & 3) * SBOX;
+                } else {
+                    if ((tid & 31) == 0) tc::bulk_wait_read();
+                    __syncwarp();
+                    box = box_du(bx);
+                }
+                stage_row32(sm + box, tid & 31, vals);
+                store_box(quarter < 2 ? &maps.yb : &maps.yk, box, 32 * cb, t0 + 32 * (quarter & 1));
+            }
             {
                 // [XQ' | XK']^T: lane = channel, columns = tokens; this warp's
                 // channels 32q.. and tokens 32(cb & 1).. into a [token][channel] box
@@ -651,27 +695,15 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                         __float2bfloat16_rn(vals[x]);
                 store_box(cb < 2 ? &maps.xq : &maps.xk, box, 32 * quarter, t0 + 32 * (cb & 1));
             }
-            {
-                // [YB'; YK']: lane = token, this warp's 32 channels 32cb..
-                float vals[32];
-                tc::tmem_ld32(tmem + lane_off + TM_G + 32 * cb, vals);
-                tc::tmem_wait_ld();
-                const uint32_t box = (quarter < 2 ? OFF_DOY : OFF_DS) + SBOX * (2 * cb + (quarter & 1));
-                stage_row32(sm + box, tid & 31, vals);
-                store_box(quarter < 2 ? &maps.yb : &maps.yk, box, 32 * cb, t0 + 32 * (quarter & 1));
-            }
-            // this warp's stores (dU, X, Y) have read their boxes
+            // this warp's stores (dU, Y, X) have read their boxes
             if ((tid & 31) == 0) tc::bulk_wait_read();
             __syncwarp();
             tc::fence_before_sync();
-            if (tid == 0 && c > 0) tc::mbar_arrive_expect_tx(bar(B_LD), ld_bytes);
-            if (compute_sync_or(*abort_s != 0)) break;
-            // the next chunk's tiles
-            if (c > 0) {
-                issue_loads(c - 1);
-                ld_out = 1;
-                ld_ph = ph ^ 1;
-            }
+            const bool stop = compute_sync_or(*abort_s != 0);
+            // the boxes where X^T was staged (also when stopping: B_LD is armed
+            // for every box of the round)
+            if (c > 0) issue_late(c - 1);
+            if (stop) break;
         }
         // nothing this CTA started may still be in flight when it exits
         if (tid == 0 && ld_out) tc::mbar_wait_bounded(bar(B_LD), ld_ph, WAIT_NS);
@@ -714,13 +746,6 @@ __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
     return x;
-}
-__device__ __forceinline__ void ld_bf16x4(const __nv_bfloat16* p, float* f) {
-    const uint2 u = *reinterpret_cast<const uint2*>(p);
-    f[0] = __uint_as_float(u.x << 16);
-    f[1] = __uint_as_float(u.x & 0xFFFF0000u);
-    f[2] = __uint_as_float(u.y << 16);
-    f[3] = __uint_as_float(u.y & 0xFFFF0000u);
 }
 __device__ __forceinline__ void st_bf16x4(__nv_bfloat16* p, const float* f) {
     *reinterpret_cast<uint2*>(p) =
