@@ -131,20 +131,20 @@ constexpr uint32_t BOX_BYTES = 64 * 128;     // one 64 x 64 bf16 TMA box
 struct BwMaps {
     CUtensorMap q, k, v, a, b, w, dout, e;  // bf16 inputs (a/b/w only for vector gates)
     CUtensorMap sst;                        // the forward's S~ tiles
-    CUtensorMap xq, xk, yk, yb, du;         // bf16 intermediates, 32 x 32 boxes
+    CUtensorMap xq, xk;                     // bf16 intermediates, 32 x 32 boxes
+    __nv_bfloat16 *yk, *yb, *du;            // bf16 intermediates written row by row
 };
 
-// Staging of the bf16 intermediates for their TMA stores: 2 KB boxes of 32
-// tokens x 32 channels (64-byte rows, 64-byte swizzle: 16-byte chunk c of row
-// r at c ^ ((r / 2) % 4)), each written and stored by one compute warp.
-// XQ', XK', YB', YK' go where [Q'; K'], [B"; K"], [dO; dY] and dS~ were, once
-// the chunk's last products are done (box 2p + h: channels 32p.., tokens
-// 32h..); dU goes into the A_qb/A_qk tile, free once the product that reads
-// it is done.
+// XQ' and XK' (lane = channel in tensor memory) are transposed through 2 KB
+// staging boxes of 32 tokens x 32 channels (64-byte rows, 64-byte swizzle:
+// 16-byte chunk c of row r at c ^ ((r / 2) % 4)), each written and stored by
+// TMA by one compute warp, in tiles that no load of the next chunk uses.
+// YB', YK' and dU (lane = token) leave from registers, one 64-byte row piece
+// per thread.
 constexpr uint32_t SBOX = 2048;   // bytes of one staging box
-__device__ __forceinline__ uint32_t box_du(int bx) { return OFF_GQ + SBOX * bx; }
-// one row of 32 channels of a box, rounded to bf16, as four 16-byte stores
-__device__ __forceinline__ void stage_row32(uint8_t* box, int r, const float* v) {
+// 32 values rounded to bf16, as four 16-byte stores to p (64-byte aligned)
+__device__ __forceinline__ void st_row32_bf16(__nv_bfloat16* p, const float* v) {
+    uint4* d = reinterpret_cast<uint4*>(p);
 #pragma unroll
     for (int c16 = 0; c16 < 4; ++c16) {
         uint4 u;
@@ -152,7 +152,7 @@ __device__ __forceinline__ void stage_row32(uint8_t* box, int r, const float* v)
         u.y = tc::pack_bf16x2(v[8 * c16 + 2], v[8 * c16 + 3]);
         u.z = tc::pack_bf16x2(v[8 * c16 + 4], v[8 * c16 + 5]);
         u.w = tc::pack_bf16x2(v[8 * c16 + 6], v[8 * c16 + 7]);
-        *reinterpret_cast<uint4*>(box + 64 * r + ((c16 ^ ((r >> 1) & 3)) << 4)) = u;
+        d[c16] = u;
     }
 }
 
@@ -369,8 +369,8 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             EXP[cb * D + lane_t] = part;
         }
         // TMA loads of chunk cc's tiles: box j = 2 * tile + panel (q, k, do, E,
-        // v, S~, b, a, w).  B_LD is armed by thread 0 before any box of the
-        // round can be issued.
+        // v, S~, b, a, w), spread over the compute warps.  B_LD is armed by
+        // thread 0 before any box of the round can be issued.
         const uint32_t ld_bytes = (10u + (va ? 2u : 0u) + (vb ? 2u : 0u) + (vw ? 2u : 0u)) *
                                       BOX_BYTES + 2u * 16384u;
         auto issue_box = [&](int j, int cc) {
@@ -397,18 +397,6 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
 #pragma unroll 1
             for (int j = warp; j < 18; j += 16) issue_box(j, cc);
         };
-        // The X / Y readout stages X^T in panel 0 of QK and BK (boxes 0, 2, 12
-        // and 14: q, k, b, a), Y where no box lands.  The other 14 boxes go out
-        // as soon as the X / Y products are done (warps 0-13, one each), these
-        // four after the stores have read their tiles (warps 0-3).
-        auto issue_early = [&](int cc) {
-            if ((tid & 31) != 0 || warp >= 14) return;
-            issue_box(warp < 2 ? 2 * warp + 1 : warp < 10 ? warp + 2 : warp < 12 ? 2 * warp - 7 : warp + 4, cc);
-        };
-        auto issue_late = [&](int cc) {
-            if ((tid & 31) != 0 || warp >= 4) return;
-            issue_box(warp < 2 ? 2 * warp : 8 + 2 * warp, cc);
-        };
         int ld_out = 0;          // (thread 0) a load round issued and not yet waited for
         uint32_t ld_ph = 0;      // its phase parity
         if (NC > 0) {
@@ -419,6 +407,8 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
         }
         // this warp's 32 x 32 box of a staged output out by TMA (rows past T
         // are not stored; a box starting past T is not issued)
+        // element offset of token tok of this (batch, head) in a [B, T, H, 128] tensor
+        auto row_off = [&](int tok) { return (((size_t)bi * T + tok) * H + hi) * D; };
         auto store_box = [&](const CUtensorMap* m, uint32_t box, int ch0, int tok0) {
             tc::fence_async_smem();
             __syncwarp();
@@ -644,13 +634,12 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                 }
                 tc::store_row32_bf16(sm + OFF_DAT + (cb >> 1) * 16384, lane_t, cb & 1, vals);
             }
-            if (quarter >= 2) {   // dU: this warp's 32 tokens x 32 channels
+            if (quarter >= 2) {   // dU: token lane_t - 64, this warp's 32 channels
                 float vals[32];
                 tc::tmem_ld32(tmem + lane_off + TM_Z + 32 * cb, vals);
                 tc::tmem_wait_ld();
-                const int bx = 2 * cb + (quarter & 1);
-                stage_row32(sm + box_du(bx), tid & 31, vals);
-                store_box(&maps.du, box_du(bx), 32 * cb, t0 + 32 * (quarter & 1));
+                const int tok = t0 + (lane_t & 63);
+                if (tok < T) st_row32_bf16(maps.du + row_off(tok) + 32 * cb, vals);
             }
             tc::fence_async_smem();
             tc::fence_before_sync();
@@ -658,34 +647,27 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
 
             // ================= C6: [YB'; YK'] and [XQ' | XK']^T out
             wait_each(B_XY, ph);
-            // the next chunk's boxes that no staged output uses
-            if (c > 0) issue_early(c - 1);
+            // the next chunk's tiles: nothing below stages into their tiles
+            if (c > 0) issue_loads(c - 1);
             {
-                // [YB'; YK']: lane = token, this warp's 32 channels 32cb..; staged
-                // where no box of the next chunk lands: the dY rows of [dO; dY]
-                // (lanes 0-63), or this warp's own dU box once its store has read it
+                // [YB'; YK']: lane = token, this warp's 32 channels 32cb..
                 float vals[32];
                 tc::tmem_ld32(tmem + lane_off + TM_G + 32 * cb, vals);
                 tc::tmem_wait_ld();
-                const int bx = 2 * cb + (quarter & 1);
-                uint32_t box;
-                if (quarter < 2) {
-                    box = OFF_DOY + (bx >> 2) * 16384 + 8192 + (bx & 3) * SBOX;
-                } else {
-                    if ((tid & 31) == 0) tc::bulk_wait_read();
-                    __syncwarp();
-                    box = box_du(bx);
-                }
-                stage_row32(sm + box, tid & 31, vals);
-                store_box(quarter < 2 ? &maps.yb : &maps.yk, box, 32 * cb, t0 + 32 * (quarter & 1));
+                const int tok = t0 + (lane_t & 63);
+                if (tok < T) st_row32_bf16((quarter < 2 ? maps.yb : maps.yk) + row_off(tok) + 32 * cb, vals);
             }
             {
                 // [XQ' | XK']^T: lane = channel, columns = tokens; this warp's
-                // channels 32q.. and tokens 32(cb & 1).. into a [token][channel] box
+                // channels 32q.. and tokens 32(cb & 1).. into a [token][channel]
+                // box, staged where no load lands: the dY rows of [dO; dY]
+                // (XQ') and the [A_qb | A_qk] tile (XK')
                 float vals[32];
                 tc::tmem_ld32(tmem + lane_off + TM_Z + 32 * cb, vals);
                 tc::tmem_wait_ld();
-                const uint32_t box = (cb < 2 ? OFF_QK : OFF_BK) + SBOX * (2 * quarter + (cb & 1));
+                const int bx = 2 * quarter + (cb & 1);
+                const uint32_t box = cb < 2 ? OFF_DOY + (bx >> 2) * 16384 + 8192 + (bx & 3) * SBOX
+                                            : OFF_GQ + bx * SBOX;
                 const int cl = tid & 31;
                 uint8_t* dst = sm + box + 2 * (cl & 7);
 #pragma unroll
@@ -695,15 +677,12 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                         __float2bfloat16_rn(vals[x]);
                 store_box(cb < 2 ? &maps.xq : &maps.xk, box, 32 * quarter, t0 + 32 * (cb & 1));
             }
-            // this warp's stores (dU, Y, X) have read their boxes
+            // this warp's X^T store has read its box (the next chunk rewrites
+            // the dY rows and the [A_qb | A_qk] tile)
             if ((tid & 31) == 0) tc::bulk_wait_read();
             __syncwarp();
             tc::fence_before_sync();
-            const bool stop = compute_sync_or(*abort_s != 0);
-            // the boxes where X^T was staged (also when stopping: B_LD is armed
-            // for every box of the round)
-            if (c > 0) issue_late(c - 1);
-            if (stop) break;
+            if (compute_sync_or(*abort_s != 0)) break;
         }
         // nothing this CTA started may still be in flight when it exits
         if (tid == 0 && ld_out) tc::mbar_wait_bounded(bar(B_LD), ld_ph, WAIT_NS);
@@ -948,10 +927,10 @@ cudaError_t launch_backward_tc(const gdr_desc& d, const void* const* in, const f
         ok = tc_map_bf16(&maps.w, in[5], B, T, H, T);
     ok = ok && tc_map_bf16_box32(&maps.xq, ws.pre[0], B, T, H) &&
          tc_map_bf16_box32(&maps.xk, ws.pre[1], B, T, H) &&
-         tc_map_bf16_box32(&maps.yk, ws.pre[2], B, T, H) &&
-         tc_map_bf16_box32(&maps.yb, ws.pre[3], B, T, H) &&
-         tc_map_bf16_box32(&maps.du, ws.pre[4], B, T, H) &&
          tc_map_state_bf16(&maps.sst, ws.states, (long long)B * H * NC);
+    maps.yk = static_cast<__nv_bfloat16*>(ws.pre[2]);
+    maps.yb = static_cast<__nv_bfloat16*>(ws.pre[3]);
+    maps.du = static_cast<__nv_bfloat16*>(ws.pre[4]);
     if (!ok) return cudaErrorInvalidValue;
 
     const bool fg2 = d.erase == GDR_GATE_FG2 || d.write == GDR_GATE_FG2;
