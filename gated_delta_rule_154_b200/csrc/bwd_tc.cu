@@ -507,6 +507,10 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
             }
             tc::tmem_wait_st();
             tc::fence_async_smem();
+            // the last chunk's XQ' / XK' stores have read their boxes (the dY
+            // rows and the [A_qb | A_qk] tile are rewritten after this barrier)
+            if ((tid & 31) == 0) tc::bulk_wait_read();
+            __syncwarp();
             tc::fence_before_sync();
             if (signal_or_stop(R_OP)) break;
 
@@ -677,10 +681,7 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
                         __float2bfloat16_rn(vals[x]);
                 store_box(cb < 2 ? &maps.xq : &maps.xk, box, 32 * quarter, t0 + 32 * (cb & 1));
             }
-            // this warp's X^T store has read its box (the next chunk rewrites
-            // the dY rows and the [A_qb | A_qk] tile)
-            if ((tid & 31) == 0) tc::bulk_wait_read();
-            __syncwarp();
+            // (the X^T stores are waited for before the next chunk's R_OP)
             tc::fence_before_sync();
             if (compute_sync_or(*abort_s != 0)) break;
         }
