@@ -53,17 +53,28 @@ def measured_traffic(name: str = "chunked_tc_gdn2_bf16_T1024.json"):
     """DRAM bytes per launch of the bench's prefill workload from the committed
     ncu counters (a JSON data file under profiles/), or None when the kernel
     sources it names changed since that capture."""
-    import hashlib
     path = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(path):
         return None, None
     rec = json.load(open(path))
-    h = hashlib.sha256()
-    for rel in rec.get("sources", []):
-        h.update(open(os.path.join(ROOT, rel), "rb").read())
-    if rec.get("source_sha256") != h.hexdigest():
+    if rec.get("code_sha256") != code_digest(rec.get("sources", [])):
         return None, rec.get("note")
     return int(rec["traffic_bytes_per_launch"]), rec.get("note")
+
+
+def code_digest(sources) -> str:
+    """sha256 of the listed sources' code with comments and blank space
+    removed: a comment edit leaves the counters attached to the code they
+    were taken from, any change to the code detaches them."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for rel in sources:
+        src = open(os.path.join(ROOT, rel)).read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
+    return h.hexdigest()
 
 
 def prefill_bytes(wl) -> int:

@@ -33,8 +33,8 @@
 // instantiation (every chunk's S~ and E in bf16, exactly the tiles its own
 // products read, and S_T in float32); bwd_tc_kernel, one CTA per (batch,
 // head) walking the chunks from the last, which carries D~ in tensor memory
-// and writes XQ', XK', YK', YB', dU (bf16, by TMA store) and per chunk
-// the G_C terms and gc; and bwd_epilogue_kernel, one warp per (batch, head,
+// and writes XQ', XK' (bf16, by TMA store), YK', YB', dU (bf16, from
+// registers) and per chunk the G_C terms and gc; and bwd_epilogue_kernel, one warp per (batch, head,
 // chunk), which forms the six gradients from them and the raw inputs (the
 // reverse cumulative sum for da).  The G_C term of a chunk is rowsum(D~ S~)
 // of the chunk after it (dS_C = g_m D~ and S_C = S~ / g_m there), and

@@ -32,14 +32,18 @@
 // kernel sets GDR_ERR_RANGE in the device error word (the float32 CUDA-core
 // kernel, chunk <= 32, has no such limit).
 //
-// One CTA (16 warps) owns one (batch, head) and walks its chunks in order;
-// S~ stays in float32 in tensor memory (lane = key channel) for the whole
-// sequence.  Raw q/k/v and vector gates arrive by TMA as 64-token x
-// 64-channel boxes, 128-byte swizzled, i.e. already in the operand layout of
-// tc_common.cuh, each prefetched as soon as its destination is free; o leaves
-// by a TMA store.  Products are tcgen05.mma issued by one thread; the decay
-// products, the UT solve and the conversions run on the CUDA cores with
-// 16-byte shared-memory accesses.
+// One CTA (16 compute warps and one issuing warp) owns one (batch, head)
+// and walks its chunks in order; S~ stays in float32 in tensor memory (lane =
+// key channel) for the whole sequence.  Raw q/k/v and vector gates arrive by
+// TMA as 64-token x 64-channel boxes, 128-byte swizzled, i.e. already in the
+// operand layout of tc_common.cuh, each prefetched as soon as its
+// destination is free; o leaves by a TMA store.  Products are tcgen05.mma
+// issued by one thread of the issuing warp; the decay products, the UT solve
+// and the conversions run on the CUDA cores with 8- and 16-byte
+// shared-memory accesses.  The compute threads wait on the TMA and product
+// barriers themselves and tell the issuing warp per warp that an operand set
+// is in place; a CTA barrier stands only where data crosses warps, and one
+// vote per chunk stops all threads together after a wait ran out.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
