@@ -149,10 +149,11 @@ __device__ __forceinline__ void issue_v(const TcMaps& m, uint32_t sbase, int t0,
         tc::tma_load_4d(sbase + OFF_U + p * 8192, &m.v, 64 * p, hi, t0, bi, bar);
 }
 
-// Arrivals that complete a "ready" barrier: one per compute warp for the
-// operand sets whose writers only need their own warp's work in place, eight
-// for R_P4 and R_O (the warps that write them), else compute thread 0 after a
-// compute barrier.
+// Arrivals that complete a "ready" barrier: one per compute warp (16) for
+// R_P2, R_P5 and R_E, whose operands each warp writes for itself; eight for
+// R_P4 and R_O (the warps that write them); one for R_OP, from compute thread
+// 0 after a compute barrier (the state scales the operand pass leaves are
+// read across warps right after it).
 __host__ __device__ constexpr uint32_t ready_count(uint32_t id);
 
 // Compute thread 0 waits on `bar`; the compute barrier that follows releases
