@@ -376,19 +376,17 @@ bwd_tc_kernel(const __grid_constant__ BwMaps maps, int B, int T, int H,
         auto issue_box = [&](int j, int cc) {
             const int t0l = cc * C;
             const uint32_t bl = bar(B_LD);
-            {
-                const int p = j & 1, x = 64 * p;
-                switch (j >> 1) {
-                case 0: tc::tma_load_4d(sbase + OFF_QK + p * 16384, &maps.q, x, hi, t0l, bi, bl); break;
-                case 1: tc::tma_load_4d(sbase + OFF_QK + p * 16384 + 8192, &maps.k, x, hi, t0l, bi, bl); break;
-                case 2: tc::tma_load_4d(sbase + OFF_DOY + p * 16384, &maps.dout, x, hi, t0l, bi, bl); break;
-                case 3: tc::tma_load_4d(sbase + OFF_EIN + p * 8192, &maps.e, x, hi, t0l, bi, bl); break;
-                case 4: tc::tma_load_4d(sbase + OFF_UIN + p * 8192, &maps.v, x, hi, t0l, bi, bl); break;
-                case 5: tc::tma_load_4d(sbase + OFF_DS + p * 16384, &maps.sst, x, 0, bh * NC + cc, 0, bl); break;
-                case 6: if (vb) tc::tma_load_4d(sbase + OFF_BK + p * 16384, &maps.b, x, hi, t0l, bi, bl); break;
-                case 7: if (va) tc::tma_load_4d(sbase + OFF_BK + p * 16384 + 8192, &maps.a, x, hi, t0l, bi, bl); break;
-                default: if (vw) tc::tma_load_4d(sbase + OFF_DE + p * 8192, &maps.w, x, hi, t0l, bi, bl); break;
-                }
+            const int p = j & 1, x = 64 * p;
+            switch (j >> 1) {
+            case 0: tc::tma_load_4d(sbase + OFF_QK + p * 16384, &maps.q, x, hi, t0l, bi, bl); break;
+            case 1: tc::tma_load_4d(sbase + OFF_QK + p * 16384 + 8192, &maps.k, x, hi, t0l, bi, bl); break;
+            case 2: tc::tma_load_4d(sbase + OFF_DOY + p * 16384, &maps.dout, x, hi, t0l, bi, bl); break;
+            case 3: tc::tma_load_4d(sbase + OFF_EIN + p * 8192, &maps.e, x, hi, t0l, bi, bl); break;
+            case 4: tc::tma_load_4d(sbase + OFF_UIN + p * 8192, &maps.v, x, hi, t0l, bi, bl); break;
+            case 5: tc::tma_load_4d(sbase + OFF_DS + p * 16384, &maps.sst, x, 0, bh * NC + cc, 0, bl); break;
+            case 6: if (vb) tc::tma_load_4d(sbase + OFF_BK + p * 16384, &maps.b, x, hi, t0l, bi, bl); break;
+            case 7: if (va) tc::tma_load_4d(sbase + OFF_BK + p * 16384 + 8192, &maps.a, x, hi, t0l, bi, bl); break;
+            default: if (vw) tc::tma_load_4d(sbase + OFF_DE + p * 8192, &maps.w, x, hi, t0l, bi, bl); break;
             }
         };
         // all 18 boxes, box j by warp j % 16
