@@ -30,6 +30,26 @@ def test_prefill_bytes_per_token_head():
     assert bench.prefill_bytes(kda) == kda.B * kda.T * kda.H * 1282 + 4 * kda.B * kda.H * 128 * 128
 
 
+def test_capture_digest_follows_code_not_comments(tmp_path, monkeypatch):
+    """The committed ncu counters stay attached to the kernel code they were
+    taken from: comments and blank space do not change the digest, code does."""
+    src = tmp_path / "k.cu"
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    src.write_text("int f(int x) {  // one\n  return x + 1; /* two */\n}\n")
+    d0 = bench.code_digest(["k.cu"])
+    src.write_text("// a header\nint f(int x)\n{\n    return x + 1;\n}\n")
+    assert bench.code_digest(["k.cu"]) == d0
+    src.write_text("int f(int x) { return x + 2; }\n")
+    assert bench.code_digest(["k.cu"]) != d0
+
+
+def test_committed_capture_matches_the_prefill_code():
+    traffic, note = bench.measured_traffic()
+    assert traffic is not None, note
+    # within a few percent of the algorithmic bytes of the bench launch
+    assert abs(traffic / bench.prefill_bytes(W.WORKLOADS["gdn2_bf16"]) - 1) < 0.05
+
+
 def test_decode_bytes_per_head_step():
     wl = W.WORKLOADS["decode_bf16"]
     assert bench.decode_bytes(wl) == wl.B * wl.H * 132864
