@@ -10,8 +10,9 @@ N(0, 0.1) initial state.  `value` is tokens/s (B*T per step) over all ranks.
 The same line carries the decode step's HBM bandwidth (batch 256, H = 32,
 d = 128, float32 state read and written in place), the roofline fraction of
 the prefill kernel, the backward pass on the same inputs (training: the
-gradients of every input, measured against the CUDA cores' float32 FMA
-peak), the float64 oracle's throughput on this host, the end-to-end figure
+gradients of every input, its issued tensor flops against the bf16 tensor
+peak, or the CUDA cores' float32 FMA peak for float32 inputs), the float64
+oracle's throughput on this host, the end-to-end figure
 through host buffers, and the SM clocks seen while timing.
 
 Under torchrun each rank runs its own B = 8 batch (weak scaling, no
