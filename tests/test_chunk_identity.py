@@ -91,3 +91,44 @@ def test_chunked_scalar_decay_and_shared_beta():
     o, s = chunked_reference(q, k, v, a, b, w, s0, 32)
     assert np.max(np.abs(o - o_ref)) / np.max(np.abs(o_ref)) < 1e-12
     assert np.max(np.abs(s - s_ref)) / np.max(np.abs(s_ref)) < 1e-12
+
+
+def _block_inverse(N, n0):
+    """T = (I + N)^{-1} for strictly lower N (size a power of two times n0)
+    by the order the kernels use: forward substitution on the n0 x n0
+    diagonal blocks, then the 2 x 2 block step T21 = -T2 (N21 T1) at every
+    doubling of the block size."""
+    n = N.shape[0]
+    T = np.zeros_like(N)
+    for i in range(0, n, n0):
+        blk = N[i:i + n0, i:i + n0]
+        for c in range(n0):
+            x = np.zeros(n0)
+            for r in range(n0):
+                x[r] = (1.0 if r == c else 0.0) - blk[r, :r] @ x[:r]
+            T[i:i + n0, i + c] = x
+    m = n0
+    while m < n:
+        for i in range(0, n, 2 * m):
+            T1, T2 = T[i:i + m, i:i + m], T[i + m:i + 2 * m, i + m:i + 2 * m]
+            T[i + m:i + 2 * m, i:i + m] = -T2 @ (N[i + m:i + 2 * m, i:i + m] @ T1)
+        m *= 2
+    return T
+
+
+@pytest.mark.parametrize("n0", [8, 16])
+def test_ut_transform_block_recursion(n0):
+    """The UT transform T = (I + A_kb)^{-1} of a 64-token chunk, evaluated as
+    the kernels do (8 x 8 substitution and block steps at 8, 16 and 32 rows;
+    16 x 16 substitution as before), equals the direct inverse, and T21 is
+    the only block that changes per level (T stays unit lower triangular)."""
+    rng = np.random.default_rng(5)
+    k = rng.normal(size=(64, 128))
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    gam = np.cumprod(np.exp(-np.log1p(np.exp(rng.normal(-4, 1, size=(64, 128))))), axis=0)
+    beta = 1 / (1 + np.exp(-rng.normal(size=(64, 128))))
+    N = np.tril((gam * k) @ (beta * k / gam).T, -1)
+    T = _block_inverse(N, n0)
+    assert np.allclose(T, np.linalg.inv(np.eye(64) + N), rtol=0, atol=1e-12)
+    assert np.array_equal(np.triu(T, 1), np.zeros((64, 64)))
+    assert np.allclose(np.diag(T), 1.0)
