@@ -227,13 +227,15 @@ def test_backward_varlen_workspace_and_checks(lib):
         _desc(B=1, T=0), 2)) == _lib.OK
 
 
-@pytest.mark.parametrize("chunk,T", [(64, 40000), (32, 32 * 1024)])
-def test_noalloc_refuses_a_problem_larger_than_its_scratch_before_any_cuda_call(lib, chunk, T):
+@pytest.mark.parametrize("dtype,T", [("bf16", 40000), ("f32", 32 * 1024)])
+def test_noalloc_refuses_a_problem_larger_than_its_scratch_before_any_cuda_call(lib, dtype, T):
     """The no-allocation backward refuses a problem whose workspace exceeds its
     64 MiB scratch with GDR_ERR_WORKSPACE, on the host, before any CUDA call
-    (so also here, without a GPU): chunk 64 takes the tensor-core path (about
-    2 KiB per token-head), chunk 32 the mma.sync one (64 KiB per 32 tokens)."""
-    desc = _lib.GdrDesc(B=1, T=T, H=1, dk=128, dv=128, chunk=chunk, in_dtype=_lib.BF16,
+    (so also here, without a GPU): bf16 at d = 128 takes the tensor-core path
+    (about 2 KiB per token-head), float32 the mma.sync one (64 KiB per 32
+    tokens and head)."""
+    desc = _lib.GdrDesc(B=1, T=T, H=1, dk=128, dv=128, chunk=64,
+                        in_dtype=_lib.BF16 if dtype == "bf16" else _lib.F32,
                         decay=_lib.GATE_VECTOR, erase=_lib.GATE_VECTOR, write=_lib.GATE_VECTOR)
     assert _lib.backward_workspace_size(desc) > _lib.NOALLOC_SCRATCH_BYTES
     p = 1 << 20   # never dereferenced
